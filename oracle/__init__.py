@@ -1,0 +1,157 @@
+"""float64 CPU oracle of the mesh rasterizer hot path (TEST INFRASTRUCTURE ONLY).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference``
+legs of ``bench.py`` may import this package.  The product path never does.
+
+The arithmetic lives in ``oracle.c`` (plain C, float64, no SIMD, no fast-math); this
+module compiles it with gcc when needed and marshals numpy arrays through ctypes.
+Each function names the step of the definition (see the header of ``oracle.c``) it
+follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc -O2, strict IEEE: no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+                               "-shared", "-fPIC", "-pthread", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i64, i32, f64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+        lib.oracle_rasterize_fwd.argtypes = [P, i64, P, i64, P, P, i32, i32, i32, f64, i32, i32,
+                                             P, i64, P, P, P, P, P, i32]
+        lib.oracle_rasterize_fwd.restype = ctypes.c_int
+        lib.oracle_silhouette_fwd.argtypes = [P, P, i64, i32, f64, P]
+        lib.oracle_silhouette_fwd.restype = None
+        lib.oracle_silhouette_bwd.argtypes = [P, P, P, i64, i32, f64, P]
+        lib.oracle_silhouette_bwd.restype = None
+        lib.oracle_rasterize_bwd.argtypes = [P, i64, P, i64, P, i32, i32, i32, i32, i32, P, P, P, P, i32]
+        lib.oracle_rasterize_bwd.restype = ctypes.c_int
+        lib.oracle_probe.argtypes = [f64, f64, P, i32, P]
+        lib.oracle_probe.restype = None
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return len(os.sched_getaffinity(0))
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def rasterize_fwd(verts, faces, first, num, H, W, blur_radius, K, perspective_correct=False,
+                  pixels=None, nthreads=None, exempt=True):
+    """Steps 1-10: per pixel the K nearest candidate faces.
+
+    Returns ``(pix_to_face int64, zbuf f64, bary f64, dists f64, exempt uint8)`` shaped
+    ``(N, H, W, K[, 3])``, or ``(P, K[, 3])`` when ``pixels`` lists flat pixel ids
+    ``(n*H + i)*W + j``.  ``exempt`` bit 0 = depth near-tie (E1), bit 1 = candidacy on
+    its threshold (E2).
+    """
+    lib = _load()
+    verts = _c(verts, np.float32)
+    faces = _c(faces, np.int64)
+    first = _c(first, np.int64)
+    num = _c(num, np.int64)
+    N = int(first.shape[0])
+    if pixels is None:
+        lead = (N, H, W)
+        pix = None
+        npix = N * H * W
+    else:
+        pix = _c(pixels, np.int64)
+        lead = (pix.shape[0],)
+        npix = pix.shape[0]
+    p2f = np.empty(lead + (K,), np.int64)
+    zbuf = np.empty(lead + (K,), np.float64)
+    bary = np.empty(lead + (K, 3), np.float64)
+    dists = np.empty(lead + (K,), np.float64)
+    ex = np.zeros(lead, np.uint8) if exempt else None
+    rc = lib.oracle_rasterize_fwd(_ptr(verts), verts.shape[0], _ptr(faces), faces.shape[0],
+                                  _ptr(first), _ptr(num), N, H, W, float(blur_radius), K,
+                                  int(bool(perspective_correct)), _ptr(pix), npix,
+                                  _ptr(p2f), _ptr(zbuf), _ptr(bary), _ptr(dists), _ptr(ex),
+                                  nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_rasterize_fwd: invalid arguments")
+    return p2f, zbuf, bary, dists, ex
+
+
+def silhouette_fwd(pix_to_face, dists, sigma):
+    """Step 11: alpha = 1 - prod(1 - sigmoid(-dist / sigma)) over valid slots."""
+    lib = _load()
+    p2f = _c(pix_to_face, np.int64)
+    d = _c(dists, np.float64)
+    K = p2f.shape[-1]
+    alpha = np.empty(p2f.shape[:-1], np.float64)
+    lib.oracle_silhouette_fwd(_ptr(p2f), _ptr(d), alpha.size, K, float(sigma), _ptr(alpha))
+    return alpha
+
+
+def silhouette_bwd(grad_alpha, pix_to_face, dists, sigma):
+    """Step 12: dL/ddists from dL/dalpha."""
+    lib = _load()
+    p2f = _c(pix_to_face, np.int64)
+    d = _c(dists, np.float64)
+    g = _c(grad_alpha, np.float64)
+    K = p2f.shape[-1]
+    out = np.empty(p2f.shape, np.float64)
+    lib.oracle_silhouette_bwd(_ptr(g), _ptr(p2f), _ptr(d), g.size, K, float(sigma), _ptr(out))
+    return out
+
+
+def rasterize_bwd(verts, faces, pix_to_face, perspective_correct=False, grad_zbuf=None,
+                  grad_bary=None, grad_dists=None, nthreads=None):
+    """Step 13: dL/dverts (V x 3, float64) from gradients of zbuf / bary / dists (any may be None)."""
+    lib = _load()
+    verts = _c(verts, np.float32)
+    faces = _c(faces, np.int64)
+    p2f = _c(pix_to_face, np.int64)
+    N, H, W, K = p2f.shape
+    gz = None if grad_zbuf is None else _c(grad_zbuf, np.float64)
+    gb = None if grad_bary is None else _c(grad_bary, np.float64)
+    gd = None if grad_dists is None else _c(grad_dists, np.float64)
+    out = np.empty(verts.shape, np.float64)
+    rc = lib.oracle_rasterize_bwd(_ptr(verts), verts.shape[0], _ptr(faces), faces.shape[0], _ptr(p2f),
+                                  N, H, W, K, int(bool(perspective_correct)), _ptr(gz), _ptr(gb), _ptr(gd),
+                                  _ptr(out), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_rasterize_bwd: invalid arguments")
+    return out
+
+
+def probe(px, py, abc, perspective_correct=False):
+    """Steps 2-9 for one pixel centre and one face; returns a dict of every intermediate."""
+    lib = _load()
+    v = _c(abc, np.float64).reshape(9)
+    out = np.empty(13, np.float64)
+    lib.oracle_probe(float(px), float(py), _ptr(v), int(bool(perspective_correct)), _ptr(out))
+    return dict(degenerate=bool(out[0]), inside=bool(out[1]), edge=int(out[2]), t=out[3], d2=out[4],
+                w=out[5:8].copy(), bary=out[8:11].copy(), z=out[11], dist=out[12])

@@ -1,0 +1,456 @@
+/*
+ * oracle.c -- plain, slow float64 CPU oracle of the mesh rasterizer hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the benchmark's
+ * CPU-baseline leg may load this library.  It shares no code, header, table or helper
+ * with the CUDA library; the two meet only through seeded inputs.
+ *
+ * What it computes (PyTorch3D paper, "Accelerating 3D Deep Learning with PyTorch3D",
+ * method summary: two-stage rasterization that keeps, for every pixel, the K nearest
+ * faces, then a second stage that blends their influence; tutorial summary, 32:56:
+ * the perspective_correct switch).  The pages give the concept only; the formulas are
+ * the textbook ones, written out below step by step:
+ *
+ *   1. pixel centre p = (-1 + (2j+1)/W, 1 - (2i+1)/H); +x right, +y up, row 0 at top.
+ *   2. a, b, c = the face's three screen-space vertices (x, y, z).
+ *      A = cross(b - a, c - a); a face with |A| <= 1e-12 is skipped (degenerate).
+ *   3. w0 = cross(b - p, c - p) / A, w1 = cross(c - p, a - p) / A,
+ *      w2 = cross(a - p, b - p) / A (each evaluated directly; no back-face culling).
+ *   4. inside = w0 >= 0 and w1 >= 0 and w2 >= 0 (closed triangle).
+ *   5. d2 = min over edges (a,b), (b,c), (c,a) of the squared distance from p to the
+ *      segment; the first minimal edge in that order wins a tie.
+ *   6. the face is a candidate iff inside or d2 <= blur_radius (squared NDC units).
+ *   7. barycentrics: perspective-correct -> u_k = w_k / z_k, bary_k = u_k / sum(u);
+ *      otherwise bary_k = w_k.  Never clipped, so they sum to 1.
+ *   8. z = sum bary_k z_k; a candidate with z < 0 is skipped (behind the camera).
+ *   9. dist = -d2 inside, +d2 outside.
+ *  10. candidates sorted by (z, face id); the first K kept; empty slots hold -1 in
+ *      pix_to_face, zbuf, bary and dists.
+ *  11. silhouette: p_k = 1 / (1 + exp(dist_k / sigma)) over valid slots,
+ *      alpha = 1 - prod_k (1 - p_k).
+ *  12. its gradient: dL/ddist_k = -dL/dalpha * prod_{j != k} (1 - p_j) * p_k (1 - p_k) / sigma.
+ *  13. rasterizer backward: the chain rule through steps 3, 5, 7, 8 and 9 with the
+ *      candidate set, the inside flag and the nearest edge held fixed.
+ *
+ * Besides the outputs, the forward marks pixels whose integer result is decided by a
+ * float64-vs-float32 rounding: (E1) two of the K+1 nearest candidates lie within 1e-6
+ * in depth; (E2) a face whose candidacy is within a margin of its threshold
+ * (|d2 - blur| < 1e-6 max(1, blur), or min w within 1e-6 of 0 when blur is 0) would
+ * rank among the first K.  These flags only steer the comparison; they change nothing.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define DEGENERATE_AREA 1e-12
+#define TIE_DEPTH 1e-6
+#define MARGIN 1e-6
+
+typedef struct { double x, y, z; } vtx;
+
+/* Everything step 2..9 yields for one (pixel, face) pair. */
+typedef struct {
+    int degenerate;    /* step 2 */
+    int inside;        /* step 4 */
+    int edge;          /* argmin edge of step 5: 0 = (a,b), 1 = (b,c), 2 = (c,a) */
+    double t;          /* segment parameter of the nearest point on that edge */
+    double d2;         /* step 5 */
+    double w[3];       /* step 3 */
+    double bary[3];    /* step 7 */
+    double z;          /* step 8 */
+    double dist;       /* step 9 */
+} pf_eval;
+
+static double cross2(double ux, double uy, double vx, double vy) { return ux * vy - uy * vx; }
+
+static void face_vertices(const float *verts, const int64_t *faces, int64_t f, vtx v[3]) {
+    for (int k = 0; k < 3; ++k) {
+        int64_t vi = faces[3 * f + k];
+        v[k].x = (double)verts[3 * vi + 0];
+        v[k].y = (double)verts[3 * vi + 1];
+        v[k].z = (double)verts[3 * vi + 2];
+    }
+}
+
+/* Squared distance from (px,py) to segment u->v, with the clamped parameter t. */
+static double segment_dist2(double px, double py, vtx u, vtx v, double *t_out) {
+    double ex = v.x - u.x, ey = v.y - u.y;
+    double len2 = ex * ex + ey * ey;
+    double t = 0.0;
+    if (len2 > 0.0) t = ((px - u.x) * ex + (py - u.y) * ey) / len2;
+    if (t < 0.0) t = 0.0;
+    if (t > 1.0) t = 1.0;
+    double qx = u.x + t * ex, qy = u.y + t * ey;
+    *t_out = t;
+    return (px - qx) * (px - qx) + (py - qy) * (py - qy);
+}
+
+/* Steps 2..9 for pixel centre (px, py) and face vertices v[0..2] = a, b, c. */
+static void evaluate(double px, double py, const vtx v[3], int persp, pf_eval *r) {
+    const vtx a = v[0], b = v[1], c = v[2];
+    memset(r, 0, sizeof(*r));
+    double A = cross2(b.x - a.x, b.y - a.y, c.x - a.x, c.y - a.y);
+    if (fabs(A) <= DEGENERATE_AREA) { r->degenerate = 1; return; }
+    r->w[0] = cross2(b.x - px, b.y - py, c.x - px, c.y - py) / A;
+    r->w[1] = cross2(c.x - px, c.y - py, a.x - px, a.y - py) / A;
+    r->w[2] = cross2(a.x - px, a.y - py, b.x - px, b.y - py) / A;
+    r->inside = r->w[0] >= 0.0 && r->w[1] >= 0.0 && r->w[2] >= 0.0;
+    double t;
+    r->d2 = segment_dist2(px, py, a, b, &t); r->edge = 0; r->t = t;
+    double d = segment_dist2(px, py, b, c, &t);
+    if (d < r->d2) { r->d2 = d; r->edge = 1; r->t = t; }
+    d = segment_dist2(px, py, c, a, &t);
+    if (d < r->d2) { r->d2 = d; r->edge = 2; r->t = t; }
+    if (persp) {
+        double u0 = r->w[0] / a.z, u1 = r->w[1] / b.z, u2 = r->w[2] / c.z;
+        double s = u0 + u1 + u2;
+        r->bary[0] = u0 / s; r->bary[1] = u1 / s; r->bary[2] = u2 / s;
+    } else {
+        r->bary[0] = r->w[0]; r->bary[1] = r->w[1]; r->bary[2] = r->w[2];
+    }
+    r->z = r->bary[0] * a.z + r->bary[1] * b.z + r->bary[2] * c.z;
+    r->dist = r->inside ? -r->d2 : r->d2;
+}
+
+static int is_candidate(const pf_eval *r, double blur) {
+    if (r->degenerate) return 0;
+    if (!(r->inside || r->d2 <= blur)) return 0;   /* step 6 */
+    if (r->z < 0.0) return 0;                      /* step 8 */
+    return 1;
+}
+
+/* (z, face id) lexicographic order of step 10. */
+static int before(double z1, int64_t f1, double z2, int64_t f2) {
+    return z1 < z2 || (z1 == z2 && f1 < f2);
+}
+
+/* ------------------------------------------------------------------ forward */
+typedef struct {
+    const float *verts; const int64_t *faces; const int64_t *first; const int64_t *num;
+    int32_t N, H, W, K, persp; double blur;
+    const int64_t *pixels; int64_t npix;
+    int64_t *p2f; double *zbuf, *bary, *dists; uint8_t *exempt;
+    int64_t next; pthread_mutex_t lock;
+} fwd_job;
+
+typedef struct { double z; int64_t f; } zf;
+
+static void rasterize_pixel(fwd_job *J, int64_t pix_id, int64_t out_slot, zf *list) {
+    const int32_t H = J->H, W = J->W, K = J->K;
+    int64_t n = pix_id / ((int64_t)H * W);
+    int64_t rem = pix_id % ((int64_t)H * W);
+    int i = (int)(rem / W), j = (int)(rem % W);
+    double px = -1.0 + (2.0 * j + 1.0) / W;     /* step 1 */
+    double py = 1.0 - (2.0 * i + 1.0) / H;
+    /* a face farther than sqrt(blur) from p along x or y can be neither inside nor
+     * within the blur radius: the reject below is exact (margin 1e-9 for sqrt rounding). */
+    double reach = sqrt(J->blur) + 1e-9;
+    int kept = 0, cap = K + 1;                   /* K+1 nearest, for the E1 check */
+    int64_t f0 = J->first[n], f1 = J->first[n] + J->num[n];
+    for (int64_t f = f0; f < f1; ++f) {
+        vtx v[3];
+        face_vertices(J->verts, J->faces, f, v);
+        double xmin = fmin(v[0].x, fmin(v[1].x, v[2].x)), xmax = fmax(v[0].x, fmax(v[1].x, v[2].x));
+        double ymin = fmin(v[0].y, fmin(v[1].y, v[2].y)), ymax = fmax(v[0].y, fmax(v[1].y, v[2].y));
+        if (px < xmin - reach || px > xmax + reach || py < ymin - reach || py > ymax + reach) continue;
+        pf_eval r;
+        evaluate(px, py, v, J->persp, &r);
+        if (!is_candidate(&r, J->blur)) continue;
+        /* insert (z, f) into the sorted list of at most K+1 entries */
+        int pos = kept;
+        while (pos > 0 && before(r.z, f, list[pos - 1].z, list[pos - 1].f)) --pos;
+        if (pos >= cap) continue;
+        int last = kept < cap ? kept : cap - 1;
+        for (int q = last; q > pos; --q) list[q] = list[q - 1];
+        list[pos].z = r.z; list[pos].f = f;
+        if (kept < cap) ++kept;
+    }
+    /* outputs: the first K entries */
+    for (int k = 0; k < K; ++k) {
+        int64_t s = out_slot * K + k;
+        if (k < kept) {
+            vtx v[3];
+            pf_eval r;
+            face_vertices(J->verts, J->faces, list[k].f, v);
+            evaluate(px, py, v, J->persp, &r);
+            J->p2f[s] = list[k].f;
+            J->zbuf[s] = r.z;
+            J->bary[3 * s + 0] = r.bary[0]; J->bary[3 * s + 1] = r.bary[1]; J->bary[3 * s + 2] = r.bary[2];
+            J->dists[s] = r.dist;
+        } else {
+            J->p2f[s] = -1;
+            J->zbuf[s] = -1.0;
+            J->bary[3 * s + 0] = J->bary[3 * s + 1] = J->bary[3 * s + 2] = -1.0;
+            J->dists[s] = -1.0;
+        }
+    }
+    if (!J->exempt) return;
+    uint8_t ex = 0;
+    /* E1: a depth near-tie among the K+1 nearest (the list is sorted) */
+    for (int k = 0; k + 1 < kept; ++k)
+        if (list[k + 1].z - list[k].z < TIE_DEPTH) ex |= 1;
+    /* E2: a face whose candidacy sits on its threshold and that would rank in the first K */
+    for (int64_t f = f0; f < f1; ++f) {
+        vtx v[3];
+        face_vertices(J->verts, J->faces, f, v);
+        double xmin = fmin(v[0].x, fmin(v[1].x, v[2].x)), xmax = fmax(v[0].x, fmax(v[1].x, v[2].x));
+        double ymin = fmin(v[0].y, fmin(v[1].y, v[2].y)), ymax = fmax(v[0].y, fmax(v[1].y, v[2].y));
+        double reach2 = reach + 1e-3;
+        if (px < xmin - reach2 || px > xmax + reach2 || py < ymin - reach2 || py > ymax + reach2) continue;
+        pf_eval r;
+        evaluate(px, py, v, J->persp, &r);
+        if (r.degenerate) continue;
+        int marginal;
+        if (J->blur > 0.0) {
+            marginal = !r.inside && fabs(r.d2 - J->blur) < MARGIN * fmax(1.0, J->blur);
+        } else {
+            double wmin = fmin(r.w[0], fmin(r.w[1], r.w[2]));
+            marginal = wmin > -MARGIN && wmin < MARGIN;
+        }
+        if (!marginal || r.z < 0.0) continue;
+        int ahead = 0;
+        for (int k = 0; k < kept; ++k)
+            if (list[k].f != f && before(list[k].z, list[k].f, r.z, f)) ++ahead;
+        if (ahead < K) ex |= 2;
+    }
+    J->exempt[out_slot] = ex;
+}
+
+static void *fwd_worker(void *arg) {
+    fwd_job *J = (fwd_job *)arg;
+    int64_t total = J->pixels ? J->npix : (int64_t)J->N * J->H * J->W;
+    zf *list = (zf *)malloc(sizeof(zf) * (size_t)(J->K + 2));
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int64_t start = J->next;
+        J->next += 64;
+        pthread_mutex_unlock(&J->lock);
+        if (start >= total) break;
+        int64_t end = start + 64 < total ? start + 64 : total;
+        for (int64_t s = start; s < end; ++s)
+            rasterize_pixel(J, J->pixels ? J->pixels[s] : s, s, list);
+    }
+    free(list);
+    return NULL;
+}
+
+static void run_threads(void *(*fn)(void *), void *job, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    for (int t = 0; t < nthreads; ++t) pthread_create(&th[t], NULL, fn, job);
+    for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
+    free(th);
+}
+
+/* Forward over all N*H*W pixels (pixels == NULL) or over the listed pixel ids
+ * (id = (n*H + i)*W + j); outputs are then P x K, in list order.  Returns 0, or -1 on
+ * invalid arguments. */
+int oracle_rasterize_fwd(const float *verts, int64_t V, const int64_t *faces, int64_t F,
+                         const int64_t *first, const int64_t *num, int32_t N, int32_t H, int32_t W,
+                         double blur, int32_t K, int32_t persp, const int64_t *pixels, int64_t npix,
+                         int64_t *p2f, double *zbuf, double *bary, double *dists, uint8_t *exempt,
+                         int32_t nthreads) {
+    if (N < 0 || H <= 0 || W <= 0 || K <= 0 || !(blur >= 0.0)) return -1;
+    for (int32_t n = 0; n < N; ++n)
+        if (first[n] < 0 || num[n] < 0 || first[n] + num[n] > F) return -1;
+    for (int64_t q = 0; q < 3 * F; ++q)
+        if (faces[q] < 0 || faces[q] >= V) return -1;
+    fwd_job J;
+    memset(&J, 0, sizeof(J));
+    J.verts = verts; J.faces = faces; J.first = first; J.num = num;
+    J.N = N; J.H = H; J.W = W; J.K = K; J.persp = persp; J.blur = blur;
+    J.pixels = pixels; J.npix = npix;
+    J.p2f = p2f; J.zbuf = zbuf; J.bary = bary; J.dists = dists; J.exempt = exempt;
+    pthread_mutex_init(&J.lock, NULL);
+    run_threads(fwd_worker, &J, nthreads);
+    pthread_mutex_destroy(&J.lock);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ silhouette */
+/* Step 11 over npix pixels of K slots each. */
+void oracle_silhouette_fwd(const int64_t *p2f, const double *dists, int64_t npix, int32_t K,
+                           double sigma, double *alpha) {
+    for (int64_t q = 0; q < npix; ++q) {
+        double keep = 1.0;   /* prod (1 - p_k) */
+        for (int k = 0; k < K; ++k) {
+            int64_t s = q * K + k;
+            if (p2f[s] < 0) continue;
+            double p = 1.0 / (1.0 + exp(dists[s] / sigma));
+            keep *= 1.0 - p;
+        }
+        alpha[q] = 1.0 - keep;
+    }
+}
+
+/* Step 12: the product over j != k is formed directly (no division). */
+void oracle_silhouette_bwd(const double *grad_alpha, const int64_t *p2f, const double *dists,
+                           int64_t npix, int32_t K, double sigma, double *grad_dists) {
+    for (int64_t q = 0; q < npix; ++q) {
+        for (int k = 0; k < K; ++k) {
+            int64_t s = q * K + k;
+            if (p2f[s] < 0) { grad_dists[s] = 0.0; continue; }
+            double others = 1.0;
+            for (int j = 0; j < K; ++j) {
+                int64_t sj = q * K + j;
+                if (j == k || p2f[sj] < 0) continue;
+                others *= 1.0 - 1.0 / (1.0 + exp(dists[sj] / sigma));
+            }
+            double p = 1.0 / (1.0 + exp(dists[s] / sigma));
+            grad_dists[s] = -grad_alpha[q] * others * p * (1.0 - p) / sigma;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ backward */
+/*
+ * Derivatives used below (v = a, b, c is vertex 0, 1, 2; only x, y enter steps 3 and 5):
+ *   C_k = cross(V1 - p, V2 - p) for (V1, V2) = (b, c), (c, a), (a, b);  w_k = C_k / A.
+ *   d cross(U - p, V - p) / dU = (V.y - p.y, -(V.x - p.x)),  / dV = (-(U.y - p.y), U.x - p.x).
+ *   d A / db = (c.y - a.y, -(c.x - a.x)),  d A / dc = (-(b.y - a.y), b.x - a.x),
+ *   d A / da = -(dA/db + dA/dc).
+ *   d w_k = (d C_k - w_k d A) / A.
+ *   Perspective: u_k = w_k / z_k, s = sum u, bary_k = u_k / s, z = 1 / s, so
+ *     d bary_m / d u_k = (delta_mk - bary_m) / s,  d z / d u_k = -z^2,
+ *     d u_k / d w_k = 1 / z_k,  d u_k / d z_k = -u_k / z_k.
+ *   Plain: bary_k = w_k, z = sum w_k z_k, so d z / d w_k = z_k and d z / d z_k = w_k.
+ *   Distance to the nearest edge u->v with nearest point q = u + t (v - u):
+ *     d d2 / du = -2 (p - q)(1 - t),  d d2 / dv = -2 (p - q) t;  dist = +-d2.
+ */
+typedef struct {
+    const float *verts; const int64_t *faces; const int64_t *p2f;
+    int32_t N, H, W, K, persp;
+    const double *gz, *gb, *gd;
+    double **partial; int64_t V;
+    int64_t next; pthread_mutex_t lock; int nthreads; int tid_next;
+} bwd_job;
+
+static void accumulate_slot(bwd_job *J, int64_t slot, double *g) {
+    int64_t f = J->p2f[slot];
+    if (f < 0) return;
+    int64_t pix = slot / J->K;
+    int64_t rem = pix % ((int64_t)J->H * J->W);
+    int i = (int)(rem / J->W), j = (int)(rem % J->W);
+    double px = -1.0 + (2.0 * j + 1.0) / J->W;
+    double py = 1.0 - (2.0 * i + 1.0) / J->H;
+    vtx v[3];
+    face_vertices(J->verts, J->faces, f, v);
+    pf_eval r;
+    evaluate(px, py, v, J->persp, &r);
+    if (r.degenerate) return;
+    int64_t vid[3] = {J->faces[3 * f], J->faces[3 * f + 1], J->faces[3 * f + 2]};
+
+    /* dists -> the two end points of the nearest edge (x, y) */
+    if (J->gd) {
+        double gdist = J->gd[slot] * (r.inside ? -1.0 : 1.0);
+        int u = r.edge, w = (r.edge + 1) % 3;
+        double qx = v[u].x + r.t * (v[w].x - v[u].x), qy = v[u].y + r.t * (v[w].y - v[u].y);
+        double rx = px - qx, ry = py - qy;
+        g[3 * vid[u] + 0] += gdist * (-2.0 * rx * (1.0 - r.t));
+        g[3 * vid[u] + 1] += gdist * (-2.0 * ry * (1.0 - r.t));
+        g[3 * vid[w] + 0] += gdist * (-2.0 * rx * r.t);
+        g[3 * vid[w] + 1] += gdist * (-2.0 * ry * r.t);
+    }
+    if (!J->gb && !J->gz) return;
+
+    double gbary[3] = {0, 0, 0}, gzb = 0.0;
+    if (J->gb) for (int m = 0; m < 3; ++m) gbary[m] = J->gb[3 * slot + m];
+    if (J->gz) gzb = J->gz[slot];
+    double gw[3], gzc[3];    /* dL/dw_k and dL/dz_k (vertex depth) */
+    if (J->persp) {
+        double u[3], s = 0.0;
+        for (int k = 0; k < 3; ++k) { u[k] = r.w[k] / v[k].z; s += u[k]; }
+        for (int k = 0; k < 3; ++k) {
+            double gu = 0.0;
+            for (int m = 0; m < 3; ++m) gu += gbary[m] * (((m == k) ? 1.0 : 0.0) - r.bary[m]) / s;
+            gu += gzb * (-r.z * r.z);
+            gw[k] = gu / v[k].z;
+            gzc[k] = gu * (-u[k] / v[k].z);
+        }
+    } else {
+        for (int k = 0; k < 3; ++k) { gw[k] = gbary[k] + gzb * v[k].z; gzc[k] = gzb * r.w[k]; }
+    }
+    /* d w_k / d (vertex x, y) */
+    const vtx a = v[0], b = v[1], c = v[2];
+    double A = cross2(b.x - a.x, b.y - a.y, c.x - a.x, c.y - a.y);
+    double dA[3][2] = {{b.y - c.y, c.x - b.x}, {c.y - a.y, -(c.x - a.x)}, {-(b.y - a.y), b.x - a.x}};
+    double dC[3][3][2];  /* dC[k][vertex][xy] */
+    memset(dC, 0, sizeof(dC));
+    int pairs[3][2] = {{1, 2}, {2, 0}, {0, 1}};
+    for (int k = 0; k < 3; ++k) {
+        int U = pairs[k][0], W2 = pairs[k][1];
+        dC[k][U][0] = v[W2].y - py;   dC[k][U][1] = -(v[W2].x - px);
+        dC[k][W2][0] = -(v[U].y - py); dC[k][W2][1] = v[U].x - px;
+    }
+    for (int k = 0; k < 3; ++k)
+        for (int q = 0; q < 3; ++q)
+            for (int e = 0; e < 2; ++e)
+                g[3 * vid[q] + e] += gw[k] * (dC[k][q][e] - r.w[k] * dA[q][e]) / A;
+    for (int k = 0; k < 3; ++k) g[3 * vid[k] + 2] += gzc[k];
+}
+
+static void *bwd_worker(void *arg) {
+    bwd_job *J = (bwd_job *)arg;
+    pthread_mutex_lock(&J->lock);
+    int tid = J->tid_next++;
+    pthread_mutex_unlock(&J->lock);
+    double *g = J->partial[tid];
+    int64_t total = (int64_t)J->N * J->H * J->W * J->K;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int64_t start = J->next;
+        J->next += 4096;
+        pthread_mutex_unlock(&J->lock);
+        if (start >= total) break;
+        int64_t end = start + 4096 < total ? start + 4096 : total;
+        for (int64_t s = start; s < end; ++s) accumulate_slot(J, s, g);
+    }
+    return NULL;
+}
+
+/* Step 13 over all N*H*W*K slots.  grad_* may be NULL (no gradient from that output).
+ * grad_verts (V x 3) is overwritten.  Returns 0, or -1 on invalid arguments. */
+int oracle_rasterize_bwd(const float *verts, int64_t V, const int64_t *faces, int64_t F,
+                         const int64_t *p2f, int32_t N, int32_t H, int32_t W, int32_t K, int32_t persp,
+                         const double *grad_zbuf, const double *grad_bary, const double *grad_dists,
+                         double *grad_verts, int32_t nthreads) {
+    if (N < 0 || H <= 0 || W <= 0 || K <= 0) return -1;
+    int64_t slots = (int64_t)N * H * W * K;
+    for (int64_t s = 0; s < slots; ++s) if (p2f[s] >= F) return -1;
+    for (int64_t q = 0; q < 3 * F; ++q) if (faces[q] < 0 || faces[q] >= V) return -1;
+    if (nthreads < 1) nthreads = 1;
+    bwd_job J;
+    memset(&J, 0, sizeof(J));
+    J.verts = verts; J.faces = faces; J.p2f = p2f;
+    J.N = N; J.H = H; J.W = W; J.K = K; J.persp = persp;
+    J.gz = grad_zbuf; J.gb = grad_bary; J.gd = grad_dists; J.V = V;
+    J.nthreads = nthreads;
+    J.partial = (double **)malloc(sizeof(double *) * (size_t)nthreads);
+    for (int t = 0; t < nthreads; ++t) J.partial[t] = (double *)calloc((size_t)(3 * V), sizeof(double));
+    pthread_mutex_init(&J.lock, NULL);
+    run_threads(bwd_worker, &J, nthreads);
+    pthread_mutex_destroy(&J.lock);
+    for (int64_t q = 0; q < 3 * V; ++q) {
+        double s = 0.0;
+        for (int t = 0; t < nthreads; ++t) s += J.partial[t][q];
+        grad_verts[q] = s;
+    }
+    for (int t = 0; t < nthreads; ++t) free(J.partial[t]);
+    free(J.partial);
+    return 0;
+}
+
+/* Per-(pixel, face) probe for tests: steps 2..9 for one pixel centre and one face. */
+void oracle_probe(double px, double py, const double *abc /* 9: a, b, c as x,y,z */, int32_t persp,
+                  double *out /* 13 values, listed below */) {
+    vtx v[3];
+    for (int k = 0; k < 3; ++k) { v[k].x = abc[3 * k]; v[k].y = abc[3 * k + 1]; v[k].z = abc[3 * k + 2]; }
+    pf_eval r;
+    evaluate(px, py, v, persp, &r);
+    /* out: [degenerate, inside, edge, t, d2, w0, w1, w2, b0, b1, b2, z, dist] */
+    out[0] = r.degenerate; out[1] = r.inside; out[2] = r.edge; out[3] = r.t; out[4] = r.d2;
+    out[5] = r.w[0]; out[6] = r.w[1]; out[7] = r.w[2];
+    out[8] = r.bary[0]; out[9] = r.bary[1]; out[10] = r.bary[2]; out[11] = r.z; out[12] = r.dist;
+}
