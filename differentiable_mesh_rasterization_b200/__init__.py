@@ -1,0 +1,243 @@
+"""Thin Python binding of ``libmeshrast.so`` (the sm_100a mesh rasterizer C ABI).
+
+Argument marshalling only: every function checks shapes, dtypes and devices of torch
+tensors, allocates the outputs with torch, and passes raw device pointers plus the
+current CUDA stream to the C entry point of the same name (``mr_*``).  All arithmetic
+runs in the library's CUDA kernels; there is no CPU path.  The library is loaded from
+this directory on first use and must have been built (``python -m
+differentiable_mesh_rasterization_b200.build``); every entry point raises ImportError
+without it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmeshrast.so")
+
+MR_KMAX = 32
+ERRORS = {-1: "invalid argument", -2: "out of memory", -3: "CUDA error", -4: "device index error"}
+
+# Entry points declared by include/meshrast.h (checked by the test-suite).
+EXPORTS = ("mr_rasterize_fwd", "mr_rasterize_silhouette_fwd", "mr_silhouette_blend_fwd",
+           "mr_silhouette_blend_bwd", "mr_rasterize_bwd", "mr_silhouette_rasterize_bwd",
+           "mr_device_status", "mr_last_error", "mr_version")
+
+
+class MeshRastError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn}: {ERRORS.get(code, code)} ({code}): {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libmeshrast.so and declare its signatures (fails loudly if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m differentiable_mesh_rasterization_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
+    sig = {
+        "mr_rasterize_fwd": [P, i64, P, i64, P, P, i32, i32, i32, f32, i32, i32, P, P, P, P, P],
+        "mr_rasterize_silhouette_fwd": [P, i64, P, i64, P, P, i32, i32, i32, f32, i32, i32, f32, P, P, P, P, P, P],
+        "mr_silhouette_blend_fwd": [P, P, i32, i32, i32, i32, f32, P, P],
+        "mr_silhouette_blend_bwd": [P, P, P, i32, i32, i32, i32, f32, P, P],
+        "mr_rasterize_bwd": [P, i64, P, i64, P, i32, i32, i32, i32, i32, P, P, P, P, P],
+        "mr_silhouette_rasterize_bwd": [P, i64, P, i64, P, P, i32, i32, i32, i32, f32, P, P, P],
+        "mr_device_status": [P],
+        "mr_last_error": [],
+        "mr_version": [],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    lib.mr_last_error.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(name: str, rc: int) -> None:
+    if rc != 0:
+        raise MeshRastError(name, rc, load_library().mr_last_error().decode())
+
+
+def _stream(dev: torch.device) -> int:
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _dev(t: torch.Tensor, dtype, name: str) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.contiguous()
+
+
+def _host_i64(a, name: str) -> np.ndarray:
+    if isinstance(a, torch.Tensor):
+        a = a.detach().cpu().numpy()
+    a = np.ascontiguousarray(a, dtype=np.int64)
+    if a.ndim != 1:
+        raise ValueError(f"{name} must be 1-D")
+    return a
+
+
+def rasterize_fwd(verts, faces, mesh_to_face_first_idx, num_faces_per_mesh, H, W, blur_radius, K,
+                  perspective_correct=False, sigma=None):
+    """Stage one (``mr_rasterize_fwd``); with ``sigma`` also the fused silhouette.
+
+    verts (V, 3) float32 CUDA, faces (F, 3) int64 CUDA; the two per-mesh index arrays live
+    on the host (numpy or CPU tensors).  Returns ``pix_to_face (N,H,W,K) int64, zbuf,
+    bary (N,H,W,K,3), dists`` and, when ``sigma`` is given, ``alpha (N,H,W)``.
+    """
+    lib = load_library()
+    verts = _dev(verts, torch.float32, "verts")
+    faces = _dev(faces, torch.int64, "faces")
+    if verts.ndim != 2 or verts.shape[1] != 3 or faces.ndim != 2 or faces.shape[1] != 3:
+        raise ValueError("verts and faces must be (V, 3) and (F, 3)")
+    first = _host_i64(mesh_to_face_first_idx, "mesh_to_face_first_idx")
+    num = _host_i64(num_faces_per_mesh, "num_faces_per_mesh")
+    if first.shape != num.shape:
+        raise ValueError("per-mesh arrays differ in length")
+    N = first.shape[0]
+    dev = verts.device
+    p2f = torch.empty((N, H, W, K), dtype=torch.int64, device=dev)
+    zbuf = torch.empty((N, H, W, K), dtype=torch.float32, device=dev)
+    bary = torch.empty((N, H, W, K, 3), dtype=torch.float32, device=dev)
+    dists = torch.empty((N, H, W, K), dtype=torch.float32, device=dev)
+    args = (_ptr(verts), verts.shape[0], _ptr(faces), faces.shape[0], first.ctypes.data, num.ctypes.data,
+            N, H, W, float(blur_radius), K, int(bool(perspective_correct)))
+    with torch.cuda.device(dev):
+        if sigma is None:
+            _check("mr_rasterize_fwd", lib.mr_rasterize_fwd(*args, _ptr(p2f), _ptr(zbuf), _ptr(bary), _ptr(dists),
+                                                            _stream(dev)))
+            return p2f, zbuf, bary, dists
+        alpha = torch.empty((N, H, W), dtype=torch.float32, device=dev)
+        _check("mr_rasterize_silhouette_fwd",
+               lib.mr_rasterize_silhouette_fwd(*args, float(sigma), _ptr(p2f), _ptr(zbuf), _ptr(bary), _ptr(dists),
+                                               _ptr(alpha), _stream(dev)))
+        return p2f, zbuf, bary, dists, alpha
+
+
+def _nhwk(p2f: torch.Tensor):
+    if p2f.ndim != 4:
+        raise ValueError("pix_to_face must be (N, H, W, K)")
+    return tuple(int(x) for x in p2f.shape)
+
+
+def silhouette_blend_fwd(pix_to_face, dists, sigma):
+    """Soft silhouette (``mr_silhouette_blend_fwd``) -> alpha (N, H, W)."""
+    lib = load_library()
+    p2f = _dev(pix_to_face, torch.int64, "pix_to_face")
+    d = _dev(dists, torch.float32, "dists")
+    N, H, W, K = _nhwk(p2f)
+    if d.shape != p2f.shape:
+        raise ValueError("dists must match pix_to_face")
+    alpha = torch.empty((N, H, W), dtype=torch.float32, device=p2f.device)
+    with torch.cuda.device(p2f.device):
+        _check("mr_silhouette_blend_fwd", lib.mr_silhouette_blend_fwd(_ptr(p2f), _ptr(d), N, H, W, K, float(sigma),
+                                                                      _ptr(alpha), _stream(p2f.device)))
+    return alpha
+
+
+def silhouette_blend_bwd(grad_alpha, pix_to_face, dists, sigma):
+    """Gradient of the soft silhouette (``mr_silhouette_blend_bwd``) -> grad_dists (N, H, W, K)."""
+    lib = load_library()
+    p2f = _dev(pix_to_face, torch.int64, "pix_to_face")
+    d = _dev(dists, torch.float32, "dists")
+    g = _dev(grad_alpha, torch.float32, "grad_alpha")
+    N, H, W, K = _nhwk(p2f)
+    if d.shape != p2f.shape or g.shape != (N, H, W):
+        raise ValueError("shape mismatch")
+    out = torch.empty_like(d)
+    with torch.cuda.device(p2f.device):
+        _check("mr_silhouette_blend_bwd", lib.mr_silhouette_blend_bwd(_ptr(g), _ptr(p2f), _ptr(d), N, H, W, K,
+                                                                      float(sigma), _ptr(out), _stream(p2f.device)))
+    return out
+
+
+def rasterize_bwd(verts, faces, pix_to_face, perspective_correct=False, grad_zbuf=None, grad_bary=None,
+                  grad_dists=None):
+    """Backward of stage one (``mr_rasterize_bwd``) -> grad_verts (V, 3) float32."""
+    lib = load_library()
+    verts = _dev(verts, torch.float32, "verts")
+    faces = _dev(faces, torch.int64, "faces")
+    p2f = _dev(pix_to_face, torch.int64, "pix_to_face")
+    N, H, W, K = _nhwk(p2f)
+    gz = None if grad_zbuf is None else _dev(grad_zbuf, torch.float32, "grad_zbuf")
+    gb = None if grad_bary is None else _dev(grad_bary, torch.float32, "grad_bary")
+    gd = None if grad_dists is None else _dev(grad_dists, torch.float32, "grad_dists")
+    for t, shp in ((gz, (N, H, W, K)), (gb, (N, H, W, K, 3)), (gd, (N, H, W, K))):
+        if t is not None and tuple(t.shape) != shp:
+            raise ValueError(f"gradient shape {tuple(t.shape)} != {shp}")
+    out = torch.empty_like(verts)
+    with torch.cuda.device(verts.device):
+        _check("mr_rasterize_bwd", lib.mr_rasterize_bwd(_ptr(verts), verts.shape[0], _ptr(faces), faces.shape[0],
+                                                        _ptr(p2f), N, H, W, K, int(bool(perspective_correct)),
+                                                        _ptr(gz), _ptr(gb), _ptr(gd), _ptr(out),
+                                                        _stream(verts.device)))
+    return out
+
+
+def silhouette_rasterize_bwd(verts, faces, pix_to_face, dists, sigma, grad_alpha):
+    """Fused silhouette + distance backward (``mr_silhouette_rasterize_bwd``) -> grad_verts (V, 3)."""
+    lib = load_library()
+    verts = _dev(verts, torch.float32, "verts")
+    faces = _dev(faces, torch.int64, "faces")
+    p2f = _dev(pix_to_face, torch.int64, "pix_to_face")
+    d = _dev(dists, torch.float32, "dists")
+    g = _dev(grad_alpha, torch.float32, "grad_alpha")
+    N, H, W, K = _nhwk(p2f)
+    if d.shape != p2f.shape or g.shape != (N, H, W):
+        raise ValueError("shape mismatch")
+    out = torch.empty_like(verts)
+    with torch.cuda.device(verts.device):
+        _check("mr_silhouette_rasterize_bwd",
+               lib.mr_silhouette_rasterize_bwd(_ptr(verts), verts.shape[0], _ptr(faces), faces.shape[0], _ptr(p2f),
+                                               _ptr(d), N, H, W, K, float(sigma), _ptr(g), _ptr(out),
+                                               _stream(verts.device)))
+    return out
+
+
+def device_status(device=None) -> None:
+    """Synchronise and raise if an asynchronous kernel skipped an out-of-range index."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _check("mr_device_status", lib.mr_device_status(_stream(dev)))
+
+
+class SilhouetteRasterizer(torch.autograd.Function):
+    """verts -> soft silhouette alpha, differentiable w.r.t. the screen-space vertices.
+
+    Forward: ``mr_rasterize_silhouette_fwd``; backward: ``mr_silhouette_rasterize_bwd``.
+    """
+
+    @staticmethod
+    def forward(ctx, verts, faces, first, num, H, W, blur_radius, K, sigma, perspective_correct=False):
+        p2f, _, _, dists, alpha = rasterize_fwd(verts, faces, first, num, H, W, blur_radius, K,
+                                                perspective_correct, sigma=sigma)
+        ctx.save_for_backward(verts, faces, p2f, dists)
+        ctx.sigma = sigma
+        return alpha
+
+    @staticmethod
+    def backward(ctx, grad_alpha):
+        verts, faces, p2f, dists = ctx.saved_tensors
+        gv = silhouette_rasterize_bwd(verts, faces, p2f, dists, ctx.sigma, grad_alpha.contiguous())
+        return gv, None, None, None, None, None, None, None, None, None

@@ -1,0 +1,105 @@
+// Host-side plumbing of the C ABI: error reporting, stream-ordered scratch, the device
+// error word and the status query.
+#include <cstdarg>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "mr_common.cuh"
+
+namespace {
+thread_local char g_last_error[512] = "";
+__device__ int g_device_error = 0;
+std::mutex g_pool_mutex;
+bool g_pool_ready[64] = {};
+}  // namespace
+
+namespace mr {
+
+void set_error(const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    set_error("%s failed: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+    return MR_ERR_CUDA;
+}
+
+// Freed scratch stays in the device's default pool instead of returning to the driver
+// at every synchronisation; the attribute is per process and per device.
+static int ensure_pool(int dev) {
+    if (dev < 0 || dev >= 64) return MR_OK;
+    std::lock_guard<std::mutex> g(g_pool_mutex);
+    if (g_pool_ready[dev]) return MR_OK;
+    cudaMemPool_t pool;
+    MR_CUDA(cudaDeviceGetDefaultMemPool(&pool, dev));
+    uint64_t keep = UINT64_MAX;
+    MR_CUDA(cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep));
+    g_pool_ready[dev] = true;
+    return MR_OK;
+}
+
+int scratch_alloc(void** p, size_t bytes, cudaStream_t s) {
+    *p = nullptr;
+    if (bytes == 0) return MR_OK;
+    int dev = 0;
+    MR_CUDA(cudaGetDevice(&dev));
+    int rc = ensure_pool(dev);
+    if (rc != MR_OK) return rc;
+    cudaError_t e = cudaMallocAsync(p, bytes, s);
+    if (e == cudaErrorMemoryAllocation) {
+        cudaGetLastError();
+        set_error("scratch allocation of %zu bytes failed", bytes);
+        return MR_ERR_OOM;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync");
+    return MR_OK;
+}
+
+void scratch_free(void* p, cudaStream_t s) {
+    if (p) cudaFreeAsync(p, s);
+}
+
+int* device_error_word() {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return static_cast<int*>(p);
+}
+
+}  // namespace mr
+
+extern "C" {
+
+const char* mr_last_error(void) { return g_last_error; }
+
+int mr_version(void) { return 10000; }
+
+int mr_device_status(void* stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int* w = mr::device_error_word();
+    if (!w) {
+        mr::set_error("cannot locate the device error word");
+        return MR_ERR_CUDA;
+    }
+    int host = 0;
+    MR_CUDA(cudaMemcpyAsync(&host, w, sizeof(int), cudaMemcpyDeviceToHost, s));
+    MR_CUDA(cudaStreamSynchronize(s));
+    if (host != 0) {
+        MR_CUDA(cudaMemsetAsync(w, 0, sizeof(int), s));
+        MR_CUDA(cudaStreamSynchronize(s));
+        mr::set_error("a kernel skipped %s",
+                      (host & mr::kErrFaceIndex) ? "a face with a vertex id outside [0, V)"
+                                                 : "a pix_to_face entry outside [-1, F)");
+        return MR_ERR_DEVICE;
+    }
+    g_last_error[0] = '\0';
+    return MR_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,57 @@
+// Shared definitions of the sm_100a mesh rasterizer library (internal header).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstdio>
+#include <string>
+
+#include "meshrast.h"
+
+namespace mr {
+
+// Screen tile of the coarse pass and of one fine-pass CTA: 16 x 16 pixels, split into
+// eight 8 x 4 warp tiles (two across, four down).
+constexpr int kBin = 16;
+constexpr int kWarpTileW = 8;
+constexpr int kWarpTileH = 4;
+constexpr int kWarpsPerBin = (kBin / kWarpTileW) * (kBin / kWarpTileH);   // 8
+constexpr int kFineThreads = kWarpsPerBin * 32;                            // 256
+constexpr double kDegenerateArea = 1e-12;
+
+// Device error bits.
+constexpr int kErrFaceIndex = 1;    // a face vertex id outside [0, V)
+constexpr int kErrSlotIndex = 2;    // a pix_to_face entry outside [-1, F)
+
+// Face geometry as written by the setup pass: the three vertices in their original
+// order (x, y, z, unused).  Exact copies of the caller's float32 values.
+struct __align__(16) FaceGeom {
+    float4 a, b, c;
+};
+
+// Inclusive pixel box of a face grown by sqrt(blur_radius), clipped to the image.
+// x0 > x1 marks a face that touches no pixel (off-screen or degenerate).
+struct __align__(16) FaceBox {
+    int x0, x1, y0, y1;
+};
+
+void set_error(const char* fmt, ...);
+int cuda_fail(cudaError_t e, const char* what);
+
+#define MR_CUDA(call)                                        \
+    do {                                                     \
+        cudaError_t e_ = (call);                             \
+        if (e_ != cudaSuccess) return ::mr::cuda_fail(e_, #call); \
+    } while (0)
+
+// Scratch allocation on the caller's stream (stream-ordered pool).
+int scratch_alloc(void** p, size_t bytes, cudaStream_t s);
+void scratch_free(void* p, cudaStream_t s);
+
+// Device-wide sticky error word (asynchronous kernels).
+int* device_error_word();
+
+inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace mr

@@ -1,0 +1,597 @@
+// Stage one of the PyTorch3D two-stage mesh rasterizer ("Accelerating 3D Deep Learning
+// with PyTorch3D", method: per-pixel K nearest faces) on sm_100a, plus the fused
+// stage-two silhouette.
+//
+// Pipeline (one CUDA stream):
+//   face setup   one thread per face: gather the three vertices, float64 signed area
+//                (degenerate test), pixel box grown by sqrt(blur_radius).
+//   bin count    one thread per (image, face) pair: count the 16x16 screen bins the box
+//                touches (warp-aggregated atomics).
+//   bin scan     exclusive scan of the per-bin counts -> list offsets and the total.
+//   (host)       one stream synchronisation to size the face lists.
+//   bin fill     second pass of the pair loop: scatter face ids into the bin lists.
+//   fine         one 256-thread CTA per bin.  Faces are staged through shared memory in
+//                chunks of 256 as bin-local float32 plane constants (computed in float64);
+//                each staged face is appended to the list of every 8x4 warp tile its box
+//                touches, so a warp only visits faces that can reach its pixels.  Each
+//                thread owns one pixel and keeps its K nearest (depth key, face id) pairs
+//                in registers, insertion-sorted.  The epilogue recomputes barycentrics,
+//                z and the signed squared distance of the K winners in float64 from the
+//                original vertices and writes them with 16-byte stores.
+#include <cfloat>
+#include <climits>
+#include <cmath>
+#include <vector>
+
+#include "mr_common.cuh"
+#include "mr_silhouette.cuh"
+
+namespace mr {
+namespace {
+
+constexpr int kChunk = kFineThreads;   // faces staged per round
+constexpr int kConstF4 = 5;            // float4 words of bin-local constants per face
+
+// ------------------------------------------------------------------ face setup
+__global__ void k_face_setup(const float* __restrict__ verts, int64_t V,
+                             const int64_t* __restrict__ faces, int64_t F, int H, int W,
+                             double reach, FaceGeom* __restrict__ geom, FaceBox* __restrict__ box,
+                             int* __restrict__ err) {
+    int64_t f = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (f >= F) return;
+    int64_t i0 = faces[3 * f], i1 = faces[3 * f + 1], i2 = faces[3 * f + 2];
+    FaceBox bx = {1, 0, 1, 0};
+    if (i0 < 0 || i0 >= V || i1 < 0 || i1 >= V || i2 < 0 || i2 >= V) {
+        atomicOr(err, kErrFaceIndex);
+        geom[f] = FaceGeom{make_float4(0, 0, 0, 0), make_float4(0, 0, 0, 0), make_float4(0, 0, 0, 0)};
+        box[f] = bx;
+        return;
+    }
+    float4 a = make_float4(verts[3 * i0], verts[3 * i0 + 1], verts[3 * i0 + 2], 0.f);
+    float4 b = make_float4(verts[3 * i1], verts[3 * i1 + 1], verts[3 * i1 + 2], 0.f);
+    float4 c = make_float4(verts[3 * i2], verts[3 * i2 + 1], verts[3 * i2 + 2], 0.f);
+    geom[f] = FaceGeom{a, b, c};
+    double ax = a.x, ay = a.y, bxx = b.x, byy = b.y, cx = c.x, cy = c.y;
+    double area2 = (bxx - ax) * (cy - ay) - (byy - ay) * (cx - ax);
+    if (fabs(area2) > kDegenerateArea) {
+        double xmin = fmin(ax, fmin(bxx, cx)) - reach, xmax = fmax(ax, fmax(bxx, cx)) + reach;
+        double ymin = fmin(ay, fmin(byy, cy)) - reach, ymax = fmax(ay, fmax(byy, cy)) + reach;
+        // pixel j has centre x = -1 + (2j+1)/W; row i has y = 1 - (2i+1)/H.  The 1e-4
+        // pixel pad keeps the box a superset under rounding.
+        double jl = ceil((xmin + 1.0) * 0.5 * W - 0.5 - 1e-4);
+        double jh = floor((xmax + 1.0) * 0.5 * W - 0.5 + 1e-4);
+        double il = ceil((1.0 - ymax) * 0.5 * H - 0.5 - 1e-4);
+        double ih = floor((1.0 - ymin) * 0.5 * H - 0.5 + 1e-4);
+        jl = fmax(jl, 0.0); il = fmax(il, 0.0);
+        jh = fmin(jh, (double)(W - 1)); ih = fmin(ih, (double)(H - 1));
+        if (jl <= jh && il <= ih) bx = FaceBox{(int)jl, (int)jh, (int)il, (int)ih};
+    }
+    box[f] = bx;
+}
+
+// ------------------------------------------------------------------ binning
+// (image, face) pairs are enumerated image by image: pair q belongs to image n with
+// pair_prefix[n] <= q < pair_prefix[n+1] and is face first[n] + q - pair_prefix[n].
+__device__ __forceinline__ int pair_image(const int64_t* prefix, int N, int64_t q) {
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= q) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+template <bool FILL>
+__global__ void k_bin_pairs(const FaceBox* __restrict__ box, const int64_t* __restrict__ prefix,
+                            const int64_t* __restrict__ first, int N, int64_t pairs, int nbx, int nby,
+                            int* __restrict__ counts, const int* __restrict__ offsets,
+                            int* __restrict__ list) {
+    const unsigned lane = threadIdx.x & 31;
+    for (int64_t q0 = (int64_t)blockIdx.x * blockDim.x; q0 < pairs; q0 += (int64_t)gridDim.x * blockDim.x) {
+        int64_t q = q0 + threadIdx.x;
+        bool live = q < pairs;
+        int n = 0;
+        int64_t f = 0;
+        FaceBox b = {1, 0, 1, 0};
+        if (live) {
+            n = pair_image(prefix, N, q);
+            f = first[n] + (q - prefix[n]);
+            b = box[f];
+        }
+        int bx0 = 0, bx1 = -1, by0 = 0, by1 = -1;
+        if (live && b.x0 <= b.x1) {
+            bx0 = b.x0 / kBin; bx1 = b.x1 / kBin; by0 = b.y0 / kBin; by1 = b.y1 / kBin;
+        }
+        // Walk the touched bins in lock-step across the warp; neighbouring faces share
+        // bins, so one atomic per distinct bin per step is issued.
+        int nx = bx1 - bx0 + 1, ny = by1 - by0 + 1;
+        int mine = (nx > 0 && ny > 0) ? nx * ny : 0;
+        int most = mine;
+        for (int o = 16; o > 0; o >>= 1) most = max(most, __shfl_xor_sync(0xffffffffu, most, o));
+        for (int s = 0; s < most; ++s) {
+            bool act = s < mine;
+            int bin = -1;
+            if (act) bin = (n * nby + by0 + s / nx) * nbx + bx0 + s % nx;
+            unsigned peers = __match_any_sync(0xffffffffu, bin);
+            if (!act) continue;
+            int leader = __ffs(peers) - 1;
+            int rank = __popc(peers & ((1u << lane) - 1));
+            int base = 0;
+            if ((int)lane == leader) base = atomicAdd(&counts[bin], __popc(peers));
+            base = __shfl_sync(peers, base, leader);
+            if (FILL) list[offsets[bin] + base + rank] = (int)f;
+        }
+    }
+}
+
+// Exclusive scan of nb counts by one 1024-thread CTA; offsets[nb] = total.
+__global__ void k_scan(const int* __restrict__ counts, int nb, int* __restrict__ offsets,
+                       long long* __restrict__ total) {
+    __shared__ long long part[1024];
+    const int t = threadIdx.x;
+    const int per = (nb + 1023) / 1024;
+    const int lo = min(nb, t * per), hi = min(nb, lo + per);
+    long long s = 0;
+    for (int i = lo; i < hi; ++i) s += counts[i];
+    part[t] = s;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+        long long v = t >= o ? part[t - o] : 0;
+        __syncthreads();
+        part[t] += v;
+        __syncthreads();
+    }
+    long long run = t ? part[t - 1] : 0;
+    for (int i = lo; i < hi; ++i) {
+        offsets[i] = (int)run;
+        run += counts[i];
+    }
+    if (t == 1023) {
+        offsets[nb] = (int)part[1023];
+        *total = part[1023];
+    }
+}
+
+// ------------------------------------------------------------------ fine pass
+// Bin-local constants of one face, computed in float64 from the exact vertices.  The
+// origin is the centre of the bin's first pixel.  The winding is made counter-clockwise
+// (b and c swapped if needed) so every edge function is positive inside.  Per edge
+// u -> v with unit direction d and length L:
+//     c(p) = -d.y * p.x + d.x * p.y + ng   signed distance to the edge line (inside > 0)
+//     s(p) =  d.x * p.x + d.y * p.y + tg   position along the edge from u
+//     squared distance to the segment = c^2 + max(-s, s - L, 0)^2.
+// The depth key is the plane through (x, y, z) -- or (x, y, -1/z) with perspective
+// correction, where 1/z is screen-affine -- as gx * p.x + gy * p.y + (k_hi + k_lo);
+// the float-float constant keeps the key within half an ulp plus the plane terms.
+template <bool PERSP>
+__device__ void face_constants(const FaceGeom& g, double ox, double oy, int fid, float4* out) {
+    double x[3] = {(double)g.a.x - ox, (double)g.b.x - ox, (double)g.c.x - ox};
+    double y[3] = {(double)g.a.y - oy, (double)g.b.y - oy, (double)g.c.y - oy};
+    double q[3];
+    if (PERSP) {
+        q[0] = -1.0 / (double)g.a.z; q[1] = -1.0 / (double)g.b.z; q[2] = -1.0 / (double)g.c.z;
+    } else {
+        q[0] = g.a.z; q[1] = g.b.z; q[2] = g.c.z;
+    }
+    double area2 = (x[1] - x[0]) * (y[2] - y[0]) - (y[1] - y[0]) * (x[2] - x[0]);
+    // depth-key plane (independent of winding)
+    double nx = (y[1] - y[0]) * (q[2] - q[0]) - (q[1] - q[0]) * (y[2] - y[0]);
+    double ny = (q[1] - q[0]) * (x[2] - x[0]) - (x[1] - x[0]) * (q[2] - q[0]);
+    double gx = -nx / area2, gy = -ny / area2;
+    double k0 = q[0] - gx * x[0] - gy * y[0];
+    float khi = (float)k0;
+    float klo = (float)(k0 - (double)khi);
+    if (area2 < 0.0) {
+        double t = x[1]; x[1] = x[2]; x[2] = t;
+        t = y[1]; y[1] = y[2]; y[2] = t;
+    }
+    float e[3][5];
+    for (int k = 0; k < 3; ++k) {
+        int k1 = k == 2 ? 0 : k + 1;
+        double ex = x[k1] - x[k], ey = y[k1] - y[k];
+        double L = sqrt(ex * ex + ey * ey);
+        double dx = ex / L, dy = ey / L;
+        e[k][0] = (float)dx;
+        e[k][1] = (float)dy;
+        e[k][2] = (float)(dy * x[k] - dx * y[k]);
+        e[k][3] = (float)(-(dx * x[k] + dy * y[k]));
+        e[k][4] = (float)L;
+    }
+    out[0] = make_float4(e[0][0], e[0][1], e[0][2], e[0][3]);
+    out[1] = make_float4(e[1][0], e[1][1], e[1][2], e[1][3]);
+    out[2] = make_float4(e[2][0], e[2][1], e[2][2], e[2][3]);
+    out[3] = make_float4(e[0][4], e[1][4], e[2][4], (float)gx);
+    out[4] = make_float4((float)gy, khi, klo, __int_as_float(fid));
+}
+
+template <int KC>
+__device__ __forceinline__ void topk_insert(float (&kk)[KC], int (&ff)[KC], float key, int fid) {
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+        bool lt = key < kk[k] || (key == kk[k] && fid < ff[k]);
+        float tk = lt ? kk[k] : key;
+        int tf = lt ? ff[k] : fid;
+        kk[k] = lt ? key : kk[k];
+        ff[k] = lt ? fid : ff[k];
+        key = tk;
+        fid = tf;
+    }
+}
+
+// Exact (float64) per-slot outputs from the original vertices: the definition written
+// out -- edge-function barycentrics, closed-triangle inside test, nearest-edge squared
+// distance, perspective renormalisation, interpolated z.
+template <bool PERSP>
+__device__ void slot_outputs(const FaceGeom& g, double px, double py, float* z_out, float* b_out,
+                             float* d_out) {
+    double ax = g.a.x, ay = g.a.y, bx = g.b.x, by = g.b.y, cx = g.c.x, cy = g.c.y;
+    double area2 = (bx - ax) * (cy - ay) - (by - ay) * (cx - ax);
+    double w0 = ((bx - px) * (cy - py) - (by - py) * (cx - px)) / area2;
+    double w1 = ((cx - px) * (ay - py) - (cy - py) * (ax - px)) / area2;
+    double w2 = ((ax - px) * (by - py) - (ay - py) * (bx - px)) / area2;
+    bool inside = w0 >= 0.0 && w1 >= 0.0 && w2 >= 0.0;
+    double d2 = DBL_MAX;
+    const double ux[3] = {ax, bx, cx}, uy[3] = {ay, by, cy};
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        int k1 = k == 2 ? 0 : k + 1;
+        double ex = ux[k1] - ux[k], ey = uy[k1] - uy[k];
+        double len2 = ex * ex + ey * ey;
+        double t = len2 > 0.0 ? ((px - ux[k]) * ex + (py - uy[k]) * ey) / len2 : 0.0;
+        t = fmin(fmax(t, 0.0), 1.0);
+        double rx = px - (ux[k] + t * ex), ry = py - (uy[k] + t * ey);
+        d2 = fmin(d2, rx * rx + ry * ry);
+    }
+    double b0 = w0, b1 = w1, b2 = w2;
+    if (PERSP) {
+        double u0 = w0 / (double)g.a.z, u1 = w1 / (double)g.b.z, u2 = w2 / (double)g.c.z;
+        double s = u0 + u1 + u2;
+        b0 = u0 / s; b1 = u1 / s; b2 = u2 / s;
+    }
+    *z_out = (float)(b0 * (double)g.a.z + b1 * (double)g.b.z + b2 * (double)g.c.z);
+    b_out[0] = (float)b0;
+    b_out[1] = (float)b1;
+    b_out[2] = (float)b2;
+    *d_out = (float)(inside ? -d2 : d2);
+}
+
+template <int KC, bool PERSP, bool SIL>
+__global__ void __launch_bounds__(kFineThreads)
+k_fine(const FaceGeom* __restrict__ geom, const FaceBox* __restrict__ box,
+       const int* __restrict__ offsets, const int* __restrict__ list, int nbx, int nby, int H, int W,
+       int K, float blur, float sigma, bool vec_ok, int64_t* __restrict__ p2f,
+       float* __restrict__ zbuf, float* __restrict__ bary, float* __restrict__ dists,
+       float* __restrict__ alpha) {
+    __shared__ float4 s_face[kChunk * kConstF4];
+    __shared__ unsigned char s_wlist[kWarpsPerBin][kChunk];
+    __shared__ int s_wcount[kWarpsPerBin];
+
+    const int bin = blockIdx.x;
+    const int bxi = bin % nbx;
+    const int byi = (bin / nbx) % nby;
+    const int n = bin / (nbx * nby);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wx = (warp & 1) * kWarpTileW, wy = (warp >> 1) * kWarpTileH;
+    const int tx = wx + (lane & 7), ty = wy + (lane >> 3);
+    const int j0 = bxi * kBin, i0 = byi * kBin;
+    const int j = j0 + tx, i = i0 + ty;
+    // bin-local pixel coordinates (origin = centre of pixel (i0, j0))
+    const float px = (float)(2.0 * tx / W);
+    const float py = (float)(-2.0 * ty / H);
+    const double ox = -1.0 + (2.0 * j0 + 1.0) / W;
+    const double oy = 1.0 - (2.0 * i0 + 1.0) / H;
+
+    float kk[KC];
+    int ff[KC];
+#pragma unroll
+    for (int k = 0; k < KC; ++k) { kk[k] = FLT_MAX; ff[k] = INT_MAX; }
+
+    const int beg = offsets[bin], cnt = offsets[bin + 1] - beg;
+    for (int c0 = 0; c0 < cnt; c0 += kChunk) {
+        if (threadIdx.x < kWarpsPerBin) s_wcount[threadIdx.x] = 0;
+        __syncthreads();
+        const int t = threadIdx.x;
+        if (c0 + t < cnt) {
+            const int fid = list[beg + c0 + t];
+            const FaceBox b = box[fid];
+            const FaceGeom g = geom[fid];
+            face_constants<PERSP>(g, ox, oy, fid, &s_face[t * kConstF4]);
+            // append to every warp tile the box touches
+#pragma unroll
+            for (int w = 0; w < kWarpsPerBin; ++w) {
+                int tj0 = j0 + (w & 1) * kWarpTileW, ti0 = i0 + (w >> 1) * kWarpTileH;
+                bool hit = b.x0 <= tj0 + kWarpTileW - 1 && b.x1 >= tj0 && b.y0 <= ti0 + kWarpTileH - 1 &&
+                           b.y1 >= ti0;
+                if (hit) {
+                    int pos = atomicAdd(&s_wcount[w], 1);
+                    s_wlist[w][pos] = (unsigned char)t;
+                }
+            }
+        }
+        __syncthreads();
+        const int nq = s_wcount[warp];
+        for (int qi = 0; qi < nq; ++qi) {
+            const float4* fc = &s_face[s_wlist[warp][qi] * kConstF4];
+            const float4 e0 = fc[0], e1 = fc[1], e2 = fc[2], e3 = fc[3], e4 = fc[4];
+            const float c0 = fmaf(-e0.y, px, fmaf(e0.x, py, e0.z));
+            const float s0 = fmaf(e0.x, px, fmaf(e0.y, py, e0.w));
+            const float c1 = fmaf(-e1.y, px, fmaf(e1.x, py, e1.z));
+            const float s1 = fmaf(e1.x, px, fmaf(e1.y, py, e1.w));
+            const float c2 = fmaf(-e2.y, px, fmaf(e2.x, py, e2.z));
+            const float s2 = fmaf(e2.x, px, fmaf(e2.y, py, e2.w));
+            const float o0 = fmaxf(fmaxf(-s0, s0 - e3.x), 0.f);
+            const float o1 = fmaxf(fmaxf(-s1, s1 - e3.y), 0.f);
+            const float o2 = fmaxf(fmaxf(-s2, s2 - e3.z), 0.f);
+            const float d0 = fmaf(o0, o0, c0 * c0);
+            const float d1 = fmaf(o1, o1, c1 * c1);
+            const float d2 = fmaf(o2, o2, c2 * c2);
+            const bool inside = fminf(c0, fminf(c1, c2)) >= 0.f;
+            const float dmin = fminf(d0, fminf(d1, d2));
+            const float key = e4.y + fmaf(e3.w, px, fmaf(e4.x, py, e4.z));
+            const bool front = PERSP ? key < 0.f : key >= 0.f;
+            if ((inside || dmin <= blur) && front && key <= kk[KC - 1])
+                topk_insert<KC>(kk, ff, key, __float_as_int(e4.w));
+        }
+        __syncthreads();
+    }
+
+    if (i >= H || j >= W) return;
+    const double pxd = -1.0 + (2.0 * j + 1.0) / W;
+    const double pyd = 1.0 - (2.0 * i + 1.0) / H;
+    const int64_t pix = ((int64_t)n * H + i) * W + j;
+    float dsil[KC];
+    bool vsil[KC];
+    if (vec_ok && (KC % 4) == 0 && K == KC) {
+#pragma unroll
+        for (int k4 = 0; k4 < KC; k4 += 4) {
+            float zz[4], bb[12], dd[4];
+            long long pf[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int k = k4 + u;
+                if (ff[k] != INT_MAX) {
+                    slot_outputs<PERSP>(geom[ff[k]], pxd, pyd, &zz[u], &bb[3 * u], &dd[u]);
+                    pf[u] = ff[k];
+                } else {
+                    zz[u] = -1.f; dd[u] = -1.f; bb[3 * u] = bb[3 * u + 1] = bb[3 * u + 2] = -1.f;
+                    pf[u] = -1;
+                }
+                dsil[k] = dd[u];
+                vsil[k] = ff[k] != INT_MAX;
+            }
+            const int64_t s = pix * KC + k4;
+            reinterpret_cast<longlong2*>(p2f + s)[0] = make_longlong2(pf[0], pf[1]);
+            reinterpret_cast<longlong2*>(p2f + s)[1] = make_longlong2(pf[2], pf[3]);
+            *reinterpret_cast<float4*>(zbuf + s) = make_float4(zz[0], zz[1], zz[2], zz[3]);
+            *reinterpret_cast<float4*>(dists + s) = make_float4(dd[0], dd[1], dd[2], dd[3]);
+            float4* bp = reinterpret_cast<float4*>(bary + 3 * s);
+            bp[0] = make_float4(bb[0], bb[1], bb[2], bb[3]);
+            bp[1] = make_float4(bb[4], bb[5], bb[6], bb[7]);
+            bp[2] = make_float4(bb[8], bb[9], bb[10], bb[11]);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < KC; ++k) {
+            if (k >= K) break;
+            const int64_t s = pix * K + k;
+            float zz, bb[3], dd;
+            if (ff[k] != INT_MAX) {
+                slot_outputs<PERSP>(geom[ff[k]], pxd, pyd, &zz, bb, &dd);
+                p2f[s] = ff[k];
+            } else {
+                zz = -1.f; dd = -1.f; bb[0] = bb[1] = bb[2] = -1.f;
+                p2f[s] = -1;
+            }
+            zbuf[s] = zz;
+            dists[s] = dd;
+            bary[3 * s] = bb[0]; bary[3 * s + 1] = bb[1]; bary[3 * s + 2] = bb[2];
+            dsil[k] = dd;
+            vsil[k] = ff[k] != INT_MAX;
+        }
+    }
+    if (SIL) alpha[pix] = silhouette_alpha<KC>(dsil, vsil, K, sigma);
+}
+
+template <int KC, bool PERSP, bool SIL>
+void launch_fine(int nbins, cudaStream_t s, const FaceGeom* geom, const FaceBox* box, const int* offsets,
+                 const int* list, int nbx, int nby, int H, int W, int K, float blur, float sigma,
+                 bool vec_ok, int64_t* p2f, float* zbuf, float* bary, float* dists, float* alpha) {
+    k_fine<KC, PERSP, SIL><<<nbins, kFineThreads, 0, s>>>(geom, box, offsets, list, nbx, nby, H, W, K, blur,
+                                                          sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
+}
+
+template <bool PERSP, bool SIL>
+void dispatch_k(int KC, int nbins, cudaStream_t s, const FaceGeom* geom, const FaceBox* box,
+                const int* offsets, const int* list, int nbx, int nby, int H, int W, int K, float blur,
+                float sigma, bool vec_ok, int64_t* p2f, float* zbuf, float* bary, float* dists,
+                float* alpha) {
+#define MR_FINE(KCV)                                                                                     \
+    launch_fine<KCV, PERSP, SIL>(nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma,     \
+                                 vec_ok, p2f, zbuf, bary, dists, alpha)
+    switch (KC) {
+        case 1: MR_FINE(1); break;
+        case 2: MR_FINE(2); break;
+        case 4: MR_FINE(4); break;
+        case 8: MR_FINE(8); break;
+        case 16: MR_FINE(16); break;
+        default: MR_FINE(32); break;
+    }
+#undef MR_FINE
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate_fwd(const float* verts, int64_t V, const int64_t* faces, int64_t F, const int64_t* first,
+                 const int64_t* num, int32_t N, int32_t H, int32_t W, float blur, int32_t K,
+                 const void* p2f, const void* zbuf, const void* bary, const void* dists) {
+    if (N < 0 || H < 1 || W < 1 || H > MR_MAX_SIDE || W > MR_MAX_SIDE) {
+        set_error("invalid image batch N=%d H=%d W=%d", N, H, W);
+        return MR_ERR_ARG;
+    }
+    if (K < 1 || K > MR_KMAX) {
+        set_error("K=%d outside 1..%d", K, MR_KMAX);
+        return MR_ERR_ARG;
+    }
+    if (!(blur >= 0.f) || !std::isfinite(blur)) {
+        set_error("blur_radius must be finite and >= 0");
+        return MR_ERR_ARG;
+    }
+    if (V < 0 || F < 0 || V > INT32_MAX || F > INT32_MAX) {
+        set_error("V=%lld F=%lld outside 0..2^31-1", (long long)V, (long long)F);
+        return MR_ERR_ARG;
+    }
+    if ((F > 0 && (!faces || !verts)) || (N > 0 && (!first || !num))) {
+        set_error("null input pointer");
+        return MR_ERR_ARG;
+    }
+    if (N > 0 && (!p2f || !zbuf || !bary || !dists)) {
+        set_error("null output pointer");
+        return MR_ERR_ARG;
+    }
+    for (int n = 0; n < N; ++n) {
+        if (first[n] < 0 || num[n] < 0 || first[n] + num[n] > F) {
+            set_error("mesh %d: faces [%lld, %lld) outside [0, F=%lld)", n, (long long)first[n],
+                      (long long)(first[n] + num[n]), (long long)F);
+            return MR_ERR_ARG;
+        }
+    }
+    return MR_OK;
+}
+
+int rasterize_impl(const float* verts, int64_t V, const int64_t* faces, int64_t F, const int64_t* first,
+                   const int64_t* num, int32_t N, int32_t H, int32_t W, float blur, int32_t K, int32_t persp,
+                   float sigma, bool sil, int64_t* p2f, float* zbuf, float* bary, float* dists, float* alpha,
+                   cudaStream_t s) {
+    int rc = validate_fwd(verts, V, faces, F, first, num, N, H, W, blur, K, p2f, zbuf, bary, dists);
+    if (rc != MR_OK) return rc;
+    if (sil && (!(sigma > 0.f) || !std::isfinite(sigma) || (N > 0 && !alpha))) {
+        set_error("silhouette needs a finite sigma > 0 and an alpha buffer");
+        return MR_ERR_ARG;
+    }
+    if (N == 0) return MR_OK;
+    const int nbx = ceil_div(W, kBin), nby = ceil_div(H, kBin);
+    const long long nbins_ll = (long long)N * nbx * nby;
+    if (nbins_ll >= INT32_MAX / 2) {
+        set_error("too many screen bins (%lld)", nbins_ll);
+        return MR_ERR_ARG;
+    }
+    const int nbins = (int)nbins_ll;
+    std::vector<int64_t> prefix(N + 1, 0);
+    for (int n = 0; n < N; ++n) prefix[n + 1] = prefix[n] + num[n];
+    const int64_t pairs = prefix[N];
+
+    // one scratch block: geometry | boxes | counts | offsets | prefix | first | total | error
+    auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
+    const size_t o_geom = 0;
+    const size_t o_box = o_geom + up(sizeof(FaceGeom) * (size_t)F);
+    const size_t o_cnt = o_box + up(sizeof(FaceBox) * (size_t)F);
+    const size_t o_off = o_cnt + up(sizeof(int) * (size_t)nbins);
+    const size_t o_pre = o_off + up(sizeof(int) * (size_t)(nbins + 1));
+    const size_t o_fst = o_pre + up(sizeof(int64_t) * (size_t)(N + 1));
+    const size_t o_tot = o_fst + up(sizeof(int64_t) * (size_t)N);
+    const size_t o_err = o_tot + 256;
+    const size_t bytes = o_err + 256;
+    char* ws = nullptr;
+    rc = scratch_alloc(reinterpret_cast<void**>(&ws), bytes, s);
+    if (rc != MR_OK) return rc;
+    FaceGeom* geom = reinterpret_cast<FaceGeom*>(ws + o_geom);
+    FaceBox* box = reinterpret_cast<FaceBox*>(ws + o_box);
+    int* counts = reinterpret_cast<int*>(ws + o_cnt);
+    int* offsets = reinterpret_cast<int*>(ws + o_off);
+    int64_t* d_prefix = reinterpret_cast<int64_t*>(ws + o_pre);
+    int64_t* d_first = reinterpret_cast<int64_t*>(ws + o_fst);
+    long long* d_total = reinterpret_cast<long long*>(ws + o_tot);
+    int* d_err = reinterpret_cast<int*>(ws + o_err);
+    int* list = nullptr;
+
+    auto fail = [&](int code) {
+        scratch_free(list, s);
+        scratch_free(ws, s);
+        return code;
+    };
+#define MR_TRY(call)                                    \
+    do {                                                \
+        cudaError_t e_ = (call);                        \
+        if (e_ != cudaSuccess) return fail(cuda_fail(e_, #call)); \
+    } while (0)
+
+    MR_TRY(cudaMemcpyAsync(d_prefix, prefix.data(), sizeof(int64_t) * (N + 1), cudaMemcpyHostToDevice, s));
+    MR_TRY(cudaMemcpyAsync(d_first, first, sizeof(int64_t) * N, cudaMemcpyHostToDevice, s));
+    MR_TRY(cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)nbins, s));
+    MR_TRY(cudaMemsetAsync(d_err, 0, sizeof(int), s));
+    const double reach = std::sqrt((double)blur) * (1.0 + 1e-6) + 1e-7;
+    if (F > 0) {
+        k_face_setup<<<(unsigned)((F + 255) / 256), 256, 0, s>>>(verts, V, faces, F, H, W, reach, geom, box, d_err);
+        MR_TRY(cudaGetLastError());
+    }
+    const int pair_blocks = (int)std::min<int64_t>((pairs + 255) / 256, 148 * 16);
+    if (pairs > 0) {
+        k_bin_pairs<false><<<pair_blocks, 256, 0, s>>>(box, d_prefix, d_first, N, pairs, nbx, nby, counts,
+                                                       nullptr, nullptr);
+        MR_TRY(cudaGetLastError());
+    }
+    k_scan<<<1, 1024, 0, s>>>(counts, nbins, offsets, d_total);
+    MR_TRY(cudaGetLastError());
+    long long host[2] = {0, 0};
+    MR_TRY(cudaMemcpyAsync(&host[0], d_total, sizeof(long long), cudaMemcpyDeviceToHost, s));
+    int herr = 0;
+    MR_TRY(cudaMemcpyAsync(&herr, d_err, sizeof(int), cudaMemcpyDeviceToHost, s));
+    MR_TRY(cudaStreamSynchronize(s));
+    const long long total = host[0];
+    if (total >= INT32_MAX) {
+        set_error("bin lists too long (%lld entries)", total);
+        return fail(MR_ERR_ARG);
+    }
+    if (total > 0) {
+        rc = scratch_alloc(reinterpret_cast<void**>(&list), sizeof(int) * (size_t)total, s);
+        if (rc != MR_OK) return fail(rc);
+        MR_TRY(cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)nbins, s));
+        k_bin_pairs<true><<<pair_blocks, 256, 0, s>>>(box, d_prefix, d_first, N, pairs, nbx, nby, counts, offsets,
+                                                      list);
+        MR_TRY(cudaGetLastError());
+    }
+    const int KC = K <= 1 ? 1 : K <= 2 ? 2 : K <= 4 ? 4 : K <= 8 ? 8 : K <= 16 ? 16 : 32;
+    const bool vec_ok = aligned16(p2f) && aligned16(zbuf) && aligned16(bary) && aligned16(dists);
+    if (persp) {
+        if (sil) dispatch_k<true, true>(KC, nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
+        else dispatch_k<true, false>(KC, nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
+    } else {
+        if (sil) dispatch_k<false, true>(KC, nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
+        else dispatch_k<false, false>(KC, nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
+    }
+    MR_TRY(cudaGetLastError());
+#undef MR_TRY
+    scratch_free(list, s);
+    scratch_free(ws, s);
+    if (herr != 0) {
+        set_error("a face references a vertex id outside [0, V=%lld); it was ignored", (long long)V);
+        return MR_ERR_DEVICE;
+    }
+    return MR_OK;
+}
+
+}  // namespace
+}  // namespace mr
+
+extern "C" {
+
+int mr_rasterize_fwd(const float* verts, int64_t V, const int64_t* faces, int64_t F,
+                     const int64_t* mesh_to_face_first_idx, const int64_t* num_faces_per_mesh, int32_t N,
+                     int32_t H, int32_t W, float blur_radius, int32_t K, int32_t perspective_correct,
+                     int64_t* pix_to_face, float* zbuf, float* bary, float* dists, void* stream) {
+    return mr::rasterize_impl(verts, V, faces, F, mesh_to_face_first_idx, num_faces_per_mesh, N, H, W, blur_radius,
+                              K, perspective_correct, 0.f, false, pix_to_face, zbuf, bary, dists, nullptr,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int mr_rasterize_silhouette_fwd(const float* verts, int64_t V, const int64_t* faces, int64_t F,
+                                const int64_t* mesh_to_face_first_idx, const int64_t* num_faces_per_mesh,
+                                int32_t N, int32_t H, int32_t W, float blur_radius, int32_t K,
+                                int32_t perspective_correct, float sigma, int64_t* pix_to_face, float* zbuf,
+                                float* bary, float* dists, float* alpha, void* stream) {
+    return mr::rasterize_impl(verts, V, faces, F, mesh_to_face_first_idx, num_faces_per_mesh, N, H, W, blur_radius,
+                              K, perspective_correct, sigma, true, pix_to_face, zbuf, bary, dists, alpha,
+                              static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,46 @@
+// Soft-silhouette arithmetic shared by the fused forward epilogue, the stand-alone
+// silhouette kernels and the fused backward (internal header).
+//
+// PyTorch3D paper, method: the second stage fuses the influence of the K faces kept per
+// pixel.  Per valid slot p_k = 1 / (1 + exp(d_k / sigma)); alpha = 1 - prod_k (1 - p_k).
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace mr {
+
+// alpha evaluated as -expm1(sum_k log(1 - p_k)) with log(1 - p_k) = -log1p(exp(-d_k / sigma)):
+// full relative accuracy both for alpha near 0 (far blur ring) and near 1 (interior).
+template <int KC>
+__device__ __forceinline__ float silhouette_alpha(const float (&d)[KC], const bool (&valid)[KC], int K,
+                                                  float sigma) {
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < KC; ++k)
+        if (k < K && valid[k]) s -= log1pf(expf(-(d[k] / sigma)));
+    return -expm1f(s);
+}
+
+// dL/dd_k = -dL/dalpha * prod_{j != k} (1 - p_j) * p_k (1 - p_k) / sigma; 0 for empty slots.
+// The product over j != k is formed directly (no division by 1 - p_k).
+template <int KC>
+__device__ __forceinline__ void silhouette_grad(const float (&d)[KC], const bool (&valid)[KC], int K, float sigma,
+                                                float grad_alpha, float (&g)[KC]) {
+    float q[KC], p[KC];
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+        const float x = d[k] / sigma;
+        q[k] = 1.f / (1.f + expf(-x));   // 1 - p_k
+        p[k] = 1.f / (1.f + expf(x));
+    }
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+        float others = 1.f;
+#pragma unroll
+        for (int j = 0; j < KC; ++j)
+            if (j != k && j < K && valid[j]) others *= q[j];
+        g[k] = (k < K && valid[k]) ? -grad_alpha * others * p[k] * q[k] / sigma : 0.f;
+    }
+}
+
+}  // namespace mr

@@ -1,0 +1,160 @@
+/*
+ * meshrast.h -- C ABI of the B200 (sm_100a) mesh rasterizer hot path.
+ *
+ * The operation is the two-stage differentiable mesh rasterizer of PyTorch3D
+ * ("Accelerating 3D Deep Learning with PyTorch3D"): stage one keeps, for every pixel,
+ * the K nearest faces (method summary: "two-stage rasterization with per-pixel K
+ * nearest faces"); stage two blends their influence into a soft silhouette; the
+ * backward pass carries pixel gradients back to the vertex positions (tutorial
+ * summary, 3:52: "backpropagation of gradients from 2D image pixels back to 3D model
+ * parameters").  The batch is heterogeneous and packed (tutorial summary, 1:00).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Screen space: verts are (x_ndc, y_ndc, z_view) per vertex, float32, row-major
+ *    V x 3.  Pixel (i, j) of an H x W image has centre x = -1 + (2j+1)/W,
+ *    y = 1 - (2i+1)/H: +x right, +y up, row 0 at the top.
+ *  - faces: int64, F x 3, global (packed) vertex ids.  Mesh n owns faces
+ *    [mesh_to_face_first_idx[n], mesh_to_face_first_idx[n] + num_faces_per_mesh[n]).
+ *  - Per-pixel outputs are N x H x W x K, slot k innermost; bary adds a trailing 3.
+ *  - pix_to_face holds the global face id, -1 for an empty slot.  Empty slots hold -1
+ *    in zbuf, in all three bary components and in dists.
+ *  - dists is the signed squared 2-D distance to the face: negative inside.
+ *  - blur_radius is a threshold on that squared distance (NDC^2 units): a face is a
+ *    candidate for a pixel iff the pixel centre is inside the closed triangle or
+ *    within squared distance blur_radius of it.  Candidates are ordered by (z, face id);
+ *    degenerate faces (|2 * area| <= 1e-12) and candidates with z < 0 are dropped.
+ *  - Pointers are DEVICE pointers unless marked HOST.  The caller owns every input and
+ *    output; the library allocates its own scratch (stream-ordered, from the device's
+ *    default memory pool, released before the call returns) and never frees caller
+ *    memory.  stream is a cudaStream_t (NULL = legacy default stream).
+ *  - Every function returns MR_OK (0) or a negative MR_ERR_* code and never aborts.
+ *    Arguments are validated on the host before any launch; on MR_ERR_ARG nothing
+ *    was launched.  mr_last_error() gives a thread-local message for the last failure.
+ *  - Device-side checks (a face vertex id outside [0, V), a pix_to_face entry outside
+ *    [-1, F)) never trap: the offending face or slot is skipped and a device error
+ *    word is set.  mr_rasterize_fwd reads it before returning; the asynchronous entry
+ *    points leave it for mr_device_status().
+ */
+#ifndef MESHRAST_H
+#define MESHRAST_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MR_OK 0
+#define MR_ERR_ARG (-1)     /* invalid argument; nothing launched */
+#define MR_ERR_OOM (-2)     /* scratch allocation failed */
+#define MR_ERR_CUDA (-3)    /* a CUDA runtime call failed (message in mr_last_error) */
+#define MR_ERR_DEVICE (-4)  /* a kernel met an out-of-range index and skipped it */
+
+#define MR_KMAX 32          /* largest K (faces kept per pixel) */
+#define MR_MAX_SIDE 32767   /* largest H or W */
+
+/*
+ * Stage one (PyTorch3D paper, method: per-pixel K nearest faces; tutorial 32:56:
+ * perspective_correct).  For each image n and pixel, the K candidate faces of mesh n
+ * nearest in z, with their z, barycentrics and signed squared distance.
+ *
+ *   verts                    V x 3 float32 (device)
+ *   faces                    F x 3 int64 (device), every id in [0, V)
+ *   mesh_to_face_first_idx   N int64 (HOST)
+ *   num_faces_per_mesh       N int64 (HOST); first + num <= F for every mesh
+ *   H, W                     1 .. MR_MAX_SIDE
+ *   blur_radius              >= 0, finite (squared NDC units)
+ *   K                        1 .. MR_KMAX
+ *   perspective_correct      0: barycentrics are the screen-space edge-function
+ *                            weights w_k; 1: u_k = w_k / z_k renormalised to sum 1.
+ *                            Barycentrics are never clipped (they sum to 1).
+ *   pix_to_face              N x H x W x K int64 (device, written)
+ *   zbuf, dists              N x H x W x K float32 (device, written)
+ *   bary                     N x H x W x K x 3 float32 (device, written)
+ *
+ * Synchronises `stream` once (to size the per-bin face lists).  Returns MR_ERR_DEVICE
+ * if a face referenced a vertex outside [0, V) (that face is then ignored).
+ */
+int mr_rasterize_fwd(const float* verts, int64_t V, const int64_t* faces, int64_t F,
+                     const int64_t* mesh_to_face_first_idx, const int64_t* num_faces_per_mesh,
+                     int32_t N, int32_t H, int32_t W, float blur_radius, int32_t K,
+                     int32_t perspective_correct, int64_t* pix_to_face, float* zbuf,
+                     float* bary, float* dists, void* stream);
+
+/*
+ * Stage one fused with the stage-two silhouette: the outputs of mr_rasterize_fwd plus
+ * alpha (N x H x W float32), bitwise equal to mr_silhouette_blend_fwd applied to the
+ * dists written here.  sigma > 0.
+ */
+int mr_rasterize_silhouette_fwd(const float* verts, int64_t V, const int64_t* faces, int64_t F,
+                                const int64_t* mesh_to_face_first_idx,
+                                const int64_t* num_faces_per_mesh, int32_t N, int32_t H,
+                                int32_t W, float blur_radius, int32_t K,
+                                int32_t perspective_correct, float sigma, int64_t* pix_to_face,
+                                float* zbuf, float* bary, float* dists, float* alpha,
+                                void* stream);
+
+/*
+ * Stage two, soft silhouette (PyTorch3D paper, method: the second stage fuses the
+ * influence of the K faces; tutorial 22:00: silhouette supervision).  Per pixel,
+ * p_k = 1 / (1 + exp(dists_k / sigma)) over slots with pix_to_face >= 0 and
+ * alpha = 1 - prod_k (1 - p_k); 0 for a pixel with no face.
+ *   pix_to_face N x H x W x K int64, dists N x H x W x K float32, alpha N x H x W float32.
+ * Asynchronous.
+ */
+int mr_silhouette_blend_fwd(const int64_t* pix_to_face, const float* dists, int32_t N,
+                            int32_t H, int32_t W, int32_t K, float sigma, float* alpha,
+                            void* stream);
+
+/*
+ * Gradient of the soft silhouette:
+ *   grad_dists_k = -grad_alpha * prod_{j != k} (1 - p_j) * p_k (1 - p_k) / sigma,
+ * 0 for empty slots.  grad_alpha N x H x W, grad_dists N x H x W x K (written).
+ * Asynchronous.
+ */
+int mr_silhouette_blend_bwd(const float* grad_alpha, const int64_t* pix_to_face,
+                            const float* dists, int32_t N, int32_t H, int32_t W, int32_t K,
+                            float sigma, float* grad_dists, void* stream);
+
+/*
+ * Backward of stage one to the screen-space vertex positions (tutorial 3:52).  For each
+ * valid slot the pixel's barycentrics, z and signed squared distance to face
+ * pix_to_face are recomputed and differentiated with the candidate set, the inside
+ * flag and the nearest edge held fixed.  grad_zbuf, grad_bary and grad_dists (shaped
+ * like zbuf, bary and dists) may each be NULL.  grad_verts (V x 3 float32) is
+ * overwritten.  Contributions are summed with float32 atomics, so the low bits of
+ * grad_verts depend on scheduling.  Asynchronous; a pix_to_face entry outside [-1, F)
+ * or a face vertex outside [0, V) is skipped and flagged for mr_device_status().
+ */
+int mr_rasterize_bwd(const float* verts, int64_t V, const int64_t* faces, int64_t F,
+                     const int64_t* pix_to_face, int32_t N, int32_t H, int32_t W, int32_t K,
+                     int32_t perspective_correct, const float* grad_zbuf, const float* grad_bary,
+                     const float* grad_dists, float* grad_verts, void* stream);
+
+/*
+ * mr_silhouette_blend_bwd followed by mr_rasterize_bwd with only grad_dists, fused so
+ * grad_dists never reaches memory.  The inside flag is read from the sign of dists
+ * (dists < 0: inside).  grad_verts (V x 3) is overwritten.  Asynchronous.
+ */
+int mr_silhouette_rasterize_bwd(const float* verts, int64_t V, const int64_t* faces, int64_t F,
+                                const int64_t* pix_to_face, const float* dists, int32_t N,
+                                int32_t H, int32_t W, int32_t K, float sigma,
+                                const float* grad_alpha, float* grad_verts, void* stream);
+
+/* Synchronises `stream`, then returns MR_ERR_DEVICE (and clears the word) if any
+ * asynchronous kernel of this library flagged an out-of-range index on the current
+ * device since the last call, else MR_OK (or MR_ERR_CUDA). */
+int mr_device_status(void* stream);
+
+/* Thread-local, NUL-terminated message for the last non-zero return ("" if none). */
+const char* mr_last_error(void);
+
+/* Library version as 10000 * major + 100 * minor + patch. */
+int mr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MESHRAST_H */

@@ -35,8 +35,9 @@
  * Besides the outputs, the forward marks pixels whose integer result is decided by a
  * float64-vs-float32 rounding: (E1) two of the K+1 nearest candidates lie within 1e-6
  * in depth; (E2) a face whose candidacy is within a margin of its threshold
- * (|d2 - blur| < 1e-6 max(1, blur), or min w within 1e-6 of 0 when blur is 0) would
- * rank among the first K.  These flags only steer the comparison; they change nothing.
+ * (|d2 - blur| < 1e-5 blur, or min w within 1e-6 of 0 when blur is 0) would rank among
+ * the first K.  The margins are tens of times the float32 error of evaluating d2 and w
+ * in bin-local coordinates.  These flags only steer the comparison; they change nothing.
  */
 #include <math.h>
 #include <pthread.h>
@@ -46,7 +47,8 @@
 
 #define DEGENERATE_AREA 1e-12
 #define TIE_DEPTH 1e-6
-#define MARGIN 1e-6
+#define MARGIN_W 1e-6       /* E2 margin on min w when blur_radius is 0 */
+#define MARGIN_BLUR 1e-5    /* E2 margin on |d2 - blur| relative to blur */
 
 typedef struct { double x, y, z; } vtx;
 
@@ -204,10 +206,10 @@ static void rasterize_pixel(fwd_job *J, int64_t pix_id, int64_t out_slot, zf *li
         if (r.degenerate) continue;
         int marginal;
         if (J->blur > 0.0) {
-            marginal = !r.inside && fabs(r.d2 - J->blur) < MARGIN * fmax(1.0, J->blur);
+            marginal = !r.inside && fabs(r.d2 - J->blur) < MARGIN_BLUR * J->blur;
         } else {
             double wmin = fmin(r.w[0], fmin(r.w[1], r.w[2]));
-            marginal = wmin > -MARGIN && wmin < MARGIN;
+            marginal = wmin > -MARGIN_W && wmin < MARGIN_W;
         }
         if (!marginal || r.z < 0.0) continue;
         int ahead = 0;
