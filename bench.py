@@ -1,0 +1,392 @@
+"""Throughput of the mesh rasterizer hot path on B200: pixel-face samples/s and Mpix/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
+
+One step is the whole hot path over one batch: stage one (face setup, coarse binning,
+fine rasterization with the fused soft silhouette) followed by the fused silhouette +
+rasterizer backward to the vertex positions, with dL/dalpha ~ N(0, 1).  The default
+workload is the 64-image 512x512 heterogeneous batch (32 icospheres of levels 3-6 and
+32 tori, K=4, sigma=1e-4).  Under torchrun every rank renders its own batch (seed offset
+by rank: weak scaling; no collective on the data path) and the reported time is the
+maximum over ranks.
+
+A pixel-face sample is a (pixel, face) pair of the same image whose pixel centre lies in
+the face's 2-D box grown by sqrt(blur_radius): the tests the method must make.  It is
+counted exactly on the host from the inputs.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "pixel-face samples/s and Mpix/s (fwd+bwd) at 1 B200; % of rasterizer roofline"
+UNIT = "pixel-face samples/s"
+C_TEST = 38                 # FP32 instructions per pixel-face test (frozen)
+FP32_LANES_PER_SM = 128
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------- counting
+def face_boxes(batch):
+    """Per (image, face) pixel boxes grown by sqrt(blur) (exact, float64), degenerate faces dropped."""
+    w = batch.workload
+    r = math.sqrt(w.blur_radius)
+    v = batch.verts.astype(np.float64)
+    out = []
+    for n in range(batch.N):
+        f0, nf = int(batch.mesh_to_face_first_idx[n]), int(batch.num_faces_per_mesh[n])
+        tri = v[batch.faces[f0:f0 + nf]]                        # (nf, 3, 3)
+        a, b, c = tri[:, 0], tri[:, 1], tri[:, 2]
+        area2 = (b[:, 0] - a[:, 0]) * (c[:, 1] - a[:, 1]) - (b[:, 1] - a[:, 1]) * (c[:, 0] - a[:, 0])
+        keep = np.abs(area2) > 1e-12
+        xmin, xmax = tri[:, :, 0].min(1) - r, tri[:, :, 0].max(1) + r
+        ymin, ymax = tri[:, :, 1].min(1) - r, tri[:, :, 1].max(1) + r
+        jl = np.maximum(np.ceil((xmin + 1) * w.W / 2 - 0.5), 0)
+        jh = np.minimum(np.floor((xmax + 1) * w.W / 2 - 0.5), w.W - 1)
+        il = np.maximum(np.ceil((1 - ymax) * w.H / 2 - 0.5), 0)
+        ih = np.minimum(np.floor((1 - ymin) * w.H / 2 - 0.5), w.H - 1)
+        ok = keep & (jl <= jh) & (il <= ih)
+        out.append((jl[ok], jh[ok], il[ok], ih[ok]))
+    return out
+
+
+def count_samples(batch, rows=None):
+    """Pixel-face samples of the batch; with ``rows`` only those image rows count."""
+    total = 0
+    for jl, jh, il, ih in face_boxes(batch):
+        width = jh - jl + 1
+        if rows is None:
+            total += int(np.sum(width * (ih - il + 1)))
+        else:
+            rr = np.asarray(rows)
+            inr = (rr[None, :] >= il[:, None]) & (rr[None, :] <= ih[:, None])
+            total += int(np.sum(width * inr.sum(1)))
+    return total
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        top = max(sm)
+        loaded = [x for x in sm if x >= 0.5 * top] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle leg
+def oracle_sample(batch, ga, seconds=15.0):
+    """A bounded sample of the workload for the CPU oracle: R evenly spaced rows of every
+    image, R chosen from a one-row calibration run so the sample takes about ``seconds``."""
+    w = batch.workload
+    t1 = run_oracle(batch, ga, np.array([w.H // 2]))
+    R = int(max(1, min(w.H, round(seconds / max(t1, 1e-3)))))
+    rows = np.unique(np.linspace(0, w.H - 1, R).round().astype(np.int64))
+    return rows, (f"{len(rows)} evenly spaced rows of each of the {batch.N} images "
+                  f"(fwd + silhouette fwd/bwd + raster bwd on those pixels)")
+
+
+def run_oracle(batch, ga, rows):
+    """Oracle fwd (no exemption diagnostics) + silhouette fwd/bwd + raster bwd on the sampled rows."""
+    import oracle
+    w = batch.workload
+    H, W, K = w.H, w.W, w.K
+    pix = ((np.arange(batch.N)[:, None, None] * H + rows[None, :, None]) * W +
+           np.arange(W)[None, None, :]).reshape(-1)
+    t0 = time.perf_counter()
+    p2f, zbuf, bary, dists, _ = oracle.rasterize_fwd(batch.verts, batch.faces, batch.mesh_to_face_first_idx,
+                                                     batch.num_faces_per_mesh, H, W, np.float32(w.blur_radius), K,
+                                                     w.perspective_correct, pixels=pix, exempt=False)
+    sig = np.float32(w.sigma)
+    oracle.silhouette_fwd(p2f, dists, sig)
+    gd = oracle.silhouette_bwd(ga.reshape(-1)[pix], p2f, dists, sig)
+    P2F = np.full((batch.N * H * W, K), -1, np.int64)
+    GD = np.zeros((batch.N * H * W, K))
+    P2F[pix] = p2f
+    GD[pix] = gd
+    oracle.rasterize_bwd(batch.verts, batch.faces, P2F.reshape(batch.N, H, W, K), w.perspective_correct,
+                         grad_dists=GD.reshape(batch.N, H, W, K))
+    return time.perf_counter() - t0
+
+
+def reference_arm(args, rank):
+    """`--impl reference`: the float64 CPU oracle on the host cores, bounded samples per step."""
+    if rank != 0:
+        return
+    from differentiable_mesh_rasterization_b200 import synthetic as syn
+    import oracle
+    oracle.build()
+    batch = syn.make_batch(args.config)
+    ga = syn.grad_alpha(batch)
+    budget = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    rows, desc = oracle_sample(batch, ga, seconds=budget)
+    samples = count_samples(batch, rows)
+    for _ in range(args.warmup):
+        run_oracle(batch, ga, rows[:1])
+    times = [run_oracle(batch, ga, rows) for _ in range(args.steps)]
+    t = sum(times)
+    w = batch.workload
+    value = samples * args.steps / t
+    cores = oracle.default_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w, args),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, args):
+    return {"workload": w.name, "description": w.description, "batch": w.N, "H": w.H, "W": w.W, "K": w.K,
+            "blur_radius": w.blur_radius, "sigma": w.sigma, "perspective_correct": w.perspective_correct,
+            "passes": "fwd+bwd" if w.backward else "fwd", "l2": "flushed (256 MiB write) between timed steps",
+            "parallelism": f"independent batch per GPU x{args.gpus}"}
+
+
+# ----------------------------------------------------------------------------- our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import differentiable_mesh_rasterization_b200 as mr
+    from differentiable_mesh_rasterization_b200 import synthetic as syn
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    batch = syn.make_batch(args.config, seed=1000 + args.config + 1000 * rank)
+    w = batch.workload
+    if w.sigma is None:
+        raise SystemExit("the benchmark step needs a soft-silhouette workload (sigma)")
+    samples = count_samples(batch)
+    verts = torch.from_numpy(batch.verts).to(dev)
+    faces = torch.from_numpy(batch.faces).to(dev)
+    ga_host = syn.grad_alpha(batch)
+    ga = torch.from_numpy(ga_host).to(dev)
+    first, num = batch.mesh_to_face_first_idx, batch.num_faces_per_mesh
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        p2f, zbuf, bary, dists, alpha = mr.rasterize_fwd(verts, faces, first, num, w.H, w.W, w.blur_radius, w.K,
+                                                         w.perspective_correct, sigma=w.sigma)
+        gv = mr.silhouette_rasterize_bwd(verts, faces, p2f, dists, w.sigma, ga)
+        return alpha, gv
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    mr.device_status(dev)
+
+    props = torch.cuda.get_device_properties(dev)
+    uuid = str(getattr(props, "uuid", "") or "")
+    uuid = ("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else uuid
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    mr.profile_enable(True)
+    with ClockSampler(uuid or None) as clocks:
+        for k in range(args.steps):
+            flush.zero_()
+            starts[k].record(stream)
+            step()
+            ends[k].record(stream)
+        torch.cuda.synchronize(dev)
+    mr.profile_enable(False)
+    if world > 1:
+        dist.barrier()
+    stages = mr.profile_read()
+    dev_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    t = torch.tensor([dev_ms, float(samples), float(w.N * w.H * w.W)], dtype=torch.float64, device=dev)
+    if world > 1:
+        tmax = t.clone()
+        dist.all_reduce(tmax[:1], op=dist.ReduceOp.MAX)
+        tsum = t.clone()
+        dist.all_reduce(tsum[1:], op=dist.ReduceOp.SUM)
+        dev_ms, tot_samples, tot_pix = float(tmax[0]), float(tsum[1]), float(tsum[2])
+    else:
+        tot_samples, tot_pix = float(samples), float(w.N * w.H * w.W)
+    sec = dev_ms / 1e3
+    value = tot_samples * args.steps / sec
+    mpix = tot_pix * args.steps / sec / 1e6
+
+    # end to end through the public API: pinned host inputs in, alpha + grad_verts out
+    h_verts = torch.from_numpy(batch.verts).pin_memory()
+    h_faces = torch.from_numpy(batch.faces).pin_memory()
+    h_ga = torch.from_numpy(ga_host).pin_memory()
+    h_alpha = torch.empty((w.N, w.H, w.W), dtype=torch.float32).pin_memory()
+    h_gv = torch.empty(batch.verts.shape, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        dv = h_verts.to(dev, non_blocking=True)
+        df = h_faces.to(dev, non_blocking=True)
+        dg = h_ga.to(dev, non_blocking=True)
+        p2f, _, _, dists, alpha = mr.rasterize_fwd(dv, df, first, num, w.H, w.W, w.blur_radius, w.K,
+                                                   w.perspective_correct, sigma=w.sigma)
+        gv = mr.silhouette_rasterize_bwd(dv, df, p2f, dists, w.sigma, dg)
+        h_alpha.copy_(alpha, non_blocking=True)
+        h_gv.copy_(gv, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        flush.zero_()
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = tot_samples * args.e2e_steps / (float(te[0]) / 1e3)
+    h2d = h_verts.numel() * 4 + h_faces.numel() * 8 + h_ga.numel() * 4
+    d2h = h_alpha.numel() * 4 + h_gv.numel() * 4
+
+    # roofline of the dominant kernel (the fine pass)
+    fine_ms, fine_n = stages["fine"]
+    fine_s = fine_ms / 1e3 / max(fine_n, 1)
+    clk = clocks.summary()
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        pass
+    sm_mhz_max = float(peaks.get("sm_max_mhz", 1965.0))
+    peak_alu = props.multi_processor_count * FP32_LANES_PER_SM * sm_mhz_max * 1e6 / 1e12   # T inst/s
+    achieved_alu = samples * C_TEST / fine_s / 1e12
+    out_bytes = w.N * w.H * w.W * (28 * w.K + 4) + int(batch.faces.shape[0]) * 64
+    hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
+    achieved_hbm = out_bytes / fine_s / 1e9
+    t_alu = samples * C_TEST / (peak_alu * 1e12)
+    t_hbm = out_bytes / (hbm_peak * 1e9)
+    if t_alu >= t_hbm:
+        roof = {"bound": "alu", "achieved": achieved_alu, "peak": peak_alu, "unit": "T FP32-inst/s",
+                "frac": achieved_alu / peak_alu, "traffic": None}
+    else:
+        roof = {"bound": "hbm", "achieved": achieved_hbm, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved_hbm / hbm_peak, "traffic": None}
+    roof.update({"kernel": "k_fine (stage-one fine pass + fused silhouette epilogue)",
+                 "fine_ms_per_launch": fine_s * 1e3, "samples_per_launch": samples, "c_test": C_TEST,
+                 "peak_note": f"alu peak = {props.multi_processor_count} SMs x 128 FP32 lanes x {sm_mhz_max:.0f} MHz "
+                              f"(unit counts and max clock); hbm peak = {hbm_peak} GB/s "
+                              f"({'of measured' if 'hbm_gbs' in peaks else 'of fallback'} copy)",
+                 "hbm_achieved_gbs": achieved_hbm, "hbm_frac_of_measured": achieved_hbm / hbm_peak,
+                 "t_roof_ms": max(t_alu, t_hbm) * 1e3, "roof_frac": max(t_alu, t_hbm) / fine_s})
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dev_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded icospheres and tori)",
+            "config": workload_config(w, args), "mpix_per_s": mpix,
+            "samples_per_step": tot_samples,
+            "stages_ms_per_step": {k: v[0] / args.steps for k, v in stages.items() if v[1]},
+            "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": float(te[0]) / args.e2e_steps},
+            "gpu_launches": int(sum(v[1] for v in stages.values())),
+            "clocks": clk}
+
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        rows, desc = oracle_sample(batch, ga_host)
+        osamp = count_samples(batch, rows)
+        tcpu = run_oracle(batch, ga_host, rows)
+        line["cpu_baseline"] = {"value": osamp / tcpu, "unit": UNIT, "cores": oracle.default_threads(),
+                                "kind": "oracle", "sample": desc, "seconds": tcpu}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -25,7 +25,9 @@ ERRORS = {-1: "invalid argument", -2: "out of memory", -3: "CUDA error", -4: "de
 # Entry points declared by include/meshrast.h (checked by the test-suite).
 EXPORTS = ("mr_rasterize_fwd", "mr_rasterize_silhouette_fwd", "mr_silhouette_blend_fwd",
            "mr_silhouette_blend_bwd", "mr_rasterize_bwd", "mr_silhouette_rasterize_bwd",
-           "mr_device_status", "mr_last_error", "mr_version")
+           "mr_device_status", "mr_last_error", "mr_version", "mr_profile_enable", "mr_profile_read")
+STAGES = ("face_setup", "bin_count", "bin_scan", "bin_fill", "fine", "silhouette_fwd", "silhouette_bwd",
+          "raster_bwd", "silhouette_raster_bwd")
 
 
 class MeshRastError(RuntimeError):
@@ -57,6 +59,8 @@ def load_library() -> ctypes.CDLL:
         "mr_device_status": [P],
         "mr_last_error": [],
         "mr_version": [],
+        "mr_profile_enable": [i32],
+        "mr_profile_read": [P, P, i32],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -220,6 +224,20 @@ def device_status(device=None) -> None:
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     with torch.cuda.device(dev):
         _check("mr_device_status", lib.mr_device_status(_stream(dev)))
+
+
+def profile_enable(on: bool = True) -> None:
+    """Start (or stop) recording CUDA events around every kernel stage (``mr_profile_enable``)."""
+    _check("mr_profile_enable", load_library().mr_profile_enable(int(bool(on))))
+
+
+def profile_read() -> dict:
+    """Summed device milliseconds and launch counts per stage since the last read."""
+    n = len(STAGES)
+    ms = np.zeros(n, np.float64)
+    cnt = np.zeros(n, np.int64)
+    _check("mr_profile_read", load_library().mr_profile_read(ms.ctypes.data, cnt.ctypes.data, n))
+    return {s: (float(ms[i]), int(cnt[i])) for i, s in enumerate(STAGES)}
 
 
 class SilhouetteRasterizer(torch.autograd.Function):

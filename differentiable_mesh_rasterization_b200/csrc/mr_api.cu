@@ -4,6 +4,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "mr_common.cuh"
 
@@ -12,6 +13,15 @@ thread_local char g_last_error[512] = "";
 __device__ int g_device_error = 0;
 std::mutex g_pool_mutex;
 bool g_pool_ready[64] = {};
+
+struct ProfEntry {
+    int stage;
+    cudaEvent_t a, b;
+};
+std::mutex g_prof_mutex;
+bool g_prof_on = false;
+std::vector<ProfEntry> g_prof_pending;
+std::vector<cudaEvent_t> g_prof_free;
 }  // namespace
 
 namespace mr {
@@ -63,6 +73,28 @@ void scratch_free(void* p, cudaStream_t s) {
     if (p) cudaFreeAsync(p, s);
 }
 
+bool profiling_enabled() { return g_prof_on; }
+
+cudaEvent_t profile_event() {
+    std::lock_guard<std::mutex> g(g_prof_mutex);
+    if (!g_prof_free.empty()) {
+        cudaEvent_t e = g_prof_free.back();
+        g_prof_free.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return e;
+}
+
+void profile_record(int stage, cudaEvent_t a, cudaEvent_t b) {
+    std::lock_guard<std::mutex> g(g_prof_mutex);
+    g_prof_pending.push_back(ProfEntry{stage, a, b});
+}
+
 int* device_error_word() {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) {
@@ -77,6 +109,41 @@ int* device_error_word() {
 extern "C" {
 
 const char* mr_last_error(void) { return g_last_error; }
+
+int mr_profile_enable(int32_t on) {
+    std::lock_guard<std::mutex> g(g_prof_mutex);
+    g_prof_on = on != 0;
+    return MR_OK;
+}
+
+int mr_profile_read(double* stage_ms, int64_t* launches, int32_t nstages) {
+    std::vector<ProfEntry> pending;
+    {
+        std::lock_guard<std::mutex> g(g_prof_mutex);
+        pending.swap(g_prof_pending);
+    }
+    for (int i = 0; i < nstages; ++i) {
+        if (stage_ms) stage_ms[i] = 0.0;
+        if (launches) launches[i] = 0;
+    }
+    int rc = MR_OK;
+    for (const ProfEntry& e : pending) {
+        float ms = 0.f;
+        cudaError_t err = cudaEventSynchronize(e.b);
+        if (err == cudaSuccess) err = cudaEventElapsedTime(&ms, e.a, e.b);
+        if (err != cudaSuccess && rc == MR_OK) rc = mr::cuda_fail(err, "cudaEventElapsedTime");
+        if (e.stage >= 0 && e.stage < nstages) {
+            if (stage_ms) stage_ms[e.stage] += ms;
+            if (launches) launches[e.stage] += 1;
+        }
+    }
+    std::lock_guard<std::mutex> g(g_prof_mutex);
+    for (const ProfEntry& e : pending) {
+        g_prof_free.push_back(e.a);
+        g_prof_free.push_back(e.b);
+    }
+    return rc;
+}
 
 int mr_version(void) { return 10000; }
 

@@ -251,6 +251,7 @@ int mr_rasterize_bwd(const float* verts, int64_t V, const int64_t* faces, int64_
         return MR_ERR_CUDA;
     }
     const int g = mr::grid_for(nslots);
+    mr::ProfScope ps(MR_STAGE_RASTER_BWD, s);
     if (perspective_correct)
         mr::k_raster_bwd<true><<<g, 256, 0, s>>>(verts, V, faces, F, pix_to_face, nslots, H, W, K, grad_zbuf, grad_bary,
                                                  grad_dists, grad_verts, err);
@@ -284,6 +285,7 @@ int mr_silhouette_rasterize_bwd(const float* verts, int64_t V, const int64_t* fa
         return MR_ERR_CUDA;
     }
     const int g = mr::grid_for(npix);
+    mr::ProfScope ps(MR_STAGE_SILHOUETTE_RASTER_BWD, s);
 #define MR_SRB(KC)                                                                                            \
     mr::k_sil_raster_bwd<KC><<<g, 256, 0, s>>>(verts, V, faces, F, pix_to_face, dists, grad_alpha, npix, H, W, K, \
                                                sigma, grad_verts, err)

@@ -52,6 +52,30 @@ void scratch_free(void* p, cudaStream_t s);
 // Device-wide sticky error word (asynchronous kernels).
 int* device_error_word();
 
+// Stage timing: while profiling is enabled, a ProfScope records a CUDA event pair
+// around the launches in its scope on stream s.
+bool profiling_enabled();
+void profile_record(int stage, cudaEvent_t start, cudaEvent_t stop);
+cudaEvent_t profile_event();
+struct ProfScope {
+    int stage;
+    cudaStream_t s;
+    cudaEvent_t a = nullptr, b = nullptr;
+    ProfScope(int st, cudaStream_t str) : stage(st), s(str) {
+        if (profiling_enabled()) {
+            a = profile_event();
+            b = profile_event();
+            if (a && b) cudaEventRecord(a, s);
+        }
+    }
+    ~ProfScope() {
+        if (a && b) {
+            cudaEventRecord(b, s);
+            profile_record(stage, a, b);
+        }
+    }
+};
+
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 }  // namespace mr

@@ -521,16 +521,21 @@ int rasterize_impl(const float* verts, int64_t V, const int64_t* faces, int64_t 
     MR_TRY(cudaMemsetAsync(d_err, 0, sizeof(int), s));
     const double reach = std::sqrt((double)blur) * (1.0 + 1e-6) + 1e-7;
     if (F > 0) {
+        ProfScope ps(MR_STAGE_FACE_SETUP, s);
         k_face_setup<<<(unsigned)((F + 255) / 256), 256, 0, s>>>(verts, V, faces, F, H, W, reach, geom, box, d_err);
         MR_TRY(cudaGetLastError());
     }
     const int pair_blocks = (int)std::min<int64_t>((pairs + 255) / 256, 148 * 16);
     if (pairs > 0) {
+        ProfScope ps(MR_STAGE_BIN_COUNT, s);
         k_bin_pairs<false><<<pair_blocks, 256, 0, s>>>(box, d_prefix, d_first, N, pairs, nbx, nby, counts,
                                                        nullptr, nullptr);
         MR_TRY(cudaGetLastError());
     }
-    k_scan<<<1, 1024, 0, s>>>(counts, nbins, offsets, d_total);
+    {
+        ProfScope ps(MR_STAGE_BIN_SCAN, s);
+        k_scan<<<1, 1024, 0, s>>>(counts, nbins, offsets, d_total);
+    }
     MR_TRY(cudaGetLastError());
     long long host[2] = {0, 0};
     MR_TRY(cudaMemcpyAsync(&host[0], d_total, sizeof(long long), cudaMemcpyDeviceToHost, s));
@@ -546,18 +551,22 @@ int rasterize_impl(const float* verts, int64_t V, const int64_t* faces, int64_t 
         rc = scratch_alloc(reinterpret_cast<void**>(&list), sizeof(int) * (size_t)total, s);
         if (rc != MR_OK) return fail(rc);
         MR_TRY(cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)nbins, s));
+        ProfScope ps(MR_STAGE_BIN_FILL, s);
         k_bin_pairs<true><<<pair_blocks, 256, 0, s>>>(box, d_prefix, d_first, N, pairs, nbx, nby, counts, offsets,
                                                       list);
         MR_TRY(cudaGetLastError());
     }
     const int KC = K <= 1 ? 1 : K <= 2 ? 2 : K <= 4 ? 4 : K <= 8 ? 8 : K <= 16 ? 16 : 32;
     const bool vec_ok = aligned16(p2f) && aligned16(zbuf) && aligned16(bary) && aligned16(dists);
+    {
+    ProfScope ps(MR_STAGE_FINE, s);
     if (persp) {
         if (sil) dispatch_k<true, true>(KC, nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
         else dispatch_k<true, false>(KC, nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
     } else {
         if (sil) dispatch_k<false, true>(KC, nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
         else dispatch_k<false, false>(KC, nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
+    }
     }
     MR_TRY(cudaGetLastError());
 #undef MR_TRY

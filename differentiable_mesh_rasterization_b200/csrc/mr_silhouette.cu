@@ -1,7 +1,6 @@
 // Stage two of the PyTorch3D rasterizer as stand-alone kernels: the soft silhouette over
 // the K faces kept per pixel and its gradient with respect to their distances.  One
-// thread per pixel; the K slots of a pixel are contiguous, read with 16-byte loads when
-// K is a multiple of 4.
+// thread per pixel (grid-stride); the K slots of a pixel are contiguous.
 #include <cmath>
 
 #include "mr_common.cuh"
@@ -82,6 +81,7 @@ int mr_silhouette_blend_fwd(const int64_t* pix_to_face, const float* dists, int3
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t npix = (int64_t)N * H * W;
     const int g = mr::grid_for(npix);
+    mr::ProfScope ps(MR_STAGE_SILHOUETTE_FWD, s);
     if (K <= 1) mr::k_silhouette_fwd<1><<<g, 256, 0, s>>>(pix_to_face, dists, npix, K, sigma, alpha);
     else if (K <= 2) mr::k_silhouette_fwd<2><<<g, 256, 0, s>>>(pix_to_face, dists, npix, K, sigma, alpha);
     else if (K <= 4) mr::k_silhouette_fwd<4><<<g, 256, 0, s>>>(pix_to_face, dists, npix, K, sigma, alpha);
@@ -99,6 +99,7 @@ int mr_silhouette_blend_bwd(const float* grad_alpha, const int64_t* pix_to_face,
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t npix = (int64_t)N * H * W;
     const int g = mr::grid_for(npix);
+    mr::ProfScope ps(MR_STAGE_SILHOUETTE_BWD, s);
 #define MR_SB(KC) mr::k_silhouette_bwd<KC><<<g, 256, 0, s>>>(grad_alpha, pix_to_face, dists, npix, K, sigma, grad_dists)
     if (K <= 1) MR_SB(1);
     else if (K <= 2) MR_SB(2);

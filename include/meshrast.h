@@ -153,6 +153,27 @@ const char* mr_last_error(void);
 /* Library version as 10000 * major + 100 * minor + patch. */
 int mr_version(void);
 
+/*
+ * Stage timing (the library's own tracing; no counterpart on the pages).  While enabled,
+ * every launch of the stages below is bracketed by two CUDA events recorded on the
+ * caller's stream; recording adds no synchronisation.  mr_profile_read() waits for the
+ * recorded events, writes the summed milliseconds and launch counts per stage into
+ * stage_ms[0..nstages) and launches[0..nstages) (either may be NULL), and forgets them.
+ * Process-wide; intended for one device and one thread at a time.
+ */
+#define MR_STAGE_FACE_SETUP 0
+#define MR_STAGE_BIN_COUNT 1
+#define MR_STAGE_BIN_SCAN 2
+#define MR_STAGE_BIN_FILL 3
+#define MR_STAGE_FINE 4
+#define MR_STAGE_SILHOUETTE_FWD 5
+#define MR_STAGE_SILHOUETTE_BWD 6
+#define MR_STAGE_RASTER_BWD 7
+#define MR_STAGE_SILHOUETTE_RASTER_BWD 8
+#define MR_NUM_STAGES 9
+int mr_profile_enable(int32_t on);
+int mr_profile_read(double* stage_ms, int64_t* launches, int32_t nstages);
+
 #ifdef __cplusplus
 }
 #endif

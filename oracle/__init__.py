@@ -129,7 +129,9 @@ def silhouette_bwd(grad_alpha, pix_to_face, dists, sigma):
 
 def rasterize_bwd(verts, faces, pix_to_face, perspective_correct=False, grad_zbuf=None,
                   grad_bary=None, grad_dists=None, nthreads=None):
-    """Step 13: dL/dverts (V x 3, float64) from gradients of zbuf / bary / dists (any may be None)."""
+    """Step 13: dL/dverts (V x 3, float64) from gradients of zbuf / bary / dists (any may be None).
+
+    Each thread keeps a private V x 3 float64 accumulator, so the default caps threads at 16."""
     lib = _load()
     verts = _c(verts, np.float32)
     faces = _c(faces, np.int64)
@@ -141,7 +143,7 @@ def rasterize_bwd(verts, faces, pix_to_face, perspective_correct=False, grad_zbu
     out = np.empty(verts.shape, np.float64)
     rc = lib.oracle_rasterize_bwd(_ptr(verts), verts.shape[0], _ptr(faces), faces.shape[0], _ptr(p2f),
                                   N, H, W, K, int(bool(perspective_correct)), _ptr(gz), _ptr(gb), _ptr(gd),
-                                  _ptr(out), nthreads or default_threads())
+                                  _ptr(out), nthreads or min(default_threads(), 16))
     if rc != 0:
         raise ValueError("oracle_rasterize_bwd: invalid arguments")
     return out
