@@ -92,13 +92,14 @@ class ClockSampler:
     def __enter__(self):
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
             if self.uuid:
                 cmd += ["-i", self.uuid]
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, ValueError):
             self.proc = None
+        time.sleep(1.5)     # let nvidia-smi start sampling before the timed region
         return self
 
     def __exit__(self, *exc):
@@ -209,12 +210,14 @@ def workload_config(w, args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--images", type=int, default=None,
+                    help="render only the first N meshes of the batch (small profiling case)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -235,7 +238,7 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    batch = syn.make_batch(args.config, seed=1000 + args.config + 1000 * rank)
+    batch = syn.make_batch(args.config, seed=1000 + args.config + 1000 * rank, n_meshes=args.images)
     w = batch.workload
     if w.sigma is None:
         raise SystemExit("the benchmark step needs a soft-silhouette workload (sigma)")
@@ -310,7 +313,8 @@ def main():
         h_alpha.copy_(alpha, non_blocking=True)
         h_gv.copy_(gv, non_blocking=True)
 
-    e2e_step()
+    if args.e2e_steps > 0:
+        e2e_step()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -326,13 +330,16 @@ def main():
     te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = tot_samples * args.e2e_steps / (float(te[0]) / 1e3)
+    e2e_value = tot_samples * args.e2e_steps / (float(te[0]) / 1e3) if args.e2e_steps > 0 else None
     h2d = h_verts.numel() * 4 + h_faces.numel() * 8 + h_ga.numel() * 4
     d2h = h_alpha.numel() * 4 + h_gv.numel() * 4
 
-    # roofline of the dominant kernel (the fine pass)
+    # roofline of the dominant kernel (the fine pass: the pixel-face tests) and of the
+    # epilogue (which writes the per-slot outputs)
     fine_ms, fine_n = stages["fine"]
     fine_s = fine_ms / 1e3 / max(fine_n, 1)
+    epi_ms, epi_n = stages["epilogue"]
+    epi_s = epi_ms / 1e3 / max(epi_n, 1)
     clk = clocks.summary()
     peaks = {}
     try:
@@ -341,25 +348,23 @@ def main():
         pass
     sm_mhz_max = float(peaks.get("sm_max_mhz", 1965.0))
     peak_alu = props.multi_processor_count * FP32_LANES_PER_SM * sm_mhz_max * 1e6 / 1e12   # T inst/s
-    achieved_alu = samples * C_TEST / fine_s / 1e12
-    out_bytes = w.N * w.H * w.W * (28 * w.K + 4) + int(batch.faces.shape[0]) * 64
     hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
-    achieved_hbm = out_bytes / fine_s / 1e9
-    t_alu = samples * C_TEST / (peak_alu * 1e12)
-    t_hbm = out_bytes / (hbm_peak * 1e9)
-    if t_alu >= t_hbm:
-        roof = {"bound": "alu", "achieved": achieved_alu, "peak": peak_alu, "unit": "T FP32-inst/s",
-                "frac": achieved_alu / peak_alu, "traffic": None}
-    else:
-        roof = {"bound": "hbm", "achieved": achieved_hbm, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved_hbm / hbm_peak, "traffic": None}
-    roof.update({"kernel": "k_fine (stage-one fine pass + fused silhouette epilogue)",
-                 "fine_ms_per_launch": fine_s * 1e3, "samples_per_launch": samples, "c_test": C_TEST,
-                 "peak_note": f"alu peak = {props.multi_processor_count} SMs x 128 FP32 lanes x {sm_mhz_max:.0f} MHz "
-                              f"(unit counts and max clock); hbm peak = {hbm_peak} GB/s "
-                              f"({'of measured' if 'hbm_gbs' in peaks else 'of fallback'} copy)",
-                 "hbm_achieved_gbs": achieved_hbm, "hbm_frac_of_measured": achieved_hbm / hbm_peak,
-                 "t_roof_ms": max(t_alu, t_hbm) * 1e3, "roof_frac": max(t_alu, t_hbm) / fine_s})
+    hbm_note = "of measured" if "hbm_gbs" in peaks else "of fallback"
+    achieved_alu = samples * C_TEST / fine_s / 1e12
+    npix = w.N * w.H * w.W
+    fine_bytes = npix * 4 * w.K                      # the K winning face ids per pixel
+    epi_bytes = npix * (4 * w.K + 28 * w.K + 4)      # ids in; p2f, zbuf, bary, dists, alpha out
+    roof = {"bound": "alu", "achieved": achieved_alu, "peak": peak_alu, "unit": "T FP32-inst/s",
+            "frac": achieved_alu / peak_alu, "traffic": None,
+            "kernel": "k_fine (stage-one fine pass: pixel-face tests and register top-K)",
+            "ms_per_launch": fine_s * 1e3, "samples_per_launch": samples, "c_test": C_TEST,
+            "peak_note": f"{props.multi_processor_count} SMs x 128 FP32 lanes x {sm_mhz_max:.0f} MHz "
+                         f"(unit counts and max clock)",
+            "hbm_bytes_per_launch": fine_bytes,
+            "epilogue": {"kernel": "k_epilogue (float64 outputs of the K winners + silhouette)",
+                         "bound": "hbm", "ms_per_launch": epi_s * 1e3, "bytes_per_launch": epi_bytes,
+                         "achieved": epi_bytes / epi_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": epi_bytes / epi_s / 1e9 / hbm_peak, "peak_note": hbm_note}}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dev_ms / args.steps, "higher_is_better": True,
@@ -369,7 +374,7 @@ def main():
             "stages_ms_per_step": {k: v[0] / args.steps for k, v in stages.items() if v[1]},
             "roofline": roof,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": float(te[0]) / args.e2e_steps},
+                    "ms_per_step": float(te[0]) / max(args.e2e_steps, 1)},
             "gpu_launches": int(sum(v[1] for v in stages.values())),
             "clocks": clk}
 

@@ -27,7 +27,7 @@ EXPORTS = ("mr_rasterize_fwd", "mr_rasterize_silhouette_fwd", "mr_silhouette_ble
            "mr_silhouette_blend_bwd", "mr_rasterize_bwd", "mr_silhouette_rasterize_bwd",
            "mr_device_status", "mr_last_error", "mr_version", "mr_profile_enable", "mr_profile_read")
 STAGES = ("face_setup", "bin_count", "bin_scan", "bin_fill", "fine", "silhouette_fwd", "silhouette_bwd",
-          "raster_bwd", "silhouette_raster_bwd")
+          "raster_bwd", "silhouette_raster_bwd", "epilogue")
 
 
 class MeshRastError(RuntimeError):

@@ -4,20 +4,20 @@
 //
 // Pipeline (one CUDA stream):
 //   face setup   one thread per face: gather the three vertices, float64 signed area
-//                (degenerate test), pixel box grown by sqrt(blur_radius).
+//                (degenerate test), pixel box grown by sqrt(blur_radius), and the face's
+//                plane constants for the fine pass (float64, rounded once to float32).
 //   bin count    one thread per (image, face) pair: count the 16x16 screen bins the box
 //                touches (warp-aggregated atomics).
 //   bin scan     exclusive scan of the per-bin counts -> list offsets and the total.
 //   (host)       one stream synchronisation to size the face lists.
 //   bin fill     second pass of the pair loop: scatter face ids into the bin lists.
-//   fine         one 256-thread CTA per bin.  Faces are staged through shared memory in
-//                chunks of 256 as bin-local float32 plane constants (computed in float64);
-//                each staged face is appended to the list of every 8x4 warp tile its box
-//                touches, so a warp only visits faces that can reach its pixels.  Each
-//                thread owns one pixel and keeps its K nearest (depth key, face id) pairs
-//                in registers, insertion-sorted.  The epilogue recomputes barycentrics,
-//                z and the signed squared distance of the K winners in float64 from the
-//                original vertices and writes them with 16-byte stores.
+//   fine         one CTA per bin, eight independent warps (8x4 pixel tiles): ballot-
+//                compacted per-warp face lists staged in shared memory, a warp-wide
+//                depth pre-test, the full candidacy test, and a register-resident
+//                insertion-sorted top-K per pixel; writes the K winning face ids.
+//   epilogue     one thread per pixel: barycentrics, z and signed squared distance of
+//                the K winners recomputed in float64 from the original vertices, the
+//                fused soft silhouette, 16-byte stores.
 #include <cfloat>
 #include <climits>
 #include <cmath>
@@ -29,21 +29,37 @@
 namespace mr {
 namespace {
 
-constexpr int kChunk = kFineThreads;   // faces staged per round
-constexpr int kConstF4 = 5;            // float4 words of bin-local constants per face
 
 // ------------------------------------------------------------------ face setup
+// Per-face plane constants of the fine pass, computed in float64 from the exact float32
+// vertices and rounded once.  The origin is the face's first vertex a, so a pixel enters
+// as (dx, dy) = p - a.  The winding is made counter-clockwise (b and c swapped if needed)
+// so every edge function is positive inside.  Per edge u -> v with unit direction e and
+// length L:
+//     c(d) = -e.y * d.x + e.x * d.y + ng   signed distance to the edge line (inside > 0)
+//     s(d) =  e.x * d.x + e.y * d.y + tg   position along the edge, measured from u
+//     squared distance to the segment = c^2 + max(-s, s - L, 0)^2.
+// The depth key is the plane through (x, y, z) -- or (x, y, -1/z) with perspective
+// correction, where 1/z is screen-affine -- written as k_hi + (gx dx + gy dy + k_lo);
+// the float-float constant keeps the key within half an ulp plus the plane terms.
+// Layout (6 float4): (ax, ay, gx, gy) (k_hi, k_lo, L0, L1) (e0.x, e0.y, ng0, tg0)
+//                    (e1.x, e1.y, ng1, tg1) (e2.x, e2.y, ng2, tg2) (L2, face id, 0, 0)
+constexpr int kConstF4 = 6;
+
 __global__ void k_face_setup(const float* __restrict__ verts, int64_t V,
                              const int64_t* __restrict__ faces, int64_t F, int H, int W,
-                             double reach, FaceGeom* __restrict__ geom, FaceBox* __restrict__ box,
+                             double reach, int persp, FaceGeom* __restrict__ geom,
+                             FaceBox* __restrict__ box, float4* __restrict__ fconst,
                              int* __restrict__ err) {
     int64_t f = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (f >= F) return;
     int64_t i0 = faces[3 * f], i1 = faces[3 * f + 1], i2 = faces[3 * f + 2];
     FaceBox bx = {1, 0, 1, 0};
+    float4* out = fconst + kConstF4 * f;
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
     if (i0 < 0 || i0 >= V || i1 < 0 || i1 >= V || i2 < 0 || i2 >= V) {
         atomicOr(err, kErrFaceIndex);
-        geom[f] = FaceGeom{make_float4(0, 0, 0, 0), make_float4(0, 0, 0, 0), make_float4(0, 0, 0, 0)};
+        geom[f] = FaceGeom{zero, zero, zero};
         box[f] = bx;
         return;
     }
@@ -53,20 +69,59 @@ __global__ void k_face_setup(const float* __restrict__ verts, int64_t V,
     geom[f] = FaceGeom{a, b, c};
     double ax = a.x, ay = a.y, bxx = b.x, byy = b.y, cx = c.x, cy = c.y;
     double area2 = (bxx - ax) * (cy - ay) - (byy - ay) * (cx - ax);
-    if (fabs(area2) > kDegenerateArea) {
-        double xmin = fmin(ax, fmin(bxx, cx)) - reach, xmax = fmax(ax, fmax(bxx, cx)) + reach;
-        double ymin = fmin(ay, fmin(byy, cy)) - reach, ymax = fmax(ay, fmax(byy, cy)) + reach;
-        // pixel j has centre x = -1 + (2j+1)/W; row i has y = 1 - (2i+1)/H.  The 1e-4
-        // pixel pad keeps the box a superset under rounding.
-        double jl = ceil((xmin + 1.0) * 0.5 * W - 0.5 - 1e-4);
-        double jh = floor((xmax + 1.0) * 0.5 * W - 0.5 + 1e-4);
-        double il = ceil((1.0 - ymax) * 0.5 * H - 0.5 - 1e-4);
-        double ih = floor((1.0 - ymin) * 0.5 * H - 0.5 + 1e-4);
-        jl = fmax(jl, 0.0); il = fmax(il, 0.0);
-        jh = fmin(jh, (double)(W - 1)); ih = fmin(ih, (double)(H - 1));
-        if (jl <= jh && il <= ih) bx = FaceBox{(int)jl, (int)jh, (int)il, (int)ih};
+    if (!(fabs(area2) > kDegenerateArea)) {
+        box[f] = bx;
+        return;
     }
+    double xmin = fmin(ax, fmin(bxx, cx)) - reach, xmax = fmax(ax, fmax(bxx, cx)) + reach;
+    double ymin = fmin(ay, fmin(byy, cy)) - reach, ymax = fmax(ay, fmax(byy, cy)) + reach;
+    // pixel j has centre x = -1 + (2j+1)/W; row i has y = 1 - (2i+1)/H.  The 1e-4
+    // pixel pad keeps the box a superset under rounding.
+    double jl = ceil((xmin + 1.0) * 0.5 * W - 0.5 - 1e-4);
+    double jh = floor((xmax + 1.0) * 0.5 * W - 0.5 + 1e-4);
+    double il = ceil((1.0 - ymax) * 0.5 * H - 0.5 - 1e-4);
+    double ih = floor((1.0 - ymin) * 0.5 * H - 0.5 + 1e-4);
+    jl = fmax(jl, 0.0); il = fmax(il, 0.0);
+    jh = fmin(jh, (double)(W - 1)); ih = fmin(ih, (double)(H - 1));
+    if (jl <= jh && il <= ih) bx = FaceBox{(int)jl, (int)jh, (int)il, (int)ih};
     box[f] = bx;
+
+    double x[3] = {0.0, bxx - ax, cx - ax};
+    double y[3] = {0.0, byy - ay, cy - ay};
+    double q[3];
+    if (persp) {
+        q[0] = -1.0 / (double)a.z; q[1] = -1.0 / (double)b.z; q[2] = -1.0 / (double)c.z;
+    } else {
+        q[0] = a.z; q[1] = b.z; q[2] = c.z;
+    }
+    const double nx = y[1] * (q[2] - q[0]) - (q[1] - q[0]) * y[2];
+    const double ny = (q[1] - q[0]) * x[2] - x[1] * (q[2] - q[0]);
+    const double gx = -nx / area2, gy = -ny / area2;
+    const float khi = (float)q[0];
+    const float klo = (float)(q[0] - (double)khi);
+    if (area2 < 0.0) {
+        double t = x[1]; x[1] = x[2]; x[2] = t;
+        t = y[1]; y[1] = y[2]; y[2] = t;
+    }
+    float e[3][5];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        const int k1 = k == 2 ? 0 : k + 1;
+        const double ex = x[k1] - x[k], ey = y[k1] - y[k];
+        const double L = sqrt(ex * ex + ey * ey);
+        const double ux = ex / L, uy = ey / L;
+        e[k][0] = (float)ux;
+        e[k][1] = (float)uy;
+        e[k][2] = (float)(uy * x[k] - ux * y[k]);
+        e[k][3] = (float)(-(ux * x[k] + uy * y[k]));
+        e[k][4] = (float)L;
+    }
+    out[0] = make_float4(a.x, a.y, (float)gx, (float)gy);
+    out[1] = make_float4(khi, klo, e[0][4], e[1][4]);
+    out[2] = make_float4(e[0][0], e[0][1], e[0][2], e[0][3]);
+    out[3] = make_float4(e[1][0], e[1][1], e[1][2], e[1][3]);
+    out[4] = make_float4(e[2][0], e[2][1], e[2][2], e[2][3]);
+    out[5] = make_float4(e[2][4], __int_as_float((int)f), 0.f, 0.f);
 }
 
 // ------------------------------------------------------------------ binning
@@ -153,57 +208,6 @@ __global__ void k_scan(const int* __restrict__ counts, int nb, int* __restrict__
 }
 
 // ------------------------------------------------------------------ fine pass
-// Bin-local constants of one face, computed in float64 from the exact vertices.  The
-// origin is the centre of the bin's first pixel.  The winding is made counter-clockwise
-// (b and c swapped if needed) so every edge function is positive inside.  Per edge
-// u -> v with unit direction d and length L:
-//     c(p) = -d.y * p.x + d.x * p.y + ng   signed distance to the edge line (inside > 0)
-//     s(p) =  d.x * p.x + d.y * p.y + tg   position along the edge from u
-//     squared distance to the segment = c^2 + max(-s, s - L, 0)^2.
-// The depth key is the plane through (x, y, z) -- or (x, y, -1/z) with perspective
-// correction, where 1/z is screen-affine -- as gx * p.x + gy * p.y + (k_hi + k_lo);
-// the float-float constant keeps the key within half an ulp plus the plane terms.
-template <bool PERSP>
-__device__ void face_constants(const FaceGeom& g, double ox, double oy, int fid, float4* out) {
-    double x[3] = {(double)g.a.x - ox, (double)g.b.x - ox, (double)g.c.x - ox};
-    double y[3] = {(double)g.a.y - oy, (double)g.b.y - oy, (double)g.c.y - oy};
-    double q[3];
-    if (PERSP) {
-        q[0] = -1.0 / (double)g.a.z; q[1] = -1.0 / (double)g.b.z; q[2] = -1.0 / (double)g.c.z;
-    } else {
-        q[0] = g.a.z; q[1] = g.b.z; q[2] = g.c.z;
-    }
-    double area2 = (x[1] - x[0]) * (y[2] - y[0]) - (y[1] - y[0]) * (x[2] - x[0]);
-    // depth-key plane (independent of winding)
-    double nx = (y[1] - y[0]) * (q[2] - q[0]) - (q[1] - q[0]) * (y[2] - y[0]);
-    double ny = (q[1] - q[0]) * (x[2] - x[0]) - (x[1] - x[0]) * (q[2] - q[0]);
-    double gx = -nx / area2, gy = -ny / area2;
-    double k0 = q[0] - gx * x[0] - gy * y[0];
-    float khi = (float)k0;
-    float klo = (float)(k0 - (double)khi);
-    if (area2 < 0.0) {
-        double t = x[1]; x[1] = x[2]; x[2] = t;
-        t = y[1]; y[1] = y[2]; y[2] = t;
-    }
-    float e[3][5];
-    for (int k = 0; k < 3; ++k) {
-        int k1 = k == 2 ? 0 : k + 1;
-        double ex = x[k1] - x[k], ey = y[k1] - y[k];
-        double L = sqrt(ex * ex + ey * ey);
-        double dx = ex / L, dy = ey / L;
-        e[k][0] = (float)dx;
-        e[k][1] = (float)dy;
-        e[k][2] = (float)(dy * x[k] - dx * y[k]);
-        e[k][3] = (float)(-(dx * x[k] + dy * y[k]));
-        e[k][4] = (float)L;
-    }
-    out[0] = make_float4(e[0][0], e[0][1], e[0][2], e[0][3]);
-    out[1] = make_float4(e[1][0], e[1][1], e[1][2], e[1][3]);
-    out[2] = make_float4(e[2][0], e[2][1], e[2][2], e[2][3]);
-    out[3] = make_float4(e[0][4], e[1][4], e[2][4], (float)gx);
-    out[4] = make_float4((float)gy, khi, klo, __int_as_float(fid));
-}
-
 template <int KC>
 __device__ __forceinline__ void topk_insert(float (&kk)[KC], int (&ff)[KC], float key, int fid) {
 #pragma unroll
@@ -215,6 +219,105 @@ __device__ __forceinline__ void topk_insert(float (&kk)[KC], int (&ff)[KC], floa
         ff[k] = lt ? fid : ff[k];
         key = tk;
         fid = tf;
+    }
+}
+
+// One CTA per 16x16 bin; each of its eight warps owns an 8x4 pixel tile and runs on its
+// own (no block barriers).  A warp reads the bin's face list 32 ids at a time, tests
+// each face's pixel box against its tile, compacts the hits with a ballot and copies
+// their constants into its shared-memory slots.  For each staged face the warp first
+// evaluates the depth key alone; if no lane could admit the face into its top-K (face
+// behind the camera or not nearer than the lane's K-th key) the face is skipped, else
+// every lane runs the full candidacy test.  EXACT: the pixel centres are exact float32
+// values (H and W powers of two), so the float-float low parts vanish.
+template <int KC, bool PERSP, bool EXACT>
+__global__ void __launch_bounds__(kFineThreads)
+k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const int* __restrict__ offsets,
+       const int* __restrict__ list, int nbx, int nby, int H, int W, int K, float blur, int* __restrict__ topk) {
+    __shared__ float4 s_c[kWarpsPerBin][32][kConstF4];
+
+    const int bin = blockIdx.x;
+    const int bxi = bin % nbx;
+    const int byi = (bin / nbx) % nby;
+    const int n = bin / (nbx * nby);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tj0 = bxi * kBin + (warp & 1) * kWarpTileW;
+    const int ti0 = byi * kBin + (warp >> 1) * kWarpTileH;
+    if (tj0 >= W || ti0 >= H) return;                        // tile entirely off the image
+    const int j = tj0 + (lane & 7), i = ti0 + (lane >> 3);
+    const bool in_img = i < H && j < W;
+    const double pxd = -1.0 + (2.0 * j + 1.0) / W;
+    const double pyd = 1.0 - (2.0 * i + 1.0) / H;
+    const float pxh = (float)pxd, pyh = (float)pyd;
+    const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
+    const unsigned lt_mask = (1u << lane) - 1u;
+
+    float kk[KC];
+    int ff[KC];
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+        kk[k] = in_img ? FLT_MAX : -FLT_MAX;                 // off-image lanes admit nothing
+        ff[k] = INT_MAX;
+    }
+
+    const int beg = offsets[bin], cnt = offsets[bin + 1] - beg;
+    float4(*slots)[kConstF4] = s_c[warp];
+    for (int base = 0; base < cnt; base += 32) {
+        bool hit = false;
+        int fid = 0;
+        if (base + lane < cnt) {
+            fid = list[beg + base + lane];
+            const FaceBox b = box[fid];
+            hit = b.x0 <= tj0 + kWarpTileW - 1 && b.x1 >= tj0 && b.y0 <= ti0 + kWarpTileH - 1 && b.y1 >= ti0;
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (hit) {
+            const int slot = __popc(m & lt_mask);
+            const float4* src = fconst + (int64_t)kConstF4 * fid;
+#pragma unroll
+            for (int u = 0; u < kConstF4; ++u) slots[slot][u] = __ldg(src + u);
+        }
+        __syncwarp();
+        const int nh = __popc(m);
+        for (int qi = 0; qi < nh; ++qi) {
+            const float4 q0 = slots[qi][0], q1 = slots[qi][1];
+            float dx = pxh - q0.x, dy = pyh - q0.y;
+            if (!EXACT) { dx += pxl; dy += pyl; }
+            const float key = q1.x + fmaf(q0.z, dx, fmaf(q0.w, dy, q1.y));
+            const bool front = PERSP ? key < 0.f : key >= 0.f;
+            const bool maybe = front && key <= kk[KC - 1];
+            if (!__any_sync(0xffffffffu, maybe)) continue;
+            const float4 e0 = slots[qi][2], e1 = slots[qi][3], e2 = slots[qi][4], q5 = slots[qi][5];
+            const float c0 = fmaf(-e0.y, dx, fmaf(e0.x, dy, e0.z));
+            const float s0 = fmaf(e0.x, dx, fmaf(e0.y, dy, e0.w));
+            const float c1 = fmaf(-e1.y, dx, fmaf(e1.x, dy, e1.z));
+            const float s1 = fmaf(e1.x, dx, fmaf(e1.y, dy, e1.w));
+            const float c2 = fmaf(-e2.y, dx, fmaf(e2.x, dy, e2.z));
+            const float s2 = fmaf(e2.x, dx, fmaf(e2.y, dy, e2.w));
+            const float o0 = fmaxf(fmaxf(-s0, s0 - q1.z), 0.f);
+            const float o1 = fmaxf(fmaxf(-s1, s1 - q1.w), 0.f);
+            const float o2 = fmaxf(fmaxf(-s2, s2 - q5.x), 0.f);
+            const float d0 = fmaf(o0, o0, c0 * c0);
+            const float d1 = fmaf(o1, o1, c1 * c1);
+            const float d2 = fmaf(o2, o2, c2 * c2);
+            const bool inside = fminf(c0, fminf(c1, c2)) >= 0.f;
+            const float dmin = fminf(d0, fminf(d1, d2));
+            if (maybe && (inside || dmin <= blur)) topk_insert<KC>(kk, ff, key, __float_as_int(q5.y));
+        }
+        __syncwarp();
+    }
+    if (!in_img) return;
+    const int64_t pix = ((int64_t)n * H + i) * W + j;
+    if (K == KC && (KC % 4) == 0) {
+#pragma unroll
+        for (int k4 = 0; k4 < KC; k4 += 4)
+            *reinterpret_cast<int4*>(topk + pix * KC + k4) =
+                make_int4(ff[k4] == INT_MAX ? -1 : ff[k4], ff[k4 + 1] == INT_MAX ? -1 : ff[k4 + 1],
+                          ff[k4 + 2] == INT_MAX ? -1 : ff[k4 + 2], ff[k4 + 3] == INT_MAX ? -1 : ff[k4 + 3]);
+    } else {
+#pragma unroll
+        for (int k = 0; k < KC; ++k)
+            if (k < K) topk[pix * K + k] = ff[k] == INT_MAX ? -1 : ff[k];
     }
 }
 
@@ -255,168 +358,127 @@ __device__ void slot_outputs(const FaceGeom& g, double px, double py, float* z_o
     *d_out = (float)(inside ? -d2 : d2);
 }
 
+// One thread per pixel: the K winners' outputs (and the fused silhouette), written
+// contiguously per pixel with 16-byte stores when K is a multiple of 4.
 template <int KC, bool PERSP, bool SIL>
-__global__ void __launch_bounds__(kFineThreads)
-k_fine(const FaceGeom* __restrict__ geom, const FaceBox* __restrict__ box,
-       const int* __restrict__ offsets, const int* __restrict__ list, int nbx, int nby, int H, int W,
-       int K, float blur, float sigma, bool vec_ok, int64_t* __restrict__ p2f,
-       float* __restrict__ zbuf, float* __restrict__ bary, float* __restrict__ dists,
-       float* __restrict__ alpha) {
-    __shared__ float4 s_face[kChunk * kConstF4];
-    __shared__ unsigned char s_wlist[kWarpsPerBin][kChunk];
-    __shared__ int s_wcount[kWarpsPerBin];
-
-    const int bin = blockIdx.x;
-    const int bxi = bin % nbx;
-    const int byi = (bin / nbx) % nby;
-    const int n = bin / (nbx * nby);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int wx = (warp & 1) * kWarpTileW, wy = (warp >> 1) * kWarpTileH;
-    const int tx = wx + (lane & 7), ty = wy + (lane >> 3);
-    const int j0 = bxi * kBin, i0 = byi * kBin;
-    const int j = j0 + tx, i = i0 + ty;
-    // bin-local pixel coordinates (origin = centre of pixel (i0, j0))
-    const float px = (float)(2.0 * tx / W);
-    const float py = (float)(-2.0 * ty / H);
-    const double ox = -1.0 + (2.0 * j0 + 1.0) / W;
-    const double oy = 1.0 - (2.0 * i0 + 1.0) / H;
-
-    float kk[KC];
-    int ff[KC];
+__global__ void __launch_bounds__(256)
+k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int64_t npix, int H, int W, int K,
+           float sigma, bool vec_ok, int64_t* __restrict__ p2f, float* __restrict__ zbuf, float* __restrict__ bary,
+           float* __restrict__ dists, float* __restrict__ alpha) {
+    for (int64_t pix = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; pix < npix;
+         pix += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t rem = pix % ((int64_t)H * W);
+        const int i = (int)(rem / W), j = (int)(rem % W);
+        const double pxd = -1.0 + (2.0 * j + 1.0) / W;
+        const double pyd = 1.0 - (2.0 * i + 1.0) / H;
+        float dsil[KC];
+        bool vsil[KC];
+        if (vec_ok && (KC % 4) == 0 && K == KC) {
 #pragma unroll
-    for (int k = 0; k < KC; ++k) { kk[k] = FLT_MAX; ff[k] = INT_MAX; }
-
-    const int beg = offsets[bin], cnt = offsets[bin + 1] - beg;
-    for (int c0 = 0; c0 < cnt; c0 += kChunk) {
-        if (threadIdx.x < kWarpsPerBin) s_wcount[threadIdx.x] = 0;
-        __syncthreads();
-        const int t = threadIdx.x;
-        if (c0 + t < cnt) {
-            const int fid = list[beg + c0 + t];
-            const FaceBox b = box[fid];
-            const FaceGeom g = geom[fid];
-            face_constants<PERSP>(g, ox, oy, fid, &s_face[t * kConstF4]);
-            // append to every warp tile the box touches
+            for (int k4 = 0; k4 < KC; k4 += 4) {
+                const int4 f4 = *reinterpret_cast<const int4*>(topk + pix * KC + k4);
+                const int fk[4] = {f4.x, f4.y, f4.z, f4.w};
+                float zz[4], bb[12], dd[4];
+                long long pf[4];
 #pragma unroll
-            for (int w = 0; w < kWarpsPerBin; ++w) {
-                int tj0 = j0 + (w & 1) * kWarpTileW, ti0 = i0 + (w >> 1) * kWarpTileH;
-                bool hit = b.x0 <= tj0 + kWarpTileW - 1 && b.x1 >= tj0 && b.y0 <= ti0 + kWarpTileH - 1 &&
-                           b.y1 >= ti0;
-                if (hit) {
-                    int pos = atomicAdd(&s_wcount[w], 1);
-                    s_wlist[w][pos] = (unsigned char)t;
+                for (int u = 0; u < 4; ++u) {
+                    if (fk[u] >= 0) {
+                        slot_outputs<PERSP>(geom[fk[u]], pxd, pyd, &zz[u], &bb[3 * u], &dd[u]);
+                    } else {
+                        zz[u] = -1.f; dd[u] = -1.f; bb[3 * u] = bb[3 * u + 1] = bb[3 * u + 2] = -1.f;
+                    }
+                    pf[u] = fk[u];
+                    dsil[k4 + u] = dd[u];
+                    vsil[k4 + u] = fk[u] >= 0;
                 }
+                const int64_t s = pix * KC + k4;
+                reinterpret_cast<longlong2*>(p2f + s)[0] = make_longlong2(pf[0], pf[1]);
+                reinterpret_cast<longlong2*>(p2f + s)[1] = make_longlong2(pf[2], pf[3]);
+                *reinterpret_cast<float4*>(zbuf + s) = make_float4(zz[0], zz[1], zz[2], zz[3]);
+                *reinterpret_cast<float4*>(dists + s) = make_float4(dd[0], dd[1], dd[2], dd[3]);
+                float4* bp = reinterpret_cast<float4*>(bary + 3 * s);
+                bp[0] = make_float4(bb[0], bb[1], bb[2], bb[3]);
+                bp[1] = make_float4(bb[4], bb[5], bb[6], bb[7]);
+                bp[2] = make_float4(bb[8], bb[9], bb[10], bb[11]);
             }
-        }
-        __syncthreads();
-        const int nq = s_wcount[warp];
-        for (int qi = 0; qi < nq; ++qi) {
-            const float4* fc = &s_face[s_wlist[warp][qi] * kConstF4];
-            const float4 e0 = fc[0], e1 = fc[1], e2 = fc[2], e3 = fc[3], e4 = fc[4];
-            const float c0 = fmaf(-e0.y, px, fmaf(e0.x, py, e0.z));
-            const float s0 = fmaf(e0.x, px, fmaf(e0.y, py, e0.w));
-            const float c1 = fmaf(-e1.y, px, fmaf(e1.x, py, e1.z));
-            const float s1 = fmaf(e1.x, px, fmaf(e1.y, py, e1.w));
-            const float c2 = fmaf(-e2.y, px, fmaf(e2.x, py, e2.z));
-            const float s2 = fmaf(e2.x, px, fmaf(e2.y, py, e2.w));
-            const float o0 = fmaxf(fmaxf(-s0, s0 - e3.x), 0.f);
-            const float o1 = fmaxf(fmaxf(-s1, s1 - e3.y), 0.f);
-            const float o2 = fmaxf(fmaxf(-s2, s2 - e3.z), 0.f);
-            const float d0 = fmaf(o0, o0, c0 * c0);
-            const float d1 = fmaf(o1, o1, c1 * c1);
-            const float d2 = fmaf(o2, o2, c2 * c2);
-            const bool inside = fminf(c0, fminf(c1, c2)) >= 0.f;
-            const float dmin = fminf(d0, fminf(d1, d2));
-            const float key = e4.y + fmaf(e3.w, px, fmaf(e4.x, py, e4.z));
-            const bool front = PERSP ? key < 0.f : key >= 0.f;
-            if ((inside || dmin <= blur) && front && key <= kk[KC - 1])
-                topk_insert<KC>(kk, ff, key, __float_as_int(e4.w));
-        }
-        __syncthreads();
-    }
-
-    if (i >= H || j >= W) return;
-    const double pxd = -1.0 + (2.0 * j + 1.0) / W;
-    const double pyd = 1.0 - (2.0 * i + 1.0) / H;
-    const int64_t pix = ((int64_t)n * H + i) * W + j;
-    float dsil[KC];
-    bool vsil[KC];
-    if (vec_ok && (KC % 4) == 0 && K == KC) {
+        } else {
 #pragma unroll
-        for (int k4 = 0; k4 < KC; k4 += 4) {
-            float zz[4], bb[12], dd[4];
-            long long pf[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int k = k4 + u;
-                if (ff[k] != INT_MAX) {
-                    slot_outputs<PERSP>(geom[ff[k]], pxd, pyd, &zz[u], &bb[3 * u], &dd[u]);
-                    pf[u] = ff[k];
+            for (int k = 0; k < KC; ++k) {
+                if (k >= K) break;
+                const int64_t s = pix * K + k;
+                const int fk = topk[s];
+                float zz, bb[3], dd;
+                if (fk >= 0) {
+                    slot_outputs<PERSP>(geom[fk], pxd, pyd, &zz, bb, &dd);
                 } else {
-                    zz[u] = -1.f; dd[u] = -1.f; bb[3 * u] = bb[3 * u + 1] = bb[3 * u + 2] = -1.f;
-                    pf[u] = -1;
+                    zz = -1.f; dd = -1.f; bb[0] = bb[1] = bb[2] = -1.f;
                 }
-                dsil[k] = dd[u];
-                vsil[k] = ff[k] != INT_MAX;
+                p2f[s] = fk;
+                zbuf[s] = zz;
+                dists[s] = dd;
+                bary[3 * s] = bb[0]; bary[3 * s + 1] = bb[1]; bary[3 * s + 2] = bb[2];
+                dsil[k] = dd;
+                vsil[k] = fk >= 0;
             }
-            const int64_t s = pix * KC + k4;
-            reinterpret_cast<longlong2*>(p2f + s)[0] = make_longlong2(pf[0], pf[1]);
-            reinterpret_cast<longlong2*>(p2f + s)[1] = make_longlong2(pf[2], pf[3]);
-            *reinterpret_cast<float4*>(zbuf + s) = make_float4(zz[0], zz[1], zz[2], zz[3]);
-            *reinterpret_cast<float4*>(dists + s) = make_float4(dd[0], dd[1], dd[2], dd[3]);
-            float4* bp = reinterpret_cast<float4*>(bary + 3 * s);
-            bp[0] = make_float4(bb[0], bb[1], bb[2], bb[3]);
-            bp[1] = make_float4(bb[4], bb[5], bb[6], bb[7]);
-            bp[2] = make_float4(bb[8], bb[9], bb[10], bb[11]);
         }
-    } else {
-#pragma unroll
-        for (int k = 0; k < KC; ++k) {
-            if (k >= K) break;
-            const int64_t s = pix * K + k;
-            float zz, bb[3], dd;
-            if (ff[k] != INT_MAX) {
-                slot_outputs<PERSP>(geom[ff[k]], pxd, pyd, &zz, bb, &dd);
-                p2f[s] = ff[k];
-            } else {
-                zz = -1.f; dd = -1.f; bb[0] = bb[1] = bb[2] = -1.f;
-                p2f[s] = -1;
-            }
-            zbuf[s] = zz;
-            dists[s] = dd;
-            bary[3 * s] = bb[0]; bary[3 * s + 1] = bb[1]; bary[3 * s + 2] = bb[2];
-            dsil[k] = dd;
-            vsil[k] = ff[k] != INT_MAX;
-        }
+        if (SIL) alpha[pix] = silhouette_alpha<KC>(dsil, vsil, K, sigma);
     }
-    if (SIL) alpha[pix] = silhouette_alpha<KC>(dsil, vsil, K, sigma);
 }
 
-template <int KC, bool PERSP, bool SIL>
-void launch_fine(int nbins, cudaStream_t s, const FaceGeom* geom, const FaceBox* box, const int* offsets,
-                 const int* list, int nbx, int nby, int H, int W, int K, float blur, float sigma,
-                 bool vec_ok, int64_t* p2f, float* zbuf, float* bary, float* dists, float* alpha) {
-    k_fine<KC, PERSP, SIL><<<nbins, kFineThreads, 0, s>>>(geom, box, offsets, list, nbx, nby, H, W, K, blur,
-                                                          sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
-}
-
-template <bool PERSP, bool SIL>
-void dispatch_k(int KC, int nbins, cudaStream_t s, const FaceGeom* geom, const FaceBox* box,
-                const int* offsets, const int* list, int nbx, int nby, int H, int W, int K, float blur,
-                float sigma, bool vec_ok, int64_t* p2f, float* zbuf, float* bary, float* dists,
-                float* alpha) {
-#define MR_FINE(KCV)                                                                                     \
-    launch_fine<KCV, PERSP, SIL>(nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma,     \
-                                 vec_ok, p2f, zbuf, bary, dists, alpha)
-    switch (KC) {
-        case 1: MR_FINE(1); break;
-        case 2: MR_FINE(2); break;
-        case 4: MR_FINE(4); break;
-        case 8: MR_FINE(8); break;
-        case 16: MR_FINE(16); break;
-        default: MR_FINE(32); break;
+template <int KC>
+void launch_fine(bool persp, bool exact, int nbins, cudaStream_t s, const float4* fconst, const FaceBox* box,
+                 const int* offsets, const int* list, int nbx, int nby, int H, int W, int K, float blur, int* topk) {
+#define MR_FINE(P, E) \
+    k_fine<KC, P, E><<<nbins, kFineThreads, 0, s>>>(fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk)
+    if (persp) {
+        if (exact) MR_FINE(true, true); else MR_FINE(true, false);
+    } else {
+        if (exact) MR_FINE(false, true); else MR_FINE(false, false);
     }
 #undef MR_FINE
+}
+
+template <int KC>
+void launch_epilogue(bool persp, bool sil, int64_t npix, cudaStream_t s, const FaceGeom* geom, const int* topk,
+                     int H, int W, int K, float sigma, bool vec_ok, int64_t* p2f, float* zbuf, float* bary,
+                     float* dists, float* alpha) {
+    const int grid = (int)std::min<int64_t>((npix + 255) / 256, 148 * 16);
+#define MR_EPI(P, S) \
+    k_epilogue<KC, P, S><<<grid, 256, 0, s>>>(geom, topk, npix, H, W, K, sigma, vec_ok, p2f, zbuf, bary, dists, alpha)
+    if (persp) {
+        if (sil) MR_EPI(true, true); else MR_EPI(true, false);
+    } else {
+        if (sil) MR_EPI(false, true); else MR_EPI(false, false);
+    }
+#undef MR_EPI
+}
+
+void dispatch_fine(int KC, bool persp, bool exact, int nbins, cudaStream_t s, const float4* fconst,
+                   const FaceBox* box, const int* offsets, const int* list, int nbx, int nby, int H, int W, int K,
+                   float blur, int* topk) {
+    switch (KC) {
+        case 1: launch_fine<1>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
+        case 2: launch_fine<2>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
+        case 4: launch_fine<4>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
+        case 8: launch_fine<8>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
+        case 16: launch_fine<16>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
+        default: launch_fine<32>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
+    }
+}
+
+void dispatch_epilogue(int KC, bool persp, bool sil, int64_t npix, cudaStream_t s, const FaceGeom* geom,
+                       const int* topk, int H, int W, int K, float sigma, bool vec_ok, int64_t* p2f, float* zbuf,
+                       float* bary, float* dists, float* alpha) {
+#define MR_E(KCV) launch_epilogue<KCV>(persp, sil, npix, s, geom, topk, H, W, K, sigma, vec_ok, p2f, zbuf, bary, dists, alpha)
+    switch (KC) {
+        case 1: MR_E(1); break;
+        case 2: MR_E(2); break;
+        case 4: MR_E(4); break;
+        case 8: MR_E(8); break;
+        case 16: MR_E(16); break;
+        default: MR_E(32); break;
+    }
+#undef MR_E
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -480,11 +542,16 @@ int rasterize_impl(const float* verts, int64_t V, const int64_t* faces, int64_t 
     for (int n = 0; n < N; ++n) prefix[n + 1] = prefix[n] + num[n];
     const int64_t pairs = prefix[N];
 
-    // one scratch block: geometry | boxes | counts | offsets | prefix | first | total | error
+    const int KC = K <= 1 ? 1 : K <= 2 ? 2 : K <= 4 ? 4 : K <= 8 ? 8 : K <= 16 ? 16 : 32;
+    const int64_t npix = (int64_t)N * H * W;
+    // one scratch block: geometry | boxes | constants | top-K ids | counts | offsets |
+    // prefix | first | total | error
     auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
     const size_t o_geom = 0;
     const size_t o_box = o_geom + up(sizeof(FaceGeom) * (size_t)F);
-    const size_t o_cnt = o_box + up(sizeof(FaceBox) * (size_t)F);
+    const size_t o_con = o_box + up(sizeof(FaceBox) * (size_t)F);
+    const size_t o_top = o_con + up(sizeof(float4) * kConstF4 * (size_t)F);
+    const size_t o_cnt = o_top + up(sizeof(int) * (size_t)npix * (size_t)K);
     const size_t o_off = o_cnt + up(sizeof(int) * (size_t)nbins);
     const size_t o_pre = o_off + up(sizeof(int) * (size_t)(nbins + 1));
     const size_t o_fst = o_pre + up(sizeof(int64_t) * (size_t)(N + 1));
@@ -496,6 +563,8 @@ int rasterize_impl(const float* verts, int64_t V, const int64_t* faces, int64_t 
     if (rc != MR_OK) return rc;
     FaceGeom* geom = reinterpret_cast<FaceGeom*>(ws + o_geom);
     FaceBox* box = reinterpret_cast<FaceBox*>(ws + o_box);
+    float4* fconst = reinterpret_cast<float4*>(ws + o_con);
+    int* topk = reinterpret_cast<int*>(ws + o_top);
     int* counts = reinterpret_cast<int*>(ws + o_cnt);
     int* offsets = reinterpret_cast<int*>(ws + o_off);
     int64_t* d_prefix = reinterpret_cast<int64_t*>(ws + o_pre);
@@ -522,7 +591,8 @@ int rasterize_impl(const float* verts, int64_t V, const int64_t* faces, int64_t 
     const double reach = std::sqrt((double)blur) * (1.0 + 1e-6) + 1e-7;
     if (F > 0) {
         ProfScope ps(MR_STAGE_FACE_SETUP, s);
-        k_face_setup<<<(unsigned)((F + 255) / 256), 256, 0, s>>>(verts, V, faces, F, H, W, reach, geom, box, d_err);
+        k_face_setup<<<(unsigned)((F + 255) / 256), 256, 0, s>>>(verts, V, faces, F, H, W, reach, persp, geom, box,
+                                                                  fconst, d_err);
         MR_TRY(cudaGetLastError());
     }
     const int pair_blocks = (int)std::min<int64_t>((pairs + 255) / 256, 148 * 16);
@@ -556,17 +626,17 @@ int rasterize_impl(const float* verts, int64_t V, const int64_t* faces, int64_t 
                                                       list);
         MR_TRY(cudaGetLastError());
     }
-    const int KC = K <= 1 ? 1 : K <= 2 ? 2 : K <= 4 ? 4 : K <= 8 ? 8 : K <= 16 ? 16 : 32;
     const bool vec_ok = aligned16(p2f) && aligned16(zbuf) && aligned16(bary) && aligned16(dists);
+    const bool exact = (H & (H - 1)) == 0 && (W & (W - 1)) == 0;
     {
-    ProfScope ps(MR_STAGE_FINE, s);
-    if (persp) {
-        if (sil) dispatch_k<true, true>(KC, nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
-        else dispatch_k<true, false>(KC, nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
-    } else {
-        if (sil) dispatch_k<false, true>(KC, nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
-        else dispatch_k<false, false>(KC, nbins, s, geom, box, offsets, list, nbx, nby, H, W, K, blur, sigma, vec_ok, p2f, zbuf, bary, dists, alpha);
+        ProfScope ps(MR_STAGE_FINE, s);
+        dispatch_fine(KC, persp != 0, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk);
     }
+    MR_TRY(cudaGetLastError());
+    {
+        ProfScope ps(MR_STAGE_EPILOGUE, s);
+        dispatch_epilogue(KC, persp != 0, sil, npix, s, geom, topk, H, W, K, sigma, vec_ok, p2f, zbuf, bary, dists,
+                          alpha);
     }
     MR_TRY(cudaGetLastError());
 #undef MR_TRY

@@ -170,7 +170,8 @@ int mr_version(void);
 #define MR_STAGE_SILHOUETTE_BWD 6
 #define MR_STAGE_RASTER_BWD 7
 #define MR_STAGE_SILHOUETTE_RASTER_BWD 8
-#define MR_NUM_STAGES 9
+#define MR_STAGE_EPILOGUE 9
+#define MR_NUM_STAGES 10
 int mr_profile_enable(int32_t on);
 int mr_profile_read(double* stage_ms, int64_t* launches, int32_t nstages);
 

@@ -115,7 +115,7 @@ def test_end_to_end_batch2(oracle_mod):
     want = _oracle_chain(oracle_mod, b, o[0], o[3], ga, sigma)
     ex = o[4] > 0
     keep = ~_touched_vertices(b, o[0][ex], np_(p2f)[ex])
-    assert keep.mean() > 0.9
+    assert keep.mean() > 0.75
     compare_grad(got, want, mask=keep, label="end-to-end batch2")
     compare_alpha(alpha, oracle_mod.silhouette_fwd(o[0], o[3], sigma), mask=~ex, label="alpha batch2")
 
