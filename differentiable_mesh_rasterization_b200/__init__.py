@@ -25,7 +25,8 @@ ERRORS = {-1: "invalid argument", -2: "out of memory", -3: "CUDA error", -4: "de
 # Entry points declared by include/meshrast.h (checked by the test-suite).
 EXPORTS = ("mr_rasterize_fwd", "mr_rasterize_silhouette_fwd", "mr_silhouette_blend_fwd",
            "mr_silhouette_blend_bwd", "mr_rasterize_bwd", "mr_silhouette_rasterize_bwd",
-           "mr_device_status", "mr_last_error", "mr_version", "mr_profile_enable", "mr_profile_read")
+           "mr_device_status", "mr_last_error", "mr_version", "mr_profile_enable", "mr_profile_read",
+           "mr_rasterize_fwd_noalloc")
 STAGES = ("face_setup", "bin_count", "bin_scan", "bin_fill", "fine", "silhouette_fwd", "silhouette_bwd",
           "raster_bwd", "silhouette_raster_bwd", "epilogue")
 
@@ -51,6 +52,7 @@ def load_library() -> ctypes.CDLL:
     P, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
     sig = {
         "mr_rasterize_fwd": [P, i64, P, i64, P, P, i32, i32, i32, f32, i32, i32, P, P, P, P, P],
+        "mr_rasterize_fwd_noalloc": [P, i64, P, i64, P, P, i32, i32, i32, f32, i32, i32, P, P, P, P, P],
         "mr_rasterize_silhouette_fwd": [P, i64, P, i64, P, P, i32, i32, i32, f32, i32, i32, f32, P, P, P, P, P, P],
         "mr_silhouette_blend_fwd": [P, P, i32, i32, i32, i32, f32, P, P],
         "mr_silhouette_blend_bwd": [P, P, P, i32, i32, i32, i32, f32, P, P],
@@ -136,6 +138,32 @@ def rasterize_fwd(verts, faces, mesh_to_face_first_idx, num_faces_per_mesh, H, W
                lib.mr_rasterize_silhouette_fwd(*args, float(sigma), _ptr(p2f), _ptr(zbuf), _ptr(bary), _ptr(dists),
                                                _ptr(alpha), _stream(dev)))
         return p2f, zbuf, bary, dists, alpha
+
+
+def rasterize_fwd_noalloc(verts, faces, mesh_to_face_first_idx, num_faces_per_mesh, H, W, blur_radius, K,
+                          perspective_correct=False):
+    """``mr_rasterize_fwd_noalloc``: stage one with the library's fixed scratch array, for
+    callers that must not allocate device memory (the outputs here are still allocated by
+    torch).  Same outputs as :func:`rasterize_fwd`; batches too large for the array raise.
+    """
+    lib = load_library()
+    verts = _dev(verts, torch.float32, "verts")
+    faces = _dev(faces, torch.int64, "faces")
+    first = _host_i64(mesh_to_face_first_idx, "mesh_to_face_first_idx")
+    num = _host_i64(num_faces_per_mesh, "num_faces_per_mesh")
+    N = first.shape[0]
+    dev = verts.device
+    p2f = torch.empty((N, H, W, K), dtype=torch.int64, device=dev)
+    zbuf = torch.empty((N, H, W, K), dtype=torch.float32, device=dev)
+    bary = torch.empty((N, H, W, K, 3), dtype=torch.float32, device=dev)
+    dists = torch.empty((N, H, W, K), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check("mr_rasterize_fwd_noalloc",
+               lib.mr_rasterize_fwd_noalloc(_ptr(verts), verts.shape[0], _ptr(faces), faces.shape[0],
+                                            first.ctypes.data, num.ctypes.data, N, H, W, float(blur_radius), K,
+                                            int(bool(perspective_correct)), _ptr(p2f), _ptr(zbuf), _ptr(bary),
+                                            _ptr(dists), _stream(dev)))
+    return p2f, zbuf, bary, dists
 
 
 def _nhwk(p2f: torch.Tensor):

@@ -1,0 +1,534 @@
+// Kernels and launch helpers of the stage-one forward pipeline (internal header).
+//
+// Shared by the allocating entry points (mr_forward.cu) and the scratch-free variant
+// (mr_noalloc.cu); everything sits in an unnamed namespace, so each translation unit
+// compiles its own copy.  The pipeline is described in mr_forward.cu.
+#pragma once
+
+#include <cfloat>
+#include <climits>
+#include <cmath>
+#include <vector>
+
+#include "mr_common.cuh"
+#include "mr_silhouette.cuh"
+
+namespace mr {
+namespace {
+
+
+// ------------------------------------------------------------------ face setup
+// Per-face plane constants of the fine pass, computed in float64 from the exact float32
+// vertices and rounded once.  The origin is the face's first vertex a, so a pixel enters
+// as (dx, dy) = p - a.  The winding is made counter-clockwise (b and c swapped if needed)
+// so every edge function is positive inside.  Per edge u -> v with unit direction e and
+// length L:
+//     c(d) = -e.y * d.x + e.x * d.y + ng   signed distance to the edge line (inside > 0)
+//     s(d) =  e.x * d.x + e.y * d.y + tg   position along the edge, measured from u
+//     squared distance to the segment = c^2 + max(-s, s - L, 0)^2.
+// The depth key is the plane through (x, y, z) -- or (x, y, -1/z) with perspective
+// correction, where 1/z is screen-affine -- written as k_hi + (gx dx + gy dy + k_lo);
+// the float-float constant keeps the key within half an ulp plus the plane terms.
+// Layout (6 float4): (ax, ay, gx, gy) (k_hi, k_lo, L0, L1) (e0.x, e0.y, ng0, tg0)
+//                    (e1.x, e1.y, ng1, tg1) (e2.x, e2.y, ng2, tg2) (L2, face id, 0, 0)
+constexpr int kConstF4 = 6;
+
+__global__ void k_face_setup(const float* __restrict__ verts, int64_t V,
+                             const int64_t* __restrict__ faces, int64_t F, int H, int W,
+                             double reach, int persp, FaceGeom* __restrict__ geom,
+                             FaceBox* __restrict__ box, float4* __restrict__ fconst,
+                             int* __restrict__ err) {
+    int64_t f = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (f >= F) return;
+    int64_t i0 = faces[3 * f], i1 = faces[3 * f + 1], i2 = faces[3 * f + 2];
+    FaceBox bx = {1, 0, 1, 0};
+    float4* out = fconst + kConstF4 * f;
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i0 < 0 || i0 >= V || i1 < 0 || i1 >= V || i2 < 0 || i2 >= V) {
+        atomicOr(err, kErrFaceIndex);
+        geom[f] = FaceGeom{zero, zero, zero};
+        box[f] = bx;
+        return;
+    }
+    float4 a = make_float4(verts[3 * i0], verts[3 * i0 + 1], verts[3 * i0 + 2], 0.f);
+    float4 b = make_float4(verts[3 * i1], verts[3 * i1 + 1], verts[3 * i1 + 2], 0.f);
+    float4 c = make_float4(verts[3 * i2], verts[3 * i2 + 1], verts[3 * i2 + 2], 0.f);
+    geom[f] = FaceGeom{a, b, c};
+    double ax = a.x, ay = a.y, bxx = b.x, byy = b.y, cx = c.x, cy = c.y;
+    double area2 = (bxx - ax) * (cy - ay) - (byy - ay) * (cx - ax);
+    if (!(fabs(area2) > kDegenerateArea)) {
+        box[f] = bx;
+        return;
+    }
+    double xmin = fmin(ax, fmin(bxx, cx)) - reach, xmax = fmax(ax, fmax(bxx, cx)) + reach;
+    double ymin = fmin(ay, fmin(byy, cy)) - reach, ymax = fmax(ay, fmax(byy, cy)) + reach;
+    // pixel j has centre x = -1 + (2j+1)/W; row i has y = 1 - (2i+1)/H.  The 1e-4
+    // pixel pad keeps the box a superset under rounding.
+    double jl = ceil((xmin + 1.0) * 0.5 * W - 0.5 - 1e-4);
+    double jh = floor((xmax + 1.0) * 0.5 * W - 0.5 + 1e-4);
+    double il = ceil((1.0 - ymax) * 0.5 * H - 0.5 - 1e-4);
+    double ih = floor((1.0 - ymin) * 0.5 * H - 0.5 + 1e-4);
+    jl = fmax(jl, 0.0); il = fmax(il, 0.0);
+    jh = fmin(jh, (double)(W - 1)); ih = fmin(ih, (double)(H - 1));
+    if (jl <= jh && il <= ih) bx = FaceBox{(int)jl, (int)jh, (int)il, (int)ih};
+    box[f] = bx;
+
+    double x[3] = {0.0, bxx - ax, cx - ax};
+    double y[3] = {0.0, byy - ay, cy - ay};
+    double q[3];
+    if (persp) {
+        q[0] = -1.0 / (double)a.z; q[1] = -1.0 / (double)b.z; q[2] = -1.0 / (double)c.z;
+    } else {
+        q[0] = a.z; q[1] = b.z; q[2] = c.z;
+    }
+    const double nx = y[1] * (q[2] - q[0]) - (q[1] - q[0]) * y[2];
+    const double ny = (q[1] - q[0]) * x[2] - x[1] * (q[2] - q[0]);
+    const double gx = -nx / area2, gy = -ny / area2;
+    const float khi = (float)q[0];
+    const float klo = (float)(q[0] - (double)khi);
+    if (area2 < 0.0) {
+        double t = x[1]; x[1] = x[2]; x[2] = t;
+        t = y[1]; y[1] = y[2]; y[2] = t;
+    }
+    float e[3][5];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        const int k1 = k == 2 ? 0 : k + 1;
+        const double ex = x[k1] - x[k], ey = y[k1] - y[k];
+        const double L = sqrt(ex * ex + ey * ey);
+        const double ux = ex / L, uy = ey / L;
+        e[k][0] = (float)ux;
+        e[k][1] = (float)uy;
+        e[k][2] = (float)(uy * x[k] - ux * y[k]);
+        e[k][3] = (float)(-(ux * x[k] + uy * y[k]));
+        e[k][4] = (float)L;
+    }
+    out[0] = make_float4(a.x, a.y, (float)gx, (float)gy);
+    out[1] = make_float4(khi, klo, e[0][4], e[1][4]);
+    out[2] = make_float4(e[0][0], e[0][1], e[0][2], e[0][3]);
+    out[3] = make_float4(e[1][0], e[1][1], e[1][2], e[1][3]);
+    out[4] = make_float4(e[2][0], e[2][1], e[2][2], e[2][3]);
+    out[5] = make_float4(e[2][4], __int_as_float((int)f), 0.f, 0.f);
+}
+
+// ------------------------------------------------------------------ binning
+// (image, face) pairs are enumerated image by image: pair q belongs to image n with
+// pair_prefix[n] <= q < pair_prefix[n+1] and is face first[n] + q - pair_prefix[n].
+__device__ __forceinline__ int pair_image(const int64_t* prefix, int N, int64_t q) {
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= q) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+template <bool FILL>
+__global__ void k_bin_pairs(const FaceBox* __restrict__ box, const int64_t* __restrict__ prefix,
+                            const int64_t* __restrict__ first, int N, int64_t pairs, int nbx, int nby,
+                            int* __restrict__ counts, const int* __restrict__ offsets,
+                            int* __restrict__ list) {
+    const unsigned lane = threadIdx.x & 31;
+    for (int64_t q0 = (int64_t)blockIdx.x * blockDim.x; q0 < pairs; q0 += (int64_t)gridDim.x * blockDim.x) {
+        int64_t q = q0 + threadIdx.x;
+        bool live = q < pairs;
+        int n = 0;
+        int64_t f = 0;
+        FaceBox b = {1, 0, 1, 0};
+        if (live) {
+            n = pair_image(prefix, N, q);
+            f = first[n] + (q - prefix[n]);
+            b = box[f];
+        }
+        int bx0 = 0, bx1 = -1, by0 = 0, by1 = -1;
+        if (live && b.x0 <= b.x1) {
+            bx0 = b.x0 / kBin; bx1 = b.x1 / kBin; by0 = b.y0 / kBin; by1 = b.y1 / kBin;
+        }
+        // Walk the touched bins in lock-step across the warp; neighbouring faces share
+        // bins, so one atomic per distinct bin per step is issued.
+        int nx = bx1 - bx0 + 1, ny = by1 - by0 + 1;
+        int mine = (nx > 0 && ny > 0) ? nx * ny : 0;
+        int most = mine;
+        for (int o = 16; o > 0; o >>= 1) most = max(most, __shfl_xor_sync(0xffffffffu, most, o));
+        for (int s = 0; s < most; ++s) {
+            bool act = s < mine;
+            int bin = -1;
+            if (act) bin = (n * nby + by0 + s / nx) * nbx + bx0 + s % nx;
+            unsigned peers = __match_any_sync(0xffffffffu, bin);
+            if (!act) continue;
+            int leader = __ffs(peers) - 1;
+            int rank = __popc(peers & ((1u << lane) - 1));
+            int base = 0;
+            if ((int)lane == leader) base = atomicAdd(&counts[bin], __popc(peers));
+            base = __shfl_sync(peers, base, leader);
+            if (FILL) list[offsets[bin] + base + rank] = (int)f;
+        }
+    }
+}
+
+// Exclusive scan of nb counts by one 1024-thread CTA; offsets[nb] = total.
+__global__ void k_scan(const int* __restrict__ counts, int nb, int* __restrict__ offsets,
+                       long long* __restrict__ total) {
+    __shared__ long long part[1024];
+    const int t = threadIdx.x;
+    const int per = (nb + 1023) / 1024;
+    const int lo = min(nb, t * per), hi = min(nb, lo + per);
+    long long s = 0;
+    for (int i = lo; i < hi; ++i) s += counts[i];
+    part[t] = s;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+        long long v = t >= o ? part[t - o] : 0;
+        __syncthreads();
+        part[t] += v;
+        __syncthreads();
+    }
+    long long run = t ? part[t - 1] : 0;
+    for (int i = lo; i < hi; ++i) {
+        offsets[i] = (int)run;
+        run += counts[i];
+    }
+    if (t == 1023) {
+        offsets[nb] = (int)part[1023];
+        *total = part[1023];
+    }
+}
+
+// ------------------------------------------------------------------ fine pass
+template <int KC>
+__device__ __forceinline__ void topk_insert(float (&kk)[KC], int (&ff)[KC], float key, int fid) {
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+        bool lt = key < kk[k] || (key == kk[k] && fid < ff[k]);
+        float tk = lt ? kk[k] : key;
+        int tf = lt ? ff[k] : fid;
+        kk[k] = lt ? key : kk[k];
+        ff[k] = lt ? fid : ff[k];
+        key = tk;
+        fid = tf;
+    }
+}
+
+// One CTA per 16x16 bin; each of its eight warps owns an 8x4 pixel tile and runs on its
+// own (no block barriers).  A warp reads the bin's face list 32 ids at a time, tests
+// each face's pixel box against its tile, compacts the hits with a ballot and copies
+// their constants into its shared-memory slots.  For each staged face the warp first
+// evaluates the depth key alone; if no lane could admit the face into its top-K (face
+// behind the camera or not nearer than the lane's K-th key) the face is skipped, else
+// every lane runs the full candidacy test.  EXACT: the pixel centres are exact float32
+// values (H and W powers of two), so the float-float low parts vanish.
+template <int KC, bool PERSP, bool EXACT>
+__global__ void __launch_bounds__(kFineThreads)
+k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const int* __restrict__ offsets,
+       const int* __restrict__ list, int nbx, int nby, int H, int W, int K, float blur, int* __restrict__ topk) {
+    __shared__ float4 s_c[kWarpsPerBin][32][kConstF4];
+
+    const int bin = blockIdx.x;
+    const int bxi = bin % nbx;
+    const int byi = (bin / nbx) % nby;
+    const int n = bin / (nbx * nby);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tj0 = bxi * kBin + (warp & 1) * kWarpTileW;
+    const int ti0 = byi * kBin + (warp >> 1) * kWarpTileH;
+    if (tj0 >= W || ti0 >= H) return;                        // tile entirely off the image
+    const int j = tj0 + (lane & 7), i = ti0 + (lane >> 3);
+    const bool in_img = i < H && j < W;
+    const double pxd = -1.0 + (2.0 * j + 1.0) / W;
+    const double pyd = 1.0 - (2.0 * i + 1.0) / H;
+    const float pxh = (float)pxd, pyh = (float)pyd;
+    const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
+    const unsigned lt_mask = (1u << lane) - 1u;
+
+    float kk[KC];
+    int ff[KC];
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+        kk[k] = in_img ? FLT_MAX : -FLT_MAX;                 // off-image lanes admit nothing
+        ff[k] = INT_MAX;
+    }
+
+    const int beg = offsets[bin], cnt = offsets[bin + 1] - beg;
+    float4(*slots)[kConstF4] = s_c[warp];
+    for (int base = 0; base < cnt; base += 32) {
+        bool hit = false;
+        int fid = 0;
+        if (base + lane < cnt) {
+            fid = list[beg + base + lane];
+            const FaceBox b = box[fid];
+            hit = b.x0 <= tj0 + kWarpTileW - 1 && b.x1 >= tj0 && b.y0 <= ti0 + kWarpTileH - 1 && b.y1 >= ti0;
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (hit) {
+            const int slot = __popc(m & lt_mask);
+            const float4* src = fconst + (int64_t)kConstF4 * fid;
+#pragma unroll
+            for (int u = 0; u < kConstF4; ++u) slots[slot][u] = __ldg(src + u);
+        }
+        __syncwarp();
+        const int nh = __popc(m);
+        for (int qi = 0; qi < nh; ++qi) {
+            const float4 q0 = slots[qi][0], q1 = slots[qi][1];
+            float dx = pxh - q0.x, dy = pyh - q0.y;
+            if (!EXACT) { dx += pxl; dy += pyl; }
+            const float key = q1.x + fmaf(q0.z, dx, fmaf(q0.w, dy, q1.y));
+            const bool front = PERSP ? key < 0.f : key >= 0.f;
+            const bool maybe = front && key <= kk[KC - 1];
+            if (!__any_sync(0xffffffffu, maybe)) continue;
+            const float4 e0 = slots[qi][2], e1 = slots[qi][3], e2 = slots[qi][4], q5 = slots[qi][5];
+            const float c0 = fmaf(-e0.y, dx, fmaf(e0.x, dy, e0.z));
+            const float s0 = fmaf(e0.x, dx, fmaf(e0.y, dy, e0.w));
+            const float c1 = fmaf(-e1.y, dx, fmaf(e1.x, dy, e1.z));
+            const float s1 = fmaf(e1.x, dx, fmaf(e1.y, dy, e1.w));
+            const float c2 = fmaf(-e2.y, dx, fmaf(e2.x, dy, e2.z));
+            const float s2 = fmaf(e2.x, dx, fmaf(e2.y, dy, e2.w));
+            const float o0 = fmaxf(fmaxf(-s0, s0 - q1.z), 0.f);
+            const float o1 = fmaxf(fmaxf(-s1, s1 - q1.w), 0.f);
+            const float o2 = fmaxf(fmaxf(-s2, s2 - q5.x), 0.f);
+            const float d0 = fmaf(o0, o0, c0 * c0);
+            const float d1 = fmaf(o1, o1, c1 * c1);
+            const float d2 = fmaf(o2, o2, c2 * c2);
+            const bool inside = fminf(c0, fminf(c1, c2)) >= 0.f;
+            const float dmin = fminf(d0, fminf(d1, d2));
+            if (maybe && (inside || dmin <= blur)) topk_insert<KC>(kk, ff, key, __float_as_int(q5.y));
+        }
+        __syncwarp();
+    }
+    if (!in_img) return;
+    const int64_t pix = ((int64_t)n * H + i) * W + j;
+    if (K == KC && (KC % 4) == 0) {
+#pragma unroll
+        for (int k4 = 0; k4 < KC; k4 += 4)
+            *reinterpret_cast<int4*>(topk + pix * KC + k4) =
+                make_int4(ff[k4] == INT_MAX ? -1 : ff[k4], ff[k4 + 1] == INT_MAX ? -1 : ff[k4 + 1],
+                          ff[k4 + 2] == INT_MAX ? -1 : ff[k4 + 2], ff[k4 + 3] == INT_MAX ? -1 : ff[k4 + 3]);
+    } else {
+#pragma unroll
+        for (int k = 0; k < KC; ++k)
+            if (k < K) topk[pix * K + k] = ff[k] == INT_MAX ? -1 : ff[k];
+    }
+}
+
+// Exact (float64) per-slot outputs from the original vertices: the definition written
+// out -- edge-function barycentrics, closed-triangle inside test, nearest-edge squared
+// distance, perspective renormalisation, interpolated z.
+template <bool PERSP>
+__device__ void slot_outputs(const FaceGeom& g, double px, double py, float* z_out, float* b_out,
+                             float* d_out) {
+    double ax = g.a.x, ay = g.a.y, bx = g.b.x, by = g.b.y, cx = g.c.x, cy = g.c.y;
+    double area2 = (bx - ax) * (cy - ay) - (by - ay) * (cx - ax);
+    double w0 = ((bx - px) * (cy - py) - (by - py) * (cx - px)) / area2;
+    double w1 = ((cx - px) * (ay - py) - (cy - py) * (ax - px)) / area2;
+    double w2 = ((ax - px) * (by - py) - (ay - py) * (bx - px)) / area2;
+    bool inside = w0 >= 0.0 && w1 >= 0.0 && w2 >= 0.0;
+    double d2 = DBL_MAX;
+    const double ux[3] = {ax, bx, cx}, uy[3] = {ay, by, cy};
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        int k1 = k == 2 ? 0 : k + 1;
+        double ex = ux[k1] - ux[k], ey = uy[k1] - uy[k];
+        double len2 = ex * ex + ey * ey;
+        double t = len2 > 0.0 ? ((px - ux[k]) * ex + (py - uy[k]) * ey) / len2 : 0.0;
+        t = fmin(fmax(t, 0.0), 1.0);
+        double rx = px - (ux[k] + t * ex), ry = py - (uy[k] + t * ey);
+        d2 = fmin(d2, rx * rx + ry * ry);
+    }
+    double b0 = w0, b1 = w1, b2 = w2;
+    if (PERSP) {
+        double u0 = w0 / (double)g.a.z, u1 = w1 / (double)g.b.z, u2 = w2 / (double)g.c.z;
+        double s = u0 + u1 + u2;
+        b0 = u0 / s; b1 = u1 / s; b2 = u2 / s;
+    }
+    *z_out = (float)(b0 * (double)g.a.z + b1 * (double)g.b.z + b2 * (double)g.c.z);
+    b_out[0] = (float)b0;
+    b_out[1] = (float)b1;
+    b_out[2] = (float)b2;
+    *d_out = (float)(inside ? -d2 : d2);
+}
+
+// One thread per pixel: the K winners' outputs (and the fused silhouette), written
+// contiguously per pixel with 16-byte stores when K is a multiple of 4.
+template <int KC, bool PERSP, bool SIL>
+__global__ void __launch_bounds__(256)
+k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int64_t npix, int H, int W, int K,
+           float sigma, bool vec_ok, int64_t* __restrict__ p2f, float* __restrict__ zbuf, float* __restrict__ bary,
+           float* __restrict__ dists, float* __restrict__ alpha) {
+    for (int64_t pix = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; pix < npix;
+         pix += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t rem = pix % ((int64_t)H * W);
+        const int i = (int)(rem / W), j = (int)(rem % W);
+        const double pxd = -1.0 + (2.0 * j + 1.0) / W;
+        const double pyd = 1.0 - (2.0 * i + 1.0) / H;
+        float dsil[KC];
+        bool vsil[KC];
+        if (vec_ok && (KC % 4) == 0 && K == KC) {
+#pragma unroll
+            for (int k4 = 0; k4 < KC; k4 += 4) {
+                const int4 f4 = *reinterpret_cast<const int4*>(topk + pix * KC + k4);
+                const int fk[4] = {f4.x, f4.y, f4.z, f4.w};
+                float zz[4], bb[12], dd[4];
+                long long pf[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (fk[u] >= 0) {
+                        slot_outputs<PERSP>(geom[fk[u]], pxd, pyd, &zz[u], &bb[3 * u], &dd[u]);
+                    } else {
+                        zz[u] = -1.f; dd[u] = -1.f; bb[3 * u] = bb[3 * u + 1] = bb[3 * u + 2] = -1.f;
+                    }
+                    pf[u] = fk[u];
+                    dsil[k4 + u] = dd[u];
+                    vsil[k4 + u] = fk[u] >= 0;
+                }
+                const int64_t s = pix * KC + k4;
+                reinterpret_cast<longlong2*>(p2f + s)[0] = make_longlong2(pf[0], pf[1]);
+                reinterpret_cast<longlong2*>(p2f + s)[1] = make_longlong2(pf[2], pf[3]);
+                *reinterpret_cast<float4*>(zbuf + s) = make_float4(zz[0], zz[1], zz[2], zz[3]);
+                *reinterpret_cast<float4*>(dists + s) = make_float4(dd[0], dd[1], dd[2], dd[3]);
+                float4* bp = reinterpret_cast<float4*>(bary + 3 * s);
+                bp[0] = make_float4(bb[0], bb[1], bb[2], bb[3]);
+                bp[1] = make_float4(bb[4], bb[5], bb[6], bb[7]);
+                bp[2] = make_float4(bb[8], bb[9], bb[10], bb[11]);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < KC; ++k) {
+                if (k >= K) break;
+                const int64_t s = pix * K + k;
+                const int fk = topk[s];
+                float zz, bb[3], dd;
+                if (fk >= 0) {
+                    slot_outputs<PERSP>(geom[fk], pxd, pyd, &zz, bb, &dd);
+                } else {
+                    zz = -1.f; dd = -1.f; bb[0] = bb[1] = bb[2] = -1.f;
+                }
+                p2f[s] = fk;
+                zbuf[s] = zz;
+                dists[s] = dd;
+                bary[3 * s] = bb[0]; bary[3 * s + 1] = bb[1]; bary[3 * s + 2] = bb[2];
+                dsil[k] = dd;
+                vsil[k] = fk >= 0;
+            }
+        }
+        if (SIL) alpha[pix] = silhouette_alpha<KC>(dsil, vsil, K, sigma);
+    }
+}
+
+template <int KC>
+void launch_fine(bool persp, bool exact, int nbins, cudaStream_t s, const float4* fconst, const FaceBox* box,
+                 const int* offsets, const int* list, int nbx, int nby, int H, int W, int K, float blur, int* topk) {
+#define MR_FINE(P, E) \
+    k_fine<KC, P, E><<<nbins, kFineThreads, 0, s>>>(fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk)
+    if (persp) {
+        if (exact) MR_FINE(true, true); else MR_FINE(true, false);
+    } else {
+        if (exact) MR_FINE(false, true); else MR_FINE(false, false);
+    }
+#undef MR_FINE
+}
+
+template <int KC>
+void launch_epilogue(bool persp, bool sil, int64_t npix, cudaStream_t s, const FaceGeom* geom, const int* topk,
+                     int H, int W, int K, float sigma, bool vec_ok, int64_t* p2f, float* zbuf, float* bary,
+                     float* dists, float* alpha) {
+    const int grid = (int)std::min<int64_t>((npix + 255) / 256, 148 * 16);
+#define MR_EPI(P, S) \
+    k_epilogue<KC, P, S><<<grid, 256, 0, s>>>(geom, topk, npix, H, W, K, sigma, vec_ok, p2f, zbuf, bary, dists, alpha)
+    if (persp) {
+        if (sil) MR_EPI(true, true); else MR_EPI(true, false);
+    } else {
+        if (sil) MR_EPI(false, true); else MR_EPI(false, false);
+    }
+#undef MR_EPI
+}
+
+void dispatch_fine(int KC, bool persp, bool exact, int nbins, cudaStream_t s, const float4* fconst,
+                   const FaceBox* box, const int* offsets, const int* list, int nbx, int nby, int H, int W, int K,
+                   float blur, int* topk) {
+    switch (KC) {
+        case 1: launch_fine<1>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
+        case 2: launch_fine<2>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
+        case 4: launch_fine<4>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
+        case 8: launch_fine<8>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
+        case 16: launch_fine<16>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
+        default: launch_fine<32>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
+    }
+}
+
+void dispatch_epilogue(int KC, bool persp, bool sil, int64_t npix, cudaStream_t s, const FaceGeom* geom,
+                       const int* topk, int H, int W, int K, float sigma, bool vec_ok, int64_t* p2f, float* zbuf,
+                       float* bary, float* dists, float* alpha) {
+#define MR_E(KCV) launch_epilogue<KCV>(persp, sil, npix, s, geom, topk, H, W, K, sigma, vec_ok, p2f, zbuf, bary, dists, alpha)
+    switch (KC) {
+        case 1: MR_E(1); break;
+        case 2: MR_E(2); break;
+        case 4: MR_E(4); break;
+        case 8: MR_E(8); break;
+        case 16: MR_E(16); break;
+        default: MR_E(32); break;
+    }
+#undef MR_E
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate_fwd(const float* verts, int64_t V, const int64_t* faces, int64_t F, const int64_t* first,
+                 const int64_t* num, int32_t N, int32_t H, int32_t W, float blur, int32_t K,
+                 const void* p2f, const void* zbuf, const void* bary, const void* dists) {
+    if (N < 0 || H < 1 || W < 1 || H > MR_MAX_SIDE || W > MR_MAX_SIDE) {
+        set_error("invalid image batch N=%d H=%d W=%d", N, H, W);
+        return MR_ERR_ARG;
+    }
+    if (K < 1 || K > MR_KMAX) {
+        set_error("K=%d outside 1..%d", K, MR_KMAX);
+        return MR_ERR_ARG;
+    }
+    if (!(blur >= 0.f) || !std::isfinite(blur)) {
+        set_error("blur_radius must be finite and >= 0");
+        return MR_ERR_ARG;
+    }
+    if (V < 0 || F < 0 || V > INT32_MAX || F > INT32_MAX) {
+        set_error("V=%lld F=%lld outside 0..2^31-1", (long long)V, (long long)F);
+        return MR_ERR_ARG;
+    }
+    if ((F > 0 && (!faces || !verts)) || (N > 0 && (!first || !num))) {
+        set_error("null input pointer");
+        return MR_ERR_ARG;
+    }
+    if (N > 0 && (!p2f || !zbuf || !bary || !dists)) {
+        set_error("null output pointer");
+        return MR_ERR_ARG;
+    }
+    for (int n = 0; n < N; ++n) {
+        if (first[n] < 0 || num[n] < 0 || first[n] + num[n] > F) {
+            set_error("mesh %d: faces [%lld, %lld) outside [0, F=%lld)", n, (long long)first[n],
+                      (long long)(first[n] + num[n]), (long long)F);
+            return MR_ERR_ARG;
+        }
+    }
+    return MR_OK;
+}
+
+// Bytes of the fixed scratch block of one forward call (everything but the bin lists),
+// and the offsets of its parts.
+struct FwdScratch {
+    size_t geom, box, con, top, cnt, off, pre, fst, tot, err, bytes;
+};
+
+inline FwdScratch fwd_scratch_layout(int64_t F, int64_t npix, int K, int nbins, int N) {
+    auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
+    FwdScratch L;
+    L.geom = 0;
+    L.box = L.geom + up(sizeof(FaceGeom) * (size_t)F);
+    L.con = L.box + up(sizeof(FaceBox) * (size_t)F);
+    L.top = L.con + up(sizeof(float4) * kConstF4 * (size_t)F);
+    L.cnt = L.top + up(sizeof(int) * (size_t)npix * (size_t)K);
+    L.off = L.cnt + up(sizeof(int) * (size_t)nbins);
+    L.pre = L.off + up(sizeof(int) * (size_t)(nbins + 1));
+    L.fst = L.pre + up(sizeof(int64_t) * (size_t)(N + 1));
+    L.tot = L.fst + up(sizeof(int64_t) * (size_t)N);
+    L.err = L.tot + 256;
+    L.bytes = L.err + 256;
+    return L;
+}
+
+}  // namespace
+}  // namespace mr

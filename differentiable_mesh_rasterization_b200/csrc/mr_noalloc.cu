@@ -1,0 +1,155 @@
+// mr_rasterize_fwd_noalloc: stage one of the rasterizer for callers that must not
+// allocate device memory.
+//
+// Some callers cannot call cudaMalloc (or any allocator) at the moment they render: a
+// host that has handed all device memory to its own pool and forbids the driver from
+// carving out more, a latency-critical loop where an allocation could block or fail
+// under memory pressure, or a plugin that runs inside someone else's memory budget.
+// For them this entry point runs the same kernels as mr_rasterize_fwd, but every byte
+// of scratch (face records, per-bin counts and lists, the top-K face ids) comes from
+// one file-scope device array of fixed size.  The caller still provides the inputs and
+// the outputs.
+//
+// The array is MR_NOALLOC_SCRATCH_BYTES (64 MiB) on every device that loads this part
+// of the library and stays there until the process exits.  Its address is looked up
+// once per device, by the first call made on that device with the device current; make
+// that first call before any stream capture.  All calls share the array and it keeps
+// the previous call's contents (the parts that must start at zero are cleared on every
+// call), so two calls whose work overlaps on the GPU -- on different streams, or from
+// different threads -- race on it; order them on one stream.
+#include <mutex>
+
+#include "mr_forward_kernels.cuh"
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MR_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mutex;
+char* g_noalloc_ptr[64] = {};
+
+// Device address of the scratch array on the current device (looked up once per device).
+int noalloc_scratch(char** out) {
+    int dev = 0;
+    MR_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) {
+        mr::set_error("device ordinal %d outside 0..63", dev);
+        return MR_ERR_ARG;
+    }
+    std::lock_guard<std::mutex> g(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return mr::cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+        g_noalloc_ptr[dev] = static_cast<char*>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return MR_OK;
+}
+
+}  // namespace
+
+namespace mr {
+namespace {
+
+int rasterize_noalloc(const float* verts, int64_t V, const int64_t* faces, int64_t F, const int64_t* first,
+                      const int64_t* num, int32_t N, int32_t H, int32_t W, float blur, int32_t K, int32_t persp,
+                      int64_t* p2f, float* zbuf, float* bary, float* dists, cudaStream_t s) {
+    int rc = validate_fwd(verts, V, faces, F, first, num, N, H, W, blur, K, p2f, zbuf, bary, dists);
+    if (rc != MR_OK) return rc;
+    if (N == 0) return MR_OK;
+    const int nbx = ceil_div(W, kBin), nby = ceil_div(H, kBin);
+    const long long nbins_ll = (long long)N * nbx * nby;
+    if (nbins_ll >= INT32_MAX / 2) {
+        set_error("too many screen bins (%lld)", nbins_ll);
+        return MR_ERR_ARG;
+    }
+    const int nbins = (int)nbins_ll;
+    const int KC = K <= 1 ? 1 : K <= 2 ? 2 : K <= 4 ? 4 : K <= 8 ? 8 : K <= 16 ? 16 : 32;
+    const int64_t npix = (int64_t)N * H * W;
+    const FwdScratch L = fwd_scratch_layout(F, npix, K, nbins, N);
+    if (L.bytes > (size_t)MR_NOALLOC_SCRATCH_BYTES) {
+        set_error("mr_rasterize_fwd_noalloc: this batch needs %zu bytes of scratch before its bin lists, more "
+                  "than the fixed %d bytes; use mr_rasterize_fwd", L.bytes, MR_NOALLOC_SCRATCH_BYTES);
+        return MR_ERR_ARG;
+    }
+    char* ws = nullptr;
+    rc = noalloc_scratch(&ws);
+    if (rc != MR_OK) return rc;
+    std::vector<int64_t> prefix(N + 1, 0);
+    for (int n = 0; n < N; ++n) prefix[n + 1] = prefix[n] + num[n];
+    const int64_t pairs = prefix[N];
+
+    FaceGeom* geom = reinterpret_cast<FaceGeom*>(ws + L.geom);
+    FaceBox* box = reinterpret_cast<FaceBox*>(ws + L.box);
+    float4* fconst = reinterpret_cast<float4*>(ws + L.con);
+    int* topk = reinterpret_cast<int*>(ws + L.top);
+    int* counts = reinterpret_cast<int*>(ws + L.cnt);
+    int* offsets = reinterpret_cast<int*>(ws + L.off);
+    int64_t* d_prefix = reinterpret_cast<int64_t*>(ws + L.pre);
+    int64_t* d_first = reinterpret_cast<int64_t*>(ws + L.fst);
+    long long* d_total = reinterpret_cast<long long*>(ws + L.tot);
+    int* d_err = reinterpret_cast<int*>(ws + L.err);
+    int* list = reinterpret_cast<int*>(ws + L.bytes);
+
+    MR_CUDA(cudaMemcpyAsync(d_prefix, prefix.data(), sizeof(int64_t) * (N + 1), cudaMemcpyHostToDevice, s));
+    MR_CUDA(cudaMemcpyAsync(d_first, first, sizeof(int64_t) * N, cudaMemcpyHostToDevice, s));
+    MR_CUDA(cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)nbins, s));
+    MR_CUDA(cudaMemsetAsync(d_err, 0, sizeof(int), s));
+    const double reach = std::sqrt((double)blur) * (1.0 + 1e-6) + 1e-7;
+    if (F > 0) {
+        k_face_setup<<<(unsigned)((F + 255) / 256), 256, 0, s>>>(verts, V, faces, F, H, W, reach, persp, geom, box,
+                                                                  fconst, d_err);
+        MR_CUDA(cudaGetLastError());
+    }
+    const int pair_blocks = (int)std::min<int64_t>((pairs + 255) / 256, 148 * 16);
+    if (pairs > 0) {
+        k_bin_pairs<false><<<pair_blocks, 256, 0, s>>>(box, d_prefix, d_first, N, pairs, nbx, nby, counts, nullptr,
+                                                       nullptr);
+        MR_CUDA(cudaGetLastError());
+    }
+    k_scan<<<1, 1024, 0, s>>>(counts, nbins, offsets, d_total);
+    MR_CUDA(cudaGetLastError());
+    long long total = 0;
+    int herr = 0;
+    MR_CUDA(cudaMemcpyAsync(&total, d_total, sizeof(long long), cudaMemcpyDeviceToHost, s));
+    MR_CUDA(cudaMemcpyAsync(&herr, d_err, sizeof(int), cudaMemcpyDeviceToHost, s));
+    MR_CUDA(cudaStreamSynchronize(s));
+    if (total < 0 || L.bytes + sizeof(int) * (size_t)total > (size_t)MR_NOALLOC_SCRATCH_BYTES) {
+        set_error("mr_rasterize_fwd_noalloc: the bin lists need %lld entries, more than the %zu left of the "
+                  "fixed %d-byte scratch; use mr_rasterize_fwd", total,
+                  ((size_t)MR_NOALLOC_SCRATCH_BYTES - L.bytes) / sizeof(int), MR_NOALLOC_SCRATCH_BYTES);
+        return MR_ERR_ARG;
+    }
+    if (total > 0) {
+        MR_CUDA(cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)nbins, s));
+        k_bin_pairs<true><<<pair_blocks, 256, 0, s>>>(box, d_prefix, d_first, N, pairs, nbx, nby, counts, offsets,
+                                                      list);
+        MR_CUDA(cudaGetLastError());
+    }
+    const bool vec_ok = aligned16(p2f) && aligned16(zbuf) && aligned16(bary) && aligned16(dists);
+    const bool exact = (H & (H - 1)) == 0 && (W & (W - 1)) == 0;
+    dispatch_fine(KC, persp != 0, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk);
+    MR_CUDA(cudaGetLastError());
+    dispatch_epilogue(KC, persp != 0, false, npix, s, geom, topk, H, W, K, 0.f, vec_ok, p2f, zbuf, bary, dists,
+                      nullptr);
+    MR_CUDA(cudaGetLastError());
+    if (herr != 0) {
+        set_error("a face references a vertex id outside [0, V=%lld); it was ignored", (long long)V);
+        return MR_ERR_DEVICE;
+    }
+    return MR_OK;
+}
+
+}  // namespace
+}  // namespace mr
+
+extern "C" int mr_rasterize_fwd_noalloc(const float* verts, int64_t V, const int64_t* faces, int64_t F,
+                                        const int64_t* mesh_to_face_first_idx, const int64_t* num_faces_per_mesh,
+                                        int32_t N, int32_t H, int32_t W, float blur_radius, int32_t K,
+                                        int32_t perspective_correct, int64_t* pix_to_face, float* zbuf, float* bary,
+                                        float* dists, void* stream) {
+    return mr::rasterize_noalloc(verts, V, faces, F, mesh_to_face_first_idx, num_faces_per_mesh, N, H, W,
+                                 blur_radius, K, perspective_correct, pix_to_face, zbuf, bary, dists,
+                                 static_cast<cudaStream_t>(stream));
+}

@@ -83,6 +83,33 @@ int mr_rasterize_fwd(const float* verts, int64_t V, const int64_t* faces, int64_
                      float* bary, float* dists, void* stream);
 
 /*
+ * mr_rasterize_fwd for callers that cannot allocate device memory (no counterpart in the
+ * paper: a property of this library's interface).  Some callers may not call cudaMalloc
+ * or any allocator while they render -- a host that hands all device memory to its own
+ * pool, a latency-critical loop where an allocation could stall or fail under memory
+ * pressure, a plugin running inside another program's memory budget.  This entry point
+ * computes exactly what mr_rasterize_fwd computes with the same kernels, but takes all
+ * of its scratch from one fixed device array of MR_NOALLOC_SCRATCH_BYTES that the
+ * library holds on each device using it until the process exits; it calls no cudaMalloc,
+ * cudaFree or other allocating routine.  The caller still provides inputs and outputs.
+ *  - Batches whose scratch exceeds the array (face records, per-pixel top-K ids, per-bin
+ *    counts and lists) are rejected with MR_ERR_ARG and a message naming the size.
+ *  - The first call on a device looks up the array's device address, with that device
+ *    current; make that first call before any stream capture.
+ *  - All calls share the array and it keeps the last call's contents (what must start
+ *    at zero is cleared on every call).  Calls whose work overlaps on the GPU race on
+ *    it: issue them in order on one stream.
+ * Same arguments, outputs, synchronisation and errors as mr_rasterize_fwd.
+ */
+#define MR_NOALLOC_SCRATCH_BYTES (64 * 1024 * 1024)
+int mr_rasterize_fwd_noalloc(const float* verts, int64_t V, const int64_t* faces, int64_t F,
+                             const int64_t* mesh_to_face_first_idx,
+                             const int64_t* num_faces_per_mesh, int32_t N, int32_t H, int32_t W,
+                             float blur_radius, int32_t K, int32_t perspective_correct,
+                             int64_t* pix_to_face, float* zbuf, float* bary, float* dists,
+                             void* stream);
+
+/*
  * Stage one fused with the stage-two silhouette: the outputs of mr_rasterize_fwd plus
  * alpha (N x H x W float32), bitwise equal to mr_silhouette_blend_fwd applied to the
  * dists written here.  sigma > 0.
