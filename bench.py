@@ -36,6 +36,7 @@ UNIT = "pixel-face samples/s"
 C_TEST = 38                 # FP32 instructions per pixel-face test (frozen)
 FP32_LANES_PER_SM = 128
 L2_FLUSH_BYTES = 256 << 20
+KERNELS_PER_STAGE = {"silhouette_raster_bwd": 2}    # main kernel + (x, y) -> (x, y, z) copy
 
 
 # ----------------------------------------------------------------------------- counting
@@ -375,7 +376,7 @@ def main():
             "roofline": roof,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": float(te[0]) / max(args.e2e_steps, 1)},
-            "gpu_launches": int(sum(v[1] for v in stages.values())),
+            "gpu_launches": int(sum(v[1] * KERNELS_PER_STAGE.get(k, 1) for k, v in stages.items())),
             "clocks": clk}
 
     if rank == 0 and not args.no_cpu_baseline:

@@ -144,77 +144,116 @@ __global__ void k_raster_bwd(const float* __restrict__ verts, int64_t V, const i
     }
 }
 
-// Fused silhouette backward + distance backward: one thread per pixel, float32.
+// Sum of c over the lanes of this warp that carry the same vertex id, added once into
+// acc[vid] with a float2 (x, y) atomic.  Inactive lanes take a unique key and drop out.
+__device__ __forceinline__ void scatter_xy(float2* __restrict__ acc, bool act, int vid, float2 c, int lane) {
+    const int key = act ? vid : -1 - lane;
+    const unsigned grp = __match_any_sync(0xffffffffu, key);
+    if (!act) return;
+    float2 sum = make_float2(0.f, 0.f);
+    for (unsigned m = grp; m; m &= m - 1) {
+        const int src = __ffs(m) - 1;
+        sum.x += __shfl_sync(grp, c.x, src);
+        sum.y += __shfl_sync(grp, c.y, src);
+    }
+    if (lane == __ffs(grp) - 1) atomicAdd(acc + vid, sum);
+}
+
+// Fused silhouette backward + distance backward: one thread per pixel (32 consecutive
+// pixels per warp), float32.  Per slot the nearest edge u -> v is recomputed and its two
+// end points receive -2 (p - q)(1 - t) and -2 (p - q) t times dL/ddist; contributions to
+// the same vertex within a warp are summed before one float2 atomic.
 template <int KC>
-__global__ void k_sil_raster_bwd(const float* __restrict__ verts, int64_t V, const int64_t* __restrict__ faces,
-                                 int64_t F, const int64_t* __restrict__ p2f, const float* __restrict__ dists,
-                                 const float* __restrict__ grad_alpha, int64_t npix, int H, int W, int K,
-                                 float sigma, float* __restrict__ gv, int* __restrict__ err) {
-    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < npix; q += (int64_t)gridDim.x * blockDim.x) {
+__global__ void __launch_bounds__(256)
+k_sil_raster_bwd(const float* __restrict__ verts, int64_t V, const int64_t* __restrict__ faces, int64_t F,
+                 const int64_t* __restrict__ p2f, const float* __restrict__ dists,
+                 const float* __restrict__ grad_alpha, int64_t npix, int H, int W, int K, float sigma,
+                 float2* __restrict__ acc, int* __restrict__ err) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t base = wid * 32; base < npix; base += nw * 32) {
+        const int64_t q = base + lane;
+        const bool live = q < npix;
         float d[KC], g[KC];
         bool v[KC];
         int64_t fk[KC];
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
-            fk[k] = k < K ? p2f[q * K + k] : -1;
+            const bool in = live && k < K;
+            fk[k] = in ? p2f[q * K + k] : -1;
             if (fk[k] < -1) atomicOr(err, kErrSlotIndex);
             v[k] = fk[k] >= 0;
-            d[k] = k < K ? dists[q * K + k] : 0.f;
+            d[k] = in ? dists[q * K + k] : 0.f;
         }
-        const float ga = grad_alpha[q];
-        if (ga == 0.f) continue;
+        const float ga = live ? grad_alpha[q] : 0.f;
         silhouette_grad<KC>(d, v, K, sigma, ga, g);
-        const int64_t rem = q % ((int64_t)H * W);
+        const int64_t rem = (live ? q : 0) % ((int64_t)H * W);
         const int i = (int)(rem / W), j = (int)(rem % W);
-        const float px = (float)(-1.0 + (2.0 * j + 1.0) / W);
-        const float py = (float)(1.0 - (2.0 * i + 1.0) / H);
+        const double pxd = -1.0 + (2.0 * j + 1.0) / W, pyd = 1.0 - (2.0 * i + 1.0) / H;
+        const float pxh = (float)pxd, pyh = (float)pyd;
+        const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
-            if (k >= K || !v[k] || g[k] == 0.f) continue;
-            const int64_t f = fk[k];
-            if (f >= F) {
-                atomicOr(err, kErrSlotIndex);
-                continue;
-            }
-            int64_t vid[3];
-            if (!load_face(faces, V, f, vid)) {
-                atomicOr(err, kErrFaceIndex);
-                continue;
-            }
-            float x[3], y[3];
+            bool act = k < K && v[k] && g[k] != 0.f;
+            int vu = 0, vv = 0;
+            float2 cu = make_float2(0.f, 0.f), cv = make_float2(0.f, 0.f);
+            if (act) {
+                int64_t vid[3];
+                if (fk[k] >= F) {
+                    atomicOr(err, kErrSlotIndex);
+                    act = false;
+                } else if (!load_face(faces, V, fk[k], vid)) {
+                    atomicOr(err, kErrFaceIndex);
+                    act = false;
+                } else {
+                    float x[3], y[3];
 #pragma unroll
-            for (int e = 0; e < 3; ++e) {
-                x[e] = verts[3 * vid[e]];
-                y[e] = verts[3 * vid[e] + 1];
-            }
-            int eu = 0;
-            float best = FLT_MAX, bt = 0.f, brx = 0.f, bry = 0.f;
+                    for (int e = 0; e < 3; ++e) {
+                        x[e] = verts[3 * vid[e]];
+                        y[e] = verts[3 * vid[e] + 1];
+                    }
+                    int eu = 0;
+                    float best = FLT_MAX, bt = 0.f, brx = 0.f, bry = 0.f;
 #pragma unroll
-            for (int e = 0; e < 3; ++e) {
-                const int e1 = e == 2 ? 0 : e + 1;
-                const float ex = x[e1] - x[e], ey = y[e1] - y[e];
-                const float ax = px - x[e], ay = py - y[e];
-                const float len2 = ex * ex + ey * ey;
-                float t = len2 > 0.f ? (ax * ex + ay * ey) / len2 : 0.f;
-                t = fminf(fmaxf(t, 0.f), 1.f);
-                const float rx = ax - t * ex, ry = ay - t * ey;
-                const float d2 = rx * rx + ry * ry;
-                if (d2 < best) { best = d2; eu = e; bt = t; brx = rx; bry = ry; }
+                    for (int e = 0; e < 3; ++e) {
+                        const int e1 = e == 2 ? 0 : e + 1;
+                        const float ex = x[e1] - x[e], ey = y[e1] - y[e];
+                        const float ax = (pxh - x[e]) + pxl, ay = (pyh - y[e]) + pyl;
+                        const float len2 = fmaf(ex, ex, ey * ey);
+                        const float t = len2 > 0.f ? __saturatef(fmaf(ax, ex, ay * ey) / len2) : 0.f;
+                        const float rx = fmaf(-t, ex, ax), ry = fmaf(-t, ey, ay);
+                        const float d2 = fmaf(rx, rx, ry * ry);
+                        if (d2 < best) { best = d2; eu = e; bt = t; brx = rx; bry = ry; }
+                    }
+                    const int ev = eu == 2 ? 0 : eu + 1;
+                    const float gdist = d[k] < 0.f ? -g[k] : g[k];
+                    const float su = -2.f * gdist * (1.f - bt), sv = -2.f * gdist * bt;
+                    cu = make_float2(su * brx, su * bry);
+                    cv = make_float2(sv * brx, sv * bry);
+                    vu = (int)vid[eu];
+                    vv = (int)vid[ev];
+                }
             }
-            const int ev = eu == 2 ? 0 : eu + 1;
-            const float gdist = d[k] < 0.f ? -g[k] : g[k];
-            const float cu = -2.f * gdist * (1.f - bt), cv = -2.f * gdist * bt;
-            atomicAdd(gv + 3 * vid[eu], cu * brx);
-            atomicAdd(gv + 3 * vid[eu] + 1, cu * bry);
-            atomicAdd(gv + 3 * vid[ev], cv * brx);
-            atomicAdd(gv + 3 * vid[ev] + 1, cv * bry);
+            scatter_xy(acc, act, vu, cu, lane);
+            scatter_xy(acc, act, vv, cv, lane);
         }
+    }
+}
+
+// grad_verts (V x 3) from the (x, y) accumulator; the silhouette has no z gradient.
+__global__ void k_xy_to_xyz(const float2* __restrict__ acc, int64_t V, float* __restrict__ gv) {
+    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < V; v += (int64_t)gridDim.x * blockDim.x) {
+        const float2 a = acc[v];
+        gv[3 * v] = a.x;
+        gv[3 * v + 1] = a.y;
+        gv[3 * v + 2] = 0.f;
     }
 }
 
 int validate_bwd(const float* verts, int64_t V, const int64_t* faces, int64_t F, const int64_t* p2f, int32_t N,
                  int32_t H, int32_t W, int32_t K, float* grad_verts) {
-    if (N < 0 || H < 1 || W < 1 || K < 1 || K > MR_KMAX || V < 0 || F < 0) {
+    if (N < 0 || H < 1 || W < 1 || K < 1 || K > MR_KMAX || V < 0 || F < 0 || V > INT32_MAX) {
         set_error("invalid shape N=%d H=%d W=%d K=%d V=%lld F=%lld", N, H, W, K, (long long)V, (long long)F);
         return MR_ERR_ARG;
     }
@@ -276,27 +315,38 @@ int mr_silhouette_rasterize_bwd(const float* verts, int64_t V, const int64_t* fa
         return MR_ERR_ARG;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (V > 0) MR_CUDA(cudaMemsetAsync(grad_verts, 0, sizeof(float) * 3 * (size_t)V, s));
     const int64_t npix = (int64_t)N * H * W;
-    if (npix == 0) return MR_OK;
+    if (npix == 0 || V == 0) {
+        if (V > 0) MR_CUDA(cudaMemsetAsync(grad_verts, 0, sizeof(float) * 3 * (size_t)V, s));
+        return MR_OK;
+    }
     int* err = mr::device_error_word();
     if (!err) {
         mr::set_error("cannot locate the device error word");
         return MR_ERR_CUDA;
     }
-    const int g = mr::grid_for(npix);
-    mr::ProfScope ps(MR_STAGE_SILHOUETTE_RASTER_BWD, s);
+    float2* acc = nullptr;
+    rc = mr::scratch_alloc(reinterpret_cast<void**>(&acc), sizeof(float2) * (size_t)V, s);
+    if (rc != MR_OK) return rc;
+    cudaError_t e = cudaMemsetAsync(acc, 0, sizeof(float2) * (size_t)V, s);
+    if (e == cudaSuccess) {
+        const int g = mr::grid_for(npix);
+        mr::ProfScope ps(MR_STAGE_SILHOUETTE_RASTER_BWD, s);
 #define MR_SRB(KC)                                                                                            \
     mr::k_sil_raster_bwd<KC><<<g, 256, 0, s>>>(verts, V, faces, F, pix_to_face, dists, grad_alpha, npix, H, W, K, \
-                                               sigma, grad_verts, err)
-    if (K <= 1) MR_SRB(1);
-    else if (K <= 2) MR_SRB(2);
-    else if (K <= 4) MR_SRB(4);
-    else if (K <= 8) MR_SRB(8);
-    else if (K <= 16) MR_SRB(16);
-    else MR_SRB(32);
+                                               sigma, acc, err)
+        if (K <= 1) MR_SRB(1);
+        else if (K <= 2) MR_SRB(2);
+        else if (K <= 4) MR_SRB(4);
+        else if (K <= 8) MR_SRB(8);
+        else if (K <= 16) MR_SRB(16);
+        else MR_SRB(32);
 #undef MR_SRB
-    MR_CUDA(cudaGetLastError());
+        mr::k_xy_to_xyz<<<mr::grid_for(V), 256, 0, s>>>(acc, V, grad_verts);
+        e = cudaGetLastError();
+    }
+    mr::scratch_free(acc, s);
+    if (e != cudaSuccess) return mr::cuda_fail(e, "silhouette-rasterizer backward launch");
     return MR_OK;
 }
 

@@ -53,13 +53,18 @@ __global__ void k_face_setup(const float* __restrict__ verts, int64_t V,
     float4 a = make_float4(verts[3 * i0], verts[3 * i0 + 1], verts[3 * i0 + 2], 0.f);
     float4 b = make_float4(verts[3 * i1], verts[3 * i1 + 1], verts[3 * i1 + 2], 0.f);
     float4 c = make_float4(verts[3 * i2], verts[3 * i2 + 1], verts[3 * i2 + 2], 0.f);
-    geom[f] = FaceGeom{a, b, c};
     double ax = a.x, ay = a.y, bxx = b.x, byy = b.y, cx = c.x, cy = c.y;
     double area2 = (bxx - ax) * (cy - ay) - (byy - ay) * (cx - ax);
     if (!(fabs(area2) > kDegenerateArea)) {
+        geom[f] = FaceGeom{a, b, c};
         box[f] = bx;
         return;
     }
+    // 1 / (2 area) as a float-float pair for the epilogue's float64 barycentrics
+    const double inv_area2 = 1.0 / area2;
+    a.w = (float)inv_area2;
+    b.w = (float)(inv_area2 - (double)a.w);
+    geom[f] = FaceGeom{a, b, c};
     double xmin = fmin(ax, fmin(bxx, cx)) - reach, xmax = fmax(ax, fmax(bxx, cx)) + reach;
     double ymin = fmin(ay, fmin(byy, cy)) - reach, ymax = fmax(ay, fmax(byy, cy)) + reach;
     // pixel j has centre x = -1 + (2j+1)/W; row i has y = 1 - (2i+1)/H.  The 1e-4
@@ -166,31 +171,41 @@ __global__ void k_bin_pairs(const FaceBox* __restrict__ box, const int64_t* __re
     }
 }
 
-// Exclusive scan of nb counts by one 1024-thread CTA; offsets[nb] = total.
-__global__ void k_scan(const int* __restrict__ counts, int nb, int* __restrict__ offsets,
-                       long long* __restrict__ total) {
-    __shared__ long long part[1024];
-    const int t = threadIdx.x;
-    const int per = (nb + 1023) / 1024;
-    const int lo = min(nb, t * per), hi = min(nb, lo + per);
-    long long s = 0;
-    for (int i = lo; i < hi; ++i) s += counts[i];
-    part[t] = s;
-    __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {
-        long long v = t >= o ? part[t - o] : 0;
+// Exclusive scan of nb counts by one 1024-thread CTA, 1024 consecutive counts per round
+// (coalesced), warp shuffles within a round and a running carry; offsets[nb] = total.
+__global__ void __launch_bounds__(1024) k_scan(const int* __restrict__ counts, int nb, int* __restrict__ offsets,
+                                               long long* __restrict__ total) {
+    __shared__ long long wsum[32];
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    long long carry = 0;
+    for (int base = 0; base < nb; base += 1024) {
+        const int i = base + t;
+        const long long v = i < nb ? counts[i] : 0;
+        long long x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) wsum[w] = x;
         __syncthreads();
-        part[t] += v;
+        if (w == 0) {
+            long long y = wsum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const long long z = __shfl_up_sync(0xffffffffu, y, o);
+                if (lane >= o) y += z;
+            }
+            wsum[lane] = y;
+        }
+        __syncthreads();
+        if (i < nb) offsets[i] = (int)(carry + (w ? wsum[w - 1] : 0) + x - v);
+        carry += wsum[31];
         __syncthreads();
     }
-    long long run = t ? part[t - 1] : 0;
-    for (int i = lo; i < hi; ++i) {
-        offsets[i] = (int)run;
-        run += counts[i];
-    }
-    if (t == 1023) {
-        offsets[nb] = (int)part[1023];
-        *total = part[1023];
+    if (t == 0) {
+        offsets[nb] = (int)carry;
+        *total = carry;
     }
 }
 
@@ -308,41 +323,53 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
     }
 }
 
-// Exact (float64) per-slot outputs from the original vertices: the definition written
-// out -- edge-function barycentrics, closed-triangle inside test, nearest-edge squared
-// distance, perspective renormalisation, interpolated z.
+// Per-slot outputs from the original vertices, the definition written out.  The
+// barycentrics and z are evaluated in float64 -- edge functions from exact float64
+// differences, times the float64 1/(2 area) kept as a float-float pair in a.w, b.w --
+// because extrapolated blur-ring faces reach |w| in the hundreds, where float32 cannot
+// hold them to 1e-5.  The squared distance only needs float32: the nearest-edge
+// distance in face-local differences is good to ~1e-10 in NDC^2.
 template <bool PERSP>
-__device__ void slot_outputs(const FaceGeom& g, double px, double py, float* z_out, float* b_out,
-                             float* d_out) {
-    double ax = g.a.x, ay = g.a.y, bx = g.b.x, by = g.b.y, cx = g.c.x, cy = g.c.y;
-    double area2 = (bx - ax) * (cy - ay) - (by - ay) * (cx - ax);
-    double w0 = ((bx - px) * (cy - py) - (by - py) * (cx - px)) / area2;
-    double w1 = ((cx - px) * (ay - py) - (cy - py) * (ax - px)) / area2;
-    double w2 = ((ax - px) * (by - py) - (ay - py) * (bx - px)) / area2;
-    bool inside = w0 >= 0.0 && w1 >= 0.0 && w2 >= 0.0;
-    double d2 = DBL_MAX;
-    const double ux[3] = {ax, bx, cx}, uy[3] = {ay, by, cy};
+__device__ __forceinline__ void slot_outputs(const FaceGeom& g, double pxd, double pyd, float pxh, float pxl,
+                                             float pyh, float pyl, float* z_out, float* b_out, float* d_out) {
+    const double inv_area2 = (double)g.a.w + (double)g.b.w;
+    const double rx0 = (double)g.a.x - pxd, ry0 = (double)g.a.y - pyd;
+    const double rx1 = (double)g.b.x - pxd, ry1 = (double)g.b.y - pyd;
+    const double rx2 = (double)g.c.x - pxd, ry2 = (double)g.c.y - pyd;
+    const double w0 = (rx1 * ry2 - ry1 * rx2) * inv_area2;
+    const double w1 = (rx2 * ry0 - ry2 * rx0) * inv_area2;
+    const double w2 = (rx0 * ry1 - ry0 * rx1) * inv_area2;
+    const bool inside = w0 >= 0.0 && w1 >= 0.0 && w2 >= 0.0;
+    const double z0 = g.a.z, z1 = g.b.z, z2 = g.c.z;
+    double b0 = w0, b1 = w1, b2 = w2, z;
+    if (PERSP) {
+        // u_k = w_k / z_k renormalised; multiplied through by z0 z1 z2 to keep one division
+        const double u0 = w0 * z1 * z2, u1 = w1 * z0 * z2, u2 = w2 * z0 * z1;
+        const double inv = 1.0 / (u0 + u1 + u2);
+        b0 = u0 * inv; b1 = u1 * inv; b2 = u2 * inv;
+        z = z0 * z1 * z2 * inv;
+    } else {
+        z = w0 * z0 + w1 * z1 + w2 * z2;
+    }
+    // squared distance to the nearest edge, float32, pixel - vertex differences
+    const float qx[3] = {(pxh - g.a.x) + pxl, (pxh - g.b.x) + pxl, (pxh - g.c.x) + pxl};
+    const float qy[3] = {(pyh - g.a.y) + pyl, (pyh - g.b.y) + pyl, (pyh - g.c.y) + pyl};
+    const float vx[3] = {g.a.x, g.b.x, g.c.x}, vy[3] = {g.a.y, g.b.y, g.c.y};
+    float d2 = FLT_MAX;
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
-        int k1 = k == 2 ? 0 : k + 1;
-        double ex = ux[k1] - ux[k], ey = uy[k1] - uy[k];
-        double len2 = ex * ex + ey * ey;
-        double t = len2 > 0.0 ? ((px - ux[k]) * ex + (py - uy[k]) * ey) / len2 : 0.0;
-        t = fmin(fmax(t, 0.0), 1.0);
-        double rx = px - (ux[k] + t * ex), ry = py - (uy[k] + t * ey);
-        d2 = fmin(d2, rx * rx + ry * ry);
+        const int k1 = k == 2 ? 0 : k + 1;
+        const float ex = vx[k1] - vx[k], ey = vy[k1] - vy[k];
+        const float len2 = fmaf(ex, ex, ey * ey);
+        const float t = len2 > 0.f ? __saturatef(fmaf(qx[k], ex, qy[k] * ey) * __frcp_rn(len2)) : 0.f;
+        const float rx = fmaf(-t, ex, qx[k]), ry = fmaf(-t, ey, qy[k]);
+        d2 = fminf(d2, fmaf(rx, rx, ry * ry));
     }
-    double b0 = w0, b1 = w1, b2 = w2;
-    if (PERSP) {
-        double u0 = w0 / (double)g.a.z, u1 = w1 / (double)g.b.z, u2 = w2 / (double)g.c.z;
-        double s = u0 + u1 + u2;
-        b0 = u0 / s; b1 = u1 / s; b2 = u2 / s;
-    }
-    *z_out = (float)(b0 * (double)g.a.z + b1 * (double)g.b.z + b2 * (double)g.c.z);
+    *z_out = (float)z;
     b_out[0] = (float)b0;
     b_out[1] = (float)b1;
     b_out[2] = (float)b2;
-    *d_out = (float)(inside ? -d2 : d2);
+    *d_out = inside ? -d2 : d2;
 }
 
 // One thread per pixel: the K winners' outputs (and the fused silhouette), written
@@ -358,6 +385,8 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int6
         const int i = (int)(rem / W), j = (int)(rem % W);
         const double pxd = -1.0 + (2.0 * j + 1.0) / W;
         const double pyd = 1.0 - (2.0 * i + 1.0) / H;
+        const float pxh = (float)pxd, pyh = (float)pyd;
+        const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
         float dsil[KC];
         bool vsil[KC];
         if (vec_ok && (KC % 4) == 0 && K == KC) {
@@ -370,7 +399,7 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int6
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     if (fk[u] >= 0) {
-                        slot_outputs<PERSP>(geom[fk[u]], pxd, pyd, &zz[u], &bb[3 * u], &dd[u]);
+                        slot_outputs<PERSP>(geom[fk[u]], pxd, pyd, pxh, pxl, pyh, pyl, &zz[u], &bb[3 * u], &dd[u]);
                     } else {
                         zz[u] = -1.f; dd[u] = -1.f; bb[3 * u] = bb[3 * u + 1] = bb[3 * u + 2] = -1.f;
                     }
@@ -396,7 +425,7 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int6
                 const int fk = topk[s];
                 float zz, bb[3], dd;
                 if (fk >= 0) {
-                    slot_outputs<PERSP>(geom[fk], pxd, pyd, &zz, bb, &dd);
+                    slot_outputs<PERSP>(geom[fk], pxd, pyd, pxh, pxl, pyh, pyl, &zz, bb, &dd);
                 } else {
                     zz = -1.f; dd = -1.f; bb[0] = bb[1] = bb[2] = -1.f;
                 }
