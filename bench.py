@@ -284,7 +284,7 @@ def main():
         dist.barrier()
     stages = mr.profile_read()
     dev_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    t = torch.tensor([dev_ms, float(samples), float(w.N * w.H * w.W)], dtype=torch.float64, device=dev)
+    t = torch.tensor([dev_ms, float(samples), float(batch.N * w.H * w.W)], dtype=torch.float64, device=dev)
     if world > 1:
         tmax = t.clone()
         dist.all_reduce(tmax[:1], op=dist.ReduceOp.MAX)
@@ -292,7 +292,7 @@ def main():
         dist.all_reduce(tsum[1:], op=dist.ReduceOp.SUM)
         dev_ms, tot_samples, tot_pix = float(tmax[0]), float(tsum[1]), float(tsum[2])
     else:
-        tot_samples, tot_pix = float(samples), float(w.N * w.H * w.W)
+        tot_samples, tot_pix = float(samples), float(batch.N * w.H * w.W)
     sec = dev_ms / 1e3
     value = tot_samples * args.steps / sec
     mpix = tot_pix * args.steps / sec / 1e6
@@ -352,7 +352,7 @@ def main():
     hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
     hbm_note = "of measured" if "hbm_gbs" in peaks else "of fallback"
     achieved_alu = samples * C_TEST / fine_s / 1e12
-    npix = w.N * w.H * w.W
+    npix = batch.N * w.H * w.W
     fine_bytes = npix * 4 * w.K                      # the K winning face ids per pixel
     epi_bytes = npix * (4 * w.K + 28 * w.K + 4)      # ids in; p2f, zbuf, bary, dists, alpha out
     roof = {"bound": "alu", "achieved": achieved_alu, "peak": peak_alu, "unit": "T FP32-inst/s",

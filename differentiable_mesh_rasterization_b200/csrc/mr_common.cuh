@@ -30,10 +30,13 @@ struct __align__(16) FaceGeom {
     float4 a, b, c;
 };
 
-// Inclusive pixel box of a face grown by sqrt(blur_radius), clipped to the image.
-// x0 > x1 marks a face that touches no pixel (off-screen or degenerate).
+// Inclusive pixel box of a face grown by sqrt(blur_radius), clipped to the image, and a
+// lower bound of the face's depth key over the pixel centres of that box.  x0 > x1 marks
+// a face that touches no pixel (off-screen or degenerate).
 struct __align__(16) FaceBox {
-    int x0, x1, y0, y1;
+    short x0, x1, y0, y1;
+    float kmin;
+    int unused;
 };
 
 void set_error(const char* fmt, ...);

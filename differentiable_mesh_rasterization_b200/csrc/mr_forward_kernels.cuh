@@ -24,13 +24,13 @@ namespace {
 // so every edge function is positive inside.  Per edge u -> v with unit direction e and
 // length L:
 //     c(d) = -e.y * d.x + e.x * d.y + ng   signed distance to the edge line (inside > 0)
-//     s(d) =  e.x * d.x + e.y * d.y + tg   position along the edge, measured from u
-//     squared distance to the segment = c^2 + max(-s, s - L, 0)^2.
+//     s(d) =  e.x * d.x + e.y * d.y + tg   position along the edge from its midpoint
+//     squared distance to the segment = c^2 + max(|s| - L/2, 0)^2.
 // The depth key is the plane through (x, y, z) -- or (x, y, -1/z) with perspective
 // correction, where 1/z is screen-affine -- written as k_hi + (gx dx + gy dy + k_lo);
 // the float-float constant keeps the key within half an ulp plus the plane terms.
-// Layout (6 float4): (ax, ay, gx, gy) (k_hi, k_lo, L0, L1) (e0.x, e0.y, ng0, tg0)
-//                    (e1.x, e1.y, ng1, tg1) (e2.x, e2.y, ng2, tg2) (L2, face id, 0, 0)
+// Layout (6 float4): (ax, ay, gx, gy) (k_hi, k_lo, L0/2, L1/2) (e0.x, e0.y, ng0, tg0)
+//                    (e1.x, e1.y, ng1, tg1) (e2.x, e2.y, ng2, tg2) (L2/2, face id, 0, 0)
 constexpr int kConstF4 = 6;
 
 __global__ void k_face_setup(const float* __restrict__ verts, int64_t V,
@@ -41,7 +41,7 @@ __global__ void k_face_setup(const float* __restrict__ verts, int64_t V,
     int64_t f = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (f >= F) return;
     int64_t i0 = faces[3 * f], i1 = faces[3 * f + 1], i2 = faces[3 * f + 2];
-    FaceBox bx = {1, 0, 1, 0};
+    FaceBox bx = {1, 0, 1, 0, 0.f, 0};
     float4* out = fconst + kConstF4 * f;
     const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
     if (i0 < 0 || i0 >= V || i1 < 0 || i1 >= V || i2 < 0 || i2 >= V) {
@@ -75,8 +75,7 @@ __global__ void k_face_setup(const float* __restrict__ verts, int64_t V,
     double ih = floor((1.0 - ymin) * 0.5 * H - 0.5 + 1e-4);
     jl = fmax(jl, 0.0); il = fmax(il, 0.0);
     jh = fmin(jh, (double)(W - 1)); ih = fmin(ih, (double)(H - 1));
-    if (jl <= jh && il <= ih) bx = FaceBox{(int)jl, (int)jh, (int)il, (int)ih};
-    box[f] = bx;
+    const bool on_screen = jl <= jh && il <= ih;
 
     double x[3] = {0.0, bxx - ax, cx - ax};
     double y[3] = {0.0, byy - ay, cy - ay};
@@ -91,6 +90,16 @@ __global__ void k_face_setup(const float* __restrict__ verts, int64_t V,
     const double gx = -nx / area2, gy = -ny / area2;
     const float khi = (float)q[0];
     const float klo = (float)(q[0] - (double)khi);
+    if (on_screen) {
+        // lowest key over the box's pixel centres (a plane: one corner), lowered by a
+        // margin well above the float32 evaluation error of the key
+        const double xl = -1.0 + (2.0 * jl + 1.0) / W - ax, xh = -1.0 + (2.0 * jh + 1.0) / W - ax;
+        const double yl = 1.0 - (2.0 * ih + 1.0) / H - ay, yh = 1.0 - (2.0 * il + 1.0) / H - ay;
+        const double tx = fmin(gx * xl, gx * xh), ty = fmin(gy * yl, gy * yh);
+        const double span = fabs(q[0]) + fmax(fabs(gx * xl), fabs(gx * xh)) + fmax(fabs(gy * yl), fabs(gy * yh));
+        bx = FaceBox{(short)jl, (short)jh, (short)il, (short)ih, __double2float_rd(q[0] + tx + ty - 1e-6 * span), 0};
+    }
+    box[f] = bx;
     if (area2 < 0.0) {
         double t = x[1]; x[1] = x[2]; x[2] = t;
         t = y[1]; y[1] = y[2]; y[2] = t;
@@ -105,8 +114,8 @@ __global__ void k_face_setup(const float* __restrict__ verts, int64_t V,
         e[k][0] = (float)ux;
         e[k][1] = (float)uy;
         e[k][2] = (float)(uy * x[k] - ux * y[k]);
-        e[k][3] = (float)(-(ux * x[k] + uy * y[k]));
-        e[k][4] = (float)L;
+        e[k][3] = (float)(-(ux * x[k] + uy * y[k]) - 0.5 * L);
+        e[k][4] = (float)(0.5 * L);
     }
     out[0] = make_float4(a.x, a.y, (float)gx, (float)gy);
     out[1] = make_float4(khi, klo, e[0][4], e[1][4]);
@@ -139,7 +148,7 @@ __global__ void k_bin_pairs(const FaceBox* __restrict__ box, const int64_t* __re
         bool live = q < pairs;
         int n = 0;
         int64_t f = 0;
-        FaceBox b = {1, 0, 1, 0};
+        FaceBox b = {1, 0, 1, 0, 0.f, 0};
         if (live) {
             n = pair_image(prefix, N, q);
             f = first[n] + (q - prefix[n]);
@@ -233,7 +242,7 @@ __device__ __forceinline__ void topk_insert(float (&kk)[KC], int (&ff)[KC], floa
 // every lane runs the full candidacy test.  EXACT: the pixel centres are exact float32
 // values (H and W powers of two), so the float-float low parts vanish.
 template <int KC, bool PERSP, bool EXACT>
-__global__ void __launch_bounds__(kFineThreads)
+__global__ void __launch_bounds__(kFineThreads, KC <= 4 ? 6 : 4)
 k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const int* __restrict__ offsets,
        const int* __restrict__ list, int nbx, int nby, int H, int W, int K, float blur, int* __restrict__ topk) {
     __shared__ float4 s_c[kWarpsPerBin][32][kConstF4];
@@ -258,19 +267,32 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
     int ff[KC];
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
-        kk[k] = in_img ? FLT_MAX : -FLT_MAX;                 // off-image lanes admit nothing
+        kk[k] = in_img ? FLT_MAX : (PERSP ? -FLT_MAX : 0.f);   // off-image lanes are never written
         ff[k] = INT_MAX;
     }
 
     const int beg = offsets[bin], cnt = offsets[bin + 1] - beg;
     float4(*slots)[kConstF4] = s_c[warp];
+    // the next batch's face id and box are loaded while the current batch is tested
+    int nfid = 0;
+    FaceBox nbox = {1, 0, 1, 0, 0.f, 0};
+    if (lane < cnt) {
+        nfid = list[beg + lane];
+        nbox = box[nfid];
+    }
     for (int base = 0; base < cnt; base += 32) {
-        bool hit = false;
-        int fid = 0;
-        if (base + lane < cnt) {
-            fid = list[beg + base + lane];
-            const FaceBox b = box[fid];
-            hit = b.x0 <= tj0 + kWarpTileW - 1 && b.x1 >= tj0 && b.y0 <= ti0 + kWarpTileH - 1 && b.y1 >= ti0;
+        const int fid = nfid;
+        const FaceBox b = nbox;
+        // tile depth cull: the farthest K-th key over the warp's pixels; a face whose lowest
+        // key over its box lies beyond it cannot enter any lane's top K
+        float zfar = in_img ? kk[KC - 1] : -FLT_MAX;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) zfar = fmaxf(zfar, __shfl_xor_sync(0xffffffffu, zfar, o));
+        const bool hit = base + lane < cnt && b.x0 <= tj0 + kWarpTileW - 1 && b.x1 >= tj0 &&
+                         b.y0 <= ti0 + kWarpTileH - 1 && b.y1 >= ti0 && b.kmin <= zfar;
+        if (base + 32 + lane < cnt) {
+            nfid = list[beg + base + 32 + lane];
+            nbox = box[nfid];
         }
         const unsigned m = __ballot_sync(0xffffffffu, hit);
         if (hit) {
@@ -286,8 +308,11 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
             float dx = pxh - q0.x, dy = pyh - q0.y;
             if (!EXACT) { dx += pxl; dy += pyl; }
             const float key = q1.x + fmaf(q0.z, dx, fmaf(q0.w, dy, q1.y));
-            const bool front = PERSP ? key < 0.f : key >= 0.f;
-            const bool maybe = front && key <= kk[KC - 1];
+            // admissible: in front of the camera and not behind the lane's K-th key.  Without
+            // perspective the keys are depths >= 0, whose float order is their bit order,
+            // so one unsigned compare does both (negative keys wrap to huge values).
+            const bool maybe = PERSP ? (key < 0.f && key <= kk[KC - 1])
+                                     : (__float_as_uint(key) <= __float_as_uint(kk[KC - 1]));
             if (!__any_sync(0xffffffffu, maybe)) continue;
             const float4 e0 = slots[qi][2], e1 = slots[qi][3], e2 = slots[qi][4], q5 = slots[qi][5];
             const float c0 = fmaf(-e0.y, dx, fmaf(e0.x, dy, e0.z));
@@ -296,9 +321,9 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
             const float s1 = fmaf(e1.x, dx, fmaf(e1.y, dy, e1.w));
             const float c2 = fmaf(-e2.y, dx, fmaf(e2.x, dy, e2.z));
             const float s2 = fmaf(e2.x, dx, fmaf(e2.y, dy, e2.w));
-            const float o0 = fmaxf(fmaxf(-s0, s0 - q1.z), 0.f);
-            const float o1 = fmaxf(fmaxf(-s1, s1 - q1.w), 0.f);
-            const float o2 = fmaxf(fmaxf(-s2, s2 - q5.x), 0.f);
+            const float o0 = fmaxf(fabsf(s0) - q1.z, 0.f);
+            const float o1 = fmaxf(fabsf(s1) - q1.w, 0.f);
+            const float o2 = fmaxf(fabsf(s2) - q5.x, 0.f);
             const float d0 = fmaf(o0, o0, c0 * c0);
             const float d1 = fmaf(o1, o1, c1 * c1);
             const float d2 = fmaf(o2, o2, c2 * c2);
@@ -375,7 +400,7 @@ __device__ __forceinline__ void slot_outputs(const FaceGeom& g, double pxd, doub
 // One thread per pixel: the K winners' outputs (and the fused silhouette), written
 // contiguously per pixel with 16-byte stores when K is a multiple of 4.
 template <int KC, bool PERSP, bool SIL>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int64_t npix, int H, int W, int K,
            float sigma, bool vec_ok, int64_t* __restrict__ p2f, float* __restrict__ zbuf, float* __restrict__ bary,
            float* __restrict__ dists, float* __restrict__ alpha) {

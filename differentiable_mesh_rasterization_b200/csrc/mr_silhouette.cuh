@@ -29,9 +29,13 @@ __device__ __forceinline__ void silhouette_grad(const float (&d)[KC], const bool
     float q[KC], p[KC];
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
+        // one exponential per slot: with e = exp(-|x|) and r = 1 / (1 + e) the two
+        // sigmoids are r and e * r, assigned by the sign of x (no overflow either way)
         const float x = d[k] / sigma;
-        q[k] = 1.f / (1.f + expf(-x));   // 1 - p_k
-        p[k] = 1.f / (1.f + expf(x));
+        const float e = expf(-fabsf(x));
+        const float r = 1.f / (1.f + e);
+        q[k] = x >= 0.f ? r : e * r;    // 1 - p_k
+        p[k] = x >= 0.f ? e * r : r;
     }
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
