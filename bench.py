@@ -207,6 +207,26 @@ def workload_config(w, args):
             "parallelism": f"independent batch per GPU x{args.gpus}"}
 
 
+# ----------------------------------------------------------------------------- ranks
+def rank_seed(config: int, rank: int) -> int:
+    """Weak scaling: every rank renders its own batch of the same workload."""
+    return 1000 + config + 1000 * rank
+
+
+def combine_ranks(dev_ms: float, samples: float, pixels: float, device=None):
+    """(max over ranks of the device time, sum of samples, sum of pixels)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([dev_ms, samples, pixels], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        tmax = t[:1].clone()
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+        tsum = t[1:].clone()
+        dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
+        return float(tmax[0]), float(tsum[0]), float(tsum[1])
+    return float(t[0]), float(t[1]), float(t[2])
+
+
 # ----------------------------------------------------------------------------- our arm
 def main():
     ap = argparse.ArgumentParser()
@@ -239,7 +259,7 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    batch = syn.make_batch(args.config, seed=1000 + args.config + 1000 * rank, n_meshes=args.images)
+    batch = syn.make_batch(args.config, seed=rank_seed(args.config, rank), n_meshes=args.images)
     w = batch.workload
     if w.sigma is None:
         raise SystemExit("the benchmark step needs a soft-silhouette workload (sigma)")
@@ -284,15 +304,7 @@ def main():
         dist.barrier()
     stages = mr.profile_read()
     dev_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    t = torch.tensor([dev_ms, float(samples), float(batch.N * w.H * w.W)], dtype=torch.float64, device=dev)
-    if world > 1:
-        tmax = t.clone()
-        dist.all_reduce(tmax[:1], op=dist.ReduceOp.MAX)
-        tsum = t.clone()
-        dist.all_reduce(tsum[1:], op=dist.ReduceOp.SUM)
-        dev_ms, tot_samples, tot_pix = float(tmax[0]), float(tsum[1]), float(tsum[2])
-    else:
-        tot_samples, tot_pix = float(samples), float(batch.N * w.H * w.W)
+    dev_ms, tot_samples, tot_pix = combine_ranks(dev_ms, float(samples), float(batch.N * w.H * w.W), dev)
     sec = dev_ms / 1e3
     value = tot_samples * args.steps / sec
     mpix = tot_pix * args.steps / sec / 1e6
