@@ -145,17 +145,9 @@ __global__ void k_raster_bwd(const float* __restrict__ verts, int64_t V, const i
     }
 }
 
-// (x, y) contribution of one slot to one vertex: a single float2 atomic.  (Summing equal
-// vertex ids across the warp first with match/shuffle was measured 1.6x slower on B200:
-// the shuffle traffic costs more than the atomics it saves.)
-__device__ __forceinline__ void scatter_xy(float2* __restrict__ acc, bool act, int vid, float2 c) {
-    if (act) atomicAdd(acc + vid, c);
-}
-
 // Fused silhouette backward + distance backward: one thread per pixel (32 consecutive
 // pixels per warp), float32.  Per slot the nearest edge u -> v is recomputed and its two
-// end points receive -2 (p - q)(1 - t) and -2 (p - q) t times dL/ddist; contributions to
-// each end point receives one float2 atomic.
+// end points receive -2 (p - q)(1 - t) and -2 (p - q) t times dL/ddist.
 template <int KC>
 __global__ void __launch_bounds__(256)
 k_sil_raster_bwd(const float* __restrict__ verts, int64_t V, const int64_t* __restrict__ faces, int64_t F,
@@ -186,11 +178,18 @@ k_sil_raster_bwd(const float* __restrict__ verts, int64_t V, const int64_t* __re
         const double pxd = -1.0 + (2.0 * j + 1.0) / W, pyd = 1.0 - (2.0 * i + 1.0) / H;
         const float pxh = (float)pxd, pyh = (float)pyd;
         const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
+        // per slot: the nearest edge's two end points and their (x, y) contributions
+        constexpr int NT = KC <= 8 ? 2 * KC : 2;
+        int tid[NT];
+        float2 tv[NT];
+        bool alive[NT];
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
             bool act = k < K && v[k] && g[k] != 0.f;
-            int vu = 0, vv = 0;
-            float2 cu = make_float2(0.f, 0.f), cv = make_float2(0.f, 0.f);
+            if constexpr (KC <= 8) {
+                tid[2 * k] = tid[2 * k + 1] = -1;
+                tv[2 * k] = tv[2 * k + 1] = make_float2(0.f, 0.f);
+            }
             if (act) {
                 int64_t vid[3];
                 if (fk[k] >= F) {
@@ -222,15 +221,36 @@ k_sil_raster_bwd(const float* __restrict__ verts, int64_t V, const int64_t* __re
                     const int ev = eu == 2 ? 0 : eu + 1;
                     const float gdist = d[k] < 0.f ? -g[k] : g[k];
                     const float su = -2.f * gdist * (1.f - bt), sv = -2.f * gdist * bt;
-                    cu = make_float2(su * brx, su * bry);
-                    cv = make_float2(sv * brx, sv * bry);
-                    vu = (int)vid[eu];
-                    vv = (int)vid[ev];
+                    if constexpr (KC <= 8) {
+                        tv[2 * k] = make_float2(su * brx, su * bry);
+                        tv[2 * k + 1] = make_float2(sv * brx, sv * bry);
+                        tid[2 * k] = (int)vid[eu];
+                        tid[2 * k + 1] = (int)vid[ev];
+                    } else {
+                        atomicAdd(acc + vid[eu], make_float2(su * brx, su * bry));
+                        atomicAdd(acc + vid[ev], make_float2(sv * brx, sv * bry));
+                        act = false;
+                    }
                 }
             }
-            scatter_xy(acc, act, vu, cu);
-            scatter_xy(acc, act, vv, cv);
+            if constexpr (KC <= 8) alive[2 * k] = alive[2 * k + 1] = act;
         }
+        // The K faces of a pixel are neighbours and often share the nearest edge's end
+        // points: sum equal vertex ids of this pixel first (the two ends of one slot
+        // always differ), then one float2 atomic per distinct vertex (up to K = 8; larger K
+        // would spend more registers on the comparisons than the atomics cost).
+#pragma unroll
+        for (int t = 2; t < (KC <= 8 ? NT : 0); ++t)
+#pragma unroll
+            for (int u = 0; u < (t & ~1); ++u)
+                if (alive[u] && alive[t] && tid[u] == tid[t]) {
+                    tv[u].x += tv[t].x;
+                    tv[u].y += tv[t].y;
+                    alive[t] = false;
+                }
+#pragma unroll
+        for (int t = 0; t < (KC <= 8 ? NT : 0); ++t)
+            if (alive[t]) atomicAdd(acc + tid[t], tv[t]);
     }
 }
 
