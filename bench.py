@@ -349,10 +349,11 @@ def main():
 
     # roofline of the dominant kernel (the fine pass: the pixel-face tests) and of the
     # epilogue (which writes the per-slot outputs)
+    # per step: the fine pass and the epilogue run as several chunk launches each
     fine_ms, fine_n = stages["fine"]
-    fine_s = fine_ms / 1e3 / max(fine_n, 1)
+    fine_s = fine_ms / 1e3 / args.steps
     epi_ms, epi_n = stages["epilogue"]
-    epi_s = epi_ms / 1e3 / max(epi_n, 1)
+    epi_s = epi_ms / 1e3 / args.steps
     clk = clocks.summary()
     peaks = {}
     try:
@@ -370,12 +371,13 @@ def main():
     roof = {"bound": "alu", "achieved": achieved_alu, "peak": peak_alu, "unit": "T FP32-inst/s",
             "frac": achieved_alu / peak_alu, "traffic": None,
             "kernel": "k_fine (stage-one fine pass: pixel-face tests and register top-K)",
-            "ms_per_launch": fine_s * 1e3, "samples_per_launch": samples, "c_test": C_TEST,
+            "ms_per_step": fine_s * 1e3, "launches_per_step": fine_n // args.steps,
+            "samples_per_step": samples, "c_test": C_TEST,
             "peak_note": f"{props.multi_processor_count} SMs x 128 FP32 lanes x {sm_mhz_max:.0f} MHz "
                          f"(unit counts and max clock)",
-            "hbm_bytes_per_launch": fine_bytes,
+            "hbm_bytes_per_step": fine_bytes,
             "epilogue": {"kernel": "k_epilogue (float64 outputs of the K winners + silhouette)",
-                         "bound": "hbm", "ms_per_launch": epi_s * 1e3, "bytes_per_launch": epi_bytes,
+                         "bound": "hbm", "ms_per_step": epi_s * 1e3, "bytes_per_step": epi_bytes,
                          "achieved": epi_bytes / epi_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
                          "frac": epi_bytes / epi_s / 1e9 / hbm_peak, "peak_note": hbm_note}}
 

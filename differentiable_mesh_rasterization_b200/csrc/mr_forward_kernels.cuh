@@ -5,6 +5,7 @@
 // compiles its own copy.  The pipeline is described in mr_forward.cu.
 #pragma once
 
+#include <algorithm>
 #include <cfloat>
 #include <climits>
 #include <cmath>
@@ -33,13 +34,11 @@ namespace {
 //                    (e1.x, e1.y, ng1, tg1) (e2.x, e2.y, ng2, tg2) (L2/2, face id, 0, 0)
 constexpr int kConstF4 = 6;
 
-__global__ void k_face_setup(const float* __restrict__ verts, int64_t V,
-                             const int64_t* __restrict__ faces, int64_t F, int H, int W,
-                             double reach, int persp, FaceGeom* __restrict__ geom,
-                             FaceBox* __restrict__ box, float4* __restrict__ fconst,
-                             int* __restrict__ err) {
-    int64_t f = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (f >= F) return;
+__device__ __forceinline__ void setup_face(const float* __restrict__ verts, int64_t V,
+                                           const int64_t* __restrict__ faces, int64_t f, int H, int W,
+                                           double reach, int persp, FaceGeom* __restrict__ geom,
+                                           FaceBox* __restrict__ box, float4* __restrict__ fconst,
+                                           int* __restrict__ err, float& qlo, float& qhi) {
     int64_t i0 = faces[3 * f], i1 = faces[3 * f + 1], i2 = faces[3 * f + 2];
     FaceBox bx = {1, 0, 1, 0, 0.f, 0};
     float4* out = fconst + kConstF4 * f;
@@ -98,6 +97,8 @@ __global__ void k_face_setup(const float* __restrict__ verts, int64_t V,
         const double tx = fmin(gx * xl, gx * xh), ty = fmin(gy * yl, gy * yh);
         const double span = fabs(q[0]) + fmax(fabs(gx * xl), fabs(gx * xh)) + fmax(fabs(gy * yl), fabs(gy * yh));
         bx = FaceBox{(short)jl, (short)jh, (short)il, (short)ih, __double2float_rd(q[0] + tx + ty - 1e-6 * span), 0};
+        qlo = (float)fmin(q[0], fmin(q[1], q[2]));
+        qhi = (float)fmax(q[0], fmax(q[1], q[2]));
     }
     box[f] = bx;
     if (area2 < 0.0) {
@@ -125,7 +126,15 @@ __global__ void k_face_setup(const float* __restrict__ verts, int64_t V,
     out[5] = make_float4(e[2][4], __int_as_float((int)f), 0.f, 0.f);
 }
 
-// ------------------------------------------------------------------ binning
+// Ordered unsigned image of a float (monotone), for atomic min / max of depth keys.
+__device__ __forceinline__ unsigned float_order(float f) {
+    const unsigned u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float order_float(unsigned u) {
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
 // (image, face) pairs are enumerated image by image: pair q belongs to image n with
 // pair_prefix[n] <= q < pair_prefix[n+1] and is face first[n] + q - pair_prefix[n].
 __device__ __forceinline__ int pair_image(const int64_t* prefix, int N, int64_t q) {
@@ -137,84 +146,170 @@ __device__ __forceinline__ int pair_image(const int64_t* prefix, int N, int64_t 
     return lo;
 }
 
+// Face setup over the (image, face) pairs (a face shared by several images is set up
+// once per image, with identical results), and each image's range of vertex depth keys
+// (ordered-unsigned minima in krange[0, N), maxima in krange[N, 2N); one atomic pair per
+// warp when the warp sits in one image).
+__global__ void k_face_setup(const float* __restrict__ verts, int64_t V, const int64_t* __restrict__ faces,
+                             const int64_t* __restrict__ prefix, const int64_t* __restrict__ first, int N,
+                             int64_t pairs, int H, int W, double reach, int persp, FaceGeom* __restrict__ geom,
+                             FaceBox* __restrict__ box, float4* __restrict__ fconst, unsigned* __restrict__ krange,
+                             int* __restrict__ err) {
+    for (int64_t q0 = (int64_t)blockIdx.x * blockDim.x; q0 < pairs; q0 += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t q = q0 + threadIdx.x;
+        const bool live = q < pairs;
+        int n = 0;
+        float qlo = FLT_MAX, qhi = -FLT_MAX;
+        if (live) {
+            n = pair_image(prefix, N, q);
+            setup_face(verts, V, faces, first[n] + (q - prefix[n]), H, W, reach, persp, geom, box, fconst, err, qlo,
+                       qhi);
+        }
+        const int n0 = __shfl_sync(0xffffffffu, n, 0);
+        if (__all_sync(0xffffffffu, !live || n == n0)) {
+            for (int o = 16; o > 0; o >>= 1) {
+                qlo = fminf(qlo, __shfl_xor_sync(0xffffffffu, qlo, o));
+                qhi = fmaxf(qhi, __shfl_xor_sync(0xffffffffu, qhi, o));
+            }
+            if ((threadIdx.x & 31) == 0 && qlo <= qhi) {
+                atomicMin(&krange[n0], float_order(qlo));
+                atomicMax(&krange[N + n0], float_order(qhi));
+            }
+        } else if (live && qlo <= qhi) {
+            atomicMin(&krange[n], float_order(qlo));
+            atomicMax(&krange[N + n], float_order(qhi));
+        }
+    }
+}
+
+// ------------------------------------------------------------------ binning
+// Each bin's face list is split into kDepthBuckets sub-lists by the face's key lower
+// bound, relative to its image's range of vertex keys, nearest bucket first.  The fine
+// pass then meets near faces first, so its depth culls reject more of the rest.
+constexpr int kDepthBuckets = 8;
+
+__device__ __forceinline__ int depth_bucket(float kmin, float lo, float hi) {
+    if (!(hi > lo)) return 0;
+    const float t = (kmin - lo) / (hi - lo) * (float)kDepthBuckets;
+    return t <= 0.f ? 0 : (t >= (float)(kDepthBuckets - 1) ? kDepthBuckets - 1 : (int)t);
+}
+
 template <bool FILL>
 __global__ void k_bin_pairs(const FaceBox* __restrict__ box, const int64_t* __restrict__ prefix,
                             const int64_t* __restrict__ first, int N, int64_t pairs, int nbx, int nby,
-                            int* __restrict__ counts, const int* __restrict__ offsets,
-                            int* __restrict__ list) {
+                            const unsigned* __restrict__ krange, int* __restrict__ counts,
+                            const int* __restrict__ offsets, int* __restrict__ list) {
     const unsigned lane = threadIdx.x & 31;
     for (int64_t q0 = (int64_t)blockIdx.x * blockDim.x; q0 < pairs; q0 += (int64_t)gridDim.x * blockDim.x) {
         int64_t q = q0 + threadIdx.x;
         bool live = q < pairs;
-        int n = 0;
+        int n = 0, bucket = 0;
         int64_t f = 0;
         FaceBox b = {1, 0, 1, 0, 0.f, 0};
         if (live) {
             n = pair_image(prefix, N, q);
             f = first[n] + (q - prefix[n]);
             b = box[f];
+            bucket = depth_bucket(b.kmin, order_float(krange[n]), order_float(krange[N + n]));
         }
         int bx0 = 0, bx1 = -1, by0 = 0, by1 = -1;
         if (live && b.x0 <= b.x1) {
             bx0 = b.x0 / kBin; bx1 = b.x1 / kBin; by0 = b.y0 / kBin; by1 = b.y1 / kBin;
         }
         // Walk the touched bins in lock-step across the warp; neighbouring faces share
-        // bins, so one atomic per distinct bin per step is issued.
+        // (bin, bucket) slots, so one atomic per distinct slot per step is issued.
         int nx = bx1 - bx0 + 1, ny = by1 - by0 + 1;
         int mine = (nx > 0 && ny > 0) ? nx * ny : 0;
         int most = mine;
         for (int o = 16; o > 0; o >>= 1) most = max(most, __shfl_xor_sync(0xffffffffu, most, o));
         for (int s = 0; s < most; ++s) {
             bool act = s < mine;
-            int bin = -1;
-            if (act) bin = (n * nby + by0 + s / nx) * nbx + bx0 + s % nx;
-            unsigned peers = __match_any_sync(0xffffffffu, bin);
+            int slot = -1;
+            if (act) slot = ((n * nby + by0 + s / nx) * nbx + bx0 + s % nx) * kDepthBuckets + bucket;
+            unsigned peers = __match_any_sync(0xffffffffu, slot);
             if (!act) continue;
             int leader = __ffs(peers) - 1;
             int rank = __popc(peers & ((1u << lane) - 1));
             int base = 0;
-            if ((int)lane == leader) base = atomicAdd(&counts[bin], __popc(peers));
+            if ((int)lane == leader) base = atomicAdd(&counts[slot], __popc(peers));
             base = __shfl_sync(peers, base, leader);
-            if (FILL) list[offsets[bin] + base + rank] = (int)f;
+            if (FILL) list[offsets[slot] + base + rank] = (int)f;
         }
     }
 }
 
-// Exclusive scan of nb counts by one 1024-thread CTA, 1024 consecutive counts per round
-// (coalesced), warp shuffles within a round and a running carry; offsets[nb] = total.
-__global__ void __launch_bounds__(1024) k_scan(const int* __restrict__ counts, int nb, int* __restrict__ offsets,
-                                               long long* __restrict__ total) {
-    __shared__ long long wsum[32];
-    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-    long long carry = 0;
-    for (int base = 0; base < nb; base += 1024) {
-        const int i = base + t;
-        const long long v = i < nb ? counts[i] : 0;
-        long long x = v;
+// Exclusive scan of nb counts in three launches: 4096-entry tiles scanned by 1024-thread
+// CTAs (coalesced, warp shuffles), the tile totals scanned by one CTA, then the tile
+// prefixes added; offsets[nb] = total.
+constexpr int kScanTile = 4096;
+
+__device__ __forceinline__ long long block_exclusive_scan(long long x, long long* wsum, long long& total) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    long long inc = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) wsum[w] = inc;
+    __syncthreads();
+    if (w == 0) {
+        long long y = lane < (int)(blockDim.x >> 5) ? wsum[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const long long y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
+            const long long z = __shfl_up_sync(0xffffffffu, y, o);
+            if (lane >= o) y += z;
         }
-        if (lane == 31) wsum[w] = x;
-        __syncthreads();
-        if (w == 0) {
-            long long y = wsum[lane];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const long long z = __shfl_up_sync(0xffffffffu, y, o);
-                if (lane >= o) y += z;
-            }
-            wsum[lane] = y;
-        }
-        __syncthreads();
-        if (i < nb) offsets[i] = (int)(carry + (w ? wsum[w - 1] : 0) + x - v);
-        carry += wsum[31];
-        __syncthreads();
+        wsum[lane] = y;
     }
-    if (t == 0) {
-        offsets[nb] = (int)carry;
-        *total = carry;
+    __syncthreads();
+    total = wsum[(blockDim.x >> 5) - 1];
+    const long long ex = (w ? wsum[w - 1] : 0) + inc - x;
+    __syncthreads();
+    return ex;
+}
+
+__global__ void __launch_bounds__(1024) k_scan_tiles(const int* __restrict__ counts, int nb, int* __restrict__ offsets,
+                                                     long long* __restrict__ tile_sum) {
+    __shared__ long long wsum[32];
+    const int base = blockIdx.x * kScanTile + threadIdx.x * 4;
+    int v[4];
+    long long sum = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        v[u] = base + u < nb ? counts[base + u] : 0;
+        sum += v[u];
+    }
+    long long total;
+    long long run = block_exclusive_scan(sum, wsum, total);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        if (base + u < nb) offsets[base + u] = (int)run;
+        run += v[u];
+    }
+    if (threadIdx.x == 0) tile_sum[blockIdx.x] = total;
+}
+
+__global__ void __launch_bounds__(1024) k_scan_tops(long long* __restrict__ tile_sum, int ntiles,
+                                                    long long* __restrict__ total_out) {
+    __shared__ long long wsum[32];
+    long long carry = 0;
+    for (int base = 0; base < ntiles; base += 1024) {
+        const int i = base + threadIdx.x;
+        const long long x = i < ntiles ? tile_sum[i] : 0;
+        long long total;
+        const long long ex = block_exclusive_scan(x, wsum, total);
+        if (i < ntiles) tile_sum[i] = carry + ex;
+        carry += total;
+    }
+    if (threadIdx.x == 0) *total_out = carry;
+}
+
+__global__ void k_scan_add(int* __restrict__ offsets, int nb, const long long* __restrict__ tile_pre,
+                           const long long* __restrict__ total) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= nb; i += gridDim.x * blockDim.x) {
+        if (i == nb) offsets[nb] = (int)*total;
+        else offsets[i] += (int)tile_pre[i / kScanTile];
     }
 }
 
@@ -271,7 +366,7 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
         ff[k] = INT_MAX;
     }
 
-    const int beg = offsets[bin], cnt = offsets[bin + 1] - beg;
+    const int beg = offsets[bin * kDepthBuckets], cnt = offsets[(bin + 1) * kDepthBuckets] - beg;
     float4(*slots)[kConstF4] = s_c[warp];
     // the next batch's face id and box are loaded while the current batch is tested
     int nfid = 0;
@@ -561,27 +656,150 @@ int validate_fwd(const float* verts, int64_t V, const int64_t* faces, int64_t F,
     return MR_OK;
 }
 
-// Bytes of the fixed scratch block of one forward call (everything but the bin lists),
-// and the offsets of its parts.
-struct FwdScratch {
-    size_t geom, box, con, top, cnt, off, pre, fst, tot, err, bytes;
+// ------------------------------------------------------------------ host pipeline
+// Sizes of one forward call and the layout of its fixed scratch block (everything but
+// the bin lists, which are sized after the count pass).
+struct FwdPlan {
+    int64_t V, F, pairs, npix;
+    int N, H, W, K, KC, persp, nbx, nby, nbins, nslots, ntiles;
+    float blur;
+    size_t geom, box, con, top, cnt, off, tsum, rng, pre, fst, tot, err, bytes;
 };
 
-inline FwdScratch fwd_scratch_layout(int64_t F, int64_t npix, int K, int nbins, int N) {
+inline int fwd_plan(int64_t V, int64_t F, const int64_t* num, int N, int H, int W, float blur, int K, int persp,
+                    FwdPlan& P) {
+    P.V = V; P.F = F; P.N = N; P.H = H; P.W = W; P.K = K; P.persp = persp; P.blur = blur;
+    P.KC = K <= 1 ? 1 : K <= 2 ? 2 : K <= 4 ? 4 : K <= 8 ? 8 : K <= 16 ? 16 : 32;
+    P.nbx = ceil_div(W, kBin);
+    P.nby = ceil_div(H, kBin);
+    const long long nbins = (long long)N * P.nbx * P.nby;
+    if (nbins * kDepthBuckets >= INT32_MAX / 2) {
+        set_error("too many screen bins (%lld)", nbins);
+        return MR_ERR_ARG;
+    }
+    P.nbins = (int)nbins;
+    P.nslots = P.nbins * kDepthBuckets;
+    P.ntiles = ceil_div(P.nslots, kScanTile);
+    P.npix = (int64_t)N * H * W;
+    P.pairs = 0;
+    for (int n = 0; n < N; ++n) P.pairs += num[n];
     auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
-    FwdScratch L;
-    L.geom = 0;
-    L.box = L.geom + up(sizeof(FaceGeom) * (size_t)F);
-    L.con = L.box + up(sizeof(FaceBox) * (size_t)F);
-    L.top = L.con + up(sizeof(float4) * kConstF4 * (size_t)F);
-    L.cnt = L.top + up(sizeof(int) * (size_t)npix * (size_t)K);
-    L.off = L.cnt + up(sizeof(int) * (size_t)nbins);
-    L.pre = L.off + up(sizeof(int) * (size_t)(nbins + 1));
-    L.fst = L.pre + up(sizeof(int64_t) * (size_t)(N + 1));
-    L.tot = L.fst + up(sizeof(int64_t) * (size_t)N);
-    L.err = L.tot + 256;
-    L.bytes = L.err + 256;
-    return L;
+    P.geom = 0;
+    P.box = P.geom + up(sizeof(FaceGeom) * (size_t)F);
+    P.con = P.box + up(sizeof(FaceBox) * (size_t)F);
+    P.top = P.con + up(sizeof(float4) * kConstF4 * (size_t)F);
+    P.cnt = P.top + up(sizeof(int) * (size_t)P.npix * (size_t)K);
+    P.off = P.cnt + up(sizeof(int) * (size_t)P.nslots);
+    P.tsum = P.off + up(sizeof(int) * (size_t)(P.nslots + 1));
+    P.rng = P.tsum + up(sizeof(long long) * (size_t)P.ntiles);
+    P.pre = P.rng + up(sizeof(unsigned) * 2 * (size_t)N);
+    P.fst = P.pre + up(sizeof(int64_t) * (size_t)(N + 1));
+    P.tot = P.fst + up(sizeof(int64_t) * (size_t)N);
+    P.err = P.tot + 256;
+    P.bytes = P.err + 256;
+    return MR_OK;
+}
+
+// Pointers into one scratch block laid out by fwd_plan.
+struct FwdBufs {
+    FaceGeom* geom;
+    FaceBox* box;
+    float4* fconst;
+    int *topk, *counts, *offsets;
+    long long* tile_sum;
+    unsigned* krange;
+    int64_t *prefix, *first;
+    long long* total;
+    int* err;
+};
+
+inline FwdBufs fwd_bufs(char* ws, const FwdPlan& P) {
+    FwdBufs B;
+    B.geom = reinterpret_cast<FaceGeom*>(ws + P.geom);
+    B.box = reinterpret_cast<FaceBox*>(ws + P.box);
+    B.fconst = reinterpret_cast<float4*>(ws + P.con);
+    B.topk = reinterpret_cast<int*>(ws + P.top);
+    B.counts = reinterpret_cast<int*>(ws + P.cnt);
+    B.offsets = reinterpret_cast<int*>(ws + P.off);
+    B.tile_sum = reinterpret_cast<long long*>(ws + P.tsum);
+    B.krange = reinterpret_cast<unsigned*>(ws + P.rng);
+    B.prefix = reinterpret_cast<int64_t*>(ws + P.pre);
+    B.first = reinterpret_cast<int64_t*>(ws + P.fst);
+    B.total = reinterpret_cast<long long*>(ws + P.tot);
+    B.err = reinterpret_cast<int*>(ws + P.err);
+    return B;
+}
+
+inline int pair_blocks(int64_t pairs) { return (int)std::min<int64_t>((pairs + 255) / 256, 148 * 16); }
+
+// Up to the bin counts: per-mesh arrays to the device, clears, face setup (with the
+// images' key ranges), bin count and scan, and the read-back of the list total and the
+// error word into host_total / host_err (valid after the stream is synchronised).
+inline cudaError_t fwd_enqueue_count(const FwdPlan& P, const FwdBufs& B, const float* verts, const int64_t* faces,
+                                     const int64_t* host_prefix, const int64_t* host_first, cudaStream_t s,
+                                     long long* host_total, int* host_err) {
+    cudaError_t e;
+    if ((e = cudaMemcpyAsync(B.prefix, host_prefix, sizeof(int64_t) * (P.N + 1), cudaMemcpyHostToDevice, s))) return e;
+    if ((e = cudaMemcpyAsync(B.first, host_first, sizeof(int64_t) * P.N, cudaMemcpyHostToDevice, s))) return e;
+    if ((e = cudaMemsetAsync(B.counts, 0, sizeof(int) * (size_t)P.nslots, s))) return e;
+    if ((e = cudaMemsetAsync(B.err, 0, sizeof(int), s))) return e;
+    // key ranges, ordered-unsigned: N minima starting at 0xffffffff, then N maxima at 0
+    if ((e = cudaMemsetAsync(B.krange, 0xff, sizeof(unsigned) * (size_t)P.N, s))) return e;
+    if ((e = cudaMemsetAsync(B.krange + P.N, 0, sizeof(unsigned) * (size_t)P.N, s))) return e;
+    const double reach = std::sqrt((double)P.blur) * (1.0 + 1e-6) + 1e-7;
+    if (P.pairs > 0) {
+        {
+            ProfScope ps(MR_STAGE_FACE_SETUP, s);
+            k_face_setup<<<pair_blocks(P.pairs), 256, 0, s>>>(verts, P.V, faces, B.prefix, B.first, P.N, P.pairs, P.H,
+                                                              P.W, reach, P.persp, B.geom, B.box, B.fconst, B.krange,
+                                                              B.err);
+        }
+        if ((e = cudaGetLastError())) return e;
+        {
+            ProfScope ps(MR_STAGE_BIN_COUNT, s);
+            k_bin_pairs<false><<<pair_blocks(P.pairs), 256, 0, s>>>(B.box, B.prefix, B.first, P.N, P.pairs, P.nbx,
+                                                                    P.nby, B.krange, B.counts, nullptr, nullptr);
+        }
+        if ((e = cudaGetLastError())) return e;
+    }
+    {
+        ProfScope ps(MR_STAGE_BIN_SCAN, s);
+        k_scan_tiles<<<P.ntiles, 1024, 0, s>>>(B.counts, P.nslots, B.offsets, B.tile_sum);
+        k_scan_tops<<<1, 1024, 0, s>>>(B.tile_sum, P.ntiles, B.total);
+        k_scan_add<<<std::min(ceil_div(P.nslots + 1, 256), 148 * 8), 256, 0, s>>>(B.offsets, P.nslots, B.tile_sum,
+                                                                                  B.total);
+    }
+    if ((e = cudaGetLastError())) return e;
+    if ((e = cudaMemcpyAsync(host_total, B.total, sizeof(long long), cudaMemcpyDeviceToHost, s))) return e;
+    return cudaMemcpyAsync(host_err, B.err, sizeof(int), cudaMemcpyDeviceToHost, s);
+}
+
+// Bin fill into `list` (total entries), fine pass and epilogue.
+inline cudaError_t fwd_enqueue_rest(const FwdPlan& P, const FwdBufs& B, int* list, long long total, bool sil,
+                                    float sigma, int64_t* p2f, float* zbuf, float* bary, float* dists, float* alpha,
+                                    cudaStream_t s) {
+    cudaError_t e;
+    if (total > 0) {
+        if ((e = cudaMemsetAsync(B.counts, 0, sizeof(int) * (size_t)P.nslots, s))) return e;
+        ProfScope ps(MR_STAGE_BIN_FILL, s);
+        k_bin_pairs<true><<<pair_blocks(P.pairs), 256, 0, s>>>(B.box, B.prefix, B.first, P.N, P.pairs, P.nbx, P.nby,
+                                                               B.krange, B.counts, B.offsets, list);
+        if ((e = cudaGetLastError())) return e;
+    }
+    const bool vec_ok = aligned16(p2f) && aligned16(zbuf) && aligned16(bary) && aligned16(dists);
+    const bool exact = (P.H & (P.H - 1)) == 0 && (P.W & (P.W - 1)) == 0;
+    {
+        ProfScope ps(MR_STAGE_FINE, s);
+        dispatch_fine(P.KC, P.persp != 0, exact, P.nbins, s, B.fconst, B.box, B.offsets, list, P.nbx, P.nby, P.H, P.W,
+                      P.K, P.blur, B.topk);
+    }
+    if ((e = cudaGetLastError())) return e;
+    {
+        ProfScope ps(MR_STAGE_EPILOGUE, s);
+        dispatch_epilogue(P.KC, P.persp != 0, sil, P.npix, s, B.geom, B.topk, P.H, P.W, P.K, sigma, vec_ok, p2f, zbuf,
+                          bary, dists, alpha);
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace

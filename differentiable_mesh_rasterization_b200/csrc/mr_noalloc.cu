@@ -58,19 +58,12 @@ int rasterize_noalloc(const float* verts, int64_t V, const int64_t* faces, int64
     int rc = validate_fwd(verts, V, faces, F, first, num, N, H, W, blur, K, p2f, zbuf, bary, dists);
     if (rc != MR_OK) return rc;
     if (N == 0) return MR_OK;
-    const int nbx = ceil_div(W, kBin), nby = ceil_div(H, kBin);
-    const long long nbins_ll = (long long)N * nbx * nby;
-    if (nbins_ll >= INT32_MAX / 2) {
-        set_error("too many screen bins (%lld)", nbins_ll);
-        return MR_ERR_ARG;
-    }
-    const int nbins = (int)nbins_ll;
-    const int KC = K <= 1 ? 1 : K <= 2 ? 2 : K <= 4 ? 4 : K <= 8 ? 8 : K <= 16 ? 16 : 32;
-    const int64_t npix = (int64_t)N * H * W;
-    const FwdScratch L = fwd_scratch_layout(F, npix, K, nbins, N);
-    if (L.bytes > (size_t)MR_NOALLOC_SCRATCH_BYTES) {
+    FwdPlan P;
+    rc = fwd_plan(V, F, num, N, H, W, blur, K, persp, P);
+    if (rc != MR_OK) return rc;
+    if (P.bytes > (size_t)MR_NOALLOC_SCRATCH_BYTES) {
         set_error("mr_rasterize_fwd_noalloc: this batch needs %zu bytes of scratch before its bin lists, more "
-                  "than the fixed %d bytes; use mr_rasterize_fwd", L.bytes, MR_NOALLOC_SCRATCH_BYTES);
+                  "than the fixed %d bytes; use mr_rasterize_fwd", P.bytes, MR_NOALLOC_SCRATCH_BYTES);
         return MR_ERR_ARG;
     }
     char* ws = nullptr;
@@ -78,62 +71,19 @@ int rasterize_noalloc(const float* verts, int64_t V, const int64_t* faces, int64
     if (rc != MR_OK) return rc;
     std::vector<int64_t> prefix(N + 1, 0);
     for (int n = 0; n < N; ++n) prefix[n + 1] = prefix[n] + num[n];
-    const int64_t pairs = prefix[N];
-
-    FaceGeom* geom = reinterpret_cast<FaceGeom*>(ws + L.geom);
-    FaceBox* box = reinterpret_cast<FaceBox*>(ws + L.box);
-    float4* fconst = reinterpret_cast<float4*>(ws + L.con);
-    int* topk = reinterpret_cast<int*>(ws + L.top);
-    int* counts = reinterpret_cast<int*>(ws + L.cnt);
-    int* offsets = reinterpret_cast<int*>(ws + L.off);
-    int64_t* d_prefix = reinterpret_cast<int64_t*>(ws + L.pre);
-    int64_t* d_first = reinterpret_cast<int64_t*>(ws + L.fst);
-    long long* d_total = reinterpret_cast<long long*>(ws + L.tot);
-    int* d_err = reinterpret_cast<int*>(ws + L.err);
-    int* list = reinterpret_cast<int*>(ws + L.bytes);
-
-    MR_CUDA(cudaMemcpyAsync(d_prefix, prefix.data(), sizeof(int64_t) * (N + 1), cudaMemcpyHostToDevice, s));
-    MR_CUDA(cudaMemcpyAsync(d_first, first, sizeof(int64_t) * N, cudaMemcpyHostToDevice, s));
-    MR_CUDA(cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)nbins, s));
-    MR_CUDA(cudaMemsetAsync(d_err, 0, sizeof(int), s));
-    const double reach = std::sqrt((double)blur) * (1.0 + 1e-6) + 1e-7;
-    if (F > 0) {
-        k_face_setup<<<(unsigned)((F + 255) / 256), 256, 0, s>>>(verts, V, faces, F, H, W, reach, persp, geom, box,
-                                                                  fconst, d_err);
-        MR_CUDA(cudaGetLastError());
-    }
-    const int pair_blocks = (int)std::min<int64_t>((pairs + 255) / 256, 148 * 16);
-    if (pairs > 0) {
-        k_bin_pairs<false><<<pair_blocks, 256, 0, s>>>(box, d_prefix, d_first, N, pairs, nbx, nby, counts, nullptr,
-                                                       nullptr);
-        MR_CUDA(cudaGetLastError());
-    }
-    k_scan<<<1, 1024, 0, s>>>(counts, nbins, offsets, d_total);
-    MR_CUDA(cudaGetLastError());
+    const FwdBufs B = fwd_bufs(ws, P);
+    int* list = reinterpret_cast<int*>(ws + P.bytes);     // the bin lists follow the fixed block
     long long total = 0;
     int herr = 0;
-    MR_CUDA(cudaMemcpyAsync(&total, d_total, sizeof(long long), cudaMemcpyDeviceToHost, s));
-    MR_CUDA(cudaMemcpyAsync(&herr, d_err, sizeof(int), cudaMemcpyDeviceToHost, s));
+    MR_CUDA(fwd_enqueue_count(P, B, verts, faces, prefix.data(), first, s, &total, &herr));
     MR_CUDA(cudaStreamSynchronize(s));
-    if (total < 0 || L.bytes + sizeof(int) * (size_t)total > (size_t)MR_NOALLOC_SCRATCH_BYTES) {
+    if (total < 0 || P.bytes + sizeof(int) * (size_t)total > (size_t)MR_NOALLOC_SCRATCH_BYTES) {
         set_error("mr_rasterize_fwd_noalloc: the bin lists need %lld entries, more than the %zu left of the "
                   "fixed %d-byte scratch; use mr_rasterize_fwd", total,
-                  ((size_t)MR_NOALLOC_SCRATCH_BYTES - L.bytes) / sizeof(int), MR_NOALLOC_SCRATCH_BYTES);
+                  ((size_t)MR_NOALLOC_SCRATCH_BYTES - P.bytes) / sizeof(int), MR_NOALLOC_SCRATCH_BYTES);
         return MR_ERR_ARG;
     }
-    if (total > 0) {
-        MR_CUDA(cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)nbins, s));
-        k_bin_pairs<true><<<pair_blocks, 256, 0, s>>>(box, d_prefix, d_first, N, pairs, nbx, nby, counts, offsets,
-                                                      list);
-        MR_CUDA(cudaGetLastError());
-    }
-    const bool vec_ok = aligned16(p2f) && aligned16(zbuf) && aligned16(bary) && aligned16(dists);
-    const bool exact = (H & (H - 1)) == 0 && (W & (W - 1)) == 0;
-    dispatch_fine(KC, persp != 0, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk);
-    MR_CUDA(cudaGetLastError());
-    dispatch_epilogue(KC, persp != 0, false, npix, s, geom, topk, H, W, K, 0.f, vec_ok, p2f, zbuf, bary, dists,
-                      nullptr);
-    MR_CUDA(cudaGetLastError());
+    MR_CUDA(fwd_enqueue_rest(P, B, list, total, false, 0.f, p2f, zbuf, bary, dists, nullptr, s));
     if (herr != 0) {
         set_error("a face references a vertex id outside [0, V=%lld); it was ignored", (long long)V);
         return MR_ERR_DEVICE;
