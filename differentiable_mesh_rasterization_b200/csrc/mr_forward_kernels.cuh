@@ -86,7 +86,7 @@ __device__ __forceinline__ void setup_face(const float* __restrict__ verts, int6
     }
     const double nx = y[1] * (q[2] - q[0]) - (q[1] - q[0]) * y[2];
     const double ny = (q[1] - q[0]) * x[2] - x[1] * (q[2] - q[0]);
-    const double gx = -nx / area2, gy = -ny / area2;
+    const double gx = -nx * inv_area2, gy = -ny * inv_area2;
     const float khi = (float)q[0];
     const float klo = (float)(q[0] - (double)khi);
     if (on_screen) {
@@ -111,7 +111,8 @@ __device__ __forceinline__ void setup_face(const float* __restrict__ verts, int6
         const int k1 = k == 2 ? 0 : k + 1;
         const double ex = x[k1] - x[k], ey = y[k1] - y[k];
         const double L = sqrt(ex * ex + ey * ey);
-        const double ux = ex / L, uy = ey / L;
+        const double inv_L = 1.0 / L;
+        const double ux = ex * inv_L, uy = ey * inv_L;
         e[k][0] = (float)ux;
         e[k][1] = (float)uy;
         e[k][2] = (float)(uy * x[k] - ux * y[k]);
