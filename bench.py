@@ -207,6 +207,26 @@ def workload_config(w, args):
             "parallelism": f"independent batch per GPU x{args.gpus}"}
 
 
+# ----------------------------------------------------------------------------- ncu traffic
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_batch5_512px.json")
+KERNEL_SOURCE = os.path.join(ROOT, "differentiable_mesh_rasterization_b200", "csrc", "mr_forward_kernels.cuh")
+
+
+def measured_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture of this workload,
+    or None when there is none or the kernel source changed since it was taken."""
+    import hashlib
+    try:
+        rec = json.load(open(TRAFFIC_FILE))
+        sha = hashlib.sha256(open(KERNEL_SOURCE, "rb").read()).hexdigest()
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_sha256") != sha:
+        return None
+    k = rec.get("kernels", {}).get(kernel)
+    return None if k is None else k["dram_read_bytes"] + k["dram_write_bytes"]
+
+
 # ----------------------------------------------------------------------------- ranks
 def rank_seed(config: int, rank: int) -> int:
     """Weak scaling: every rank renders its own batch of the same workload."""
@@ -368,8 +388,9 @@ def main():
     npix = batch.N * w.H * w.W
     fine_bytes = npix * 4 * w.K                      # the K winning face ids per pixel
     epi_bytes = npix * (4 * w.K + 28 * w.K + 4)      # ids in; p2f, zbuf, bary, dists, alpha out
+    full_batch = args.images is None and args.config == 5
     roof = {"bound": "alu", "achieved": achieved_alu, "peak": peak_alu, "unit": "T FP32-inst/s",
-            "frac": achieved_alu / peak_alu, "traffic": None,
+            "frac": achieved_alu / peak_alu, "traffic": measured_traffic("k_fine") if full_batch else None,
             "kernel": "k_fine (stage-one fine pass: pixel-face tests and register top-K)",
             "ms_per_step": fine_s * 1e3, "launches_per_step": fine_n // args.steps,
             "samples_per_step": samples, "c_test": C_TEST,
@@ -379,7 +400,8 @@ def main():
             "epilogue": {"kernel": "k_epilogue (float64 outputs of the K winners + silhouette)",
                          "bound": "hbm", "ms_per_step": epi_s * 1e3, "bytes_per_step": epi_bytes,
                          "achieved": epi_bytes / epi_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": epi_bytes / epi_s / 1e9 / hbm_peak, "peak_note": hbm_note}}
+                         "frac": epi_bytes / epi_s / 1e9 / hbm_peak, "peak_note": hbm_note,
+                         "traffic": measured_traffic("k_epilogue") if full_batch else None}}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dev_ms / args.steps, "higher_is_better": True,
