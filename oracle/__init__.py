@@ -50,6 +50,14 @@ def _load():
         lib.oracle_rasterize_bwd.restype = ctypes.c_int
         lib.oracle_probe.argtypes = [f64, f64, P, i32, P]
         lib.oracle_probe.restype = None
+        lib.oracle_interpolate_fwd.argtypes = [P, P, i64, i32, P, P, i32, P]
+        lib.oracle_interpolate_fwd.restype = None
+        lib.oracle_interpolate_bwd.argtypes = [P, P, i64, i32, P, P, i64, i32, P, P, P]
+        lib.oracle_interpolate_bwd.restype = None
+        lib.oracle_blend_fwd.argtypes = [P, P, P, P, i64, i32, i32, P, f64, f64, f64, f64, P]
+        lib.oracle_blend_fwd.restype = None
+        lib.oracle_blend_bwd.argtypes = [P, P, P, P, i64, i32, i32, P, f64, f64, f64, f64, P, P, P, P]
+        lib.oracle_blend_bwd.restype = None
         _lib = lib
     return _lib
 
@@ -157,3 +165,69 @@ def probe(px, py, abc, perspective_correct=False):
     lib.oracle_probe(float(px), float(py), _ptr(v), int(bool(perspective_correct)), _ptr(out))
     return dict(degenerate=bool(out[0]), inside=bool(out[1]), edge=int(out[2]), t=out[3], d2=out[4],
                 w=out[5:8].copy(), bary=out[8:11].copy(), z=out[11], dist=out[12])
+
+
+def interpolate_fwd(pix_to_face, bary, faces, attr):
+    """Step 14: per-slot attributes sum_m bary_m attr[v_m]; shape p2f.shape + (D,)."""
+    lib = _load()
+    p2f = _c(pix_to_face, np.int64)
+    b = _c(bary, np.float64)
+    f = _c(faces, np.int64)
+    a = _c(attr, np.float64)
+    K, D = p2f.shape[-1], a.shape[1]
+    npix = p2f.size // K
+    out = np.empty(p2f.shape + (D,), np.float64)
+    lib.oracle_interpolate_fwd(_ptr(p2f), _ptr(b), npix, K, _ptr(f), _ptr(a), D, _ptr(out))
+    return out
+
+
+def interpolate_bwd(pix_to_face, bary, faces, attr, grad_out):
+    """Step 15: (grad_attr V x D, grad_bary like bary)."""
+    lib = _load()
+    p2f = _c(pix_to_face, np.int64)
+    b = _c(bary, np.float64)
+    f = _c(faces, np.int64)
+    a = _c(attr, np.float64)
+    g = _c(grad_out, np.float64)
+    K, D = p2f.shape[-1], a.shape[1]
+    npix = p2f.size // K
+    ga = np.empty(a.shape, np.float64)
+    gb = np.empty(b.shape, np.float64)
+    lib.oracle_interpolate_bwd(_ptr(p2f), _ptr(b), npix, K, _ptr(f), _ptr(a), a.shape[0], D, _ptr(g), _ptr(ga),
+                               _ptr(gb))
+    return ga, gb
+
+
+def blend_fwd(pix_to_face, colors, dists, zbuf, background, sigma, gamma, znear, zfar):
+    """Step 16: soft RGB blend -> (..., D + 1) colour channels then alpha."""
+    lib = _load()
+    p2f = _c(pix_to_face, np.int64)
+    c = _c(colors, np.float64)
+    d = _c(dists, np.float64)
+    z = _c(zbuf, np.float64)
+    bg = _c(background, np.float64)
+    K, D = p2f.shape[-1], c.shape[-1]
+    npix = p2f.size // K
+    out = np.empty(p2f.shape[:-1] + (D + 1,), np.float64)
+    lib.oracle_blend_fwd(_ptr(p2f), _ptr(c), _ptr(d), _ptr(z), npix, K, D, _ptr(bg), float(sigma), float(gamma),
+                         float(znear), float(zfar), _ptr(out))
+    return out
+
+
+def blend_bwd(pix_to_face, colors, dists, zbuf, background, sigma, gamma, znear, zfar, grad_rgba):
+    """Step 17: (grad_colors, grad_dists, grad_zbuf)."""
+    lib = _load()
+    p2f = _c(pix_to_face, np.int64)
+    c = _c(colors, np.float64)
+    d = _c(dists, np.float64)
+    z = _c(zbuf, np.float64)
+    bg = _c(background, np.float64)
+    g = _c(grad_rgba, np.float64)
+    K, D = p2f.shape[-1], c.shape[-1]
+    npix = p2f.size // K
+    gc = np.empty(c.shape, np.float64)
+    gd = np.empty(d.shape, np.float64)
+    gz = np.empty(z.shape, np.float64)
+    lib.oracle_blend_bwd(_ptr(p2f), _ptr(c), _ptr(d), _ptr(z), npix, K, D, _ptr(bg), float(sigma), float(gamma),
+                         float(znear), float(zfar), _ptr(g), _ptr(gc), _ptr(gd), _ptr(gz))
+    return gc, gd, gz

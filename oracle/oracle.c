@@ -31,6 +31,8 @@
  *  12. its gradient: dL/ddist_k = -dL/dalpha * prod_{j != k} (1 - p_j) * p_k (1 - p_k) / sigma.
  *  13. rasterizer backward: the chain rule through steps 3, 5, 7, 8 and 9 with the
  *      candidate set, the inside flag and the nearest edge held fixed.
+ *  14-17. stage-two shading (attribute interpolation, soft RGB blend) and their
+ *      gradients; see the section at the end of this file.
  *
  * Besides the outputs, the forward marks pixels whose integer result is decided by a
  * float64-vs-float32 rounding: (E1) two of the K+1 nearest candidates lie within 1e-6
@@ -455,4 +457,147 @@ void oracle_probe(double px, double py, const double *abc /* 9: a, b, c as x,y,z
     out[0] = r.degenerate; out[1] = r.inside; out[2] = r.edge; out[3] = r.t; out[4] = r.d2;
     out[5] = r.w[0]; out[6] = r.w[1]; out[7] = r.w[2];
     out[8] = r.bary[0]; out[9] = r.bary[1]; out[10] = r.bary[2]; out[11] = r.z; out[12] = r.dist;
+}
+
+/* ------------------------------------------------------------------ stage two: shading */
+/*
+ * Gouraud shading and the soft RGB blend (PyTorch3D paper, method: pluggable Gouraud and
+ * Phong shaders over the K faces kept per pixel; the soft aggregation is SoftRas's, the
+ * renderer the paper compares against).  Written out:
+ *
+ *  14. interpolation: for a valid slot with face f = (v0, v1, v2) and barycentrics b,
+ *      out[d] = sum_m b_m attr[v_m][d]; empty slots give 0.
+ *  15. its gradient: d attr[v_m][d] += b_m g[d]; d b_m = sum_d attr[v_m][d] g[d].
+ *  16. soft RGB blend over the valid slots of a pixel, with colours c_k (D channels),
+ *      signed distances d_k and depths z_k:
+ *        p_k = 1 / (1 + exp(d_k / sigma))                      coverage weight
+ *        s_k = (zfar - z_k) / (zfar - znear)                   normalised nearness
+ *        m   = max(max_k s_k, eps)        (eps = 1e-10; shift for stability only)
+ *        w_k = p_k exp((s_k - m) / gamma),  w_b = exp((eps - m) / gamma)
+ *        rgb = (sum_k w_k c_k + w_b bg) / (sum_k w_k + w_b)
+ *        alpha = 1 - prod_k (1 - p_k)
+ *  17. its gradient, with m held fixed (rgb does not depend on it):
+ *        d c_k = w_k / D g,  d w_k = (c_k - rgb) . g / D,
+ *        d d_k = d w_k * w_k * (-(1 - p_k) / sigma) + (alpha part as in step 12),
+ *        d z_k = d w_k * w_k * (-1 / (gamma (zfar - znear))).
+ */
+#define BLEND_EPS 1e-10
+
+/* Step 14 over npix pixels of K slots: attr V x D, bary (npix x K x 3), out npix x K x D. */
+void oracle_interpolate_fwd(const int64_t *p2f, const double *bary, int64_t npix, int32_t K,
+                            const int64_t *faces, const double *attr, int32_t D, double *out) {
+    for (int64_t s = 0; s < npix * K; ++s) {
+        int64_t f = p2f[s];
+        for (int d = 0; d < D; ++d) {
+            double v = 0.0;
+            if (f >= 0)
+                for (int m = 0; m < 3; ++m) v += bary[3 * s + m] * attr[faces[3 * f + m] * D + d];
+            out[s * D + d] = v;
+        }
+    }
+}
+
+/* Step 15: grad_attr (V x D) is overwritten; grad_bary (npix x K x 3) may be NULL. */
+void oracle_interpolate_bwd(const int64_t *p2f, const double *bary, int64_t npix, int32_t K,
+                            const int64_t *faces, const double *attr, int64_t V, int32_t D,
+                            const double *grad_out, double *grad_attr, double *grad_bary) {
+    memset(grad_attr, 0, sizeof(double) * (size_t)(V * D));
+    for (int64_t s = 0; s < npix * K; ++s) {
+        int64_t f = p2f[s];
+        for (int m = 0; m < 3; ++m) {
+            double gb = 0.0;
+            if (f >= 0) {
+                int64_t v = faces[3 * f + m];
+                for (int d = 0; d < D; ++d) {
+                    grad_attr[v * D + d] += bary[3 * s + m] * grad_out[s * D + d];
+                    gb += attr[v * D + d] * grad_out[s * D + d];
+                }
+            }
+            if (grad_bary) grad_bary[3 * s + m] = gb;
+        }
+    }
+}
+
+/* Step 16: colors npix x K x D, out rgba npix x (D + 1) (colour channels, then alpha). */
+void oracle_blend_fwd(const int64_t *p2f, const double *colors, const double *dists, const double *zbuf,
+                      int64_t npix, int32_t K, int32_t D, const double *background, double sigma,
+                      double gamma, double znear, double zfar, double *out) {
+    for (int64_t q = 0; q < npix; ++q) {
+        double m = BLEND_EPS, keep = 1.0;
+        for (int k = 0; k < K; ++k) {
+            int64_t s = q * K + k;
+            if (p2f[s] < 0) continue;
+            double sk = (zfar - zbuf[s]) / (zfar - znear);
+            if (sk > m) m = sk;
+        }
+        double den = exp((BLEND_EPS - m) / gamma);
+        for (int d = 0; d < D; ++d) out[q * (D + 1) + d] = den * background[d];
+        for (int k = 0; k < K; ++k) {
+            int64_t s = q * K + k;
+            if (p2f[s] < 0) continue;
+            double p = 1.0 / (1.0 + exp(dists[s] / sigma));
+            double sk = (zfar - zbuf[s]) / (zfar - znear);
+            double w = p * exp((sk - m) / gamma);
+            den += w;
+            for (int d = 0; d < D; ++d) out[q * (D + 1) + d] += w * colors[s * D + d];
+            keep *= 1.0 - p;
+        }
+        for (int d = 0; d < D; ++d) out[q * (D + 1) + d] /= den;
+        out[q * (D + 1) + D] = 1.0 - keep;
+    }
+}
+
+/* Step 17: grad_rgba npix x (D + 1); writes grad_colors (npix x K x D), grad_dists and
+ * grad_zbuf (npix x K); any output may be NULL. */
+void oracle_blend_bwd(const int64_t *p2f, const double *colors, const double *dists, const double *zbuf,
+                      int64_t npix, int32_t K, int32_t D, const double *background, double sigma,
+                      double gamma, double znear, double zfar, const double *grad_rgba,
+                      double *grad_colors, double *grad_dists, double *grad_zbuf) {
+    double *rgb = (double *)malloc(sizeof(double) * (size_t)(D + 1));
+    for (int64_t q = 0; q < npix; ++q) {
+        oracle_blend_fwd(p2f + q * K, colors + q * K * D, dists + q * K, zbuf + q * K, 1, K, D, background,
+                         sigma, gamma, znear, zfar, rgb);
+        double m = BLEND_EPS;
+        for (int k = 0; k < K; ++k) {
+            int64_t s = q * K + k;
+            if (p2f[s] < 0) continue;
+            double sk = (zfar - zbuf[s]) / (zfar - znear);
+            if (sk > m) m = sk;
+        }
+        double den = exp((BLEND_EPS - m) / gamma);
+        for (int k = 0; k < K; ++k) {
+            int64_t s = q * K + k;
+            if (p2f[s] < 0) continue;
+            double p = 1.0 / (1.0 + exp(dists[s] / sigma));
+            den += p * exp(((zfar - zbuf[s]) / (zfar - znear) - m) / gamma);
+        }
+        const double *g = grad_rgba + q * (D + 1);
+        for (int k = 0; k < K; ++k) {
+            int64_t s = q * K + k;
+            if (p2f[s] < 0) {
+                if (grad_colors) for (int d = 0; d < D; ++d) grad_colors[s * D + d] = 0.0;
+                if (grad_dists) grad_dists[s] = 0.0;
+                if (grad_zbuf) grad_zbuf[s] = 0.0;
+                continue;
+            }
+            double p = 1.0 / (1.0 + exp(dists[s] / sigma));
+            double w = p * exp(((zfar - zbuf[s]) / (zfar - znear) - m) / gamma);
+            double gw = 0.0;
+            for (int d = 0; d < D; ++d) {
+                if (grad_colors) grad_colors[s * D + d] = w / den * g[d];
+                gw += (colors[s * D + d] - rgb[d]) * g[d] / den;
+            }
+            /* alpha = 1 - prod (1 - p_j): d alpha / d p_k = prod_{j != k} (1 - p_j) */
+            double others = 1.0;
+            for (int j = 0; j < K; ++j) {
+                int64_t sj = q * K + j;
+                if (j == k || p2f[sj] < 0) continue;
+                others *= 1.0 - 1.0 / (1.0 + exp(dists[sj] / sigma));
+            }
+            double dp_dd = -p * (1.0 - p) / sigma;
+            if (grad_dists) grad_dists[s] = gw * w * (-(1.0 - p) / sigma) + g[D] * others * dp_dd;
+            if (grad_zbuf) grad_zbuf[s] = gw * w * (-1.0 / (gamma * (zfar - znear)));
+        }
+    }
+    free(rgb);
 }
