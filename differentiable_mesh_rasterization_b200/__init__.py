@@ -26,9 +26,10 @@ ERRORS = {-1: "invalid argument", -2: "out of memory", -3: "CUDA error", -4: "de
 EXPORTS = ("mr_rasterize_fwd", "mr_rasterize_silhouette_fwd", "mr_silhouette_blend_fwd",
            "mr_silhouette_blend_bwd", "mr_rasterize_bwd", "mr_silhouette_rasterize_bwd",
            "mr_device_status", "mr_last_error", "mr_version", "mr_profile_enable", "mr_profile_read",
-           "mr_rasterize_fwd_noalloc")
+           "mr_rasterize_fwd_noalloc", "mr_interpolate_fwd", "mr_interpolate_bwd", "mr_blend_fwd", "mr_blend_bwd")
 STAGES = ("face_setup", "bin_count", "bin_scan", "bin_fill", "fine", "silhouette_fwd", "silhouette_bwd",
-          "raster_bwd", "silhouette_raster_bwd", "epilogue")
+          "raster_bwd", "silhouette_raster_bwd", "epilogue", "interpolate_fwd", "interpolate_bwd", "blend_fwd",
+          "blend_bwd")
 
 
 class MeshRastError(RuntimeError):
@@ -61,6 +62,10 @@ def load_library() -> ctypes.CDLL:
         "mr_device_status": [P],
         "mr_last_error": [],
         "mr_version": [],
+        "mr_interpolate_fwd": [P, P, i64, i32, P, i64, P, i64, i32, P, P],
+        "mr_interpolate_bwd": [P, P, i64, i32, P, i64, P, i64, i32, P, P, P, P],
+        "mr_blend_fwd": [P, P, P, P, i64, i32, i32, P, f32, f32, f32, f32, P, P],
+        "mr_blend_bwd": [P, P, P, P, i64, i32, i32, P, f32, f32, f32, f32, P, P, P, P, P],
         "mr_profile_enable": [i32],
         "mr_profile_read": [P, P, i32],
     }
@@ -244,6 +249,82 @@ def silhouette_rasterize_bwd(verts, faces, pix_to_face, dists, sigma, grad_alpha
                                                _ptr(d), N, H, W, K, float(sigma), _ptr(g), _ptr(out),
                                                _stream(verts.device)))
     return out
+
+
+def interpolate_fwd(pix_to_face, bary, faces, attr):
+    """Per-slot vertex attributes (``mr_interpolate_fwd``): (N, H, W, K, D) float32."""
+    lib = load_library()
+    p2f = _dev(pix_to_face, torch.int64, "pix_to_face")
+    b = _dev(bary, torch.float32, "bary")
+    f = _dev(faces, torch.int64, "faces")
+    a = _dev(attr, torch.float32, "attr")
+    if a.ndim != 2 or tuple(b.shape) != tuple(p2f.shape) + (3,):
+        raise ValueError("attr must be (V, D) and bary (N, H, W, K, 3)")
+    K, D = p2f.shape[-1], a.shape[1]
+    out = torch.empty(tuple(p2f.shape) + (D,), dtype=torch.float32, device=p2f.device)
+    with torch.cuda.device(p2f.device):
+        _check("mr_interpolate_fwd", lib.mr_interpolate_fwd(_ptr(p2f), _ptr(b), p2f.numel() // K, K, _ptr(f), f.shape[0],
+                                                            _ptr(a), a.shape[0], D, _ptr(out), _stream(p2f.device)))
+    return out
+
+
+def interpolate_bwd(pix_to_face, bary, faces, attr, grad_out):
+    """Gradient of the interpolation (``mr_interpolate_bwd``) -> (grad_attr (V, D), grad_bary)."""
+    lib = load_library()
+    p2f = _dev(pix_to_face, torch.int64, "pix_to_face")
+    b = _dev(bary, torch.float32, "bary")
+    f = _dev(faces, torch.int64, "faces")
+    a = _dev(attr, torch.float32, "attr")
+    g = _dev(grad_out, torch.float32, "grad_out")
+    K, D = p2f.shape[-1], a.shape[1]
+    if tuple(g.shape) != tuple(p2f.shape) + (D,):
+        raise ValueError("grad_out shape mismatch")
+    ga = torch.empty_like(a)
+    gb = torch.empty_like(b)
+    with torch.cuda.device(p2f.device):
+        _check("mr_interpolate_bwd", lib.mr_interpolate_bwd(_ptr(p2f), _ptr(b), p2f.numel() // K, K, _ptr(f), f.shape[0],
+                                                            _ptr(a), a.shape[0], D, _ptr(g), _ptr(ga), _ptr(gb),
+                                                            _stream(p2f.device)))
+    return ga, gb
+
+
+def _blend_args(pix_to_face, colors, dists, zbuf, background):
+    p2f = _dev(pix_to_face, torch.int64, "pix_to_face")
+    c = _dev(colors, torch.float32, "colors")
+    d = _dev(dists, torch.float32, "dists")
+    z = _dev(zbuf, torch.float32, "zbuf")
+    K, D = p2f.shape[-1], c.shape[-1]
+    if tuple(c.shape[:-1]) != tuple(p2f.shape) or d.shape != p2f.shape or z.shape != p2f.shape:
+        raise ValueError("colors / dists / zbuf must match pix_to_face")
+    bg = np.ascontiguousarray(np.asarray(background, dtype=np.float32).reshape(-1))
+    if bg.shape[0] != D:
+        raise ValueError("background must have one value per colour channel")
+    return p2f, c, d, z, bg, K, D
+
+
+def blend_fwd(pix_to_face, colors, dists, zbuf, background, sigma, gamma, znear, zfar):
+    """Soft RGB blend (``mr_blend_fwd``) -> rgba (N, H, W, D + 1)."""
+    lib = load_library()
+    p2f, c, d, z, bg, K, D = _blend_args(pix_to_face, colors, dists, zbuf, background)
+    out = torch.empty(tuple(p2f.shape[:-1]) + (D + 1,), dtype=torch.float32, device=p2f.device)
+    with torch.cuda.device(p2f.device):
+        _check("mr_blend_fwd", lib.mr_blend_fwd(_ptr(p2f), _ptr(c), _ptr(d), _ptr(z), p2f.numel() // K, K, D,
+                                                bg.ctypes.data, float(sigma), float(gamma), float(znear), float(zfar),
+                                                _ptr(out), _stream(p2f.device)))
+    return out
+
+
+def blend_bwd(pix_to_face, colors, dists, zbuf, background, sigma, gamma, znear, zfar, grad_rgba):
+    """Gradient of the blend (``mr_blend_bwd``) -> (grad_colors, grad_dists, grad_zbuf)."""
+    lib = load_library()
+    p2f, c, d, z, bg, K, D = _blend_args(pix_to_face, colors, dists, zbuf, background)
+    g = _dev(grad_rgba, torch.float32, "grad_rgba")
+    gc, gd, gz = torch.empty_like(c), torch.empty_like(d), torch.empty_like(z)
+    with torch.cuda.device(p2f.device):
+        _check("mr_blend_bwd", lib.mr_blend_bwd(_ptr(p2f), _ptr(c), _ptr(d), _ptr(z), p2f.numel() // K, K, D,
+                                                bg.ctypes.data, float(sigma), float(gamma), float(znear), float(zfar),
+                                                _ptr(g), _ptr(gc), _ptr(gd), _ptr(gz), _stream(p2f.device)))
+    return gc, gd, gz
 
 
 def device_status(device=None) -> None:

@@ -169,6 +169,41 @@ int mr_silhouette_rasterize_bwd(const float* verts, int64_t V, const int64_t* fa
                                 int32_t H, int32_t W, int32_t K, float sigma,
                                 const float* grad_alpha, float* grad_verts, void* stream);
 
+/*
+ * Stage-two shading (PyTorch3D paper, method: pluggable Gouraud and Phong shaders over
+ * the K faces kept per pixel; SoftRas, the renderer the paper compares against, is the
+ * source of the soft aggregation).  pix_to_face / bary / dists / zbuf are the stage-one
+ * outputs (npix = N*H*W pixels of K slots).  All asynchronous.
+ *
+ * mr_interpolate_fwd: out (npix x K x D float32) = sum_m bary_m attr[v_m] over the face's
+ *   vertices v_m, 0 for empty slots (Gouraud: attr = per-vertex colours or normals).
+ *   attr: V x D float32 (device).
+ * mr_interpolate_bwd: grad_attr (V x D, overwritten; float32 atomics) and grad_bary
+ *   (npix x K x 3, may be NULL) from grad_out (npix x K x D).
+ * mr_blend_fwd: soft RGB blend of per-slot colours (npix x K x D, D <= MR_BLEND_DMAX) into
+ *   rgba (npix x (D + 1) float32: D colour channels, then alpha):
+ *     p_k = 1 / (1 + exp(dists_k / sigma)),  s_k = (zfar - zbuf_k) / (zfar - znear),
+ *     m = max(max_k s_k, 1e-10),  w_k = p_k exp((s_k - m) / gamma),  w_b = exp((1e-10 - m) / gamma),
+ *     rgb = (sum_k w_k colour_k + w_b background) / (sum_k w_k + w_b),  alpha = 1 - prod_k (1 - p_k).
+ *   background: D floats (HOST).  sigma, gamma > 0, zfar > znear.
+ * mr_blend_bwd: grad_colors (npix x K x D), grad_dists and grad_zbuf (npix x K) from
+ *   grad_rgba (npix x (D + 1)); each output may be NULL; empty slots get 0.
+ */
+#define MR_BLEND_DMAX 8
+int mr_interpolate_fwd(const int64_t* pix_to_face, const float* bary, int64_t npix, int32_t K,
+                       const int64_t* faces, int64_t F, const float* attr, int64_t V, int32_t D,
+                       float* out, void* stream);
+int mr_interpolate_bwd(const int64_t* pix_to_face, const float* bary, int64_t npix, int32_t K,
+                       const int64_t* faces, int64_t F, const float* attr, int64_t V, int32_t D,
+                       const float* grad_out, float* grad_attr, float* grad_bary, void* stream);
+int mr_blend_fwd(const int64_t* pix_to_face, const float* colors, const float* dists,
+                 const float* zbuf, int64_t npix, int32_t K, int32_t D, const float* background,
+                 float sigma, float gamma, float znear, float zfar, float* rgba, void* stream);
+int mr_blend_bwd(const int64_t* pix_to_face, const float* colors, const float* dists,
+                 const float* zbuf, int64_t npix, int32_t K, int32_t D, const float* background,
+                 float sigma, float gamma, float znear, float zfar, const float* grad_rgba,
+                 float* grad_colors, float* grad_dists, float* grad_zbuf, void* stream);
+
 /* Synchronises `stream`, then returns MR_ERR_DEVICE (and clears the word) if any
  * asynchronous kernel of this library flagged an out-of-range index on the current
  * device since the last call, else MR_OK (or MR_ERR_CUDA). */
@@ -198,7 +233,11 @@ int mr_version(void);
 #define MR_STAGE_RASTER_BWD 7
 #define MR_STAGE_SILHOUETTE_RASTER_BWD 8
 #define MR_STAGE_EPILOGUE 9
-#define MR_NUM_STAGES 10
+#define MR_STAGE_INTERPOLATE_FWD 10
+#define MR_STAGE_INTERPOLATE_BWD 11
+#define MR_STAGE_BLEND_FWD 12
+#define MR_STAGE_BLEND_BWD 13
+#define MR_NUM_STAGES 14
 int mr_profile_enable(int32_t on);
 int mr_profile_read(double* stage_ms, int64_t* launches, int32_t nstages);
 
