@@ -32,12 +32,13 @@ __device__ __forceinline__ bool load_face(const int64_t* __restrict__ faces, int
     return vid[0] >= 0 && vid[0] < V && vid[1] >= 0 && vid[1] < V && vid[2] >= 0 && vid[2] < V;
 }
 
-// General backward: one thread per slot, float64 arithmetic.
+// General backward: one thread per slot, float64 arithmetic; each of the face's vertices
+// receives one float4 (x, y, z, 0) atomic into a padded accumulator.
 template <bool PERSP>
 __global__ void k_raster_bwd(const float* __restrict__ verts, int64_t V, const int64_t* __restrict__ faces,
                              int64_t F, const int64_t* __restrict__ p2f, int64_t nslots, int H, int W, int K,
                              const float* __restrict__ gz, const float* __restrict__ gb,
-                             const float* __restrict__ gd, float* __restrict__ gv, int* __restrict__ err) {
+                             const float* __restrict__ gd, float4* __restrict__ acc, int* __restrict__ err) {
     for (int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; s < nslots; s += (int64_t)gridDim.x * blockDim.x) {
         const int64_t f = p2f[s];
         if (f == -1) continue;
@@ -139,9 +140,18 @@ __global__ void k_raster_bwd(const float* __restrict__ verts, int64_t V, const i
         }
 #pragma unroll
         for (int q = 0; q < 3; ++q)
-#pragma unroll
-            for (int e = 0; e < 3; ++e)
-                if (g[q][e] != 0.0) atomicAdd(gv + 3 * vid[q] + e, (float)g[q][e]);
+            if (g[q][0] != 0.0 || g[q][1] != 0.0 || g[q][2] != 0.0)
+                atomicAdd(acc + vid[q], make_float4((float)g[q][0], (float)g[q][1], (float)g[q][2], 0.f));
+    }
+}
+
+// grad_verts (V x 3) from the padded (x, y, z, 0) accumulator.
+__global__ void k_xyzw_to_xyz(const float4* __restrict__ acc, int64_t V, float* __restrict__ gv) {
+    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < V; v += (int64_t)gridDim.x * blockDim.x) {
+        const float4 a = acc[v];
+        gv[3 * v] = a.x;
+        gv[3 * v + 1] = a.y;
+        gv[3 * v + 2] = a.z;
     }
 }
 
@@ -294,23 +304,35 @@ int mr_rasterize_bwd(const float* verts, int64_t V, const int64_t* faces, int64_
     int rc = mr::validate_bwd(verts, V, faces, F, pix_to_face, N, H, W, K, grad_verts);
     if (rc != MR_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (V > 0) MR_CUDA(cudaMemsetAsync(grad_verts, 0, sizeof(float) * 3 * (size_t)V, s));
     const int64_t nslots = (int64_t)N * H * W * K;
-    if (nslots == 0 || (!grad_zbuf && !grad_bary && !grad_dists)) return MR_OK;
+    if (V == 0) return MR_OK;
+    if (nslots == 0 || (!grad_zbuf && !grad_bary && !grad_dists)) {
+        MR_CUDA(cudaMemsetAsync(grad_verts, 0, sizeof(float) * 3 * (size_t)V, s));
+        return MR_OK;
+    }
     int* err = mr::device_error_word();
     if (!err) {
         mr::set_error("cannot locate the device error word");
         return MR_ERR_CUDA;
     }
-    const int g = mr::grid_for(nslots);
-    mr::ProfScope ps(MR_STAGE_RASTER_BWD, s);
-    if (perspective_correct)
-        mr::k_raster_bwd<true><<<g, 256, 0, s>>>(verts, V, faces, F, pix_to_face, nslots, H, W, K, grad_zbuf, grad_bary,
-                                                 grad_dists, grad_verts, err);
-    else
-        mr::k_raster_bwd<false><<<g, 256, 0, s>>>(verts, V, faces, F, pix_to_face, nslots, H, W, K, grad_zbuf,
-                                                  grad_bary, grad_dists, grad_verts, err);
-    MR_CUDA(cudaGetLastError());
+    float4* acc = nullptr;
+    rc = mr::scratch_alloc(reinterpret_cast<void**>(&acc), sizeof(float4) * (size_t)V, s);
+    if (rc != MR_OK) return rc;
+    cudaError_t e = cudaMemsetAsync(acc, 0, sizeof(float4) * (size_t)V, s);
+    if (e == cudaSuccess) {
+        const int g = mr::grid_for(nslots);
+        mr::ProfScope ps(MR_STAGE_RASTER_BWD, s);
+        if (perspective_correct)
+            mr::k_raster_bwd<true><<<g, 256, 0, s>>>(verts, V, faces, F, pix_to_face, nslots, H, W, K, grad_zbuf,
+                                                     grad_bary, grad_dists, acc, err);
+        else
+            mr::k_raster_bwd<false><<<g, 256, 0, s>>>(verts, V, faces, F, pix_to_face, nslots, H, W, K, grad_zbuf,
+                                                      grad_bary, grad_dists, acc, err);
+        mr::k_xyzw_to_xyz<<<mr::grid_for(V), 256, 0, s>>>(acc, V, grad_verts);
+        e = cudaGetLastError();
+    }
+    mr::scratch_free(acc, s);
+    if (e != cudaSuccess) return mr::cuda_fail(e, "rasterizer backward launch");
     return MR_OK;
 }
 

@@ -56,10 +56,14 @@ __global__ void k_interpolate_fwd(const int64_t* __restrict__ p2f, const float* 
     }
 }
 
+// Gradient of the interpolation.  For D <= 4 the attribute gradient is summed into a
+// padded V x 4 accumulator with one float4 atomic per (slot, vertex) (three per slot
+// instead of 3 D scalar ones), then copied out; wider attributes use scalar atomics.
+template <bool VEC4>
 __global__ void k_interpolate_bwd(const int64_t* __restrict__ p2f, const float* __restrict__ bary, int64_t nslots,
                                   const int64_t* __restrict__ faces, int64_t F, const float* __restrict__ attr,
                                   int64_t V, int D, const float* __restrict__ grad_out, float* __restrict__ grad_attr,
-                                  float* __restrict__ grad_bary, int* __restrict__ err) {
+                                  float4* __restrict__ acc4, float* __restrict__ grad_bary, int* __restrict__ err) {
     for (int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; s < nslots; s += (int64_t)gridDim.x * blockDim.x) {
         const int64_t f = p2f[s];
         int64_t v[3];
@@ -74,13 +78,23 @@ __global__ void k_interpolate_bwd(const int64_t* __restrict__ p2f, const float* 
         float gb[3] = {0.f, 0.f, 0.f};
         if (ok) {
             const float b[3] = {bary[3 * s], bary[3 * s + 1], bary[3 * s + 2]};
-            for (int d = 0; d < D; ++d) {
-                const float g = grad_out[s * D + d];
-                if (g == 0.f) continue;
+            if (VEC4) {
+                float g[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int d = 0; d < D; ++d) g[d] = grad_out[s * D + d];
 #pragma unroll
                 for (int m = 0; m < 3; ++m) {
-                    gb[m] = fmaf(attr[v[m] * D + d], g, gb[m]);
-                    if (b[m] != 0.f) atomicAdd(grad_attr + v[m] * D + d, b[m] * g);
+                    for (int d = 0; d < D; ++d) gb[m] = fmaf(attr[v[m] * D + d], g[d], gb[m]);
+                    atomicAdd(acc4 + v[m], make_float4(b[m] * g[0], b[m] * g[1], b[m] * g[2], b[m] * g[3]));
+                }
+            } else {
+                for (int d = 0; d < D; ++d) {
+                    const float g = grad_out[s * D + d];
+                    if (g == 0.f) continue;
+#pragma unroll
+                    for (int m = 0; m < 3; ++m) {
+                        gb[m] = fmaf(attr[v[m] * D + d], g, gb[m]);
+                        if (b[m] != 0.f) atomicAdd(grad_attr + v[m] * D + d, b[m] * g);
+                    }
                 }
             }
         }
@@ -89,6 +103,14 @@ __global__ void k_interpolate_bwd(const int64_t* __restrict__ p2f, const float* 
             grad_bary[3 * s + 1] = gb[1];
             grad_bary[3 * s + 2] = gb[2];
         }
+    }
+}
+
+__global__ void k_acc4_to_rows(const float4* __restrict__ acc4, int64_t V, int D, float* __restrict__ out) {
+    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < V; v += (int64_t)gridDim.x * blockDim.x) {
+        const float4 a = acc4[v];
+        const float x[4] = {a.x, a.y, a.z, a.w};
+        for (int d = 0; d < D; ++d) out[v * D + d] = x[d];
     }
 }
 
@@ -248,20 +270,38 @@ int mr_interpolate_bwd(const int64_t* pix_to_face, const float* bary, int64_t np
         return MR_ERR_ARG;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (V > 0) MR_CUDA(cudaMemsetAsync(grad_attr, 0, sizeof(float) * (size_t)(V * D), s));
     const int64_t nslots = npix * K;
-    if (nslots == 0) return MR_OK;
+    if (nslots == 0 || V == 0) {
+        if (V > 0) MR_CUDA(cudaMemsetAsync(grad_attr, 0, sizeof(float) * (size_t)(V * D), s));
+        return MR_OK;
+    }
     int* err = mr::device_error_word();
     if (!err) {
         mr::set_error("cannot locate the device error word");
         return MR_ERR_CUDA;
     }
-    {
+    if (D > 4) {
+        MR_CUDA(cudaMemsetAsync(grad_attr, 0, sizeof(float) * (size_t)(V * D), s));
         mr::ProfScope ps(MR_STAGE_INTERPOLATE_BWD, s);
-        mr::k_interpolate_bwd<<<mr::grid_for(nslots), 256, 0, s>>>(pix_to_face, bary, nslots, faces, F, attr, V, D,
-                                                                  grad_out, grad_attr, grad_bary, err);
+        mr::k_interpolate_bwd<false><<<mr::grid_for(nslots), 256, 0, s>>>(pix_to_face, bary, nslots, faces, F, attr, V,
+                                                                         D, grad_out, grad_attr, nullptr, grad_bary,
+                                                                         err);
+        MR_CUDA(cudaGetLastError());
+        return MR_OK;
     }
-    MR_CUDA(cudaGetLastError());
+    float4* acc = nullptr;
+    int rc = mr::scratch_alloc(reinterpret_cast<void**>(&acc), sizeof(float4) * (size_t)V, s);
+    if (rc != MR_OK) return rc;
+    cudaError_t e = cudaMemsetAsync(acc, 0, sizeof(float4) * (size_t)V, s);
+    if (e == cudaSuccess) {
+        mr::ProfScope ps(MR_STAGE_INTERPOLATE_BWD, s);
+        mr::k_interpolate_bwd<true><<<mr::grid_for(nslots), 256, 0, s>>>(pix_to_face, bary, nslots, faces, F, attr, V,
+                                                                        D, grad_out, nullptr, acc, grad_bary, err);
+        mr::k_acc4_to_rows<<<mr::grid_for(V), 256, 0, s>>>(acc, V, D, grad_attr);
+        e = cudaGetLastError();
+    }
+    mr::scratch_free(acc, s);
+    if (e != cudaSuccess) return mr::cuda_fail(e, "interpolation backward");
     return MR_OK;
 }
 
