@@ -149,6 +149,8 @@ class MeshBatch:
     workload: Workload
     seed: int
     kinds: list = field(default_factory=list)   # per mesh: ("ico", level) or ("torus", R, S)
+    world: np.ndarray | None = None     # (sum V, 3) float32: world positions (camera at (0, 0, 2.7))
+    normals: np.ndarray | None = None   # (sum V, 3) float32: unit normals of the unperturbed shape
 
     @property
     def N(self) -> int:
@@ -158,7 +160,7 @@ class MeshBatch:
 def _pack(meshes: list[tuple[np.ndarray, np.ndarray]]):
     verts, faces, ff, nf, vf, nv = [], [], [], [], [], []
     vo = fo = 0
-    for v, f in meshes:
+    for v, f, *_ in meshes:
         verts.append(v)
         faces.append(f + vo)
         ff.append(fo); nf.append(f.shape[0]); vf.append(vo); nv.append(v.shape[0])
@@ -200,21 +202,30 @@ def make_batch(config: int, seed: int | None = None, n_meshes: int | None = None
         if config == 5 and n >= N // 2:
             R, S = int(rs[n - N // 2, 0]), int(rs[n - N // 2, 1])
             v, f = torus(R, S)
+            ring = v.copy()
+            ring[:, 2] = 0.0
+            ring /= np.linalg.norm(ring, axis=1, keepdims=True)
+            nrm = (v - ring) / np.linalg.norm(v - ring, axis=1, keepdims=True)   # away from the tube's core
             kinds.append(("torus", R, S))
         else:
             v, f = icosphere(int(levels[n]))
+            nrm = v.copy()                                                     # unit sphere: normal = position
             kinds.append(("ico", int(levels[n])))
         if noise > 0:
             v = v * (1.0 + noise * rng.standard_normal((v.shape[0], 1)))
         if config == 3:
             v = v * rng.uniform(0.6, 1.0)
         if config in (2, 3, 5):
-            v = v @ random_rotation(rng).T
+            R3 = random_rotation(rng)
+            v = v @ R3.T
+            nrm = nrm @ R3.T
         if config == 5:
             v = v + rng.uniform(-0.2, 0.2, size=3)
-        meshes.append((project(v), f))
+        meshes.append((project(v), f, v, nrm))
     verts, faces, ff, nf, vf, nv = _pack(meshes)
-    return MeshBatch(verts, faces, ff, nf, vf, nv, w, seed, kinds)
+    world = np.concatenate([m[2] for m in meshes]).astype(np.float32)
+    normals = np.concatenate([m[3] for m in meshes]).astype(np.float32)
+    return MeshBatch(verts, faces, ff, nf, vf, nv, w, seed, kinds, world, normals)
 
 
 def grad_alpha(batch: MeshBatch) -> np.ndarray:

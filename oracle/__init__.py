@@ -58,6 +58,14 @@ def _load():
         lib.oracle_blend_fwd.restype = None
         lib.oracle_blend_bwd.argtypes = [P, P, P, P, i64, i32, i32, P, f64, f64, f64, f64, P, P, P, P]
         lib.oracle_blend_bwd.restype = None
+        lib.oracle_phong_fwd.argtypes = [P, P, P, i64, P, P, P]
+        lib.oracle_phong_fwd.restype = None
+        lib.oracle_phong_bwd.argtypes = [P, P, P, i64, P, P, P, P, P]
+        lib.oracle_phong_bwd.restype = None
+        lib.oracle_phong_shade_fwd.argtypes = [P, P, i64, i32, P, P, P, P, P, P, P]
+        lib.oracle_phong_shade_fwd.restype = None
+        lib.oracle_phong_shade_bwd.argtypes = [P, P, i64, i32, P, P, P, P, i64, P, P, P, P, P, P]
+        lib.oracle_phong_shade_bwd.restype = None
         _lib = lib
     return _lib
 
@@ -231,3 +239,68 @@ def blend_bwd(pix_to_face, colors, dists, zbuf, background, sigma, gamma, znear,
     lib.oracle_blend_bwd(_ptr(p2f), _ptr(c), _ptr(d), _ptr(z), npix, K, D, _ptr(bg), float(sigma), float(gamma),
                          float(znear), float(zfar), _ptr(g), _ptr(gc), _ptr(gd), _ptr(gz))
     return gc, gd, gz
+
+
+PHONG_PARAMS = ("light_location", "camera_position", "ambient", "diffuse", "specular", "shininess")
+
+
+def phong_params(light_location, camera_position, ambient, diffuse, specular, shininess):
+    """The 16 lighting numbers of steps 18-21: L, C, ambient, diffuse, specular colours, shininess."""
+    return np.concatenate([np.asarray(x, np.float64).reshape(-1) for x in
+                           (light_location, camera_position, ambient, diffuse, specular, [shininess])])
+
+
+def phong_fwd(points, normals, albedo, params):
+    """Step 18 at M points: (colours M x 3, flags M: |cos| < 1e-6)."""
+    lib = _load()
+    P, N, c = (_c(x, np.float64).reshape(-1, 3) for x in (points, normals, albedo))
+    prm = _c(params, np.float64)
+    out = np.empty(P.shape, np.float64)
+    flags = np.empty(P.shape[0], np.uint8)
+    lib.oracle_phong_fwd(_ptr(P), _ptr(N), _ptr(c), P.shape[0], _ptr(prm), _ptr(out), _ptr(flags))
+    return out, flags.astype(bool)
+
+
+def phong_bwd(points, normals, albedo, params, grad):
+    """Step 19: (grad_points, grad_normals, grad_albedo), each M x 3."""
+    lib = _load()
+    P, N, c, g = (_c(x, np.float64).reshape(-1, 3) for x in (points, normals, albedo, grad))
+    prm = _c(params, np.float64)
+    gP, gN, gc = (np.empty(P.shape, np.float64) for _ in range(3))
+    lib.oracle_phong_bwd(_ptr(P), _ptr(N), _ptr(c), P.shape[0], _ptr(prm), _ptr(g), _ptr(gP), _ptr(gN), _ptr(gc))
+    return gP, gN, gc
+
+
+def phong_shade_fwd(pix_to_face, bary, faces, points, normals, albedo, params):
+    """Step 20: per-slot Phong colours (p2f.shape + (3,)) and flags (p2f.shape)."""
+    lib = _load()
+    p2f = _c(pix_to_face, np.int64)
+    b = _c(bary, np.float64)
+    f = _c(faces, np.int64)
+    P, N, c = (_c(x, np.float64).reshape(-1, 3) for x in (points, normals, albedo))
+    prm = _c(params, np.float64)
+    K = p2f.shape[-1]
+    npix = p2f.size // K
+    out = np.empty(p2f.shape + (3,), np.float64)
+    flags = np.empty(p2f.shape, np.uint8)
+    lib.oracle_phong_shade_fwd(_ptr(p2f), _ptr(b), npix, K, _ptr(f), _ptr(P), _ptr(N), _ptr(c), _ptr(prm),
+                               _ptr(out), _ptr(flags))
+    return out, flags.astype(bool)
+
+
+def phong_shade_bwd(pix_to_face, bary, faces, points, normals, albedo, params, grad):
+    """Step 21: (grad_points, grad_normals, grad_albedo) per vertex and grad_bary."""
+    lib = _load()
+    p2f = _c(pix_to_face, np.int64)
+    b = _c(bary, np.float64)
+    f = _c(faces, np.int64)
+    P, N, c = (_c(x, np.float64).reshape(-1, 3) for x in (points, normals, albedo))
+    prm = _c(params, np.float64)
+    g = _c(grad, np.float64)
+    K = p2f.shape[-1]
+    npix = p2f.size // K
+    gP, gN, gc = (np.empty(P.shape, np.float64) for _ in range(3))
+    gb = np.empty(b.shape, np.float64)
+    lib.oracle_phong_shade_bwd(_ptr(p2f), _ptr(b), npix, K, _ptr(f), _ptr(P), _ptr(N), _ptr(c), P.shape[0],
+                               _ptr(prm), _ptr(g), _ptr(gP), _ptr(gN), _ptr(gc), _ptr(gb))
+    return gP, gN, gc, gb

@@ -31,8 +31,8 @@
  *  12. its gradient: dL/ddist_k = -dL/dalpha * prod_{j != k} (1 - p_j) * p_k (1 - p_k) / sigma.
  *  13. rasterizer backward: the chain rule through steps 3, 5, 7, 8 and 9 with the
  *      candidate set, the inside flag and the nearest edge held fixed.
- *  14-17. stage-two shading (attribute interpolation, soft RGB blend) and their
- *      gradients; see the section at the end of this file.
+ *  14-21. stage-two shading (attribute interpolation, soft RGB blend, Phong lighting)
+ *      and their gradients; see the two sections at the end of this file.
  *
  * Besides the outputs, the forward marks pixels whose integer result is decided by a
  * float64-vs-float32 rounding: (E1) two of the K+1 nearest candidates lie within 1e-6
@@ -600,4 +600,187 @@ void oracle_blend_bwd(const int64_t *p2f, const double *colors, const double *di
         }
     }
     free(rgb);
+}
+
+/* ------------------------------------------------------------------ stage two: Phong lighting */
+/*
+ * The Phong reflection model (the PyTorch3D paper names Gouraud and Phong shading and
+ * several lights and materials but prints no formula; this is the textbook model of
+ * Phong 1975 with one point light, written out).  At a surface point P with normal N,
+ * albedo c, light position L and camera position C (one params row of 16 numbers:
+ * L[3], C[3], ambient[3], diffuse[3], specular[3], shininess; each colour is the
+ * product of the light's and the material's colour):
+ *
+ *  18. n = N / |N|, l = (L - P) / |L - P|, v = (C - P) / |C - P|, cos = n . l,
+ *      r = 2 cos n - l (l mirrored about n), rv = r . v,
+ *      diffuse term  t_d = max(cos, 0),
+ *      specular term t_s = rv^shininess when cos > 0 and rv > 0, else 0,
+ *      colour = (ambient + diffuse t_d) * c + specular t_s   (per channel).
+ *      Gouraud shading evaluates this at the vertices and interpolates the colours
+ *      (step 14); Phong shading interpolates P, N and c per fragment (step 14) and
+ *      evaluates it there (step 20).
+ *  19. its gradient: the chain rule through step 18 with the two switches (cos > 0,
+ *      rv > 0) held; the normalisation x / |x| has Jacobian (I - x^ x^T) / |x|.
+ *  20. Phong shading of the K slots of each pixel: step 14 for P, N and c, then step 18;
+ *      empty slots give 0.  Its gradient (step 21) is step 19 followed by step 15 for
+ *      each of the three attributes; grad_bary sums the three.
+ *
+ * The specular term jumps where cos crosses 0 while rv > 0, so a point with
+ * |cos| < 1e-6 is flagged (its colour is decided by rounding).
+ */
+#define PHONG_MARGIN 1e-6
+
+typedef struct {
+    double n[3], l[3], v[3];
+    double ln, lv, lc;           /* |N|, |L - P|, |C - P| */
+    double cos, rv, td, ts, nv, lvd;
+    int lit, shiny;
+} phong_state;
+
+static double dot3(const double *a, const double *b) { return a[0] * b[0] + a[1] * b[1] + a[2] * b[2]; }
+
+static void phong_eval(const double *P, const double *N, const double *prm, phong_state *S) {
+    double dl[3], dv[3];
+    for (int e = 0; e < 3; ++e) {
+        dl[e] = prm[e] - P[e];
+        dv[e] = prm[3 + e] - P[e];
+    }
+    S->ln = sqrt(dot3(N, N));
+    S->lv = sqrt(dot3(dl, dl));
+    S->lc = sqrt(dot3(dv, dv));
+    for (int e = 0; e < 3; ++e) {
+        S->n[e] = N[e] / S->ln;
+        S->l[e] = dl[e] / S->lv;
+        S->v[e] = dv[e] / S->lc;
+    }
+    S->cos = dot3(S->n, S->l);
+    S->nv = dot3(S->n, S->v);
+    S->lvd = dot3(S->l, S->v);
+    S->rv = 2.0 * S->cos * S->nv - S->lvd;
+    S->lit = S->cos > 0.0;
+    S->shiny = S->lit && S->rv > 0.0;
+    S->td = S->lit ? S->cos : 0.0;
+    S->ts = S->shiny ? pow(S->rv, prm[15]) : 0.0;
+}
+
+/* Step 18 over M points (each row of P, N, c holds 3 numbers); flags may be NULL. */
+void oracle_phong_fwd(const double *P, const double *N, const double *c, int64_t M, const double *prm,
+                      double *out, uint8_t *flags) {
+    for (int64_t i = 0; i < M; ++i) {
+        phong_state S;
+        phong_eval(P + 3 * i, N + 3 * i, prm, &S);
+        for (int e = 0; e < 3; ++e) out[3 * i + e] = (prm[6 + e] + prm[9 + e] * S.td) * c[3 * i + e] + prm[12 + e] * S.ts;
+        if (flags) flags[i] = fabs(S.cos) < PHONG_MARGIN;
+    }
+}
+
+/* d x^ given d(x^) for x^ = x / |x|: (g - (g . x^) x^) / |x|. */
+static void unit_bwd(const double *xh, double len, const double *g, double *gx) {
+    double t = dot3(g, xh);
+    for (int e = 0; e < 3; ++e) gx[e] = (g[e] - t * xh[e]) / len;
+}
+
+/* Step 19 for one point: gP, gN, gc (3 each) from the colour gradient g. */
+static void phong_point_bwd(const double *P, const double *N, const double *c, const double *prm, const double *g,
+                            double *gP, double *gN, double *gc) {
+    phong_state S;
+    phong_eval(P, N, prm, &S);
+    double g_td = 0.0, g_ts = 0.0;
+    for (int e = 0; e < 3; ++e) {
+        gc[e] = g[e] * (prm[6 + e] + prm[9 + e] * S.td);
+        g_td += g[e] * prm[9 + e] * c[e];
+        g_ts += g[e] * prm[12 + e];
+    }
+    double g_cos = S.lit ? g_td : 0.0;
+    double g_rv = S.shiny ? g_ts * prm[15] * pow(S.rv, prm[15] - 1.0) : 0.0;
+    /* rv = 2 cos nv - lv */
+    g_cos += g_rv * 2.0 * S.nv;
+    double g_nv = g_rv * 2.0 * S.cos, g_lv = -g_rv;
+    double gn[3], gl[3], gv[3];
+    for (int e = 0; e < 3; ++e) {
+        gn[e] = g_cos * S.l[e] + g_nv * S.v[e];
+        gl[e] = g_cos * S.n[e] + g_lv * S.v[e];
+        gv[e] = g_nv * S.n[e] + g_lv * S.l[e];
+    }
+    double gdl[3], gdv[3];
+    unit_bwd(S.n, S.ln, gn, gN);
+    unit_bwd(S.l, S.lv, gl, gdl);
+    unit_bwd(S.v, S.lc, gv, gdv);
+    for (int e = 0; e < 3; ++e) gP[e] = -gdl[e] - gdv[e];
+}
+
+/* Step 19 over M points; each output (M x 3) may be NULL. */
+void oracle_phong_bwd(const double *P, const double *N, const double *c, int64_t M, const double *prm,
+                      const double *grad, double *gP, double *gN, double *gc) {
+    for (int64_t i = 0; i < M; ++i) {
+        double a[3], b[3], d[3];
+        phong_point_bwd(P + 3 * i, N + 3 * i, c + 3 * i, prm, grad + 3 * i, a, b, d);
+        for (int e = 0; e < 3; ++e) {
+            if (gP) gP[3 * i + e] = a[e];
+            if (gN) gN[3 * i + e] = b[e];
+            if (gc) gc[3 * i + e] = d[e];
+        }
+    }
+}
+
+/* One slot's interpolated P, N, c (step 14 with D = 3, three times). */
+static void slot_attributes(const int64_t *faces, int64_t f, const double *bary, const double *vP, const double *vN,
+                            const double *vc, double *P, double *N, double *c) {
+    for (int e = 0; e < 3; ++e) P[e] = N[e] = c[e] = 0.0;
+    for (int m = 0; m < 3; ++m) {
+        int64_t v = faces[3 * f + m];
+        for (int e = 0; e < 3; ++e) {
+            P[e] += bary[m] * vP[3 * v + e];
+            N[e] += bary[m] * vN[3 * v + e];
+            c[e] += bary[m] * vc[3 * v + e];
+        }
+    }
+}
+
+/* Step 20: colors (npix x K x 3); flags (npix x K) may be NULL. */
+void oracle_phong_shade_fwd(const int64_t *p2f, const double *bary, int64_t npix, int32_t K, const int64_t *faces,
+                            const double *vP, const double *vN, const double *vc, const double *prm, double *out,
+                            uint8_t *flags) {
+    for (int64_t s = 0; s < npix * K; ++s) {
+        int64_t f = p2f[s];
+        if (flags) flags[s] = 0;
+        if (f < 0) {
+            out[3 * s] = out[3 * s + 1] = out[3 * s + 2] = 0.0;
+            continue;
+        }
+        double P[3], N[3], c[3];
+        slot_attributes(faces, f, bary + 3 * s, vP, vN, vc, P, N, c);
+        oracle_phong_fwd(P, N, c, 1, prm, out + 3 * s, flags ? flags + s : NULL);
+    }
+}
+
+/* Step 21: gradients into the vertex attributes (V x 3 each, overwritten) and grad_bary
+ * (npix x K x 3, may be NULL). */
+void oracle_phong_shade_bwd(const int64_t *p2f, const double *bary, int64_t npix, int32_t K, const int64_t *faces,
+                            const double *vP, const double *vN, const double *vc, int64_t V, const double *prm,
+                            const double *grad, double *gvP, double *gvN, double *gvc, double *grad_bary) {
+    memset(gvP, 0, sizeof(double) * 3 * (size_t)V);
+    memset(gvN, 0, sizeof(double) * 3 * (size_t)V);
+    memset(gvc, 0, sizeof(double) * 3 * (size_t)V);
+    for (int64_t s = 0; s < npix * K; ++s) {
+        int64_t f = p2f[s];
+        if (f < 0) {
+            if (grad_bary) grad_bary[3 * s] = grad_bary[3 * s + 1] = grad_bary[3 * s + 2] = 0.0;
+            continue;
+        }
+        double P[3], N[3], c[3], gP[3], gN[3], gc[3];
+        slot_attributes(faces, f, bary + 3 * s, vP, vN, vc, P, N, c);
+        phong_point_bwd(P, N, c, prm, grad + 3 * s, gP, gN, gc);
+        for (int m = 0; m < 3; ++m) {
+            int64_t v = faces[3 * f + m];
+            double b = bary[3 * s + m], gb = 0.0;
+            for (int e = 0; e < 3; ++e) {
+                gvP[3 * v + e] += b * gP[e];
+                gvN[3 * v + e] += b * gN[e];
+                gvc[3 * v + e] += b * gc[e];
+                gb += vP[3 * v + e] * gP[e] + vN[3 * v + e] * gN[e] + vc[3 * v + e] * gc[e];
+            }
+            if (grad_bary) grad_bary[3 * s + m] = gb;
+        }
+    }
 }
