@@ -249,60 +249,91 @@ def combine_ranks(dev_ms: float, samples: float, pixels: float, device=None):
 
 # ----------------------------------------------------------------------------- shading row
 def shading_step_timing(mr, torch, dev, stream, batch, verts, faces, first, num, flush, args, hbm_peak, hbm_note):
-    """Gouraud RGB step on the same batch: stage one (no silhouette), interpolation of
-    per-vertex colours, soft RGB blend, and the backward of all three to vertex colours
-    and positions.  Timed like the main step (L2 flushed, CUDA events, stage timing)."""
+    """The two stage-two RGB steps on the same batch, each timed like the main step (L2
+    flushed, CUDA events, stage timing):
+
+    gouraud_rgb: stage one (no silhouette), Phong lighting at the vertices, interpolation
+        of the lit colours, soft RGB blend; backward of all of it to the world positions,
+        normals and albedo of the vertices and to the screen-space vertices.
+    phong_rgb: stage one, per-fragment Phong shading (interpolation of position, normal and
+        albedo fused with the lighting), soft RGB blend; backward likewise.
+    """
     from differentiable_mesh_rasterization_b200 import synthetic as syn
     w = batch.workload
-    vcol = torch.from_numpy(syn.random_grads((batch.verts.shape[0], 3), 11)).abs().clamp(max=1.0).to(dev)
+    V = batch.verts.shape[0]
+    P = torch.from_numpy(batch.world).to(dev)
+    N = torch.from_numpy(batch.normals).to(dev)
+    alb = torch.from_numpy(syn.random_grads((V, 3), 11)).abs().clamp(max=1.0).to(dev)
+    prm = mr.phong_params([1.0, 1.5, 3.0], [0.0, 0.0, 2.7], [0.1, 0.1, 0.15], [0.6, 0.55, 0.5], [0.3, 0.3, 0.3],
+                          32.0)
     bg = [1.0, 1.0, 1.0]
     kw = dict(sigma=w.sigma, gamma=1e-2, znear=1.0, zfar=10.0)
     g = torch.from_numpy(syn.random_grads((batch.N, w.H, w.W, 4), 12)).to(dev)
 
-    def step():
-        p2f, zbuf, bary, dists = mr.rasterize_fwd(verts, faces, first, num, w.H, w.W, w.blur_radius, w.K,
-                                                  w.perspective_correct)
+    def frags():
+        return mr.rasterize_fwd(verts, faces, first, num, w.H, w.W, w.blur_radius, w.K, w.perspective_correct)
+
+    def gouraud():
+        p2f, zbuf, bary, dists = frags()
+        vcol = mr.phong_fwd(P, N, alb, prm)
         col = mr.interpolate_fwd(p2f, bary, faces, vcol)
         mr.blend_fwd(p2f, col, dists, zbuf, bg, **kw)
         gcol, gd, gz = mr.blend_bwd(p2f, col, dists, zbuf, bg, grad_rgba=g, **kw)
-        _, gbary = mr.interpolate_bwd(p2f, bary, faces, vcol, gcol)
+        gvcol, gbary = mr.interpolate_bwd(p2f, bary, faces, vcol, gcol)
+        mr.phong_bwd(P, N, alb, prm, gvcol)
         mr.rasterize_bwd(verts, faces, p2f, w.perspective_correct, grad_zbuf=gz, grad_bary=gbary, grad_dists=gd)
 
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize(dev)
-    steps = max(3, args.steps // 5)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    mr.profile_read()
-    mr.profile_enable(True)
-    for k in range(steps):
-        flush.zero_()
-        starts[k].record(stream)
-        step()
-        ends[k].record(stream)
-    torch.cuda.synchronize(dev)
-    mr.profile_enable(False)
-    st = mr.profile_read()
-    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / steps
+    def phong():
+        p2f, zbuf, bary, dists = frags()
+        col = mr.phong_shade_fwd(p2f, bary, faces, P, N, alb, prm)
+        mr.blend_fwd(p2f, col, dists, zbuf, bg, **kw)
+        gcol, gd, gz = mr.blend_bwd(p2f, col, dists, zbuf, bg, grad_rgba=g, **kw)
+        _, _, _, gbary = mr.phong_shade_bwd(p2f, bary, faces, P, N, alb, prm, gcol)
+        mr.rasterize_bwd(verts, faces, p2f, w.perspective_correct, grad_zbuf=gz, grad_bary=gbary, grad_dists=gd)
+
     npix = batch.N * w.H * w.W
     K = w.K
-    # algorithmic bytes of the stage-two kernels (slot = K per pixel; colours D = 3)
+    # algorithmic bytes of the stage-two kernels (slot = K per pixel; colours D = 3): each
+    # per-slot input read once, each output written once; vertex gathers hit L2 and are
+    # not counted
     algo = {"interpolate_fwd": npix * K * (8 + 12 + 12), "blend_fwd": npix * (K * (8 + 12 + 4 + 4) + 16),
             "blend_bwd": npix * (K * (8 + 12 + 4 + 4) + 16 + K * (12 + 4 + 4)),
-            "interpolate_bwd": npix * K * (8 + 12 + 12 + 12)}
-    stages = {}
-    for name, (t, n) in st.items():
-        if n:
-            ent = {"ms_per_step": t / steps}
-            if name in algo:
-                ent["hbm_frac"] = algo[name] / (t / steps / 1e3) / 1e9 / hbm_peak
-            stages[name] = ent
-    return {"ms_per_step": ms, "samples_per_s": float(count_samples(batch)) / (ms / 1e3),
-            "mpix_per_s": npix / (ms / 1e3) / 1e6, "steps": steps, "stages": stages,
-            "hbm_peak_note": hbm_note,
-            "note": "Gouraud: stage one + per-vertex colour interpolation + soft RGB blend (gamma 1e-2), fwd+bwd "
-                    "to vertex colours and positions; same workload, L2 flushed per step"}
+            "interpolate_bwd": npix * K * (8 + 12 + 12 + 12),
+            "phong_shade_fwd": npix * K * (8 + 12 + 12), "phong_shade_bwd": npix * K * (8 + 12 + 12 + 12)}
+
+    def timed(step, note):
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize(dev)
+        steps = max(3, args.steps // 5)
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        mr.profile_read()
+        mr.profile_enable(True)
+        for k in range(steps):
+            flush.zero_()
+            starts[k].record(stream)
+            step()
+            ends[k].record(stream)
+        torch.cuda.synchronize(dev)
+        mr.profile_enable(False)
+        st = mr.profile_read()
+        ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / steps
+        stages = {}
+        for name, (t, n) in st.items():
+            if n:
+                ent = {"ms_per_step": t / steps}
+                if name in algo:
+                    ent["hbm_frac"] = algo[name] / (t / steps / 1e3) / 1e9 / hbm_peak
+                stages[name] = ent
+        return {"ms_per_step": ms, "samples_per_s": float(count_samples(batch)) / (ms / 1e3),
+                "mpix_per_s": npix / (ms / 1e3) / 1e6, "steps": steps, "stages": stages,
+                "hbm_peak_note": hbm_note, "note": note + "; same workload, L2 flushed per step"}
+
+    return {"gouraud_rgb": timed(gouraud, "Gouraud: stage one + Phong lighting at the vertices + colour "
+                                          "interpolation + soft RGB blend (gamma 1e-2), fwd+bwd"),
+            "phong_rgb": timed(phong, "Phong: stage one + per-fragment interpolation and lighting (fused) + "
+                                      "soft RGB blend (gamma 1e-2), fwd+bwd")}
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -315,7 +346,7 @@ def main():
     ap.add_argument("--config", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--no-shading", action="store_true", help="skip the Gouraud RGB measurement")
+    ap.add_argument("--no-shading", action="store_true", help="skip the Gouraud and Phong RGB measurements")
     ap.add_argument("--images", type=int, default=None,
                     help="render only the first N meshes of the batch (small profiling case)")
     args = ap.parse_args()
@@ -475,8 +506,8 @@ def main():
             "clocks": clk}
 
     if not args.no_shading:
-        line["next_rows"] = {"gouraud_rgb": shading_step_timing(mr, torch, dev, stream, batch, verts, faces, first, num,
-                                                                flush, args, hbm_peak, hbm_note)}
+        line["next_rows"] = shading_step_timing(mr, torch, dev, stream, batch, verts, faces, first, num, flush,
+                                                args, hbm_peak, hbm_note)
 
     if rank == 0 and not args.no_cpu_baseline:
         import oracle

@@ -26,10 +26,11 @@ ERRORS = {-1: "invalid argument", -2: "out of memory", -3: "CUDA error", -4: "de
 EXPORTS = ("mr_rasterize_fwd", "mr_rasterize_silhouette_fwd", "mr_silhouette_blend_fwd",
            "mr_silhouette_blend_bwd", "mr_rasterize_bwd", "mr_silhouette_rasterize_bwd",
            "mr_device_status", "mr_last_error", "mr_version", "mr_profile_enable", "mr_profile_read",
-           "mr_rasterize_fwd_noalloc", "mr_interpolate_fwd", "mr_interpolate_bwd", "mr_blend_fwd", "mr_blend_bwd")
+           "mr_rasterize_fwd_noalloc", "mr_interpolate_fwd", "mr_interpolate_bwd", "mr_blend_fwd", "mr_blend_bwd",
+           "mr_phong_fwd", "mr_phong_bwd", "mr_phong_shade_fwd", "mr_phong_shade_bwd")
 STAGES = ("face_setup", "bin_count", "bin_scan", "bin_fill", "fine", "silhouette_fwd", "silhouette_bwd",
           "raster_bwd", "silhouette_raster_bwd", "epilogue", "interpolate_fwd", "interpolate_bwd", "blend_fwd",
-          "blend_bwd")
+          "blend_bwd", "phong_fwd", "phong_bwd", "phong_shade_fwd", "phong_shade_bwd")
 
 
 class MeshRastError(RuntimeError):
@@ -66,6 +67,10 @@ def load_library() -> ctypes.CDLL:
         "mr_interpolate_bwd": [P, P, i64, i32, P, i64, P, i64, i32, P, P, P, P],
         "mr_blend_fwd": [P, P, P, P, i64, i32, i32, P, f32, f32, f32, f32, P, P],
         "mr_blend_bwd": [P, P, P, P, i64, i32, i32, P, f32, f32, f32, f32, P, P, P, P, P],
+        "mr_phong_fwd": [P, P, P, i64, P, P, P],
+        "mr_phong_bwd": [P, P, P, i64, P, P, P, P, P, P],
+        "mr_phong_shade_fwd": [P, P, i64, i32, P, i64, P, P, P, i64, P, P, P],
+        "mr_phong_shade_bwd": [P, P, i64, i32, P, i64, P, P, P, i64, P, P, P, P, P, P, P],
         "mr_profile_enable": [i32],
         "mr_profile_read": [P, P, i32],
     }
@@ -286,6 +291,91 @@ def interpolate_bwd(pix_to_face, bary, faces, attr, grad_out):
                                                             _ptr(a), a.shape[0], D, _ptr(g), _ptr(ga), _ptr(gb),
                                                             _stream(p2f.device)))
     return ga, gb
+
+
+PHONG_NPARAMS = 16
+
+
+def phong_params(light_location, camera_position, ambient, diffuse, specular, shininess) -> np.ndarray:
+    """The 16 host floats of the lighting calls: L, C, ambient, diffuse, specular colours, shininess."""
+    prm = np.concatenate([np.asarray(x, np.float32).reshape(-1) for x in
+                          (light_location, camera_position, ambient, diffuse, specular, [shininess])])
+    if prm.shape[0] != PHONG_NPARAMS:
+        raise ValueError("light/camera positions and the three colours take 3 values each")
+    return np.ascontiguousarray(prm)
+
+
+def _points3(name, *ts):
+    out = [_dev(t, torch.float32, name) for t in ts]
+    if any(t.ndim != 2 or t.shape[1] != 3 or t.shape[0] != out[0].shape[0] for t in out):
+        raise ValueError(f"{name}: points, normals and albedo must all be (M, 3)")
+    return out
+
+
+def phong_fwd(points, normals, albedo, params):
+    """Phong lighting at M points (``mr_phong_fwd``) -> colours (M, 3)."""
+    lib = load_library()
+    P, N, c = _points3("phong_fwd", points, normals, albedo)
+    prm = np.ascontiguousarray(params, dtype=np.float32)
+    out = torch.empty_like(P)
+    with torch.cuda.device(P.device):
+        _check("mr_phong_fwd", lib.mr_phong_fwd(_ptr(P), _ptr(N), _ptr(c), P.shape[0], prm.ctypes.data, _ptr(out),
+                                                _stream(P.device)))
+    return out
+
+
+def phong_bwd(points, normals, albedo, params, grad_colors):
+    """Gradient of the lighting (``mr_phong_bwd``) -> (grad_points, grad_normals, grad_albedo)."""
+    lib = load_library()
+    P, N, c, g = _points3("phong_bwd", points, normals, albedo, grad_colors)
+    prm = np.ascontiguousarray(params, dtype=np.float32)
+    gP, gN, gc = (torch.empty_like(P) for _ in range(3))
+    with torch.cuda.device(P.device):
+        _check("mr_phong_bwd", lib.mr_phong_bwd(_ptr(P), _ptr(N), _ptr(c), P.shape[0], prm.ctypes.data, _ptr(g),
+                                                _ptr(gP), _ptr(gN), _ptr(gc), _stream(P.device)))
+    return gP, gN, gc
+
+
+def phong_shade_fwd(pix_to_face, bary, faces, points, normals, albedo, params):
+    """Per-fragment Phong shading (``mr_phong_shade_fwd``) -> colours (N, H, W, K, 3)."""
+    lib = load_library()
+    p2f = _dev(pix_to_face, torch.int64, "pix_to_face")
+    b = _dev(bary, torch.float32, "bary")
+    f = _dev(faces, torch.int64, "faces")
+    P, N, c = _points3("phong_shade_fwd", points, normals, albedo)
+    if tuple(b.shape) != tuple(p2f.shape) + (3,):
+        raise ValueError("bary must be pix_to_face.shape + (3,)")
+    prm = np.ascontiguousarray(params, dtype=np.float32)
+    K = p2f.shape[-1]
+    out = torch.empty(tuple(p2f.shape) + (3,), dtype=torch.float32, device=p2f.device)
+    with torch.cuda.device(p2f.device):
+        _check("mr_phong_shade_fwd", lib.mr_phong_shade_fwd(_ptr(p2f), _ptr(b), p2f.numel() // K, K, _ptr(f),
+                                                            f.shape[0], _ptr(P), _ptr(N), _ptr(c), P.shape[0],
+                                                            prm.ctypes.data, _ptr(out), _stream(p2f.device)))
+    return out
+
+
+def phong_shade_bwd(pix_to_face, bary, faces, points, normals, albedo, params, grad_colors):
+    """Gradient of the Phong shading (``mr_phong_shade_bwd``) ->
+    (grad_points, grad_normals, grad_albedo, grad_bary)."""
+    lib = load_library()
+    p2f = _dev(pix_to_face, torch.int64, "pix_to_face")
+    b = _dev(bary, torch.float32, "bary")
+    f = _dev(faces, torch.int64, "faces")
+    P, N, c = _points3("phong_shade_bwd", points, normals, albedo)
+    g = _dev(grad_colors, torch.float32, "grad_colors")
+    if tuple(b.shape) != tuple(p2f.shape) + (3,) or g.shape != b.shape:
+        raise ValueError("bary and grad_colors must be pix_to_face.shape + (3,)")
+    prm = np.ascontiguousarray(params, dtype=np.float32)
+    K = p2f.shape[-1]
+    gP, gN, gc = (torch.empty_like(P) for _ in range(3))
+    gb = torch.empty_like(b)
+    with torch.cuda.device(p2f.device):
+        _check("mr_phong_shade_bwd", lib.mr_phong_shade_bwd(_ptr(p2f), _ptr(b), p2f.numel() // K, K, _ptr(f),
+                                                            f.shape[0], _ptr(P), _ptr(N), _ptr(c), P.shape[0],
+                                                            prm.ctypes.data, _ptr(g), _ptr(gP), _ptr(gN), _ptr(gc),
+                                                            _ptr(gb), _stream(p2f.device)))
+    return gP, gN, gc, gb
 
 
 def _blend_args(pix_to_face, colors, dists, zbuf, background):

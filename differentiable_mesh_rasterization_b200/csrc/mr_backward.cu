@@ -32,116 +32,186 @@ __device__ __forceinline__ bool load_face(const int64_t* __restrict__ faces, int
     return vid[0] >= 0 && vid[0] < V && vid[1] >= 0 && vid[1] < V && vid[2] >= 0 && vid[2] < V;
 }
 
-// General backward: one thread per slot, float64 arithmetic; each of the face's vertices
-// receives one float4 (x, y, z, 0) atomic into a padded accumulator.
+// Chain rule of one slot's barycentric and depth outputs into its three vertices'
+// (x, y, z), in arithmetic type T.  r = vertex - pixel centre, w = the edge-function
+// weights C_k / A, invA = 1 / A; g[vertex][x, y, z] is added to.
+template <typename T, bool PERSP>
+__device__ __forceinline__ void bary_z_grad(const T (&rx)[3], const T (&ry)[3], const T (&w)[3], T invA,
+                                            const float (&x)[3], const float (&y)[3], const float (&z)[3],
+                                            const float (&gbar)[3], float gzz, float (&g)[3][3]) {
+    T gw[3];
+    if constexpr (PERSP) {
+        T u[3], S = 0;
+#pragma unroll
+        for (int e = 0; e < 3; ++e) { u[e] = w[e] / (T)z[e]; S += u[e]; }
+        const T iS = (T)1 / S;
+        const T dot = ((T)gbar[0] * u[0] + (T)gbar[1] * u[1] + (T)gbar[2] * u[2]) * iS;
+#pragma unroll
+        for (int e = 0; e < 3; ++e) {
+            const T gu = ((T)gbar[e] - dot) * iS - (T)gzz * iS * iS;
+            gw[e] = gu / (T)z[e];
+            g[e][2] -= (float)(gu * u[e] / (T)z[e]);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 3; ++e) {
+            gw[e] = (T)gzz * (T)z[e] + (T)gbar[e];
+            g[e][2] += (float)((T)gzz * w[e]);
+        }
+    }
+    const T G = gw[0] * w[0] + gw[1] * w[1] + gw[2] * w[2];
+    // d A / d vertex and sum_k gw_k d C_k / d vertex (C_k = cross of two rows of r)
+    const T dA[3][2] = {{(T)y[1] - (T)y[2], (T)x[2] - (T)x[1]}, {(T)y[2] - (T)y[0], (T)x[0] - (T)x[2]},
+                        {(T)y[0] - (T)y[1], (T)x[1] - (T)x[0]}};
+    const T dc[3][2] = {{gw[2] * ry[1] - gw[1] * ry[2], gw[1] * rx[2] - gw[2] * rx[1]},
+                        {gw[0] * ry[2] - gw[2] * ry[0], gw[2] * rx[0] - gw[0] * rx[2]},
+                        {gw[1] * ry[0] - gw[0] * ry[1], gw[0] * rx[1] - gw[1] * rx[0]}};
+#pragma unroll
+    for (int e = 0; e < 3; ++e) {
+        g[e][0] += (float)((dc[e][0] - G * dA[e][0]) * invA);
+        g[e][1] += (float)((dc[e][1] - G * dA[e][1]) * invA);
+    }
+}
+
+// One slot's contributions g[vertex][x, y, z] to its face's three vertices (x, y, z:
+// their screen-space coordinates), added to g; false for a degenerate face.  The distance part runs in float32 in face-local
+// coordinates (vertex minus pixel centre, the centre given as a double and as a float
+// pair; near-tied edges re-decided in float64), the barycentric and depth part in float64
+// (its terms scale with 1/A and cancel for slivers seen edge-on).
 template <bool PERSP>
-__global__ void k_raster_bwd(const float* __restrict__ verts, int64_t V, const int64_t* __restrict__ faces,
-                             int64_t F, const int64_t* __restrict__ p2f, int64_t nslots, int H, int W, int K,
-                             const float* __restrict__ gz, const float* __restrict__ gb,
-                             const float* __restrict__ gd, float4* __restrict__ acc, int* __restrict__ err) {
-    for (int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; s < nslots; s += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t f = p2f[s];
-        if (f == -1) continue;
-        if (f < -1 || f >= F) {
-            atomicOr(err, kErrSlotIndex);
-            continue;
-        }
-        int64_t vid[3];
-        if (!load_face(faces, V, f, vid)) {
-            atomicOr(err, kErrFaceIndex);
-            continue;
-        }
-        const int64_t pix = s / K;
-        const int64_t rem = pix % ((int64_t)H * W);
-        const int i = (int)(rem / W), j = (int)(rem % W);
-        const double px = -1.0 + (2.0 * j + 1.0) / W;
-        const double py = 1.0 - (2.0 * i + 1.0) / H;
-        double x[3], y[3], z[3];
+__device__ __forceinline__ bool slot_grad(const float (&x)[3], const float (&y)[3], const float (&z)[3], double pxd,
+                                          double pyd, float pxh, float pyh, float pxl, float pyl, int64_t s,
+                                          const float* __restrict__ gz, const float* __restrict__ gb,
+                                          const float* __restrict__ gd, float (&g)[3][3]) {
+    float rx[3], ry[3];
 #pragma unroll
-        for (int q = 0; q < 3; ++q) {
-            x[q] = verts[3 * vid[q]];
-            y[q] = verts[3 * vid[q] + 1];
-            z[q] = verts[3 * vid[q] + 2];
-        }
-        const double A = (x[1] - x[0]) * (y[2] - y[0]) - (y[1] - y[0]) * (x[2] - x[0]);
-        if (fabs(A) <= kDegenerateArea) continue;
-        double rx[3], ry[3];   // vertex - pixel
+    for (int e = 0; e < 3; ++e) {
+        rx[e] = (x[e] - pxh) - pxl;   // vertex - pixel centre
+        ry[e] = (y[e] - pyh) - pyl;
+    }
+    const double Ad = ((double)x[1] - x[0]) * ((double)y[2] - y[0]) - ((double)y[1] - y[0]) * ((double)x[2] - x[0]);
+    if (fabs(Ad) <= kDegenerateArea) return false;
+    // edge-function weights in float64: the barycentric chain below divides by A and
+    // cancels large terms for slivers seen edge-on, which float32 cannot carry
+    double rxd[3], ryd[3], wd[3];
 #pragma unroll
-        for (int q = 0; q < 3; ++q) { rx[q] = x[q] - px; ry[q] = y[q] - py; }
-        double w[3];
-        w[0] = (rx[1] * ry[2] - ry[1] * rx[2]) / A;
-        w[1] = (rx[2] * ry[0] - ry[2] * rx[0]) / A;
-        w[2] = (rx[0] * ry[1] - ry[0] * rx[1]) / A;
-        const bool inside = w[0] >= 0.0 && w[1] >= 0.0 && w[2] >= 0.0;
-        double g[3][3] = {{0, 0, 0}, {0, 0, 0}, {0, 0, 0}};   // [vertex][x, y, z]
-        if (gd) {
-            int eu = 0;
-            double best = DBL_MAX, bt = 0.0;
+    for (int e = 0; e < 3; ++e) { rxd[e] = x[e] - pxd; ryd[e] = y[e] - pyd; }
+    const double iAd = 1.0 / Ad;
+    wd[0] = (rxd[1] * ryd[2] - ryd[1] * rxd[2]) * iAd;
+    wd[1] = (rxd[2] * ryd[0] - ryd[2] * rxd[0]) * iAd;
+    wd[2] = (rxd[0] * ryd[1] - ryd[0] * rxd[1]) * iAd;
+    if (gd) {
+        const float gds = gd[s];
+        if (gds != 0.f) {
+            const bool inside = wd[0] >= 0.0 && wd[1] >= 0.0 && wd[2] >= 0.0;
+            int eu = 0, vbest = -1, vsecond = -2;   // nearest point's vertex (-1: inside an edge)
+            float best = FLT_MAX, second = FLT_MAX, bt = 0.f, bdx = 0.f, bdy = 0.f;
 #pragma unroll
-            for (int k = 0; k < 3; ++k) {
-                const int k1 = k == 2 ? 0 : k + 1;
-                const double ex = x[k1] - x[k], ey = y[k1] - y[k];
-                const double len2 = ex * ex + ey * ey;
-                double t = len2 > 0.0 ? ((px - x[k]) * ex + (py - y[k]) * ey) / len2 : 0.0;
-                t = fmin(fmax(t, 0.0), 1.0);
-                const double dx = px - (x[k] + t * ex), dy = py - (y[k] + t * ey);
-                const double d2 = dx * dx + dy * dy;
-                if (d2 < best) { best = d2; eu = k; bt = t; }
+            for (int e = 0; e < 3; ++e) {
+                const int e1 = e == 2 ? 0 : e + 1;
+                const float ex = x[e1] - x[e], ey = y[e1] - y[e];
+                const float ax = -rx[e], ay = -ry[e];        // pixel - edge start
+                const float len2 = fmaf(ex, ex, ey * ey);
+                const float t = len2 > 0.f ? __saturatef(fmaf(ax, ex, ay * ey) / len2) : 0.f;
+                const float dx = fmaf(-t, ex, ax), dy = fmaf(-t, ey, ay);   // pixel - nearest point
+                const float d2 = fmaf(dx, dx, dy * dy);
+                const int vtx = t == 0.f ? e : (t == 1.f ? e1 : -1 - e);
+                if (d2 < best) {
+                    second = best;
+                    vsecond = vbest;
+                    best = d2; eu = e; bt = t; bdx = dx; bdy = dy;
+                    vbest = vtx;
+                } else if (d2 < second) {
+                    second = d2;
+                    vsecond = vtx;
+                }
+            }
+            // Two edges almost equally near (the pixel sits on an angle bisector
+            // inside the face): float32 may pick the other edge than the exact
+            // distances do, and the two picks feed different vertices.  Decide
+            // such near-ties again in float64 (rare).  Two edges whose nearest
+            // point is the same shared vertex are no tie: both feed that vertex.
+            if (second - best <= 1e-5f * best && !(vbest >= 0 && vbest == vsecond)) {
+                double bd = DBL_MAX;
+#pragma unroll
+                for (int e = 0; e < 3; ++e) {
+                    const int e1 = e == 2 ? 0 : e + 1;
+                    const double ex = (double)x[e1] - x[e], ey = (double)y[e1] - y[e];
+                    const double ax = pxd - x[e], ay = pyd - y[e];
+                    const double len2 = ex * ex + ey * ey;
+                    double t = len2 > 0.0 ? (ax * ex + ay * ey) / len2 : 0.0;
+                    t = fmin(fmax(t, 0.0), 1.0);
+                    const double dx = ax - t * ex, dy = ay - t * ey;
+                    const double d2 = dx * dx + dy * dy;
+                    if (d2 < bd) { bd = d2; eu = e; bt = (float)t; bdx = (float)dx; bdy = (float)dy; }
+                }
             }
             const int ev = eu == 2 ? 0 : eu + 1;
-            const double gdist = (double)gd[s] * (inside ? -1.0 : 1.0);
-            const double qx = x[eu] + bt * (x[ev] - x[eu]), qy = y[eu] + bt * (y[ev] - y[eu]);
-            const double dx = px - qx, dy = py - qy;
-            g[eu][0] += gdist * (-2.0 * dx * (1.0 - bt));
-            g[eu][1] += gdist * (-2.0 * dy * (1.0 - bt));
-            g[ev][0] += gdist * (-2.0 * dx * bt);
-            g[ev][1] += gdist * (-2.0 * dy * bt);
+            const float gdist = inside ? -gds : gds;
+            const float su = -2.f * gdist * (1.f - bt), sv = -2.f * gdist * bt;
+            g[eu][0] += su * bdx;
+            g[eu][1] += su * bdy;
+            g[ev][0] += sv * bdx;
+            g[ev][1] += sv * bdy;
         }
-        if (gb || gz) {
-            double gbar[3] = {0, 0, 0};
-            if (gb) { gbar[0] = gb[3 * s]; gbar[1] = gb[3 * s + 1]; gbar[2] = gb[3 * s + 2]; }
-            const double gzz = gz ? (double)gz[s] : 0.0;
-            double gw[3];
-            if (PERSP) {
-                double u[3], S = 0.0;
+    }
+    if (gb || gz) {
+        float gbar[3] = {0.f, 0.f, 0.f};
+        if (gb) { gbar[0] = gb[3 * s]; gbar[1] = gb[3 * s + 1]; gbar[2] = gb[3 * s + 2]; }
+        const float gzz = gz ? gz[s] : 0.f;
+        bary_z_grad<double, PERSP>(rxd, ryd, wd, iAd, x, y, z, gbar, gzz, g);
+    }
+    return true;
+}
+
+// General backward: one thread per pixel, its K slots in turn; each valid slot's
+// contributions (slot_grad) go out as one float4 atomic per vertex into a padded
+// (x, y, z, 0) accumulator.  Measured alternatives that lost on this scatter: summing
+// equal vertex ids within a pixel, or along a run of lanes, before the atomics; issuing
+// the K slots' gathers phase by phase (more registers, fewer resident warps); packing the
+// valid slots of a warp's pixels into a shared-memory queue so that no lane idles.
+template <int KC, bool PERSP>
+__global__ void __launch_bounds__(256)
+k_raster_bwd(const float* __restrict__ verts, int64_t V, const int64_t* __restrict__ faces, int64_t F,
+             const int64_t* __restrict__ p2f, int64_t npix, int H, int W, int K, const float* __restrict__ gz,
+             const float* __restrict__ gb, const float* __restrict__ gd, float4* __restrict__ acc,
+             int* __restrict__ err) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < npix; q += stride) {
+        const int64_t rem = q % ((int64_t)H * W);
+        const int i = (int)(rem / W), j = (int)(rem % W);
+        const double pxd = -1.0 + (2.0 * j + 1.0) / W, pyd = 1.0 - (2.0 * i + 1.0) / H;
+        const float pxh = (float)pxd, pyh = (float)pyd;
+        const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
 #pragma unroll
-                for (int k = 0; k < 3; ++k) { u[k] = w[k] / z[k]; S += u[k]; }
-                double bar[3] = {u[0] / S, u[1] / S, u[2] / S};
-                const double zz = 1.0 / S;
-                const double dot = gbar[0] * bar[0] + gbar[1] * bar[1] + gbar[2] * bar[2];
-#pragma unroll
-                for (int k = 0; k < 3; ++k) {
-                    const double gu = (gbar[k] - dot) / S - gzz * zz * zz;
-                    gw[k] = gu / z[k];
-                    g[k][2] += -gu * u[k] / z[k];
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < 3; ++k) {
-                    gw[k] = gbar[k] + gzz * z[k];
-                    g[k][2] += gzz * w[k];
-                }
+        for (int k = 0; k < KC; ++k) {
+            if (k >= K) break;
+            const int64_t s = q * K + k;
+            const int64_t f = p2f[s];
+            if (f == -1) continue;
+            if (f < -1 || f >= F) {
+                atomicOr(err, kErrSlotIndex);
+                continue;
             }
-            const double G = gw[0] * w[0] + gw[1] * w[1] + gw[2] * w[2];
-            const double dA[3][2] = {{y[1] - y[2], x[2] - x[1]}, {y[2] - y[0], x[0] - x[2]}, {y[0] - y[1], x[1] - x[0]}};
-            // sum_k gw_k dC_k / d(vertex)
-            double dc[3][2];
-            dc[0][0] = gw[1] * (-ry[2]) + gw[2] * (ry[1]);
-            dc[0][1] = gw[1] * (rx[2]) + gw[2] * (-rx[1]);
-            dc[1][0] = gw[0] * (ry[2]) + gw[2] * (-ry[0]);
-            dc[1][1] = gw[0] * (-rx[2]) + gw[2] * (rx[0]);
-            dc[2][0] = gw[0] * (-ry[1]) + gw[1] * (ry[0]);
-            dc[2][1] = gw[0] * (rx[1]) + gw[1] * (-rx[0]);
-#pragma unroll
-            for (int q = 0; q < 3; ++q) {
-                g[q][0] += (dc[q][0] - G * dA[q][0]) / A;
-                g[q][1] += (dc[q][1] - G * dA[q][1]) / A;
+            int64_t vid[3];
+            if (!load_face(faces, V, f, vid)) {
+                atomicOr(err, kErrFaceIndex);
+                continue;
             }
+            float x[3], y[3], z[3];
+#pragma unroll
+            for (int e = 0; e < 3; ++e) {
+                x[e] = verts[3 * vid[e]];
+                y[e] = verts[3 * vid[e] + 1];
+                z[e] = verts[3 * vid[e] + 2];
+            }
+            float g[3][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};   // [vertex][x, y, z]
+            if (!slot_grad<PERSP>(x, y, z, pxd, pyd, pxh, pyh, pxl, pyl, s, gz, gb, gd, g)) continue;
+#pragma unroll
+            for (int e = 0; e < 3; ++e)
+                if (g[e][0] != 0.f || g[e][1] != 0.f || g[e][2] != 0.f)
+                    atomicAdd(acc + vid[e], make_float4(g[e][0], g[e][1], g[e][2], 0.f));
         }
-#pragma unroll
-        for (int q = 0; q < 3; ++q)
-            if (g[q][0] != 0.0 || g[q][1] != 0.0 || g[q][2] != 0.0)
-                atomicAdd(acc + vid[q], make_float4((float)g[q][0], (float)g[q][1], (float)g[q][2], 0.f));
     }
 }
 
@@ -291,7 +361,6 @@ int validate_bwd(const float* verts, int64_t V, const int64_t* faces, int64_t F,
     return MR_OK;
 }
 
-inline int grid_for(int64_t n) { return (int)std::min<int64_t>((n + 255) / 256, 148 * 32); }
 
 }  // namespace
 }  // namespace mr
@@ -320,14 +389,26 @@ int mr_rasterize_bwd(const float* verts, int64_t V, const int64_t* faces, int64_
     if (rc != MR_OK) return rc;
     cudaError_t e = cudaMemsetAsync(acc, 0, sizeof(float4) * (size_t)V, s);
     if (e == cudaSuccess) {
-        const int g = mr::grid_for(nslots);
+        const int64_t npix = (int64_t)N * H * W;
+        const int g = mr::grid_for(npix);
         mr::ProfScope ps(MR_STAGE_RASTER_BWD, s);
-        if (perspective_correct)
-            mr::k_raster_bwd<true><<<g, 256, 0, s>>>(verts, V, faces, F, pix_to_face, nslots, H, W, K, grad_zbuf,
-                                                     grad_bary, grad_dists, acc, err);
-        else
-            mr::k_raster_bwd<false><<<g, 256, 0, s>>>(verts, V, faces, F, pix_to_face, nslots, H, W, K, grad_zbuf,
-                                                      grad_bary, grad_dists, acc, err);
+#define MR_RB(KC, PC)                                                                                           \
+    mr::k_raster_bwd<KC, PC><<<g, 256, 0, s>>>(verts, V, faces, F, pix_to_face, npix, H, W, K, grad_zbuf, grad_bary, \
+                                               grad_dists, acc, err)
+#define MR_RB_K(PC)               \
+    if (K <= 1) MR_RB(1, PC);     \
+    else if (K <= 2) MR_RB(2, PC); \
+    else if (K <= 4) MR_RB(4, PC); \
+    else if (K <= 8) MR_RB(8, PC); \
+    else if (K <= 16) MR_RB(16, PC); \
+    else MR_RB(32, PC)
+        if (perspective_correct) {
+            MR_RB_K(true);
+        } else {
+            MR_RB_K(false);
+        }
+#undef MR_RB_K
+#undef MR_RB
         mr::k_xyzw_to_xyz<<<mr::grid_for(V), 256, 0, s>>>(acc, V, grad_verts);
         e = cudaGetLastError();
     }

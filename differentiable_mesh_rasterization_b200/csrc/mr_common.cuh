@@ -52,6 +52,10 @@ int cuda_fail(cudaError_t e, const char* what);
 int scratch_alloc(void** p, size_t bytes, cudaStream_t s);
 void scratch_free(void* p, cudaStream_t s);
 
+// Grid of 256-thread blocks for a grid-stride loop over n items: at most 32 blocks per
+// SM of the 148.
+inline int grid_for(int64_t n) { return (int)(n < 148 * 32 * 256 ? (n + 255) / 256 : 148 * 32); }
+
 // Device-wide sticky error word (asynchronous kernels).
 int* device_error_word();
 

@@ -211,7 +211,6 @@ __global__ void k_blend_bwd(const int64_t* __restrict__ p2f, const float* __rest
     }
 }
 
-inline int grid_for(int64_t n) { return (int)std::min<int64_t>((n + 255) / 256, 148 * 32); }
 
 int check_blend(int64_t npix, int K, int D, float sigma, float gamma, float znear, float zfar) {
     if (npix < 0 || K < 1 || K > MR_KMAX || D < 1 || D > MR_BLEND_DMAX) {

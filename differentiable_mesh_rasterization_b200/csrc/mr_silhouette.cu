@@ -67,7 +67,6 @@ int validate(int32_t N, int32_t H, int32_t W, int32_t K, float sigma, const void
     return MR_OK;
 }
 
-inline int grid_for(int64_t n) { return (int)std::min<int64_t>((n + 255) / 256, 148 * 32); }
 
 }  // namespace
 }  // namespace mr

@@ -204,6 +204,47 @@ int mr_blend_bwd(const int64_t* pix_to_face, const float* colors, const float* d
                  float sigma, float gamma, float znear, float zfar, const float* grad_rgba,
                  float* grad_colors, float* grad_dists, float* grad_zbuf, void* stream);
 
+/*
+ * Phong lighting (PyTorch3D paper, "Accelerating 3D Deep Learning with PyTorch3D", method:
+ * Gouraud and Phong shaders with several lights and materials; the pages print no formula,
+ * so this is the textbook Phong reflection model with one point light).  params: 16 floats
+ * (HOST) = light position L[3], camera position C[3], ambient[3], diffuse[3], specular[3]
+ * (each the product of the light's and the material's colour), shininess (>= 1).  At a point
+ * P with normal N (any length > 0) and albedo c:
+ *   n = N/|N|, l = (L-P)/|L-P|, v = (C-P)/|C-P|, cos = n.l, rv = (2 cos n - l).v,
+ *   colour = (ambient + diffuse max(cos, 0)) c + specular [cos > 0 and rv > 0] rv^shininess.
+ * Gouraud shading lights the vertices (mr_phong_fwd with M = V) and interpolates the colours
+ * with mr_interpolate_fwd; Phong shading lights every fragment (mr_phong_shade_fwd).
+ *
+ * mr_phong_fwd: colors (M x 3) at M points; points, normals, albedo: M x 3 float32 (device).
+ * mr_phong_bwd: grad_points, grad_normals, grad_albedo (M x 3 each, may be NULL) from
+ *   grad_colors (M x 3); the two switches are held fixed.
+ * mr_phong_shade_fwd: per slot of npix pixels x K, interpolates P, N and c from the face's
+ *   vertices (points, normals, albedo: V x 3) with bary, then lights them: colors
+ *   (npix x K x 3), 0 for empty slots.  One pass; the interpolated attributes never reach
+ *   memory.
+ * mr_phong_shade_bwd: grad_points, grad_normals, grad_albedo (V x 3 each, overwritten;
+ *   float32 atomics) and grad_bary (npix x K x 3, may be NULL) from grad_colors.
+ * Errors: MR_ERR_ARG for negative sizes, K outside [1, MR_KMAX], a NULL required pointer,
+ * non-finite params or shininess < 1; out-of-range face or vertex ids are flagged in the
+ * device error word (mr_device_status) and the slot is skipped.
+ */
+#define MR_PHONG_NPARAMS 16
+int mr_phong_fwd(const float* points, const float* normals, const float* albedo, int64_t M,
+                 const float* params, float* colors, void* stream);
+int mr_phong_bwd(const float* points, const float* normals, const float* albedo, int64_t M,
+                 const float* params, const float* grad_colors, float* grad_points,
+                 float* grad_normals, float* grad_albedo, void* stream);
+int mr_phong_shade_fwd(const int64_t* pix_to_face, const float* bary, int64_t npix, int32_t K,
+                       const int64_t* faces, int64_t F, const float* points, const float* normals,
+                       const float* albedo, int64_t V, const float* params, float* colors,
+                       void* stream);
+int mr_phong_shade_bwd(const int64_t* pix_to_face, const float* bary, int64_t npix, int32_t K,
+                       const int64_t* faces, int64_t F, const float* points, const float* normals,
+                       const float* albedo, int64_t V, const float* params, const float* grad_colors,
+                       float* grad_points, float* grad_normals, float* grad_albedo, float* grad_bary,
+                       void* stream);
+
 /* Synchronises `stream`, then returns MR_ERR_DEVICE (and clears the word) if any
  * asynchronous kernel of this library flagged an out-of-range index on the current
  * device since the last call, else MR_OK (or MR_ERR_CUDA). */
@@ -237,7 +278,11 @@ int mr_version(void);
 #define MR_STAGE_INTERPOLATE_BWD 11
 #define MR_STAGE_BLEND_FWD 12
 #define MR_STAGE_BLEND_BWD 13
-#define MR_NUM_STAGES 14
+#define MR_STAGE_PHONG_FWD 14
+#define MR_STAGE_PHONG_BWD 15
+#define MR_STAGE_PHONG_SHADE_FWD 16
+#define MR_STAGE_PHONG_SHADE_BWD 17
+#define MR_NUM_STAGES 18
 int mr_profile_enable(int32_t on);
 int mr_profile_read(double* stage_ms, int64_t* launches, int32_t nstages);
 

@@ -109,3 +109,182 @@ def test_gouraud_render_end_to_end(oracle_mod):
     assert keep.mean() > 0.75
     compare_grad(np_(gvcol)[keep], ovcol[keep], label="grad vertex colours")
     compare_grad(np_(gv)[keep], ogv[keep], label="grad vertices")
+
+
+LIGHT = dict(light_location=[1.0, 1.5, 3.0], camera_position=[0.0, 0.0, 2.7], ambient=[0.1, 0.1, 0.15],
+             diffuse=[0.6, 0.55, 0.5], specular=[0.3, 0.3, 0.3])
+
+
+def _params(shininess):
+    return mr.phong_params(shininess=shininess, **LIGHT)
+
+
+def _light_tol(shininess):
+    """Float32 rounding allowance of the lighting of one point: the attributes (below 2 in
+    magnitude) are rounded once after interpolation, and the lighting magnifies an
+    attribute error by at most about 1 + shininess (the specular power's slope)."""
+    return 4.0 * (1.0 + shininess) * 2.0 ** -23
+
+
+def _rounding_allowance(oracle_mod, p2f, bary, faces, vP, vN, vc, prm64, g):
+    """What rounding the interpolated position, normal and albedo to float32 changes in the
+    oracle's own lighting and gradient, slot by slot; spread to the vertices like the
+    gradient itself (sum over slots of |b_m| |change|) and to grad_bary (sum over the
+    attributes of |attr_m| . |change|).
+
+    The CUDA path interpolates exactly and rounds once to float32 there.  Where the
+    lighting is ill-conditioned (a blur-ring point extrapolated with barycentrics of
+    magnitude ~40 to within a few hundredths of the camera or the light), that rounding
+    alone moves the result beyond the relative tolerance.  Returns (per-slot colour
+    change, [per-vertex change of grad P, N, c], per-slot change of grad_bary)."""
+    valid = p2f >= 0
+    b32 = np.asarray(bary, np.float32)
+    X = [oracle_mod.interpolate_fwd(p2f, bary, faces, a)[valid] for a in (vP, vN, vc)]
+    R = [oracle_mod.interpolate_fwd(p2f, b32, faces, a)[valid].astype(np.float32) for a in (vP, vN, vc)]
+    gv = np.asarray(g, np.float64)[valid]
+    col = np.zeros(p2f.shape + (3,))
+    col[valid] = np.abs(oracle_mod.phong_fwd(*X, prm64)[0] - oracle_mod.phong_fwd(*R, prm64)[0])
+    zeros = np.zeros((np.asarray(vP).shape[0], 3))
+    f = np.asarray(faces)[np.where(valid, p2f, 0)]
+    per_vertex, gb = [], np.zeros(p2f.shape + (3,))
+    for attr, a, r in zip((vP, vN, vc), oracle_mod.phong_bwd(*X, prm64, gv), oracle_mod.phong_bwd(*R, prm64, gv)):
+        sp = np.zeros(p2f.shape + (3,))
+        sp[valid] = np.abs(a - r)
+        per_vertex.append(oracle_mod.interpolate_bwd(p2f, np.abs(bary), faces, zeros, sp)[0])
+        gb += (np.abs(np.asarray(attr, np.float64)[f]) * sp[..., None, :]).sum(-1)
+    gb[~valid] = 0.0
+    return col, per_vertex, gb
+
+
+@pytest.mark.parametrize("shininess", [8.0, 64.0])
+def test_phong_lighting_matches_oracle(oracle_mod, shininess):
+    rng = np.random.default_rng(3)
+    M = 100_003
+    P = rng.uniform(-1, 1, size=(M, 3)).astype(np.float32)
+    N = rng.normal(size=(M, 3)).astype(np.float32)
+    c = rng.uniform(size=(M, 3)).astype(np.float32)
+    prm = _params(shininess)
+    got = np_(mr.phong_fwd(cuda(P), cuda(N), cuda(c), prm))
+    want, flags = oracle_mod.phong_fwd(P, N, c, prm.astype(np.float64))
+    ok = ~flags
+    err = np.abs(got[ok] - want[ok]) - (1e-4 * np.abs(want[ok]) + 1e-6)
+    assert err.max() <= 0, f"colours off by {err.max():.3g} beyond tolerance"
+    g = rng.normal(size=(M, 3)).astype(np.float32)
+    gP, gN, gc = mr.phong_bwd(cuda(P), cuda(N), cuda(c), prm, cuda(g))
+    wP, wN, wc = oracle_mod.phong_bwd(P, N, c, prm.astype(np.float64), g)
+    compare_grad(np_(gP)[ok], wP[ok], label="grad_points")
+    compare_grad(np_(gN)[ok], wN[ok], label="grad_normals")
+    compare_grad(np_(gc)[ok], wc[ok], label="grad_albedo")
+
+
+def test_phong_shading_matches_oracle(oracle_mod, frags):
+    b, p2f, zbuf, bary, dists, _ = frags
+    rng = np.random.default_rng(4)
+    alb = rng.uniform(size=(b.verts.shape[0], 3)).astype(np.float32)
+    prm = _params(16.0)
+    args = (b.world, b.normals, alb)
+    got = np_(mr.phong_shade_fwd(cuda(p2f), cuda(bary), cuda(b.faces), *(cuda(a) for a in args), prm))
+    want, flags = oracle_mod.phong_shade_fwd(p2f, bary, b.faces, *args, prm.astype(np.float64))
+    ok = ~flags
+    assert ok.mean() > 0.99
+    g = rng.normal(size=want.shape).astype(np.float32)
+    g[flags] = 0.0          # a flagged slot's switch is decided by rounding: no gradient through it
+    col_a, vert_a, gb_a = _rounding_allowance(oracle_mod, p2f, bary, b.faces, *args, prm.astype(np.float64), g)
+    tol = 1e-4 * np.abs(want) + 1e-6 + _light_tol(16.0) + 4.0 * col_a
+    err = (np.abs(got - want) - tol)[ok]
+    assert err.max() <= 0, f"colours off by {err.max():.3g} beyond tolerance"
+    assert np.all(got[p2f < 0] == 0)
+    outs = mr.phong_shade_bwd(cuda(p2f), cuda(bary), cuda(b.faces), *(cuda(a) for a in args), prm, cuda(g))
+    wants = oracle_mod.phong_shade_bwd(p2f, bary, b.faces, *args, prm.astype(np.float64), g)
+    for name, x, y, a in zip(("grad_points", "grad_normals", "grad_albedo", "grad_bary"), outs, wants,
+                             vert_a + [gb_a]):
+        compare_grad(x, y, label=name, extra=4.0 * a)
+
+
+def test_phong_render_end_to_end(oracle_mod):
+    """verts -> fragments -> per-fragment Phong colours -> soft RGB blend -> loss and back to
+    the world positions, normals and albedo, and to the screen-space vertices."""
+    b = syn.make_batch(2)
+    w = b.workload
+    rng = np.random.default_rng(5)
+    alb = rng.uniform(size=(b.verts.shape[0], 3)).astype(np.float32)
+    prm = _params(32.0)
+    bg = np.array([0.0, 0.0, 0.0], np.float32)
+    kw = dict(sigma=1e-4, gamma=1e-2, znear=1.0, zfar=10.0)
+    v, f = cuda(b.verts), cuda(b.faces)
+    P, N, A = cuda(b.world), cuda(b.normals), cuda(alb)
+    p2f, zbuf, bary, dists = mr.rasterize_fwd(v, f, b.mesh_to_face_first_idx, b.num_faces_per_mesh, w.H, w.W,
+                                              w.blur_radius, w.K)
+    col = mr.phong_shade_fwd(p2f, bary, f, P, N, A, prm)
+    rgba = mr.blend_fwd(p2f, col, dists, zbuf, bg, **kw)
+    g = syn.random_grads(tuple(rgba.shape), 8)
+    gcol, gd, gz = mr.blend_bwd(p2f, col, dists, zbuf, bg, grad_rgba=cuda(g), **kw)
+    gP, gN, gA, gbary = mr.phong_shade_bwd(p2f, bary, f, P, N, A, prm, gcol)
+    gv = mr.rasterize_bwd(v, f, p2f, False, grad_zbuf=gz, grad_bary=gbary, grad_dists=gd)
+    mr.device_status()
+
+    o = oracle_mod.rasterize_fwd(b.verts, b.faces, b.mesh_to_face_first_idx, b.num_faces_per_mesh, w.H, w.W,
+                                 np.float32(w.blur_radius), w.K, False)
+    op2f, oz, ob, od, ex = o
+    prm64 = prm.astype(np.float64)
+    ocol, oflags = oracle_mod.phong_shade_fwd(op2f, ob, b.faces, b.world, b.normals, alb, prm64)
+    orgba = oracle_mod.blend_fwd(op2f, ocol, od, oz, bg, **kw)
+    ok = (ex == 0) & ~oflags.any(-1)
+    oc, odd, ozz = oracle_mod.blend_bwd(op2f, ocol, od, oz, bg, grad_rgba=g, **kw)
+    col_a, vert_a, gb_a = _rounding_allowance(oracle_mod, op2f, ob, b.faces, b.world, b.normals, alb, prm64, oc)
+    extra = 4.0 * col_a.max(axis=(-2, -1))[..., None]
+    err = (np.abs(np_(rgba) - orgba) - (1e-4 * np.abs(orgba) + 1e-5 + _light_tol(32.0) + extra))[ok]
+    assert err.max() <= 0, f"rgba off by {err.max():.3g}"
+    oP, oN, oA, obary = oracle_mod.phong_shade_bwd(op2f, ob, b.faces, b.world, b.normals, alb, prm64, oc)
+    ogv = oracle_mod.rasterize_bwd(b.verts, b.faces, op2f, False, grad_zbuf=ozz, grad_bary=obary, grad_dists=odd)
+    fs = np.unique(np.concatenate([op2f[~ok].reshape(-1), np_(p2f)[~ok].reshape(-1)]))
+    keep = np.ones(b.verts.shape[0], bool)
+    fs = fs[fs >= 0]
+    keep[b.faces[fs].reshape(-1)] = False
+    assert keep.mean() > 0.75
+    for name, x, y, a in (("grad points", gP, oP, vert_a[0]), ("grad normals", gN, oN, vert_a[1]),
+                          ("grad albedo", gA, oA, vert_a[2])):
+        compare_grad(np_(x)[keep], y[keep], label=name, extra=4.0 * a[keep])
+    # grad_bary of the ill-conditioned slots (see _rounding_allowance) reaches the screen
+    # vertices through 1/area factors: their faces' vertices are left out there
+    ill = gb_a.max(-1) > 1e-4 * np.sqrt(np.mean(obary ** 2))
+    keep_v = keep.copy()
+    keep_v[b.faces[np.unique(op2f[ill])].reshape(-1)] = False
+    assert keep_v.mean() > 0.75
+    compare_grad(np_(gv)[keep_v], ogv[keep_v], label="grad vertices")
+
+
+def test_gouraud_lighting_at_vertices_end_to_end(oracle_mod):
+    """Gouraud shading with lighting: Phong at the vertices, then interpolation and blend."""
+    b = syn.make_batch(2, n_meshes=4)
+    w = b.workload
+    rng = np.random.default_rng(6)
+    alb = rng.uniform(size=(b.verts.shape[0], 3)).astype(np.float32)
+    prm = _params(8.0)
+    bg = np.array([1.0, 1.0, 1.0], np.float32)
+    kw = dict(sigma=1e-4, gamma=1e-2, znear=1.0, zfar=10.0)
+    P, N, A = cuda(b.world), cuda(b.normals), cuda(alb)
+    vcol = mr.phong_fwd(P, N, A, prm)
+    o = oracle_mod.rasterize_fwd(b.verts, b.faces, b.mesh_to_face_first_idx, b.num_faces_per_mesh, w.H, w.W,
+                                 np.float32(w.blur_radius), w.K, False)
+    op2f, oz, ob, od, ex = o
+    p2f, zb, bb, dd = cuda(op2f), cuda(oz, np.float32), cuda(ob, np.float32), cuda(od, np.float32)
+    col = mr.interpolate_fwd(p2f, bb, cuda(b.faces), vcol)
+    rgba = mr.blend_fwd(p2f, col, dd, zb, bg, **kw)
+    g = syn.random_grads(tuple(rgba.shape), 9)
+    gcol, _, _ = mr.blend_bwd(p2f, col, dd, zb, bg, grad_rgba=cuda(g), **kw)
+    gvcol, _ = mr.interpolate_bwd(p2f, bb, cuda(b.faces), vcol, gcol)
+    gP, gN, gA = mr.phong_bwd(P, N, A, prm, gvcol)
+
+    prm64 = prm.astype(np.float64)
+    ovcol, vflags = oracle_mod.phong_fwd(b.world, b.normals, alb, prm64)
+    ocol = oracle_mod.interpolate_fwd(op2f, ob.astype(np.float32), b.faces, ovcol)
+    orgba = oracle_mod.blend_fwd(op2f, ocol, od.astype(np.float32), oz.astype(np.float32), bg, **kw)
+    err = np.abs(np_(rgba) - orgba) - (1e-4 * np.abs(orgba) + 1e-5)
+    assert err.max() <= 0, f"rgba off by {err.max():.3g}"
+    oc, _, _ = oracle_mod.blend_bwd(op2f, ocol, od.astype(np.float32), oz.astype(np.float32), bg, grad_rgba=g, **kw)
+    ogv, _ = oracle_mod.interpolate_bwd(op2f, ob.astype(np.float32), b.faces, ovcol, oc)
+    oP, oN, oA = oracle_mod.phong_bwd(b.world, b.normals, alb, prm64, ogv)
+    keep = ~vflags
+    for name, x, y in (("grad points", gP, oP), ("grad normals", gN, oN), ("grad albedo", gA, oA)):
+        compare_grad(np_(x)[keep], y[keep], label=name)
