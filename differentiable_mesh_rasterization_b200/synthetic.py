@@ -238,3 +238,96 @@ def grad_alpha(batch: MeshBatch) -> np.ndarray:
 def random_grads(shape: tuple, seed: int) -> np.ndarray:
     """Generic seeded N(0, 1) float32 array (upstream gradients for tests)."""
     return np.random.Generator(np.random.PCG64(seed)).standard_normal(shape).astype(np.float32)
+
+
+# --------------------------------------------------------------------------- point clouds
+@dataclass
+class PointWorkload:
+    name: str
+    mesh_config: int        # the mesh batch whose vertices are the clouds
+    H: int
+    W: int
+    K: int
+    radius: float           # NDC units
+    C: int                  # feature channels
+    description: str
+
+
+POINT_WORKLOADS: dict[int, PointWorkload] = {
+    2: PointWorkload("pts_ico234_b8_137px_K8", 2, 137, 137, 8, 0.02, 3,
+                     "vertices of mesh batch 2 (8 clouds, 642-2562 points), 137x137, K=8, radius 0.02, RGB"),
+    5: PointWorkload("pts_ico36_torus_b64_512px_K8", 5, 512, 512, 8, 0.01, 3,
+                     "vertices of mesh batch 5 (64 clouds, 642-55,418 points, 1.18 M in all), 512x512, K=8, "
+                     "radius 0.01, RGB"),
+}
+
+
+@dataclass
+class PointBatch:
+    """A packed heterogeneous batch of screen-space point clouds with per-point features."""
+    points: np.ndarray              # (P, 3) float32: x_ndc, y_ndc, z_view
+    cloud_first_idx: np.ndarray     # (N,) int64
+    num_points_per_cloud: np.ndarray  # (N,) int64
+    features: np.ndarray            # (P, C) float32 in [0, 1)
+    workload: PointWorkload
+
+    @property
+    def N(self) -> int:
+        return int(self.num_points_per_cloud.shape[0])
+
+
+def make_point_batch(config: int, n_clouds: int | None = None) -> PointBatch:
+    """Point clouds made of the vertices of mesh batch ``config`` (same draws), with
+    features ~ U[0, 1) from ``PCG64(2000 + config)``."""
+    w = POINT_WORKLOADS[config]
+    b = make_batch(w.mesh_config, n_meshes=n_clouds)
+    rng = np.random.Generator(np.random.PCG64(2000 + config))
+    feats = rng.uniform(size=(b.verts.shape[0], w.C)).astype(np.float32)
+    return PointBatch(b.verts, b.mesh_to_vert_first_idx.copy(), b.num_verts_per_mesh.copy(), feats, w)
+
+
+@dataclass
+class KnnWorkload:
+    name: str
+    mesh_config: int
+    K: int
+    jitter: float
+    description: str
+
+
+KNN_WORKLOADS: dict[int, KnnWorkload] = {
+    2: KnnWorkload("knn_ico234_b8_K8", 2, 8, 0.01,
+                   "8 clouds (world vertices of mesh batch 2, 642-2562 points) against their jittered copies, D=3, K=8"),
+    5: KnnWorkload("knn_ico36_torus_b64_K8", 5, 8, 0.01,
+                   "64 clouds (world vertices of mesh batch 5, 642-55,418 points, 1.18 M in all) against their "
+                   "jittered copies, D=3, K=8"),
+}
+
+
+@dataclass
+class KnnBatch:
+    """Two packed heterogeneous sets of 3-D clouds: queries p1 and references p2 (cloud n of
+    p1 searches cloud n of p2)."""
+    p1: np.ndarray
+    first1: np.ndarray
+    num1: np.ndarray
+    p2: np.ndarray
+    first2: np.ndarray
+    num2: np.ndarray
+    workload: KnnWorkload
+
+    @property
+    def N(self) -> int:
+        return int(self.num1.shape[0])
+
+
+def make_knn_batch(config: int, n_clouds: int | None = None) -> KnnBatch:
+    """References: the world vertices of mesh batch ``config``; queries: the same points
+    moved by N(0, jitter^2) per coordinate from ``PCG64(3000 + config)``."""
+    w = KNN_WORKLOADS[config]
+    b = make_batch(w.mesh_config, n_meshes=n_clouds)
+    rng = np.random.Generator(np.random.PCG64(3000 + config))
+    p2 = b.world.astype(np.float32)
+    p1 = (p2 + w.jitter * rng.standard_normal(p2.shape)).astype(np.float32)
+    f, n = b.mesh_to_vert_first_idx.copy(), b.num_verts_per_mesh.copy()
+    return KnnBatch(p1, f, n, p2, f.copy(), n.copy(), w)

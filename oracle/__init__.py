@@ -66,6 +66,18 @@ def _load():
         lib.oracle_phong_shade_fwd.restype = None
         lib.oracle_phong_shade_bwd.argtypes = [P, P, i64, i32, P, P, P, P, i64, P, P, P, P, P, P]
         lib.oracle_phong_shade_bwd.restype = None
+        lib.oracle_rasterize_points.argtypes = [P, i64, P, P, i32, i32, i32, f64, i32, P, P, P, P]
+        lib.oracle_rasterize_points.restype = ctypes.c_int
+        lib.oracle_rasterize_points_bwd.argtypes = [P, i64, P, i32, i32, i32, i32, P, P, P]
+        lib.oracle_rasterize_points_bwd.restype = None
+        lib.oracle_composite_points.argtypes = [P, P, i64, i32, P, i32, f64, i32, P]
+        lib.oracle_composite_points.restype = None
+        lib.oracle_composite_points_bwd.argtypes = [P, P, i64, i32, P, i64, i32, f64, i32, P, P, P]
+        lib.oracle_composite_points_bwd.restype = None
+        lib.oracle_knn.argtypes = [P, P, P, P, P, P, i32, i32, i32, P, P, P]
+        lib.oracle_knn.restype = ctypes.c_int
+        lib.oracle_knn_bwd.argtypes = [P, i64, P, i64, i32, i32, P, P, P, P]
+        lib.oracle_knn_bwd.restype = None
         _lib = lib
     return _lib
 
@@ -304,3 +316,98 @@ def phong_shade_bwd(pix_to_face, bary, faces, points, normals, albedo, params, g
     lib.oracle_phong_shade_bwd(_ptr(p2f), _ptr(b), npix, K, _ptr(f), _ptr(P), _ptr(N), _ptr(c), P.shape[0],
                                _ptr(prm), _ptr(g), _ptr(gP), _ptr(gN), _ptr(gc), _ptr(gb))
     return gP, gN, gc, gb
+
+
+def rasterize_points(points, cloud_first_idx, num_points_per_cloud, H, W, radius, K):
+    """Step 22: (idx, zbuf, dists) of shape (N, H, W, K) and flags (N, H, W)."""
+    lib = _load()
+    pts = _c(points, np.float32)
+    first = _c(cloud_first_idx, np.int64)
+    num = _c(num_points_per_cloud, np.int64)
+    N = first.shape[0]
+    idx = np.empty((N, H, W, K), np.int64)
+    zbuf = np.empty((N, H, W, K), np.float64)
+    dists = np.empty((N, H, W, K), np.float64)
+    flags = np.empty((N, H, W), np.uint8)
+    rc = lib.oracle_rasterize_points(_ptr(pts), pts.shape[0], _ptr(first), _ptr(num), N, H, W, float(radius), K,
+                                     _ptr(idx), _ptr(zbuf), _ptr(dists), _ptr(flags))
+    if rc != 0:
+        raise ValueError("oracle_rasterize_points: invalid arguments")
+    return idx, zbuf, dists, flags.astype(bool)
+
+
+def rasterize_points_bwd(points, idx, grad_zbuf=None, grad_dists=None):
+    """Step 23: grad_points (P, 3)."""
+    lib = _load()
+    pts = _c(points, np.float32)
+    ix = _c(idx, np.int64)
+    N, H, W, K = ix.shape
+    gz = None if grad_zbuf is None else _c(grad_zbuf, np.float64)
+    gd = None if grad_dists is None else _c(grad_dists, np.float64)
+    out = np.empty((pts.shape[0], 3), np.float64)
+    lib.oracle_rasterize_points_bwd(_ptr(pts), pts.shape[0], _ptr(ix), N, H, W, K, _ptr(gz), _ptr(gd), _ptr(out))
+    return out
+
+
+COMPOSITE_MODES = {"alpha": 0, "norm_weighted": 1}
+
+
+def composite_points(idx, dists, features, radius, mode="alpha"):
+    """Steps 24-25: composited features, idx.shape[:-1] + (C,)."""
+    lib = _load()
+    ix = _c(idx, np.int64)
+    d = _c(dists, np.float64)
+    f = _c(features, np.float64)
+    K, C = ix.shape[-1], f.shape[1]
+    npix = ix.size // K
+    out = np.empty(ix.shape[:-1] + (C,), np.float64)
+    lib.oracle_composite_points(_ptr(ix), _ptr(d), npix, K, _ptr(f), C, float(radius), COMPOSITE_MODES[mode],
+                                _ptr(out))
+    return out
+
+
+def composite_points_bwd(idx, dists, features, radius, grad_out, mode="alpha"):
+    """Step 26: (grad_features (P, C), grad_dists like dists)."""
+    lib = _load()
+    ix = _c(idx, np.int64)
+    d = _c(dists, np.float64)
+    f = _c(features, np.float64)
+    g = _c(grad_out, np.float64)
+    K, C = ix.shape[-1], f.shape[1]
+    npix = ix.size // K
+    gf = np.empty(f.shape, np.float64)
+    gd = np.empty(d.shape, np.float64)
+    lib.oracle_composite_points_bwd(_ptr(ix), _ptr(d), npix, K, _ptr(f), f.shape[0], C, float(radius),
+                                    COMPOSITE_MODES[mode], _ptr(g), _ptr(gf), _ptr(gd))
+    return gf, gd
+
+
+def knn(p1, first1, num1, p2, first2, num2, K):
+    """Step 27: (idx (P1, K) global ids into p2, dists (P1, K), flags (P1,))."""
+    lib = _load()
+    a = _c(p1, np.float32)
+    b = _c(p2, np.float32)
+    f1, n1, f2, n2 = (_c(x, np.int64) for x in (first1, num1, first2, num2))
+    D = a.shape[1]
+    idx = np.empty((a.shape[0], K), np.int64)
+    dists = np.empty((a.shape[0], K), np.float64)
+    flags = np.zeros(a.shape[0], np.uint8)
+    rc = lib.oracle_knn(_ptr(a), _ptr(f1), _ptr(n1), _ptr(b), _ptr(f2), _ptr(n2), f1.shape[0], D, K, _ptr(idx),
+                        _ptr(dists), _ptr(flags))
+    if rc != 0:
+        raise ValueError("oracle_knn: invalid arguments")
+    return idx, dists, flags.astype(bool)
+
+
+def knn_bwd(p1, p2, idx, grad_dists):
+    """Step 28: (grad_p1, grad_p2)."""
+    lib = _load()
+    a = _c(p1, np.float32)
+    b = _c(p2, np.float32)
+    ix = _c(idx, np.int64)
+    g = _c(grad_dists, np.float64)
+    D, K = a.shape[1], ix.shape[1]
+    g1 = np.empty(a.shape, np.float64)
+    g2 = np.empty(b.shape, np.float64)
+    lib.oracle_knn_bwd(_ptr(a), a.shape[0], _ptr(b), b.shape[0], D, K, _ptr(ix), _ptr(g), _ptr(g1), _ptr(g2))
+    return g1, g2

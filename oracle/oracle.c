@@ -784,3 +784,260 @@ void oracle_phong_shade_bwd(const int64_t *p2f, const double *bary, int64_t npix
         }
     }
 }
+
+/* ------------------------------------------------------------------ point clouds */
+/*
+ * The point-cloud renderer and the batched K-nearest-neighbour search (PyTorch3D paper:
+ * the renderer handles point clouds as well as meshes, with the same two stages, and a
+ * custom heterogeneous-batch KNN kernel; the pages print no formula, so the definitions
+ * below are the plain ones that match the mesh path).  Points are in screen space
+ * (x_ndc, y_ndc, z) like the mesh vertices; cloud n is points [first_n, first_n + num_n)
+ * and is drawn into image n.
+ *
+ *  22. point rasterization: pixel centre p as in step 1; point m of cloud n is a
+ *      candidate iff z_m >= 0 and d2 = (p_x - x_m)^2 + (p_y - y_m)^2 <= r^2 (r = the
+ *      radius in NDC units); candidates sorted by (z, point id), the first K kept:
+ *      idx (global point id), zbuf = z_m, dists = d2; empty slots hold -1 in all three.
+ *  23. its gradient: d dists / d (x_m, y_m) = -2 (p - (x_m, y_m)); d zbuf / d z_m = 1.
+ *  24. alpha compositing over a pixel's valid slots in order, with per-point features
+ *      f_m (C channels) and a_k = 1 - dists_k / r^2:
+ *        out = sum_k a_k T_k f_{idx_k},  T_k = prod_{j < k} (1 - a_j).
+ *  25. norm-weighted compositing: out = sum_k a_k f_{idx_k} / max(sum_k a_k, 1e-4).
+ *  26. their gradients into the features and the dists (the products over j != k are
+ *      formed directly; no division by 1 - a_k).
+ *  27. batched KNN: for query point i of cloud n of the first set (D coordinates each),
+ *      the squared Euclidean distance to every point j of cloud n of the second set; the
+ *      K smallest, ordered by (distance, j); idx = the global (packed) id of j, dists the
+ *      distance; when cloud n of the second set has fewer than K points the rest hold
+ *      -1 in both.
+ *  28. its gradient: d dist / d q = 2 (q - r_j), d dist / d r_j = -2 (q - r_j).
+ *
+ * Flags: step 22 marks pixels where a point within a margin of the radius
+ * (|d2 - r^2| < 1e-5 r^2) would rank among the first K; step 27 marks queries whose
+ * K-th and (K+1)-th distances lie within 1e-6 (relative) of each other, or whose first
+ * K contain such a near tie (the order of near-equal distances is decided by rounding).
+ */
+#define POINT_MARGIN 1e-5
+#define KNN_TIE 1e-6
+#define NORM_FLOOR 1e-4
+
+typedef struct {
+    double key;
+    int64_t id;
+    double aux;
+} kv;
+
+static int kv_before(const kv *a, const kv *b) { return a->key < b->key || (a->key == b->key && a->id < b->id); }
+
+/* insertion into a sorted list of at most cap entries; returns the new length */
+static int kv_insert(kv *list, int n, int cap, kv e) {
+    int pos = n;
+    while (pos > 0 && kv_before(&e, &list[pos - 1])) --pos;
+    if (pos >= cap) return n;
+    int last = n < cap ? n : cap - 1;
+    for (int t = last; t > pos; --t) list[t] = list[t - 1];
+    list[pos] = e;
+    return n < cap ? n + 1 : n;
+}
+
+/* Step 22 for the N images; idx, zbuf, dists are N x H x W x K; flags N x H x W (may be NULL). */
+int oracle_rasterize_points(const float *pts, int64_t P, const int64_t *first, const int64_t *num, int32_t N,
+                            int32_t H, int32_t W, double radius, int32_t K, int64_t *idx, double *zbuf,
+                            double *dists, uint8_t *flags) {
+    if (N < 0 || H < 1 || W < 1 || K < 1 || radius < 0) return -1;
+    double r2 = radius * radius;
+    kv *list = (kv *)malloc(sizeof(kv) * (size_t)(K + 1));
+    for (int32_t n = 0; n < N; ++n)
+        for (int32_t i = 0; i < H; ++i)
+            for (int32_t j = 0; j < W; ++j) {
+                double px = -1.0 + (2.0 * j + 1.0) / W, py = 1.0 - (2.0 * i + 1.0) / H;
+                int cnt = 0;
+                int near_margin = 0;
+                kv marg;
+                marg.key = 0.0;
+                marg.id = 0;
+                marg.aux = 0.0;
+                for (int64_t m = first[n]; m < first[n] + num[n]; ++m) {
+                    if (m < 0 || m >= P) continue;
+                    double x = pts[3 * m], y = pts[3 * m + 1], z = pts[3 * m + 2];
+                    if (z < 0.0) continue;
+                    double d2 = (px - x) * (px - x) + (py - y) * (py - y);
+                    if (fabs(d2 - r2) < POINT_MARGIN * r2) {
+                        /* decided by rounding: remember the nearest such point */
+                        kv e = {z, m, d2};
+                        if (!near_margin || kv_before(&e, &marg)) marg = e;
+                        near_margin = 1;
+                    }
+                    if (d2 > r2) continue;
+                    kv e = {z, m, d2};
+                    cnt = kv_insert(list, cnt, K, e);
+                }
+                int64_t o = (((int64_t)n * H + i) * W + j) * K;
+                for (int k = 0; k < K; ++k) {
+                    idx[o + k] = k < cnt ? list[k].id : -1;
+                    zbuf[o + k] = k < cnt ? list[k].key : -1.0;
+                    dists[o + k] = k < cnt ? list[k].aux : -1.0;
+                }
+                if (flags) {
+                    int f = 0;
+                    if (near_margin) f = cnt < K || kv_before(&marg, &list[K - 1]) || marg.id == list[K - 1].id;
+                    flags[((int64_t)n * H + i) * W + j] = (uint8_t)f;
+                }
+            }
+    free(list);
+    return 0;
+}
+
+/* Step 23: grad_points (P x 3) overwritten; grad_zbuf / grad_dists may be NULL. */
+void oracle_rasterize_points_bwd(const float *pts, int64_t P, const int64_t *idx, int32_t N, int32_t H, int32_t W,
+                                 int32_t K, const double *grad_zbuf, const double *grad_dists, double *grad) {
+    memset(grad, 0, sizeof(double) * 3 * (size_t)P);
+    for (int32_t n = 0; n < N; ++n)
+        for (int32_t i = 0; i < H; ++i)
+            for (int32_t j = 0; j < W; ++j) {
+                double px = -1.0 + (2.0 * j + 1.0) / W, py = 1.0 - (2.0 * i + 1.0) / H;
+                int64_t o = (((int64_t)n * H + i) * W + j) * K;
+                for (int k = 0; k < K; ++k) {
+                    int64_t m = idx[o + k];
+                    if (m < 0) continue;
+                    if (grad_dists) {
+                        grad[3 * m] += grad_dists[o + k] * -2.0 * (px - pts[3 * m]);
+                        grad[3 * m + 1] += grad_dists[o + k] * -2.0 * (py - pts[3 * m + 1]);
+                    }
+                    if (grad_zbuf) grad[3 * m + 2] += grad_zbuf[o + k];
+                }
+            }
+}
+
+/* Steps 24-25: mode 0 alpha, 1 norm-weighted; features P x C; out npix x C. */
+void oracle_composite_points(const int64_t *idx, const double *dists, int64_t npix, int32_t K, const double *feat,
+                             int32_t C, double radius, int32_t mode, double *out) {
+    double r2 = radius * radius;
+    for (int64_t q = 0; q < npix; ++q) {
+        double T = 1.0, wsum = 0.0;
+        for (int c = 0; c < C; ++c) out[q * C + c] = 0.0;
+        for (int k = 0; k < K; ++k) {
+            int64_t m = idx[q * K + k];
+            if (m < 0) continue;
+            double a = 1.0 - dists[q * K + k] / r2;
+            double w = mode == 0 ? a * T : a;
+            for (int c = 0; c < C; ++c) out[q * C + c] += w * feat[m * C + c];
+            T *= 1.0 - a;
+            wsum += a;
+        }
+        if (mode == 1) {
+            double den = wsum > NORM_FLOOR ? wsum : NORM_FLOOR;
+            for (int c = 0; c < C; ++c) out[q * C + c] /= den;
+        }
+    }
+}
+
+/* Step 26: grad_feat (P x C) overwritten, grad_dists (npix x K) written (0 for empty slots). */
+void oracle_composite_points_bwd(const int64_t *idx, const double *dists, int64_t npix, int32_t K,
+                                 const double *feat, int64_t P, int32_t C, double radius, int32_t mode,
+                                 const double *grad_out, double *grad_feat, double *grad_dists) {
+    double r2 = radius * radius;
+    double *fo = (double *)malloc(sizeof(double) * (size_t)C);   /* the normalised output */
+    memset(grad_feat, 0, sizeof(double) * (size_t)(P * C));
+    for (int64_t q = 0; q < npix; ++q) {
+        const double *g = grad_out + q * C;
+        double wsum = 0.0;
+        for (int k = 0; k < K; ++k)
+            if (idx[q * K + k] >= 0) wsum += 1.0 - dists[q * K + k] / r2;
+        double den = wsum > NORM_FLOOR ? wsum : NORM_FLOOR;
+        for (int c = 0; c < C; ++c) fo[c] = 0.0;
+        if (mode == 1)
+            for (int k = 0; k < K; ++k) {
+                int64_t m = idx[q * K + k];
+                if (m < 0) continue;
+                double a = 1.0 - dists[q * K + k] / r2;
+                for (int c = 0; c < C; ++c) fo[c] += a * feat[m * C + c] / den;
+            }
+        for (int k = 0; k < K; ++k) {
+            int64_t m = idx[q * K + k];
+            if (m < 0) {
+                grad_dists[q * K + k] = 0.0;
+                continue;
+            }
+            double a = 1.0 - dists[q * K + k] / r2;
+            double ga = 0.0;
+            if (mode == 0) {
+                /* out = sum_l a_l prod_{j<l} (1 - a_j) f_l */
+                double Tk = 1.0;
+                for (int j = 0; j < k; ++j)
+                    if (idx[q * K + j] >= 0) Tk *= 1.0 - (1.0 - dists[q * K + j] / r2);
+                for (int c = 0; c < C; ++c) {
+                    grad_feat[m * C + c] += a * Tk * g[c];
+                    ga += Tk * feat[m * C + c] * g[c];
+                }
+                for (int l = k + 1; l < K; ++l) {
+                    int64_t ml = idx[q * K + l];
+                    if (ml < 0) continue;
+                    double al = 1.0 - dists[q * K + l] / r2;
+                    double Tl_wo_k = 1.0;   /* prod_{j < l, j != k} (1 - a_j) */
+                    for (int j = 0; j < l; ++j)
+                        if (j != k && idx[q * K + j] >= 0) Tl_wo_k *= 1.0 - (1.0 - dists[q * K + j] / r2);
+                    for (int c = 0; c < C; ++c) ga -= al * Tl_wo_k * feat[ml * C + c] * g[c];
+                }
+            } else {
+                for (int c = 0; c < C; ++c) grad_feat[m * C + c] += a / den * g[c];
+                if (wsum > NORM_FLOOR)
+                    for (int c = 0; c < C; ++c) ga += (feat[m * C + c] - fo[c]) / den * g[c];
+                else
+                    for (int c = 0; c < C; ++c) ga += feat[m * C + c] / den * g[c];
+            }
+            grad_dists[q * K + k] = ga * (-1.0 / r2);
+        }
+    }
+    free(fo);
+}
+
+/* Step 27: queries (P1 x D, clouds first1/num1), references (P2 x D, first2/num2);
+ * idx, dists P1 x K; flags P1 (may be NULL). */
+int oracle_knn(const float *p1, const int64_t *first1, const int64_t *num1, const float *p2, const int64_t *first2,
+               const int64_t *num2, int32_t N, int32_t D, int32_t K, int64_t *idx, double *dists, uint8_t *flags) {
+    if (N < 0 || D < 1 || K < 1) return -1;
+    kv *list = (kv *)malloc(sizeof(kv) * (size_t)(K + 1));
+    for (int32_t n = 0; n < N; ++n)
+        for (int64_t i = first1[n]; i < first1[n] + num1[n]; ++i) {
+            int cnt = 0;
+            for (int64_t j = first2[n]; j < first2[n] + num2[n]; ++j) {
+                double d = 0.0;
+                for (int e = 0; e < D; ++e) {
+                    double t = (double)p1[i * D + e] - (double)p2[j * D + e];
+                    d += t * t;
+                }
+                kv x = {d, j, 0.0};
+                cnt = kv_insert(list, cnt, K + 1, x);   /* K + 1 kept to see the boundary */
+            }
+            for (int k = 0; k < K; ++k) {
+                idx[i * K + k] = k < cnt ? list[k].id : -1;
+                dists[i * K + k] = k < cnt ? list[k].key : -1.0;
+            }
+            if (flags) {
+                int f = 0;
+                for (int k = 0; k + 1 < cnt && k < K; ++k)
+                    if (list[k + 1].key - list[k].key <= KNN_TIE * list[k + 1].key) f = 1;
+                flags[i] = (uint8_t)f;
+            }
+        }
+    free(list);
+    return 0;
+}
+
+/* Step 28: grad_p1 (P1 x D) and grad_p2 (P2 x D) overwritten. */
+void oracle_knn_bwd(const float *p1, int64_t P1, const float *p2, int64_t P2, int32_t D, int32_t K,
+                    const int64_t *idx, const double *grad_dists, double *grad_p1, double *grad_p2) {
+    memset(grad_p1, 0, sizeof(double) * (size_t)(P1 * D));
+    memset(grad_p2, 0, sizeof(double) * (size_t)(P2 * D));
+    for (int64_t i = 0; i < P1; ++i)
+        for (int k = 0; k < K; ++k) {
+            int64_t j = idx[i * K + k];
+            if (j < 0) continue;
+            for (int e = 0; e < D; ++e) {
+                double t = 2.0 * ((double)p1[i * D + e] - (double)p2[j * D + e]) * grad_dists[i * K + k];
+                grad_p1[i * D + e] += t;
+                grad_p2[j * D + e] -= t;
+            }
+        }
+}
