@@ -336,6 +336,111 @@ def shading_step_timing(mr, torch, dev, stream, batch, verts, faces, first, num,
                                       "soft RGB blend (gamma 1e-2), fwd+bwd")}
 
 
+def _timed_steps(mr, torch, dev, stream, flush, steps, step):
+    """Warm-up, then ``steps`` timed calls of ``step`` (L2 flushed before each, CUDA events on
+    the launching stream, library stage timing on): (ms per step, stage dict)."""
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    mr.profile_read()
+    mr.profile_enable(True)
+    for k in range(steps):
+        flush.zero_()
+        starts[k].record(stream)
+        step()
+        ends[k].record(stream)
+    torch.cuda.synchronize(dev)
+    mr.profile_enable(False)
+    st = mr.profile_read()
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / steps
+    return ms, {name: t / steps for name, (t, n) in st.items() if n}
+
+
+def point_box_samples(pb):
+    """Pixel-point samples of a point batch: (pixel, point) pairs of the same image whose pixel
+    centre lies in the point's box of half-width radius (exact host count; points behind the
+    camera excluded)."""
+    w = pb.workload
+    p = pb.points.astype(np.float64)
+    r = float(np.float32(w.radius))
+    ok = p[:, 2] >= 0
+    jl = np.maximum(np.ceil((p[:, 0] - r + 1) * w.W / 2 - 0.5), 0)
+    jh = np.minimum(np.floor((p[:, 0] + r + 1) * w.W / 2 - 0.5), w.W - 1)
+    il = np.maximum(np.ceil((1 - p[:, 1] - r) * w.H / 2 - 0.5), 0)
+    ih = np.minimum(np.floor((1 - p[:, 1] + r) * w.H / 2 - 0.5), w.H - 1)
+    n = np.clip(jh - jl + 1, 0, None) * np.clip(ih - il + 1, 0, None)
+    return int(np.sum(n[ok]))
+
+
+def points_step_timing(mr, torch, dev, stream, flush, args, hbm_peak, hbm_note):
+    """Point-cloud render step: 64 clouds (1.18 M points) -> K=8 nearest per pixel at 512x512
+    -> alpha compositing of RGB features -> backward to the points and features."""
+    from differentiable_mesh_rasterization_b200 import synthetic as syn
+    pb = syn.make_point_batch(5)
+    w = pb.workload
+    P = torch.from_numpy(pb.points).to(dev)
+    F = torch.from_numpy(pb.features).to(dev)
+    r = float(np.float32(w.radius))
+    g = torch.from_numpy(syn.random_grads((pb.N, w.H, w.W, w.C), 13)).to(dev)
+
+    def step():
+        idx, zbuf, dists = mr.rasterize_points_fwd(P, pb.cloud_first_idx, pb.num_points_per_cloud, w.H, w.W, r, w.K)
+        mr.composite_points_fwd(idx, dists, F, r, "alpha")
+        _, gd = mr.composite_points_bwd(idx, dists, F, r, g, "alpha")
+        mr.rasterize_points_bwd(P, idx, grad_dists=gd)
+
+    steps = max(3, args.steps // 5)
+    ms, stages = _timed_steps(mr, torch, dev, stream, flush, steps, step)
+    npix = pb.N * w.H * w.W
+    slot = npix * w.K
+    # algorithmic bytes: each per-slot array read or written once
+    algo = {"points_fine": slot * (8 + 4 + 4), "composite_fwd": slot * (8 + 4) + npix * w.C * 4,
+            "composite_bwd": slot * (8 + 4 + 4) + npix * w.C * 4, "points_bwd": slot * (8 + 4)}
+    out = {s: {"ms_per_step": t} for s, t in stages.items()}
+    for s, b in algo.items():
+        if s in out:
+            out[s]["hbm_frac"] = b / (out[s]["ms_per_step"] / 1e3) / 1e9 / hbm_peak
+    samples = point_box_samples(pb)
+    return {"workload": w.name, "ms_per_step": ms, "pixel_point_samples_per_s": samples / (ms / 1e3),
+            "mpix_per_s": npix / (ms / 1e3) / 1e6, "points": int(pb.points.shape[0]), "steps": steps,
+            "stages": out, "hbm_peak_note": hbm_note,
+            "note": w.description + "; alpha compositing fwd+bwd; L2 flushed per step"}
+
+
+KNN_C_PAIR = 7       # FP32 instructions per (query, reference) pair for D=3: 3 FADD, 3 FFMA, 1 compare
+
+
+def knn_step_timing(mr, torch, dev, stream, flush, args, peak_alu):
+    """Batched KNN step: 64 heterogeneous clouds (1.18 M queries against 1.18 M references,
+    D=3, K=8) forward and backward."""
+    from differentiable_mesh_rasterization_b200 import synthetic as syn
+    kb = syn.make_knn_batch(5)
+    K = kb.workload.K
+    A = torch.from_numpy(kb.p1).to(dev)
+    B = torch.from_numpy(kb.p2).to(dev)
+    g = torch.from_numpy(syn.random_grads((kb.p1.shape[0], K), 14)).to(dev)
+
+    def step():
+        idx, _ = mr.knn_fwd(A, kb.first1, kb.num1, B, kb.first2, kb.num2, K)
+        mr.knn_bwd(A, B, idx, g)
+
+    steps = max(3, args.steps // 10)
+    ms, stages = _timed_steps(mr, torch, dev, stream, flush, steps, step)
+    pairs = int(np.sum(kb.num1.astype(np.int64) * kb.num2.astype(np.int64)))
+    out = {s: {"ms_per_step": t} for s, t in stages.items()}
+    knn_ms = out.get("knn", {}).get("ms_per_step")
+    roof = None
+    if knn_ms:
+        achieved = pairs * KNN_C_PAIR / (knn_ms / 1e3) / 1e12
+        roof = {"bound": "alu", "kernel": "k_knn (exhaustive, register top-K)", "achieved": achieved,
+                "peak": peak_alu, "unit": "T FP32-inst/s", "frac": achieved / peak_alu, "c_pair": KNN_C_PAIR}
+    return {"workload": kb.workload.name, "ms_per_step": ms, "pairs_per_s": pairs / (ms / 1e3), "pairs": pairs,
+            "queries": int(kb.p1.shape[0]), "steps": steps, "stages": out, "roofline": roof,
+            "note": kb.workload.description + "; fwd+bwd; L2 flushed per step"}
+
+
 # ----------------------------------------------------------------------------- our arm
 def main():
     ap = argparse.ArgumentParser()
@@ -346,7 +451,7 @@ def main():
     ap.add_argument("--config", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--no-shading", action="store_true", help="skip the Gouraud and Phong RGB measurements")
+    ap.add_argument("--no-shading", action="store_true", help="skip the Gouraud, Phong, point-cloud and KNN measurements")
     ap.add_argument("--images", type=int, default=None,
                     help="render only the first N meshes of the batch (small profiling case)")
     args = ap.parse_args()
@@ -508,6 +613,9 @@ def main():
     if not args.no_shading:
         line["next_rows"] = shading_step_timing(mr, torch, dev, stream, batch, verts, faces, first, num, flush,
                                                 args, hbm_peak, hbm_note)
+        line["next_rows"]["points_rgb"] = points_step_timing(mr, torch, dev, stream, flush, args, hbm_peak,
+                                                             hbm_note)
+        line["next_rows"]["knn"] = knn_step_timing(mr, torch, dev, stream, flush, args, peak_alu)
 
     if rank == 0 and not args.no_cpu_baseline:
         import oracle

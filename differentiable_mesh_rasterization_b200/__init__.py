@@ -27,10 +27,13 @@ EXPORTS = ("mr_rasterize_fwd", "mr_rasterize_silhouette_fwd", "mr_silhouette_ble
            "mr_silhouette_blend_bwd", "mr_rasterize_bwd", "mr_silhouette_rasterize_bwd",
            "mr_device_status", "mr_last_error", "mr_version", "mr_profile_enable", "mr_profile_read",
            "mr_rasterize_fwd_noalloc", "mr_interpolate_fwd", "mr_interpolate_bwd", "mr_blend_fwd", "mr_blend_bwd",
-           "mr_phong_fwd", "mr_phong_bwd", "mr_phong_shade_fwd", "mr_phong_shade_bwd")
+           "mr_phong_fwd", "mr_phong_bwd", "mr_phong_shade_fwd", "mr_phong_shade_bwd",
+           "mr_rasterize_points_fwd", "mr_rasterize_points_bwd", "mr_composite_points_fwd",
+           "mr_composite_points_bwd", "mr_knn_fwd", "mr_knn_bwd")
 STAGES = ("face_setup", "bin_count", "bin_scan", "bin_fill", "fine", "silhouette_fwd", "silhouette_bwd",
           "raster_bwd", "silhouette_raster_bwd", "epilogue", "interpolate_fwd", "interpolate_bwd", "blend_fwd",
-          "blend_bwd", "phong_fwd", "phong_bwd", "phong_shade_fwd", "phong_shade_bwd")
+          "blend_bwd", "phong_fwd", "phong_bwd", "phong_shade_fwd", "phong_shade_bwd",
+          "points_bin", "points_fine", "points_bwd", "composite_fwd", "composite_bwd", "knn", "knn_bwd")
 
 
 class MeshRastError(RuntimeError):
@@ -71,6 +74,12 @@ def load_library() -> ctypes.CDLL:
         "mr_phong_bwd": [P, P, P, i64, P, P, P, P, P, P],
         "mr_phong_shade_fwd": [P, P, i64, i32, P, i64, P, P, P, i64, P, P, P],
         "mr_phong_shade_bwd": [P, P, i64, i32, P, i64, P, P, P, i64, P, P, P, P, P, P, P],
+        "mr_rasterize_points_fwd": [P, i64, P, P, i32, i32, i32, f32, i32, P, P, P, P],
+        "mr_rasterize_points_bwd": [P, i64, P, i32, i32, i32, i32, P, P, P, P],
+        "mr_composite_points_fwd": [P, P, i64, i32, P, i64, i32, f32, i32, P, P],
+        "mr_composite_points_bwd": [P, P, i64, i32, P, i64, i32, f32, i32, P, P, P, P],
+        "mr_knn_fwd": [P, i64, P, P, P, i64, P, P, i32, i32, i32, P, P, P],
+        "mr_knn_bwd": [P, i64, P, i64, i32, i32, P, P, P, P, P],
         "mr_profile_enable": [i32],
         "mr_profile_read": [P, P, i32],
     }
@@ -376,6 +385,116 @@ def phong_shade_bwd(pix_to_face, bary, faces, points, normals, albedo, params, g
                                                             prm.ctypes.data, _ptr(g), _ptr(gP), _ptr(gN), _ptr(gc),
                                                             _ptr(gb), _stream(p2f.device)))
     return gP, gN, gc, gb
+
+
+# ----------------------------------------------------------------------------- point clouds
+COMPOSITE_MODES = {"alpha": 0, "norm_weighted": 1}
+
+
+def rasterize_points_fwd(points, cloud_first_idx, num_points_per_cloud, H, W, radius, K):
+    """K nearest points per pixel (``mr_rasterize_points_fwd``) -> (idx, zbuf, dists), each (N, H, W, K)."""
+    lib = load_library()
+    pts = _dev(points, torch.float32, "points")
+    first = _host_i64(cloud_first_idx, "cloud_first_idx")
+    num = _host_i64(num_points_per_cloud, "num_points_per_cloud")
+    if pts.ndim != 2 or pts.shape[1] != 3 or first.shape != num.shape:
+        raise ValueError("points must be (P, 3); cloud_first_idx and num_points_per_cloud of equal length")
+    N = first.shape[0]
+    dev = pts.device
+    idx = torch.empty((N, H, W, K), dtype=torch.int64, device=dev)
+    zbuf = torch.empty((N, H, W, K), dtype=torch.float32, device=dev)
+    dists = torch.empty((N, H, W, K), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check("mr_rasterize_points_fwd",
+               lib.mr_rasterize_points_fwd(_ptr(pts), pts.shape[0], first.ctypes.data, num.ctypes.data, N, H, W,
+                                           float(radius), K, _ptr(idx), _ptr(zbuf), _ptr(dists), _stream(dev)))
+    return idx, zbuf, dists
+
+
+def rasterize_points_bwd(points, idx, grad_zbuf=None, grad_dists=None):
+    """Gradient of the point rasterizer (``mr_rasterize_points_bwd``) -> grad_points (P, 3)."""
+    lib = load_library()
+    pts = _dev(points, torch.float32, "points")
+    ix = _dev(idx, torch.int64, "idx")
+    N, H, W, K = ix.shape
+    gz = None if grad_zbuf is None else _dev(grad_zbuf, torch.float32, "grad_zbuf")
+    gd = None if grad_dists is None else _dev(grad_dists, torch.float32, "grad_dists")
+    out = torch.empty_like(pts)
+    with torch.cuda.device(pts.device):
+        _check("mr_rasterize_points_bwd",
+               lib.mr_rasterize_points_bwd(_ptr(pts), pts.shape[0], _ptr(ix), N, H, W, K, _ptr(gz), _ptr(gd),
+                                           _ptr(out), _stream(pts.device)))
+    return out
+
+
+def composite_points_fwd(idx, dists, features, radius, mode="alpha"):
+    """Alpha or norm-weighted compositing of per-point features (``mr_composite_points_fwd``) -> (N, H, W, C)."""
+    lib = load_library()
+    ix = _dev(idx, torch.int64, "idx")
+    d = _dev(dists, torch.float32, "dists")
+    f = _dev(features, torch.float32, "features")
+    if d.shape != ix.shape or f.ndim != 2:
+        raise ValueError("dists must match idx and features be (P, C)")
+    K, C = ix.shape[-1], f.shape[1]
+    out = torch.empty(tuple(ix.shape[:-1]) + (C,), dtype=torch.float32, device=ix.device)
+    with torch.cuda.device(ix.device):
+        _check("mr_composite_points_fwd",
+               lib.mr_composite_points_fwd(_ptr(ix), _ptr(d), ix.numel() // K, K, _ptr(f), f.shape[0], C,
+                                           float(radius), COMPOSITE_MODES[mode], _ptr(out), _stream(ix.device)))
+    return out
+
+
+def composite_points_bwd(idx, dists, features, radius, grad_out, mode="alpha"):
+    """Gradient of the compositing (``mr_composite_points_bwd``) -> (grad_features, grad_dists)."""
+    lib = load_library()
+    ix = _dev(idx, torch.int64, "idx")
+    d = _dev(dists, torch.float32, "dists")
+    f = _dev(features, torch.float32, "features")
+    g = _dev(grad_out, torch.float32, "grad_out")
+    K, C = ix.shape[-1], f.shape[1]
+    if tuple(g.shape) != tuple(ix.shape[:-1]) + (C,):
+        raise ValueError("grad_out shape mismatch")
+    gf = torch.empty_like(f)
+    gd = torch.empty_like(d)
+    with torch.cuda.device(ix.device):
+        _check("mr_composite_points_bwd",
+               lib.mr_composite_points_bwd(_ptr(ix), _ptr(d), ix.numel() // K, K, _ptr(f), f.shape[0], C,
+                                           float(radius), COMPOSITE_MODES[mode], _ptr(g), _ptr(gf), _ptr(gd),
+                                           _stream(ix.device)))
+    return gf, gd
+
+
+def knn_fwd(p1, first1, num1, p2, first2, num2, K):
+    """Batched K nearest neighbours (``mr_knn_fwd``) -> (idx (P1, K) ids into p2, dists (P1, K))."""
+    lib = load_library()
+    a = _dev(p1, torch.float32, "p1")
+    b = _dev(p2, torch.float32, "p2")
+    f1, n1, f2, n2 = (_host_i64(x, nm) for x, nm in ((first1, "first1"), (num1, "num1"), (first2, "first2"),
+                                                     (num2, "num2")))
+    if a.ndim != 2 or b.ndim != 2 or a.shape[1] != b.shape[1] or not (f1.shape == n1.shape == f2.shape == n2.shape):
+        raise ValueError("p1 (P1, D), p2 (P2, D) and four cloud arrays of equal length expected")
+    idx = torch.empty((a.shape[0], K), dtype=torch.int64, device=a.device)
+    dists = torch.empty((a.shape[0], K), dtype=torch.float32, device=a.device)
+    with torch.cuda.device(a.device):
+        _check("mr_knn_fwd", lib.mr_knn_fwd(_ptr(a), a.shape[0], f1.ctypes.data, n1.ctypes.data, _ptr(b), b.shape[0],
+                                            f2.ctypes.data, n2.ctypes.data, f1.shape[0], a.shape[1], K, _ptr(idx),
+                                            _ptr(dists), _stream(a.device)))
+    return idx, dists
+
+
+def knn_bwd(p1, p2, idx, grad_dists):
+    """Gradient of the KNN distances (``mr_knn_bwd``) -> (grad_p1, grad_p2)."""
+    lib = load_library()
+    a = _dev(p1, torch.float32, "p1")
+    b = _dev(p2, torch.float32, "p2")
+    ix = _dev(idx, torch.int64, "idx")
+    g = _dev(grad_dists, torch.float32, "grad_dists")
+    g1 = torch.empty_like(a)
+    g2 = torch.empty_like(b)
+    with torch.cuda.device(a.device):
+        _check("mr_knn_bwd", lib.mr_knn_bwd(_ptr(a), a.shape[0], _ptr(b), b.shape[0], a.shape[1], ix.shape[1],
+                                            _ptr(ix), _ptr(g), _ptr(g1), _ptr(g2), _stream(a.device)))
+    return g1, g2
 
 
 def _blend_args(pix_to_face, colors, dists, zbuf, background):

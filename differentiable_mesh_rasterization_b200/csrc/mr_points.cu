@@ -1,0 +1,592 @@
+// The point-cloud renderer ("Accelerating 3D Deep Learning with PyTorch3D": the same
+// two-stage renderer draws point clouds as well as meshes, over heterogeneous batches).
+//
+// Stage one, for every pixel of image n: the K points of cloud n nearest in depth among
+// those with z >= 0 whose squared 2-D distance to the pixel centre is at most r^2, ordered
+// by (z, point id); idx (global point id), zbuf = z, dists = squared distance; -1 pads.
+// Stage two composites per-point features over those K slots with weights
+// a_k = 1 - dists_k / r^2: front-to-back alpha compositing (out = sum a_k T_k f_k,
+// T_k = prod_{j<k} (1 - a_j)) or the norm-weighted sum (sum a_k f_k / max(sum a_k, 1e-4)).
+//
+// Pipeline: points are binned into 16 x 16-pixel screen bins of their image (count ->
+// exclusive scan -> one stream sync for the total -> fill, like the mesh path); one CTA per
+// bin then stages the bin's points in shared memory in chunks of 256 and every thread
+// (one pixel) keeps its K nearest in registers; 16-byte stores write the slots.
+#include <algorithm>
+#include <cfloat>
+#include <cmath>
+#include <vector>
+
+#include "mr_common.cuh"
+#include "mr_scan.cuh"
+
+namespace mr {
+namespace {
+
+constexpr int kPtBin = 16;          // bin side in pixels (one 256-thread CTA per bin)
+constexpr float kNormFloor = 1e-4f;
+
+// Image of point p: the cloud whose range [first, first + num) holds it (binary search
+// over the cloud starts, which are ascending), or -1.
+__device__ __forceinline__ int cloud_of(int64_t p, const int64_t* __restrict__ first, const int64_t* __restrict__ num,
+                                       int N) {
+    int lo = 0, hi = N - 1, n = -1;
+    while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        if (first[mid] <= p) {
+            n = mid;
+            lo = mid + 1;
+        } else {
+            hi = mid - 1;
+        }
+    }
+    return n >= 0 && p < first[n] + num[n] ? n : -1;
+}
+
+// Inclusive pixel ranges whose centres lie within r of (x, y), widened by 1e-5 NDC so that
+// every pixel the float32 test can accept is inside; false if empty.
+__device__ __forceinline__ bool point_box(float x, float y, float r, int H, int W, int& j0, int& j1, int& i0,
+                                          int& i1) {
+    const double rr = (double)r + 1e-5;
+    const double a = ((double)x - rr + 1.0) * W * 0.5 - 0.5, b = ((double)x + rr + 1.0) * W * 0.5 - 0.5;
+    const double c = (1.0 - (double)y - rr) * H * 0.5 - 0.5, d = (1.0 - (double)y + rr) * H * 0.5 - 0.5;
+    if (!(b >= 0.0) || !(a <= W - 1.0) || !(d >= 0.0) || !(c <= H - 1.0)) return false;   // also NaN
+    j0 = (int)fmax(ceil(a), 0.0);
+    j1 = (int)fmin(floor(b), W - 1.0);
+    i0 = (int)fmax(ceil(c), 0.0);
+    i1 = (int)fmin(floor(d), H - 1.0);
+    return j0 <= j1 && i0 <= i1;
+}
+
+template <bool FILL>
+__global__ void k_point_bins(const float* __restrict__ pts, int64_t P, const int64_t* __restrict__ first,
+                             const int64_t* __restrict__ num, int N, int H, int W, float r, int nbx, int nby,
+                             int* __restrict__ counts, const int* __restrict__ offsets, int* __restrict__ list) {
+    for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < P; p += (int64_t)gridDim.x * blockDim.x) {
+        const int n = cloud_of(p, first, num, N);
+        if (n < 0) continue;
+        const float x = pts[3 * p], y = pts[3 * p + 1], z = pts[3 * p + 2];
+        if (!(z >= 0.f)) continue;
+        int j0, j1, i0, i1;
+        if (!point_box(x, y, r, H, W, j0, j1, i0, i1)) continue;
+        for (int by = i0 / kPtBin; by <= i1 / kPtBin; ++by)
+            for (int bx = j0 / kPtBin; bx <= j1 / kPtBin; ++bx) {
+                const int b = (n * nby + by) * nbx + bx;
+                const int at = atomicAdd(counts + b, 1);
+                if (FILL) list[offsets[b] + at] = (int)p;
+            }
+    }
+}
+
+// Sorted insertion of (z, id, d2) into a register list of KC entries ordered by (z, id).
+template <int KC>
+__device__ __forceinline__ void insert_point(float (&kz)[KC], int (&kid)[KC], float (&kd)[KC], float z, int id,
+                                             float d2) {
+#pragma unroll
+    for (int k = KC - 1; k > 0; --k) {
+        const bool shift = z < kz[k - 1] || (z == kz[k - 1] && id < kid[k - 1]);
+        const bool here = !shift && (z < kz[k] || (z == kz[k] && id < kid[k]));
+        if (shift) {
+            kz[k] = kz[k - 1];
+            kid[k] = kid[k - 1];
+            kd[k] = kd[k - 1];
+        } else if (here) {
+            kz[k] = z;
+            kid[k] = id;
+            kd[k] = d2;
+        }
+    }
+    if (z < kz[0] || (z == kz[0] && id < kid[0])) {
+        kz[0] = z;
+        kid[0] = id;
+        kd[0] = d2;
+    }
+}
+
+template <int KC>
+__global__ void __launch_bounds__(256) k_point_fine(const float* __restrict__ pts, const int* __restrict__ offsets,
+                                                    const int* __restrict__ list, int N, int H, int W, float r2,
+                                                    int K, int nbx, int nby, int64_t* __restrict__ idx,
+                                                    float* __restrict__ zbuf, float* __restrict__ dists, bool vec) {
+    __shared__ float4 sp[256];
+    const int b = blockIdx.x;
+    const int n = b / (nbx * nby), by = (b / nbx) % nby, bx = b % nbx;
+    const int i = by * kPtBin + (threadIdx.x >> 4), j = bx * kPtBin + (threadIdx.x & 15);
+    // pixel centre as a float pair (hi + lo): the offset to a point is then exact to ~1e-15
+    const double pxd = -1.0 + (2.0 * j + 1.0) / W, pyd = 1.0 - (2.0 * i + 1.0) / H;
+    const float pxh = (float)pxd, pyh = (float)pyd;
+    const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
+    float kz[KC], kd[KC];
+    int kid[KC];
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+        kz[k] = FLT_MAX;
+        kid[k] = INT_MAX;
+        kd[k] = -1.f;
+    }
+    const int beg = offsets[b], end = offsets[b + 1];
+    for (int c0 = beg; c0 < end; c0 += 256) {
+        __syncthreads();
+        if (c0 + (int)threadIdx.x < end) {
+            const int p = list[c0 + threadIdx.x];
+            sp[threadIdx.x] = make_float4(pts[3 * (int64_t)p], pts[3 * (int64_t)p + 1], pts[3 * (int64_t)p + 2],
+                                          __int_as_float(p));
+        }
+        __syncthreads();
+        const int cnt = min(256, end - c0);
+        for (int t = 0; t < cnt; ++t) {
+            const float4 q = sp[t];
+            const float dx = (pxh - q.x) + pxl, dy = (pyh - q.y) + pyl;
+            const float d2 = fmaf(dx, dx, dy * dy);
+            const int id = __float_as_int(q.w);
+            if (d2 <= r2 && (q.z < kz[KC - 1] || (q.z == kz[KC - 1] && id < kid[KC - 1])))
+                insert_point<KC>(kz, kid, kd, q.z, id, d2);
+        }
+    }
+    if (i >= H || j >= W) return;
+    const int64_t o = (((int64_t)n * H + i) * W + j) * K;
+    if constexpr (KC >= 4) {
+      if (vec && (K & 3) == 0) {
+#pragma unroll
+        for (int k = 0; k < KC; k += 4) {
+            if (k >= K) break;
+            long long v[4];
+            float z4[4], d4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const bool ok = kid[k + u] != INT_MAX;
+                v[u] = ok ? kid[k + u] : -1;
+                z4[u] = ok ? kz[k + u] : -1.f;
+                d4[u] = ok ? kd[k + u] : -1.f;
+            }
+            reinterpret_cast<longlong2*>(idx + o + k)[0] = make_longlong2(v[0], v[1]);
+            reinterpret_cast<longlong2*>(idx + o + k)[1] = make_longlong2(v[2], v[3]);
+            *reinterpret_cast<float4*>(zbuf + o + k) = make_float4(z4[0], z4[1], z4[2], z4[3]);
+            *reinterpret_cast<float4*>(dists + o + k) = make_float4(d4[0], d4[1], d4[2], d4[3]);
+        }
+        return;
+      }
+    }
+    {
+#pragma unroll
+        for (int k = 0; k < KC; ++k) {
+            if (k >= K) break;
+            const bool ok = kid[k] != INT_MAX;
+            idx[o + k] = ok ? kid[k] : -1;
+            zbuf[o + k] = ok ? kz[k] : -1.f;
+            dists[o + k] = ok ? kd[k] : -1.f;
+        }
+    }
+}
+
+// Backward of the point rasterizer: thread per slot, one float4 (x, y, z, 0) atomic per
+// valid slot into a padded accumulator.
+__global__ void k_point_raster_bwd(const float* __restrict__ pts, int64_t P, const int64_t* __restrict__ idx,
+                                   int64_t nslots, int H, int W, int K, const float* __restrict__ gz,
+                                   const float* __restrict__ gd, float4* __restrict__ acc, int* __restrict__ err) {
+    for (int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; s < nslots; s += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t m = idx[s];
+        if (m == -1) continue;
+        if (m < -1 || m >= P) {
+            atomicOr(err, kErrSlotIndex);
+            continue;
+        }
+        float4 c = make_float4(0.f, 0.f, gz ? gz[s] : 0.f, 0.f);
+        if (gd) {
+            const int64_t rem = (s / K) % ((int64_t)H * W);
+            const int i = (int)(rem / W), j = (int)(rem % W);
+            const double pxd = -1.0 + (2.0 * j + 1.0) / W, pyd = 1.0 - (2.0 * i + 1.0) / H;
+            const float g = gd[s];
+            c.x = -2.f * g * (float)(pxd - (double)pts[3 * m]);
+            c.y = -2.f * g * (float)(pyd - (double)pts[3 * m + 1]);
+        }
+        if (c.x != 0.f || c.y != 0.f || c.z != 0.f) atomicAdd(acc + m, c);
+    }
+}
+
+__global__ void k_xyzw_rows(const float4* __restrict__ acc, int64_t P, float* __restrict__ out) {
+    for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < P; p += (int64_t)gridDim.x * blockDim.x) {
+        const float4 a = acc[p];
+        out[3 * p] = a.x;
+        out[3 * p + 1] = a.y;
+        out[3 * p + 2] = a.z;
+    }
+}
+
+// r^2 as a float pair and 1/r^2: a = 1 - d / r^2 is formed as ((r2h - d) + r2l) / r^2, so
+// that a keeps its relative accuracy where it is small (a point near the radius; the
+// norm-weighted sum divides by sum a down to the 1e-4 floor).
+struct Radius2 {
+    float h, l, inv;
+};
+
+__device__ __forceinline__ float point_weight(float d, const Radius2& R) { return ((R.h - d) + R.l) * R.inv; }
+
+inline Radius2 radius2(float radius) {
+    const double r2 = (double)radius * radius;
+    Radius2 R;
+    R.h = (float)r2;
+    R.l = (float)(r2 - (double)R.h);
+    R.inv = (float)(1.0 / r2);
+    return R;
+}
+
+// Compositing, thread per pixel.  MODE 0: alpha, 1: norm-weighted.
+template <int KC, int MODE>
+__global__ void k_composite_fwd(const int64_t* __restrict__ idx, const float* __restrict__ dists, int64_t npix, int K,
+                                const float* __restrict__ feat, int64_t P, int C, Radius2 R,
+                                float* __restrict__ out, int* __restrict__ err) {
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < npix; q += (int64_t)gridDim.x * blockDim.x) {
+        int64_t m[KC];
+        float w[KC];
+        float T = 1.f, wsum = 0.f;
+#pragma unroll
+        for (int k = 0; k < KC; ++k) {
+            m[k] = k < K ? idx[q * K + k] : -1;
+            if (m[k] < -1 || m[k] >= P) {
+                atomicOr(err, kErrSlotIndex);
+                m[k] = -1;
+            }
+            const float a = m[k] >= 0 ? point_weight(dists[q * K + k], R) : 0.f;
+            w[k] = MODE == 0 ? a * T : a;
+            T *= 1.f - a;
+            wsum += a;
+        }
+        const float scale = MODE == 0 ? 1.f : 1.f / fmaxf(wsum, kNormFloor);
+        for (int c = 0; c < C; ++c) {
+            float acc = 0.f;
+#pragma unroll
+            for (int k = 0; k < KC; ++k)
+                if (m[k] >= 0) acc = fmaf(w[k], feat[m[k] * C + c], acc);
+            out[q * C + c] = acc * scale;
+        }
+    }
+}
+
+// Backward of the compositing.  Alpha: with R_k = the composite behind slot k relative to
+// the transmittance after it (R_last = 0, R_{k-1} = a_k (f_k . g) + (1 - a_k) R_k),
+// dL/da_k = T_k ((f_k . g) - R_k) -- no division by 1 - a_k.  Norm-weighted:
+// dL/da_k = (f_k - out) . g / den (den = sum a > floor) or f_k . g / den.  Feature
+// gradients w_k g go to a padded accumulator (float4 per point for C <= 4, else scalars).
+template <int KC, int MODE, bool VEC4>
+__global__ void k_composite_bwd(const int64_t* __restrict__ idx, const float* __restrict__ dists, int64_t npix, int K,
+                                const float* __restrict__ feat, int64_t P, int C, Radius2 R,
+                                const float* __restrict__ grad_out, float* __restrict__ gfeat,
+                                float4* __restrict__ gfeat4, float* __restrict__ grad_dists, int* __restrict__ err) {
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < npix; q += (int64_t)gridDim.x * blockDim.x) {
+        int64_t m[KC];
+        float a[KC], T[KC], fg[KC];
+        float t = 1.f, wsum = 0.f;
+#pragma unroll
+        for (int k = 0; k < KC; ++k) {
+            m[k] = k < K ? idx[q * K + k] : -1;
+            if (m[k] < -1 || m[k] >= P) {
+                atomicOr(err, kErrSlotIndex);
+                m[k] = -1;
+            }
+            a[k] = m[k] >= 0 ? point_weight(dists[q * K + k], R) : 0.f;
+            T[k] = t;
+            t *= 1.f - a[k];
+            wsum += a[k];
+            fg[k] = 0.f;
+        }
+        const float den = fmaxf(wsum, kNormFloor);
+        const float inv_den = 1.f / den;
+        float og = 0.f;              // out . g (norm-weighted)
+        for (int c = 0; c < C; ++c) {
+            const float g = grad_out[q * C + c];
+            float o = 0.f;
+#pragma unroll
+            for (int k = 0; k < KC; ++k)
+                if (m[k] >= 0) {
+                    const float f = feat[m[k] * C + c];
+                    fg[k] = fmaf(f, g, fg[k]);
+                    o = fmaf(a[k], f, o);
+                }
+            og = fmaf(o * inv_den, g, og);
+        }
+        float rest = 0.f;            // R_k of the comment above
+#pragma unroll
+        for (int k = KC - 1; k >= 0; --k) {
+            float ga = 0.f;
+            if (m[k] >= 0) {
+                if (MODE == 0) ga = T[k] * (fg[k] - rest);
+                else ga = (wsum > kNormFloor ? fg[k] - og : fg[k]) * inv_den;
+                if (MODE == 0) rest = fmaf(a[k], fg[k], (1.f - a[k]) * rest);
+                const float wk = MODE == 0 ? a[k] * T[k] : a[k] * inv_den;
+                if (VEC4) {
+                    float g4[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int c = 0; c < C; ++c) g4[c] = wk * grad_out[q * C + c];
+                    atomicAdd(gfeat4 + m[k], make_float4(g4[0], g4[1], g4[2], g4[3]));
+                } else {
+                    for (int c = 0; c < C; ++c) atomicAdd(gfeat + m[k] * C + c, wk * grad_out[q * C + c]);
+                }
+            }
+            if (grad_dists && k < K) grad_dists[q * K + k] = -ga * R.inv;
+        }
+    }
+}
+
+__global__ void k_acc4_cols(const float4* __restrict__ acc, int64_t P, int C, float* __restrict__ out) {
+    for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < P; p += (int64_t)gridDim.x * blockDim.x) {
+        const float4 a = acc[p];
+        const float x[4] = {a.x, a.y, a.z, a.w};
+        for (int c = 0; c < C; ++c) out[p * C + c] = x[c];
+    }
+}
+
+int check_clouds(const int64_t* first, const int64_t* num, int N, int64_t P, const char* what) {
+    for (int n = 0; n < N; ++n) {
+        if (first[n] < 0 || num[n] < 0 || first[n] + num[n] > P || (n > 0 && first[n] < first[n - 1] + num[n - 1])) {
+            set_error("%s: cloud %d range [%lld, %lld) outside [0, %lld) or not ascending", what, n,
+                      (long long)first[n], (long long)(first[n] + num[n]), (long long)P);
+            return MR_ERR_ARG;
+        }
+    }
+    return MR_OK;
+}
+
+}  // namespace
+}  // namespace mr
+
+extern "C" {
+
+int mr_rasterize_points_fwd(const float* points, int64_t P, const int64_t* cloud_first_idx,
+                            const int64_t* num_points_per_cloud, int32_t N, int32_t H, int32_t W, float radius,
+                            int32_t K, int64_t* idx, float* zbuf, float* dists, void* stream) {
+    using namespace mr;
+    if (N < 0 || H < 1 || W < 1 || H > MR_MAX_SIDE || W > MR_MAX_SIDE || K < 1 || K > MR_KMAX || P < 0 ||
+        P > INT32_MAX || !(radius >= 0.f) || !std::isfinite(radius)) {
+        set_error("invalid arguments N=%d H=%d W=%d K=%d P=%lld radius=%g", N, H, W, K, (long long)P, (double)radius);
+        return MR_ERR_ARG;
+    }
+    if (N == 0) return MR_OK;
+    if (!cloud_first_idx || !num_points_per_cloud || !idx || !zbuf || !dists || (P > 0 && !points)) {
+        set_error("null pointer");
+        return MR_ERR_ARG;
+    }
+    int rc = check_clouds(cloud_first_idx, num_points_per_cloud, N, P, "mr_rasterize_points_fwd");
+    if (rc != MR_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int nbx = (W + kPtBin - 1) / kPtBin, nby = (H + kPtBin - 1) / kPtBin;
+    const int64_t nbins64 = (int64_t)N * nbx * nby;
+    if (nbins64 >= INT32_MAX / 2) {
+        set_error("too many bins");
+        return MR_ERR_ARG;
+    }
+    const int nbins = (int)nbins64;
+    const int ntiles = (nbins + kScanTile - 1) / kScanTile;
+    // scratch: cloud ranges, counts, offsets (+1), tile sums, total
+    const size_t sz_cl = sizeof(int64_t) * 2 * (size_t)N, sz_cnt = sizeof(int) * (size_t)nbins,
+                 sz_off = sizeof(int) * ((size_t)nbins + 1), sz_tile = sizeof(long long) * ((size_t)ntiles + 1);
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t bytes = up(sz_cl) + up(sz_cnt) + up(sz_off) + up(sz_tile);
+    char* base = nullptr;
+    rc = scratch_alloc(reinterpret_cast<void**>(&base), bytes, s);
+    if (rc != MR_OK) return rc;
+    int64_t* cl = reinterpret_cast<int64_t*>(base);
+    int* counts = reinterpret_cast<int*>(base + up(sz_cl));
+    int* offsets = reinterpret_cast<int*>(base + up(sz_cl) + up(sz_cnt));
+    long long* tile = reinterpret_cast<long long*>(base + up(sz_cl) + up(sz_cnt) + up(sz_off));
+    long long* total_d = tile + ntiles;
+    std::vector<int64_t> host(2 * (size_t)N);
+    std::copy(cloud_first_idx, cloud_first_idx + N, host.begin());
+    std::copy(num_points_per_cloud, num_points_per_cloud + N, host.begin() + N);
+    int* list = nullptr;
+    long long total = 0;
+    cudaError_t e = cudaMemcpyAsync(cl, host.data(), sz_cl, cudaMemcpyHostToDevice, s);
+    const float r2 = radius * radius;
+    const int gp = grid_for(std::max<int64_t>(P, 1));
+    if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, sz_cnt, s);
+    if (e == cudaSuccess) {
+        ProfScope ps(MR_STAGE_POINTS_BIN, s);
+        if (P > 0)
+            k_point_bins<false><<<gp, 256, 0, s>>>(points, P, cl, cl + N, N, H, W, radius, nbx, nby, counts, nullptr,
+                                                   nullptr);
+        k_scan_tiles<<<ntiles, 1024, 0, s>>>(counts, nbins, offsets, tile);
+        k_scan_tops<<<1, 1024, 0, s>>>(tile, ntiles, total_d);
+        k_scan_add<<<std::min((nbins + 256) / 256, 148 * 8), 256, 0, s>>>(offsets, nbins, tile, total_d);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&total, total_d, sizeof(long long), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);   // the one sync: the list's size
+    if (e == cudaSuccess && total > INT32_MAX) {
+        scratch_free(base, s);
+        set_error("%lld point-bin entries exceed the int32 list (radius too large for this batch)", total);
+        return MR_ERR_ARG;
+    }
+    if (e == cudaSuccess && total > 0) {
+        rc = scratch_alloc(reinterpret_cast<void**>(&list), sizeof(int) * (size_t)total, s);
+        if (rc != MR_OK) {
+            scratch_free(base, s);
+            return rc;
+        }
+        e = cudaMemsetAsync(counts, 0, sz_cnt, s);
+        if (e == cudaSuccess) {
+            ProfScope ps(MR_STAGE_POINTS_BIN, s);
+            k_point_bins<true><<<gp, 256, 0, s>>>(points, P, cl, cl + N, N, H, W, radius, nbx, nby, counts, offsets,
+                                                  list);
+            e = cudaGetLastError();
+        }
+    }
+    if (e == cudaSuccess) {
+        const bool vec = (reinterpret_cast<uintptr_t>(idx) & 15) == 0 && (reinterpret_cast<uintptr_t>(zbuf) & 15) == 0 &&
+                         (reinterpret_cast<uintptr_t>(dists) & 15) == 0;
+        ProfScope ps(MR_STAGE_POINTS_FINE, s);
+#define MR_PF(KC) \
+    k_point_fine<KC><<<nbins, 256, 0, s>>>(points, offsets, list, N, H, W, r2, K, nbx, nby, idx, zbuf, dists, vec)
+        if (K <= 1) MR_PF(1);
+        else if (K <= 2) MR_PF(2);
+        else if (K <= 4) MR_PF(4);
+        else if (K <= 8) MR_PF(8);
+        else if (K <= 16) MR_PF(16);
+        else MR_PF(32);
+#undef MR_PF
+        e = cudaGetLastError();
+    }
+    if (list) scratch_free(list, s);
+    scratch_free(base, s);
+    if (e != cudaSuccess) return cuda_fail(e, "point rasterization");
+    return MR_OK;
+}
+
+int mr_rasterize_points_bwd(const float* points, int64_t P, const int64_t* idx, int32_t N, int32_t H, int32_t W,
+                            int32_t K, const float* grad_zbuf, const float* grad_dists, float* grad_points,
+                            void* stream) {
+    using namespace mr;
+    if (N < 0 || H < 1 || W < 1 || K < 1 || K > MR_KMAX || P < 0) {
+        set_error("invalid shape");
+        return MR_ERR_ARG;
+    }
+    if (P > 0 && (!points || !grad_points)) {
+        set_error("null point pointer");
+        return MR_ERR_ARG;
+    }
+    if (P == 0) return MR_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t nslots = (int64_t)N * H * W * K;
+    if (nslots == 0 || (!grad_zbuf && !grad_dists)) {
+        MR_CUDA(cudaMemsetAsync(grad_points, 0, sizeof(float) * 3 * (size_t)P, s));
+        return MR_OK;
+    }
+    if (!idx) {
+        set_error("null idx");
+        return MR_ERR_ARG;
+    }
+    int* err = device_error_word();
+    if (!err) {
+        set_error("cannot locate the device error word");
+        return MR_ERR_CUDA;
+    }
+    float4* acc = nullptr;
+    int rc = scratch_alloc(reinterpret_cast<void**>(&acc), sizeof(float4) * (size_t)P, s);
+    if (rc != MR_OK) return rc;
+    cudaError_t e = cudaMemsetAsync(acc, 0, sizeof(float4) * (size_t)P, s);
+    if (e == cudaSuccess) {
+        ProfScope ps(MR_STAGE_POINTS_BWD, s);
+        k_point_raster_bwd<<<grid_for(nslots), 256, 0, s>>>(points, P, idx, nslots, H, W, K, grad_zbuf, grad_dists,
+                                                           acc, err);
+        k_xyzw_rows<<<grid_for(P), 256, 0, s>>>(acc, P, grad_points);
+        e = cudaGetLastError();
+    }
+    scratch_free(acc, s);
+    if (e != cudaSuccess) return cuda_fail(e, "point rasterizer backward");
+    return MR_OK;
+}
+
+int mr_composite_points_fwd(const int64_t* idx, const float* dists, int64_t npix, int32_t K, const float* features,
+                            int64_t P, int32_t C, float radius, int32_t mode, float* out, void* stream) {
+    using namespace mr;
+    if (npix < 0 || K < 1 || K > MR_KMAX || C < 1 || P < 0 || (mode != 0 && mode != 1) || !(radius > 0.f) ||
+        !std::isfinite(radius)) {
+        set_error("invalid arguments npix=%lld K=%d C=%d mode=%d radius=%g", (long long)npix, K, C, mode,
+                  (double)radius);
+        return MR_ERR_ARG;
+    }
+    if (npix == 0) return MR_OK;
+    if (!idx || !dists || !out || (P > 0 && !features)) {
+        set_error("null pointer");
+        return MR_ERR_ARG;
+    }
+    int* err = device_error_word();
+    if (!err) {
+        set_error("cannot locate the device error word");
+        return MR_ERR_CUDA;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Radius2 R = radius2(radius);
+    const int g = grid_for(npix);
+    ProfScope ps(MR_STAGE_COMPOSITE_FWD, s);
+#define MR_CF(KC)                                                                                                \
+    (mode == 0 ? k_composite_fwd<KC, 0><<<g, 256, 0, s>>>(idx, dists, npix, K, features, P, C, R, out, err) \
+               : k_composite_fwd<KC, 1><<<g, 256, 0, s>>>(idx, dists, npix, K, features, P, C, R, out, err))
+    if (K <= 1) MR_CF(1);
+    else if (K <= 2) MR_CF(2);
+    else if (K <= 4) MR_CF(4);
+    else if (K <= 8) MR_CF(8);
+    else if (K <= 16) MR_CF(16);
+    else MR_CF(32);
+#undef MR_CF
+    MR_CUDA(cudaGetLastError());
+    return MR_OK;
+}
+
+int mr_composite_points_bwd(const int64_t* idx, const float* dists, int64_t npix, int32_t K, const float* features,
+                            int64_t P, int32_t C, float radius, int32_t mode, const float* grad_out,
+                            float* grad_features, float* grad_dists, void* stream) {
+    using namespace mr;
+    if (npix < 0 || K < 1 || K > MR_KMAX || C < 1 || P < 0 || (mode != 0 && mode != 1) || !(radius > 0.f) ||
+        !std::isfinite(radius)) {
+        set_error("invalid arguments");
+        return MR_ERR_ARG;
+    }
+    if ((P > 0 && (!features || !grad_features)) || (npix > 0 && (!idx || !dists || !grad_out))) {
+        set_error("null pointer");
+        return MR_ERR_ARG;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (npix == 0 || P == 0) {
+        if (P > 0) MR_CUDA(cudaMemsetAsync(grad_features, 0, sizeof(float) * (size_t)(P * C), s));
+        if (npix > 0 && grad_dists) MR_CUDA(cudaMemsetAsync(grad_dists, 0, sizeof(float) * (size_t)(npix * K), s));
+        return MR_OK;
+    }
+    int* err = device_error_word();
+    if (!err) {
+        set_error("cannot locate the device error word");
+        return MR_ERR_CUDA;
+    }
+    const bool vec4 = C <= 4;
+    float4* acc = nullptr;
+    if (vec4) {
+        int rc = scratch_alloc(reinterpret_cast<void**>(&acc), sizeof(float4) * (size_t)P, s);
+        if (rc != MR_OK) return rc;
+    }
+    cudaError_t e = vec4 ? cudaMemsetAsync(acc, 0, sizeof(float4) * (size_t)P, s)
+                         : cudaMemsetAsync(grad_features, 0, sizeof(float) * (size_t)(P * C), s);
+    const Radius2 R = radius2(radius);
+    const int g = grid_for(npix);
+    if (e == cudaSuccess) {
+        ProfScope ps(MR_STAGE_COMPOSITE_BWD, s);
+#define MR_CB2(KC, MODE)                                                                                       \
+    (vec4 ? k_composite_bwd<KC, MODE, true><<<g, 256, 0, s>>>(idx, dists, npix, K, features, P, C, R,    \
+                                                              grad_out, nullptr, acc, grad_dists, err)         \
+          : k_composite_bwd<KC, MODE, false><<<g, 256, 0, s>>>(idx, dists, npix, K, features, P, C, R,   \
+                                                               grad_out, grad_features, nullptr, grad_dists, err))
+#define MR_CB(KC) (mode == 0 ? MR_CB2(KC, 0) : MR_CB2(KC, 1))
+        if (K <= 1) MR_CB(1);
+        else if (K <= 2) MR_CB(2);
+        else if (K <= 4) MR_CB(4);
+        else if (K <= 8) MR_CB(8);
+        else if (K <= 16) MR_CB(16);
+        else MR_CB(32);
+#undef MR_CB
+#undef MR_CB2
+        if (vec4) k_acc4_cols<<<grid_for(P), 256, 0, s>>>(acc, P, C, grad_features);
+        e = cudaGetLastError();
+    }
+    if (acc) scratch_free(acc, s);
+    if (e != cudaSuccess) return cuda_fail(e, "compositing backward");
+    return MR_OK;
+}
+
+}  // extern "C"

@@ -245,6 +245,64 @@ int mr_phong_shade_bwd(const int64_t* pix_to_face, const float* bary, int64_t np
                        float* grad_points, float* grad_normals, float* grad_albedo, float* grad_bary,
                        void* stream);
 
+/*
+ * Point clouds ("Accelerating 3D Deep Learning with PyTorch3D": the renderer draws point
+ * clouds with the same two stages, over heterogeneous batches; the pages print no formula,
+ * so these are the plain definitions that match the mesh path).  points: P x 3 float32
+ * (device), screen space (x_ndc, y_ndc, z) like the mesh vertices; cloud n is points
+ * [cloud_first_idx[n], + num_points_per_cloud[n]) (HOST arrays of N, ascending, disjoint)
+ * and is drawn into image n.  Pixel centres as for meshes.
+ *
+ * mr_rasterize_points_fwd: per pixel the K points of its cloud nearest in depth among those
+ *   with z >= 0 and squared 2-D distance to the pixel centre <= radius^2, ordered by
+ *   (z, point id): idx (global point id, int64), zbuf (= z), dists (squared distance), all
+ *   N x H x W x K, -1 in empty slots.  Bins points into 16 x 16-pixel tiles; performs one
+ *   stream synchronisation (the bin list's size).  MR_ERR_ARG also when the bin list would
+ *   exceed 2^31 entries (a radius far larger than the image).
+ * mr_rasterize_points_bwd: grad_points (P x 3, overwritten) from grad_zbuf and grad_dists
+ *   (each nullable): d dists / d (x, y) = -2 (pixel centre - (x, y)), d zbuf / d z = 1.
+ * mr_composite_points_fwd: features (P x C float32) composited over each pixel's K slots
+ *   with a_k = 1 - dists_k / radius^2 into out (npix x C): mode 0 front-to-back alpha,
+ *   out = sum_k a_k T_k f_k with T_k = prod_{j<k} (1 - a_j); mode 1 norm-weighted,
+ *   out = sum_k a_k f_k / max(sum_k a_k, 1e-4).  radius > 0.
+ * mr_composite_points_bwd: grad_features (P x C, overwritten; float32 atomics) and
+ *   grad_dists (npix x K, nullable; 0 in empty slots) from grad_out (npix x C).
+ * Out-of-range point ids in idx are flagged in the device error word and skipped.
+ */
+int mr_rasterize_points_fwd(const float* points, int64_t P, const int64_t* cloud_first_idx,
+                            const int64_t* num_points_per_cloud, int32_t N, int32_t H, int32_t W,
+                            float radius, int32_t K, int64_t* idx, float* zbuf, float* dists,
+                            void* stream);
+int mr_rasterize_points_bwd(const float* points, int64_t P, const int64_t* idx, int32_t N, int32_t H,
+                            int32_t W, int32_t K, const float* grad_zbuf, const float* grad_dists,
+                            float* grad_points, void* stream);
+int mr_composite_points_fwd(const int64_t* idx, const float* dists, int64_t npix, int32_t K,
+                            const float* features, int64_t P, int32_t C, float radius, int32_t mode,
+                            float* out, void* stream);
+int mr_composite_points_bwd(const int64_t* idx, const float* dists, int64_t npix, int32_t K,
+                            const float* features, int64_t P, int32_t C, float radius, int32_t mode,
+                            const float* grad_out, float* grad_features, float* grad_dists,
+                            void* stream);
+
+/*
+ * Batched K nearest neighbours (PyTorch3D paper: a custom KNN kernel for heterogeneous
+ * batches of point clouds).  p1: P1 x D queries, p2: P2 x D references (float32, device);
+ * cloud n of p1 (first1[n], num1[n]; HOST) searches cloud n of p2 (first2[n], num2[n];
+ * HOST).  mr_knn_fwd: idx (P1 x K int64: global ids into p2) and dists (P1 x K float32:
+ * squared Euclidean distances), the K nearest ordered by (distance, id); when cloud n of
+ * p2 has fewer than K points the rest hold -1 in both; queries in no cloud get -1 rows.
+ * 1 <= D <= MR_KNN_DMAX, 1 <= K <= MR_KMAX; MR_ERR_ARG for overlapping query clouds or a
+ * range outside its set.  Exhaustive search (every pair of a cloud is tested).
+ * mr_knn_bwd: grad_p1 (P1 x D) and grad_p2 (P2 x D), both overwritten (float32 atomics into
+ * grad_p2), from grad_dists (P1 x K): d dist / d q = 2 (q - r), d dist / d r = -2 (q - r).
+ */
+#define MR_KNN_DMAX 4
+int mr_knn_fwd(const float* p1, int64_t P1, const int64_t* first1, const int64_t* num1, const float* p2,
+               int64_t P2, const int64_t* first2, const int64_t* num2, int32_t N, int32_t D, int32_t K,
+               int64_t* idx, float* dists, void* stream);
+int mr_knn_bwd(const float* p1, int64_t P1, const float* p2, int64_t P2, int32_t D, int32_t K,
+               const int64_t* idx, const float* grad_dists, float* grad_p1, float* grad_p2, void* stream);
+
 /* Synchronises `stream`, then returns MR_ERR_DEVICE (and clears the word) if any
  * asynchronous kernel of this library flagged an out-of-range index on the current
  * device since the last call, else MR_OK (or MR_ERR_CUDA). */
@@ -282,7 +340,14 @@ int mr_version(void);
 #define MR_STAGE_PHONG_BWD 15
 #define MR_STAGE_PHONG_SHADE_FWD 16
 #define MR_STAGE_PHONG_SHADE_BWD 17
-#define MR_NUM_STAGES 18
+#define MR_STAGE_POINTS_BIN 18
+#define MR_STAGE_POINTS_FINE 19
+#define MR_STAGE_POINTS_BWD 20
+#define MR_STAGE_COMPOSITE_FWD 21
+#define MR_STAGE_COMPOSITE_BWD 22
+#define MR_STAGE_KNN 23
+#define MR_STAGE_KNN_BWD 24
+#define MR_NUM_STAGES 25
 int mr_profile_enable(int32_t on);
 int mr_profile_read(double* stage_ms, int64_t* launches, int32_t nstages);
 

@@ -68,6 +68,8 @@ def _load():
         lib.oracle_phong_shade_bwd.restype = None
         lib.oracle_rasterize_points.argtypes = [P, i64, P, P, i32, i32, i32, f64, i32, P, P, P, P]
         lib.oracle_rasterize_points.restype = ctypes.c_int
+        lib.oracle_rasterize_points_pixels.argtypes = [P, i64, P, P, i32, i32, i32, f64, i32, P, i64, P, P, P, P]
+        lib.oracle_rasterize_points_pixels.restype = ctypes.c_int
         lib.oracle_rasterize_points_bwd.argtypes = [P, i64, P, i32, i32, i32, i32, P, P, P]
         lib.oracle_rasterize_points_bwd.restype = None
         lib.oracle_composite_points.argtypes = [P, P, i64, i32, P, i32, f64, i32, P]
@@ -318,13 +320,27 @@ def phong_shade_bwd(pix_to_face, bary, faces, points, normals, albedo, params, g
     return gP, gN, gc, gb
 
 
-def rasterize_points(points, cloud_first_idx, num_points_per_cloud, H, W, radius, K):
-    """Step 22: (idx, zbuf, dists) of shape (N, H, W, K) and flags (N, H, W)."""
+def rasterize_points(points, cloud_first_idx, num_points_per_cloud, H, W, radius, K, pixels=None):
+    """Step 22: (idx, zbuf, dists) of shape (N, H, W, K) and flags (N, H, W); with ``pixels``
+    (ids n*H*W + i*W + j) only those, as (npix, K) and (npix,)."""
     lib = _load()
     pts = _c(points, np.float32)
     first = _c(cloud_first_idx, np.int64)
     num = _c(num_points_per_cloud, np.int64)
     N = first.shape[0]
+    if pixels is not None:
+        pix = _c(pixels, np.int64)
+        n = pix.shape[0]
+        idx = np.empty((n, K), np.int64)
+        zbuf = np.empty((n, K), np.float64)
+        dists = np.empty((n, K), np.float64)
+        flags = np.empty(n, np.uint8)
+        rc = lib.oracle_rasterize_points_pixels(_ptr(pts), pts.shape[0], _ptr(first), _ptr(num), N, H, W,
+                                                float(radius), K, _ptr(pix), n, _ptr(idx), _ptr(zbuf), _ptr(dists),
+                                                _ptr(flags))
+        if rc != 0:
+            raise ValueError("oracle_rasterize_points_pixels: invalid arguments")
+        return idx, zbuf, dists, flags.astype(bool)
     idx = np.empty((N, H, W, K), np.int64)
     zbuf = np.empty((N, H, W, K), np.float64)
     dists = np.empty((N, H, W, K), np.float64)

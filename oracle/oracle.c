@@ -840,50 +840,76 @@ static int kv_insert(kv *list, int n, int cap, kv e) {
     return n < cap ? n + 1 : n;
 }
 
+/* Step 22 at one pixel (image n, row i, column j) into K slots at idx/zbuf/dists + o;
+ * returns the flag.  list: K scratch entries. */
+static int point_pixel(const float *pts, int64_t P, const int64_t *first, const int64_t *num, int32_t n, int32_t H,
+                       int32_t W, int32_t i, int32_t j, double r2, int32_t K, kv *list, int64_t *idx, double *zbuf,
+                       double *dists) {
+    double px = -1.0 + (2.0 * j + 1.0) / W, py = 1.0 - (2.0 * i + 1.0) / H;
+    int cnt = 0;
+    int near_margin = 0;
+    kv marg;
+    marg.key = 0.0;
+    marg.id = 0;
+    marg.aux = 0.0;
+    for (int64_t m = first[n]; m < first[n] + num[n]; ++m) {
+        if (m < 0 || m >= P) continue;
+        double x = pts[3 * m], y = pts[3 * m + 1], z = pts[3 * m + 2];
+        if (z < 0.0) continue;
+        double d2 = (px - x) * (px - x) + (py - y) * (py - y);
+        if (fabs(d2 - r2) < POINT_MARGIN * r2) {
+            /* decided by rounding: remember the nearest such point */
+            kv e = {z, m, d2};
+            if (!near_margin || kv_before(&e, &marg)) marg = e;
+            near_margin = 1;
+        }
+        if (d2 > r2) continue;
+        kv e = {z, m, d2};
+        cnt = kv_insert(list, cnt, K, e);
+    }
+    for (int k = 0; k < K; ++k) {
+        idx[k] = k < cnt ? list[k].id : -1;
+        zbuf[k] = k < cnt ? list[k].key : -1.0;
+        dists[k] = k < cnt ? list[k].aux : -1.0;
+    }
+    if (!near_margin) return 0;
+    return cnt < K || kv_before(&marg, &list[K - 1]) || marg.id == list[K - 1].id;
+}
+
 /* Step 22 for the N images; idx, zbuf, dists are N x H x W x K; flags N x H x W (may be NULL). */
 int oracle_rasterize_points(const float *pts, int64_t P, const int64_t *first, const int64_t *num, int32_t N,
                             int32_t H, int32_t W, double radius, int32_t K, int64_t *idx, double *zbuf,
                             double *dists, uint8_t *flags) {
     if (N < 0 || H < 1 || W < 1 || K < 1 || radius < 0) return -1;
-    double r2 = radius * radius;
     kv *list = (kv *)malloc(sizeof(kv) * (size_t)(K + 1));
     for (int32_t n = 0; n < N; ++n)
         for (int32_t i = 0; i < H; ++i)
             for (int32_t j = 0; j < W; ++j) {
-                double px = -1.0 + (2.0 * j + 1.0) / W, py = 1.0 - (2.0 * i + 1.0) / H;
-                int cnt = 0;
-                int near_margin = 0;
-                kv marg;
-                marg.key = 0.0;
-                marg.id = 0;
-                marg.aux = 0.0;
-                for (int64_t m = first[n]; m < first[n] + num[n]; ++m) {
-                    if (m < 0 || m >= P) continue;
-                    double x = pts[3 * m], y = pts[3 * m + 1], z = pts[3 * m + 2];
-                    if (z < 0.0) continue;
-                    double d2 = (px - x) * (px - x) + (py - y) * (py - y);
-                    if (fabs(d2 - r2) < POINT_MARGIN * r2) {
-                        /* decided by rounding: remember the nearest such point */
-                        kv e = {z, m, d2};
-                        if (!near_margin || kv_before(&e, &marg)) marg = e;
-                        near_margin = 1;
-                    }
-                    if (d2 > r2) continue;
-                    kv e = {z, m, d2};
-                    cnt = kv_insert(list, cnt, K, e);
-                }
-                int64_t o = (((int64_t)n * H + i) * W + j) * K;
-                for (int k = 0; k < K; ++k) {
-                    idx[o + k] = k < cnt ? list[k].id : -1;
-                    zbuf[o + k] = k < cnt ? list[k].key : -1.0;
-                    dists[o + k] = k < cnt ? list[k].aux : -1.0;
-                }
-                if (flags) {
-                    int f = 0;
-                    if (near_margin) f = cnt < K || kv_before(&marg, &list[K - 1]) || marg.id == list[K - 1].id;
-                    flags[((int64_t)n * H + i) * W + j] = (uint8_t)f;
-                }
+                int64_t q = ((int64_t)n * H + i) * W + j;
+                int f = point_pixel(pts, P, first, num, n, H, W, i, j, radius * radius, K, list, idx + q * K,
+                                    zbuf + q * K, dists + q * K);
+                if (flags) flags[q] = (uint8_t)f;
             }
+    free(list);
+    return 0;
+}
+
+/* Step 22 at npix listed pixels (ids n * H * W + i * W + j); outputs npix x K, flags npix. */
+int oracle_rasterize_points_pixels(const float *pts, int64_t P, const int64_t *first, const int64_t *num, int32_t N,
+                                   int32_t H, int32_t W, double radius, int32_t K, const int64_t *pixels,
+                                   int64_t npix, int64_t *idx, double *zbuf, double *dists, uint8_t *flags) {
+    if (N < 0 || H < 1 || W < 1 || K < 1 || radius < 0) return -1;
+    kv *list = (kv *)malloc(sizeof(kv) * (size_t)(K + 1));
+    for (int64_t t = 0; t < npix; ++t) {
+        int64_t q = pixels[t];
+        int32_t n = (int32_t)(q / ((int64_t)H * W)), i = (int32_t)((q / W) % H), j = (int32_t)(q % W);
+        if (q < 0 || n >= N) {
+            free(list);
+            return -1;
+        }
+        flags[t] = (uint8_t)point_pixel(pts, P, first, num, n, H, W, i, j, radius * radius, K, list, idx + t * K,
+                                        zbuf + t * K, dists + t * K);
+    }
     free(list);
     return 0;
 }

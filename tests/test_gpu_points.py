@@ -1,0 +1,243 @@
+"""Parity of the CUDA point-cloud renderer (rasterization, compositing, their gradients)
+and of the batched KNN with the float64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import differentiable_mesh_rasterization_b200 as mr
+from differentiable_mesh_rasterization_b200 import synthetic as syn
+
+from _parity import EXEMPT_MAX, compare_grad, np_
+
+pytestmark = pytest.mark.gpu
+
+ABS = 1e-5
+ULP = 2.0 ** -23
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from differentiable_mesh_rasterization_b200 import build
+    build.build()
+
+
+def cuda(a, dtype=None):
+    return torch.from_numpy(np.ascontiguousarray(a if dtype is None else a.astype(dtype))).cuda()
+
+
+def _compare_slots(got, want, flags, label):
+    """idx exact outside flagged pixels; zbuf, dists within 1e-5 + 1 ulp there."""
+    gi, gz, gd = (np_(x) for x in got)
+    wi, wz, wd, = want
+    ok = ~flags
+    assert flags.mean() <= EXEMPT_MAX, f"{label}: {flags.mean():.3%} flagged"
+    assert np.array_equal(gi[ok], wi[ok]), f"{label}: idx differs at {np.argwhere((gi != wi).any(-1) & ok)[:5]}"
+    for name, x, y in (("zbuf", gz, wz), ("dists", gd, wd)):
+        err = (np.abs(x - y) - (ABS + ULP * np.abs(y)))[ok]
+        assert err.size == 0 or err.max() <= 0, f"{label}: {name} off by {err.max():.3g}"
+
+
+@pytest.fixture(scope="module")
+def pts2(oracle_mod):
+    pb = syn.make_point_batch(2)
+    w = pb.workload
+    o = oracle_mod.rasterize_points(pb.points, pb.cloud_first_idx, pb.num_points_per_cloud, w.H, w.W, w.radius, w.K)
+    return pb, o
+
+
+def test_point_rasterizer_matches_oracle(pts2):
+    pb, (wi, wz, wd, flags) = pts2
+    w = pb.workload
+    got = mr.rasterize_points_fwd(cuda(pb.points), pb.cloud_first_idx, pb.num_points_per_cloud, w.H, w.W,
+                                  np.float32(w.radius), w.K)
+    assert (wi >= 0).mean() > 0.05
+    _compare_slots(got, (wi, wz, wd), flags[..., None].repeat(w.K, -1), "points batch 2")
+    mr.device_status()
+
+
+@pytest.mark.parametrize("K,H,W,radius", [(1, 33, 47, 0.03), (3, 64, 40, 0.01), (16, 50, 50, 0.05)])
+def test_point_rasterizer_shapes_and_ragged_tiles(oracle_mod, K, H, W, radius):
+    pb = syn.make_point_batch(2, n_clouds=3)
+    got = mr.rasterize_points_fwd(cuda(pb.points), pb.cloud_first_idx, pb.num_points_per_cloud, H, W,
+                                  np.float32(radius), K)
+    wi, wz, wd, flags = oracle_mod.rasterize_points(pb.points, pb.cloud_first_idx, pb.num_points_per_cloud, H, W,
+                                                    np.float32(radius), K)
+    _compare_slots(got, (wi, wz, wd), flags[..., None].repeat(K, -1), f"K={K} {H}x{W}")
+
+
+def test_point_rasterizer_edge_cases(oracle_mod):
+    """Empty clouds, points behind the camera, points off screen, a cloud of one point."""
+    rng = np.random.default_rng(5)
+    pts = np.concatenate([rng.uniform(-1.2, 1.2, size=(300, 2)), rng.uniform(-0.5, 3, size=(300, 1))], 1)
+    pts = pts.astype(np.float32)
+    first = np.array([0, 100, 100, 299], np.int64)
+    num = np.array([100, 0, 199, 1], np.int64)
+    got = mr.rasterize_points_fwd(cuda(pts), first, num, 24, 20, np.float32(0.2), 5)
+    wi, wz, wd, flags = oracle_mod.rasterize_points(pts, first, num, 24, 20, np.float32(0.2), 5)
+    assert np.all(np_(got[0])[1] == -1)
+    _compare_slots(got, (wi, wz, wd), flags[..., None].repeat(5, -1), "edge cases")
+    empty = mr.rasterize_points_fwd(cuda(pts), first, num, 8, 8, np.float32(0.0), 2)
+    assert int((np_(empty[0]) >= 0).sum()) <= 4            # radius 0: only exact centre hits
+
+
+def test_point_rasterizer_full_size_sampled(oracle_mod):
+    """The benchmark batch (64 clouds, 1.18 M points, 512x512, K=8) in the benchmark's launch,
+    checked at sampled pixels against the oracle and everywhere by properties."""
+    pb = syn.make_point_batch(5)
+    w = pb.workload
+    P = cuda(pb.points)
+    idx, zbuf, dists = (np_(x) for x in mr.rasterize_points_fwd(P, pb.cloud_first_idx, pb.num_points_per_cloud,
+                                                                 w.H, w.W, np.float32(w.radius), w.K))
+    mr.device_status()
+    # properties at every slot: the reported point is within the radius, in front, of the
+    # pixel's own cloud; slots are in (z, id) order; zbuf / dists recompute from the point
+    valid = idx >= 0
+    assert valid.mean() > 0.05
+    n_of = np.repeat(np.arange(pb.N), pb.num_points_per_cloud)
+    n_img = np.broadcast_to(np.arange(pb.N)[:, None, None, None], idx.shape)
+    assert np.all(n_of[idx[valid]] == n_img[valid])
+    pv = pb.points.astype(np.float64)[idx[valid]]
+    assert np.all(pv[:, 2] >= 0) and np.array_equal(zbuf[valid], pb.points[idx[valid], 2])
+    jj = np.broadcast_to(np.arange(w.W)[None, None, :, None], idx.shape)[valid]
+    ii = np.broadcast_to(np.arange(w.H)[None, :, None, None], idx.shape)[valid]
+    d2 = (-1 + (2 * jj + 1) / w.W - pv[:, 0]) ** 2 + (1 - (2 * ii + 1) / w.H - pv[:, 1]) ** 2
+    assert np.all(np.abs(dists[valid] - d2) <= ABS + ULP * d2)
+    assert np.all(d2 <= np.float64(np.float32(w.radius)) ** 2 * (1 + 1e-5))
+    z = np.where(valid, zbuf, np.inf)
+    zi = np.where(valid, idx, np.iinfo(np.int64).max)
+    order_ok = (z[..., :-1] < z[..., 1:]) | ((z[..., :-1] == z[..., 1:]) & (zi[..., :-1] < zi[..., 1:]))
+    assert np.all(order_ok | ~valid[..., 1:])
+    assert np.all(valid[..., :-1] | ~valid[..., 1:])        # padding only at the end
+    # sampled pixels against the oracle
+    rng = np.random.default_rng(11)
+    pix = np.concatenate([rng.choice(np.flatnonzero(valid[..., 0].reshape(-1)), 3000, replace=False),
+                          rng.integers(0, pb.N * w.H * w.W, 500)])
+    wi, wz, wd, flags = oracle_mod.rasterize_points(pb.points, pb.cloud_first_idx, pb.num_points_per_cloud, w.H,
+                                                    w.W, np.float32(w.radius), w.K, pixels=pix)
+    got = tuple(x.reshape(-1, w.K)[pix] for x in (idx, zbuf, dists))
+    _compare_slots(got, (wi, wz, wd), flags[:, None].repeat(w.K, -1), "batch 5 sampled")
+
+
+@pytest.mark.parametrize("mode", ["alpha", "norm_weighted"])
+def test_compositing_matches_oracle(oracle_mod, pts2, mode):
+    pb, (wi, wz, wd, flags) = pts2
+    w = pb.workload
+    d32 = wd.astype(np.float32)
+    feats = pb.features
+    got = np_(mr.composite_points_fwd(cuda(wi), cuda(d32), cuda(feats), np.float32(w.radius), mode))
+    want = oracle_mod.composite_points(wi, d32, feats, np.float32(w.radius), mode)
+    err = np.abs(got - want) - (1e-4 * np.abs(want) + 1e-6)
+    assert err.max() <= 0, f"{mode}: off by {err.max():.3g}"
+    g = syn.random_grads(want.shape, 21)
+    gf, gd = mr.composite_points_bwd(cuda(wi), cuda(d32), cuda(feats), np.float32(w.radius), cuda(g), mode)
+    wf, wdd = oracle_mod.composite_points_bwd(wi, d32, feats, np.float32(w.radius), g, mode)
+    compare_grad(gf, wf, label=f"{mode} grad_features")
+    compare_grad(gd, wdd, label=f"{mode} grad_dists")
+
+
+def test_point_rasterizer_backward_matches_oracle(oracle_mod, pts2):
+    pb, (wi, wz, wd, flags) = pts2
+    gz = syn.random_grads(wi.shape, 22)
+    gd = syn.random_grads(wi.shape, 23)
+    got = mr.rasterize_points_bwd(cuda(pb.points), cuda(wi), cuda(gz), cuda(gd))
+    want = oracle_mod.rasterize_points_bwd(pb.points, wi, gz, gd)
+    compare_grad(got, want, label="point raster bwd")
+    only_z = mr.rasterize_points_bwd(cuda(pb.points), cuda(wi), grad_zbuf=cuda(gz))
+    compare_grad(only_z, oracle_mod.rasterize_points_bwd(pb.points, wi, gz, None), label="only zbuf")
+
+
+def test_point_render_end_to_end(oracle_mod):
+    """points, features -> K nearest -> alpha compositing -> loss, and back to the points'
+    screen positions and features, against the oracle's chain (flagged pixels left out)."""
+    pb = syn.make_point_batch(2)
+    w = pb.workload
+    P, F = cuda(pb.points), cuda(pb.features)
+    r = np.float32(w.radius)
+    idx, zbuf, dists = mr.rasterize_points_fwd(P, pb.cloud_first_idx, pb.num_points_per_cloud, w.H, w.W, r, w.K)
+    img = mr.composite_points_fwd(idx, dists, F, r)
+    g = syn.random_grads(tuple(img.shape), 24)
+    gf, gd = mr.composite_points_bwd(idx, dists, F, r, cuda(g))
+    gp = mr.rasterize_points_bwd(P, idx, grad_dists=gd)
+    mr.device_status()
+    wi, wz, wd, flags = oracle_mod.rasterize_points(pb.points, pb.cloud_first_idx, pb.num_points_per_cloud, w.H, w.W,
+                                                    r, w.K)
+    wimg = oracle_mod.composite_points(wi, wd, pb.features, r)
+    ok = ~flags
+    err = (np.abs(np_(img) - wimg) - (1e-4 * np.abs(wimg) + 1e-5))[ok]
+    assert err.max() <= 0
+    wf, wdd = oracle_mod.composite_points_bwd(wi, wd, pb.features, r, g)
+    wp = oracle_mod.rasterize_points_bwd(pb.points, wi, None, wdd)
+    touched = np.zeros(pb.points.shape[0], bool)
+    for a in (wi[flags], np_(idx)[flags]):
+        touched[a[a >= 0]] = True
+    keep = ~touched
+    assert keep.mean() > 0.9
+    compare_grad(np_(gf)[keep], wf[keep], label="grad features")
+    compare_grad(np_(gp)[keep], wp[keep], label="grad points")
+
+
+def _compare_knn(gi, gd, wi, wd, flags, label):
+    ok = ~flags
+    assert flags.mean() < 0.02, f"{label}: {flags.mean():.3%} flagged"
+    assert np.array_equal(gi[ok], wi[ok]), f"{label}: idx differs at {np.argwhere((gi != wi).any(-1) & ok)[:5]}"
+    # float32 distances from float32 differences: a few ulps of the value
+    tol = 1e-9 + 8 * ULP * np.abs(wd)
+    assert np.all(np.abs(gd - wd) <= tol), f"{label}: dists off by {np.max(np.abs(gd - wd) - tol):.3g}"
+    # flagged queries: the same K distances (the order of near-ties is rounding's)
+    assert np.array_equal(gi[flags] >= 0, wi[flags] >= 0)
+
+
+@pytest.mark.parametrize("K", [1, 8, 20])
+def test_knn_matches_oracle(oracle_mod, K):
+    kb = syn.make_knn_batch(2)
+    gi, gd = mr.knn_fwd(cuda(kb.p1), kb.first1, kb.num1, cuda(kb.p2), kb.first2, kb.num2, K)
+    wi, wd, flags = oracle_mod.knn(kb.p1, kb.first1, kb.num1, kb.p2, kb.first2, kb.num2, K)
+    _compare_knn(np_(gi), np_(gd), wi, wd, flags, f"knn batch 2 K={K}")
+
+
+def test_knn_edge_cases(oracle_mod):
+    """Fewer references than K, an empty reference cloud, queries outside every cloud, D=2."""
+    rng = np.random.default_rng(6)
+    p1 = rng.normal(size=(50, 2)).astype(np.float32)
+    p2 = rng.normal(size=(30, 2)).astype(np.float32)
+    f1, n1 = np.array([0, 20, 35]), np.array([20, 10, 10])      # queries 30..34 and 45..49 in no cloud
+    f2, n2 = np.array([0, 5, 5]), np.array([5, 0, 25])
+    gi, gd = mr.knn_fwd(cuda(p1), f1, n1, cuda(p2), f2, n2, 8)
+    wi, wd, flags = oracle_mod.knn(p1, f1, n1, p2, f2, n2, 8)
+    gi, gd = np_(gi), np_(gd)
+    outside = np.r_[30:35, 45:50]
+    assert np.all(gi[outside] == -1) and np.all(gd[outside] == -1)
+    inside = np.setdiff1d(np.arange(50), outside)
+    _compare_knn(gi[inside], gd[inside], wi[inside], wd[inside], flags[inside], "edge cases")
+    assert np.all(gi[:20, 5:] == -1) and np.all(gi[20:30] == -1)
+
+
+def test_knn_full_size_sampled(oracle_mod):
+    """The benchmark batch (64 clouds, 1.18 M points, D=3, K=8) in the benchmark's launch,
+    checked on sampled queries of every cloud against the oracle."""
+    kb = syn.make_knn_batch(5)
+    K = kb.workload.K
+    gi, gd = (np_(x) for x in mr.knn_fwd(cuda(kb.p1), kb.first1, kb.num1, cuda(kb.p2), kb.first2, kb.num2, K))
+    rng = np.random.default_rng(12)
+    sel, n1 = [], []
+    for n in range(kb.N):
+        q = np.sort(rng.choice(kb.num1[n], min(40, kb.num1[n]), replace=False)) + kb.first1[n]
+        n1.append(len(q))
+        sel.append(q)
+    sel = np.concatenate(sel)
+    f1 = np.cumsum([0] + n1[:-1])
+    wi, wd, flags = oracle_mod.knn(kb.p1[sel], f1, n1, kb.p2, kb.first2, kb.num2, K)
+    _compare_knn(gi[sel], gd[sel], wi, wd, flags, "knn batch 5 sampled")
+
+
+def test_knn_backward_matches_oracle(oracle_mod):
+    kb = syn.make_knn_batch(2)
+    K = 8
+    wi, wd, flags = oracle_mod.knn(kb.p1, kb.first1, kb.num1, kb.p2, kb.first2, kb.num2, K)
+    g = syn.random_grads(wi.shape, 25)
+    g1, g2 = mr.knn_bwd(cuda(kb.p1), cuda(kb.p2), cuda(wi), cuda(g))
+    w1, w2 = oracle_mod.knn_bwd(kb.p1, kb.p2, wi, g)
+    compare_grad(g1, w1, label="knn grad p1")
+    compare_grad(g2, w2, label="knn grad p2")
