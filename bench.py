@@ -330,10 +330,14 @@ def shading_step_timing(mr, torch, dev, stream, batch, verts, faces, first, num,
                 "mpix_per_s": npix / (ms / 1e3) / 1e6, "steps": steps, "stages": stages,
                 "hbm_peak_note": hbm_note, "note": note + "; same workload, L2 flushed per step"}
 
-    return {"gouraud_rgb": timed(gouraud, "Gouraud: stage one + Phong lighting at the vertices + colour "
-                                          "interpolation + soft RGB blend (gamma 1e-2), fwd+bwd"),
-            "phong_rgb": timed(phong, "Phong: stage one + per-fragment interpolation and lighting (fused) + "
-                                      "soft RGB blend (gamma 1e-2), fwd+bwd")}
+    out = {}
+    if "gouraud" in args.rows:
+        out["gouraud_rgb"] = timed(gouraud, "Gouraud: stage one + Phong lighting at the vertices + colour "
+                                            "interpolation + soft RGB blend (gamma 1e-2), fwd+bwd")
+    if "phong" in args.rows:
+        out["phong_rgb"] = timed(phong, "Phong: stage one + per-fragment interpolation and lighting (fused) + "
+                                        "soft RGB blend (gamma 1e-2), fwd+bwd")
+    return out
 
 
 def _timed_steps(mr, torch, dev, stream, flush, steps, step):
@@ -378,7 +382,7 @@ def points_step_timing(mr, torch, dev, stream, flush, args, hbm_peak, hbm_note):
     """Point-cloud render step: 64 clouds (1.18 M points) -> K=8 nearest per pixel at 512x512
     -> alpha compositing of RGB features -> backward to the points and features."""
     from differentiable_mesh_rasterization_b200 import synthetic as syn
-    pb = syn.make_point_batch(5)
+    pb = syn.make_point_batch(5, n_clouds=args.images)
     w = pb.workload
     P = torch.from_numpy(pb.points).to(dev)
     F = torch.from_numpy(pb.features).to(dev)
@@ -416,7 +420,7 @@ def knn_step_timing(mr, torch, dev, stream, flush, args, peak_alu):
     """Batched KNN step: 64 heterogeneous clouds (1.18 M queries against 1.18 M references,
     D=3, K=8) forward and backward."""
     from differentiable_mesh_rasterization_b200 import synthetic as syn
-    kb = syn.make_knn_batch(5)
+    kb = syn.make_knn_batch(5, n_clouds=args.images)
     K = kb.workload.K
     A = torch.from_numpy(kb.p1).to(dev)
     B = torch.from_numpy(kb.p2).to(dev)
@@ -452,8 +456,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-shading", action="store_true", help="skip the Gouraud, Phong, point-cloud and KNN measurements")
+    ap.add_argument("--rows", default="gouraud,phong,points,knn",
+                    help="comma-separated next-row measurements after the main step (gouraud, phong, points, knn)")
     ap.add_argument("--images", type=int, default=None,
-                    help="render only the first N meshes of the batch (small profiling case)")
+                    help="render only the first N meshes of the batch, clouds of the point and KNN batches "
+                         "(small profiling case)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -610,12 +617,18 @@ def main():
             "gpu_launches": int(sum(v[1] * KERNELS_PER_STAGE.get(k, 1) for k, v in stages.items())),
             "clocks": clk}
 
-    if not args.no_shading:
-        line["next_rows"] = shading_step_timing(mr, torch, dev, stream, batch, verts, faces, first, num, flush,
-                                                args, hbm_peak, hbm_note)
-        line["next_rows"]["points_rgb"] = points_step_timing(mr, torch, dev, stream, flush, args, hbm_peak,
-                                                             hbm_note)
-        line["next_rows"]["knn"] = knn_step_timing(mr, torch, dev, stream, flush, args, peak_alu)
+    if args.no_shading:
+        args.rows = ""
+    rows = {}
+    if "gouraud" in args.rows or "phong" in args.rows:
+        rows.update(shading_step_timing(mr, torch, dev, stream, batch, verts, faces, first, num, flush, args, hbm_peak,
+                                        hbm_note))
+    if "points" in args.rows:
+        rows["points_rgb"] = points_step_timing(mr, torch, dev, stream, flush, args, hbm_peak, hbm_note)
+    if "knn" in args.rows:
+        rows["knn"] = knn_step_timing(mr, torch, dev, stream, flush, args, peak_alu)
+    if rows:
+        line["next_rows"] = rows
 
     if rank == 0 and not args.no_cpu_baseline:
         import oracle

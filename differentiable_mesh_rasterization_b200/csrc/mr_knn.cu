@@ -4,12 +4,14 @@
 // For query i of cloud n of the first set, the squared Euclidean distance to every point j
 // of cloud n of the second set; the K smallest, ordered by (distance, j).
 //
-// Exhaustive search, tiled: a CTA owns 256 queries of one cloud (one per thread, the
-// query in registers) and streams the reference cloud through shared memory in chunks of
-// 1024 points; each thread keeps its K best in registers and tests a reference against
-// its current K-th distance before inserting.  The distance is formed from coordinate
-// differences (not |q|^2 + |r|^2 - 2 q.r, which cancels for near neighbours).  Tiles are
-// issued largest reference cloud first, so the long tiles start early.
+// Exact search, tiled: a CTA owns 256 queries of one cloud (one per thread, the query in
+// registers) and streams the reference cloud through shared memory in chunks of 1024
+// points, with the bounding box of every group of 32 references; a warp skips a group
+// whose box lies beyond the K-th distance of all its 32 queries (exact: the box bounds
+// every distance in it), otherwise each thread tests the 32 references, four distances at
+// a time, against its current K-th distance and keeps its K best in registers.  The
+// distance is formed from coordinate differences (not |q|^2 + |r|^2 - 2 q.r, which cancels
+// for near neighbours).  Tiles are issued largest reference cloud first.
 #include <algorithm>
 #include <cfloat>
 #include <climits>
@@ -54,11 +56,14 @@ template <int KC, int D>
 __global__ void __launch_bounds__(kKnnQueries) k_knn(const float* __restrict__ p1, const float* __restrict__ p2,
                                                      const KnnTile* __restrict__ tiles, int K,
                                                      int64_t* __restrict__ idx, float* __restrict__ dists) {
+    constexpr int kGroups = kKnnChunk / 32;
     __shared__ float4 sr[kKnnChunk];
+    __shared__ float4 blo[kGroups], bhi[kGroups];     // box of each group of 32 references
     const KnnTile T = tiles[blockIdx.x];
+    const int lane = threadIdx.x & 31;
     const int64_t qi = T.q0 + threadIdx.x;
     const bool live = threadIdx.x < T.qn;
-    float q[D];
+    float q[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int e = 0; e < D; ++e) q[e] = live ? p1[qi * D + e] : 0.f;
     float kd[KC];
@@ -71,25 +76,69 @@ __global__ void __launch_bounds__(kKnnQueries) k_knn(const float* __restrict__ p
     for (int64_t c0 = 0; c0 < T.rn; c0 += kKnnChunk) {
         __syncthreads();
         const int cnt = (int)min((int64_t)kKnnChunk, T.rn - c0);
-        for (int t = threadIdx.x; t < cnt; t += kKnnQueries) {
-            const int64_t r = T.r0 + c0 + t;
+        // each warp loads groups of 32 references and their bounding box
+        for (int t = threadIdx.x; t < kKnnChunk; t += kKnnQueries) {
+            const bool in = t < cnt;
             float v[4] = {0.f, 0.f, 0.f, 0.f};
+            if (in) {
+                const int64_t r = T.r0 + c0 + t;
 #pragma unroll
-            for (int e = 0; e < D; ++e) v[e] = p2[r * D + e];
+                for (int e = 0; e < D; ++e) v[e] = p2[r * D + e];
+            }
             sr[t] = make_float4(v[0], v[1], v[2], v[3]);
+            float lo[4], hi[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                lo[e] = in ? v[e] : FLT_MAX;
+                hi[e] = in ? v[e] : -FLT_MAX;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int e = 0; e < D; ++e) {
+                    lo[e] = fminf(lo[e], __shfl_xor_sync(0xffffffffu, lo[e], o));
+                    hi[e] = fmaxf(hi[e], __shfl_xor_sync(0xffffffffu, hi[e], o));
+                }
+            if (lane == 0) {
+                blo[t >> 5] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+                bhi[t >> 5] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+            }
         }
         __syncthreads();
         const int id0 = (int)(T.r0 + c0);
-        for (int t = 0; t < cnt; ++t) {
-            const float4 r = sr[t];
-            const float rv[4] = {r.x, r.y, r.z, r.w};
-            float d = 0.f;
+        const int ngroups = (cnt + 31) >> 5;
+        for (int gi = 0; gi < ngroups; ++gi) {
+            // skip the group when its box is farther than this lane's K-th distance, for
+            // every lane of the warp (the bound is shrunk by 2^-20 against rounding)
+            const float4 lo4 = blo[gi], hi4 = bhi[gi];
+            const float lo[4] = {lo4.x, lo4.y, lo4.z, lo4.w}, hi[4] = {hi4.x, hi4.y, hi4.z, hi4.w};
+            float lb = 0.f;
 #pragma unroll
             for (int e = 0; e < D; ++e) {
-                const float u = q[e] - rv[e];
-                d = fmaf(u, u, d);
+                const float gap = fmaxf(fmaxf(lo[e] - q[e], q[e] - hi[e]), 0.f);
+                lb = fmaf(gap, gap, lb);
             }
-            if (d < kd[KC - 1]) insert_nn<KC>(kd, ki, d, id0 + t);   // ids ascend: ties keep the earlier
+            const bool far = !live || lb * (1.f - 0x1p-20f) > kd[KC - 1];
+            if (__all_sync(0xffffffffu, far)) continue;
+            const int t0 = gi * 32, t1 = min(t0 + 32, cnt);
+            for (int t = t0; t < t1; t += 4) {
+                float d4[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 r = sr[min(t + u, kKnnChunk - 1)];
+                    const float rv[4] = {r.x, r.y, r.z, r.w};
+                    float d = 0.f;
+#pragma unroll
+                    for (int e = 0; e < D; ++e) {
+                        const float w = q[e] - rv[e];
+                        d = fmaf(w, w, d);
+                    }
+                    d4[u] = t + u < t1 ? d : FLT_MAX;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)   // ids ascend: a tie keeps the earlier id
+                    if (d4[u] < kd[KC - 1]) insert_nn<KC>(kd, ki, d4[u], id0 + t + u);
+            }
         }
     }
     if (!live) return;

@@ -103,79 +103,89 @@ __device__ __forceinline__ void insert_point(float (&kz)[KC], int (&kid)[KC], fl
     }
 }
 
+// One pixel's K slots from its register list (16-byte stores when K is a multiple of 4 and
+// the outputs are 16-byte aligned).
+template <int KC>
+__device__ __forceinline__ void write_point_slots(const float (&kz)[KC], const int (&kid)[KC], const float (&kd)[KC],
+                                                  int K, int64_t o, bool vec, int64_t* __restrict__ idx,
+                                                  float* __restrict__ zbuf, float* __restrict__ dists) {
+    if constexpr (KC >= 4) {
+        if (vec && (K & 3) == 0) {
+#pragma unroll
+            for (int k = 0; k < KC; k += 4) {
+                if (k >= K) break;
+                long long v[4];
+                float z4[4], d4[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const bool ok = kid[k + u] != INT_MAX;
+                    v[u] = ok ? kid[k + u] : -1;
+                    z4[u] = ok ? kz[k + u] : -1.f;
+                    d4[u] = ok ? kd[k + u] : -1.f;
+                }
+                reinterpret_cast<longlong2*>(idx + o + k)[0] = make_longlong2(v[0], v[1]);
+                reinterpret_cast<longlong2*>(idx + o + k)[1] = make_longlong2(v[2], v[3]);
+                *reinterpret_cast<float4*>(zbuf + o + k) = make_float4(z4[0], z4[1], z4[2], z4[3]);
+                *reinterpret_cast<float4*>(dists + o + k) = make_float4(d4[0], d4[1], d4[2], d4[3]);
+            }
+            return;
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+        if (k >= K) break;
+        const bool ok = kid[k] != INT_MAX;
+        idx[o + k] = ok ? kid[k] : -1;
+        zbuf[o + k] = ok ? kz[k] : -1.f;
+        dists[o + k] = ok ? kd[k] : -1.f;
+    }
+}
+
+// Fine pass: a CTA of 256 threads (one per pixel of a 16 x 16 bin) walks the bins
+// b = blockIdx.x, + gridDim.x, ... (most bins of a batch hold few or no points, so a CTA
+// per bin would spend its time being scheduled).
 template <int KC>
 __global__ void __launch_bounds__(256) k_point_fine(const float* __restrict__ pts, const int* __restrict__ offsets,
-                                                    const int* __restrict__ list, int N, int H, int W, float r2,
+                                                    const int* __restrict__ list, int nbins, int H, int W, float r2,
                                                     int K, int nbx, int nby, int64_t* __restrict__ idx,
                                                     float* __restrict__ zbuf, float* __restrict__ dists, bool vec) {
     __shared__ float4 sp[256];
-    const int b = blockIdx.x;
-    const int n = b / (nbx * nby), by = (b / nbx) % nby, bx = b % nbx;
-    const int i = by * kPtBin + (threadIdx.x >> 4), j = bx * kPtBin + (threadIdx.x & 15);
-    // pixel centre as a float pair (hi + lo): the offset to a point is then exact to ~1e-15
-    const double pxd = -1.0 + (2.0 * j + 1.0) / W, pyd = 1.0 - (2.0 * i + 1.0) / H;
-    const float pxh = (float)pxd, pyh = (float)pyd;
-    const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
-    float kz[KC], kd[KC];
-    int kid[KC];
-#pragma unroll
-    for (int k = 0; k < KC; ++k) {
-        kz[k] = FLT_MAX;
-        kid[k] = INT_MAX;
-        kd[k] = -1.f;
-    }
-    const int beg = offsets[b], end = offsets[b + 1];
-    for (int c0 = beg; c0 < end; c0 += 256) {
-        __syncthreads();
-        if (c0 + (int)threadIdx.x < end) {
-            const int p = list[c0 + threadIdx.x];
-            sp[threadIdx.x] = make_float4(pts[3 * (int64_t)p], pts[3 * (int64_t)p + 1], pts[3 * (int64_t)p + 2],
-                                          __int_as_float(p));
-        }
-        __syncthreads();
-        const int cnt = min(256, end - c0);
-        for (int t = 0; t < cnt; ++t) {
-            const float4 q = sp[t];
-            const float dx = (pxh - q.x) + pxl, dy = (pyh - q.y) + pyl;
-            const float d2 = fmaf(dx, dx, dy * dy);
-            const int id = __float_as_int(q.w);
-            if (d2 <= r2 && (q.z < kz[KC - 1] || (q.z == kz[KC - 1] && id < kid[KC - 1])))
-                insert_point<KC>(kz, kid, kd, q.z, id, d2);
-        }
-    }
-    if (i >= H || j >= W) return;
-    const int64_t o = (((int64_t)n * H + i) * W + j) * K;
-    if constexpr (KC >= 4) {
-      if (vec && (K & 3) == 0) {
-#pragma unroll
-        for (int k = 0; k < KC; k += 4) {
-            if (k >= K) break;
-            long long v[4];
-            float z4[4], d4[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const bool ok = kid[k + u] != INT_MAX;
-                v[u] = ok ? kid[k + u] : -1;
-                z4[u] = ok ? kz[k + u] : -1.f;
-                d4[u] = ok ? kd[k + u] : -1.f;
-            }
-            reinterpret_cast<longlong2*>(idx + o + k)[0] = make_longlong2(v[0], v[1]);
-            reinterpret_cast<longlong2*>(idx + o + k)[1] = make_longlong2(v[2], v[3]);
-            *reinterpret_cast<float4*>(zbuf + o + k) = make_float4(z4[0], z4[1], z4[2], z4[3]);
-            *reinterpret_cast<float4*>(dists + o + k) = make_float4(d4[0], d4[1], d4[2], d4[3]);
-        }
-        return;
-      }
-    }
-    {
+    for (int b = blockIdx.x; b < nbins; b += gridDim.x) {
+        const int n = b / (nbx * nby), by = (b / nbx) % nby, bx = b % nbx;
+        const int i = by * kPtBin + (threadIdx.x >> 4), j = bx * kPtBin + (threadIdx.x & 15);
+        // pixel centre as a float pair (hi + lo): the offset to a point is then exact to ~1e-15
+        const double pxd = -1.0 + (2.0 * j + 1.0) / W, pyd = 1.0 - (2.0 * i + 1.0) / H;
+        const float pxh = (float)pxd, pyh = (float)pyd;
+        const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
+        float kz[KC], kd[KC];
+        int kid[KC];
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
-            if (k >= K) break;
-            const bool ok = kid[k] != INT_MAX;
-            idx[o + k] = ok ? kid[k] : -1;
-            zbuf[o + k] = ok ? kz[k] : -1.f;
-            dists[o + k] = ok ? kd[k] : -1.f;
+            kz[k] = FLT_MAX;
+            kid[k] = INT_MAX;
+            kd[k] = -1.f;
         }
+        const int beg = offsets[b], end = offsets[b + 1];
+        for (int c0 = beg; c0 < end; c0 += 256) {
+            __syncthreads();
+            if (c0 + (int)threadIdx.x < end) {
+                const int p = list[c0 + threadIdx.x];
+                sp[threadIdx.x] = make_float4(pts[3 * (int64_t)p], pts[3 * (int64_t)p + 1],
+                                              pts[3 * (int64_t)p + 2], __int_as_float(p));
+            }
+            __syncthreads();
+            const int cnt = min(256, end - c0);
+            for (int t = 0; t < cnt; ++t) {
+                const float4 q = sp[t];
+                const float dx = (pxh - q.x) + pxl, dy = (pyh - q.y) + pyl;
+                const float d2 = fmaf(dx, dx, dy * dy);
+                const int id = __float_as_int(q.w);
+                if (d2 <= r2 && (q.z < kz[KC - 1] || (q.z == kz[KC - 1] && id < kid[KC - 1])))
+                    insert_point<KC>(kz, kid, kd, q.z, id, d2);
+            }
+        }
+        if (i < H && j < W)
+            write_point_slots<KC>(kz, kid, kd, K, (((int64_t)n * H + i) * W + j) * K, vec, idx, zbuf, dists);
     }
 }
 
@@ -433,8 +443,9 @@ int mr_rasterize_points_fwd(const float* points, int64_t P, const int64_t* cloud
         const bool vec = (reinterpret_cast<uintptr_t>(idx) & 15) == 0 && (reinterpret_cast<uintptr_t>(zbuf) & 15) == 0 &&
                          (reinterpret_cast<uintptr_t>(dists) & 15) == 0;
         ProfScope ps(MR_STAGE_POINTS_FINE, s);
+        const int grid = std::min(nbins, 148 * 8);
 #define MR_PF(KC) \
-    k_point_fine<KC><<<nbins, 256, 0, s>>>(points, offsets, list, N, H, W, r2, K, nbx, nby, idx, zbuf, dists, vec)
+    k_point_fine<KC><<<grid, 256, 0, s>>>(points, offsets, list, nbins, H, W, r2, K, nbx, nby, idx, zbuf, dists, vec)
         if (K <= 1) MR_PF(1);
         else if (K <= 2) MR_PF(2);
         else if (K <= 4) MR_PF(4);
