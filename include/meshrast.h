@@ -291,8 +291,10 @@ int mr_composite_points_bwd(const int64_t* idx, const float* dists, int64_t npix
  * HOST).  mr_knn_fwd: idx (P1 x K int64: global ids into p2) and dists (P1 x K float32:
  * squared Euclidean distances), the K nearest ordered by (distance, id); when cloud n of
  * p2 has fewer than K points the rest hold -1 in both; queries in no cloud get -1 rows.
- * 1 <= D <= MR_KNN_DMAX, 1 <= K <= MR_KMAX; MR_ERR_ARG for overlapping query clouds or a
- * range outside its set.  Exhaustive search (every pair of a cloud is tested).
+ * 1 <= D <= MR_KNN_DMAX, 1 <= K <= MR_KMAX, P1, P2 < 2^31; MR_ERR_ARG for overlapping query
+ * clouds or a range outside its set.  Exact (every reference of the cloud is either tested
+ * or bounded away by the box of its group); allocates scratch of about 24 bytes per point
+ * of each set, stream-ordered.
  * mr_knn_bwd: grad_p1 (P1 x D) and grad_p2 (P2 x D), both overwritten (float32 atomics into
  * grad_p2), from grad_dists (P1 x K): d dist / d q = 2 (q - r), d dist / d r = -2 (q - r).
  */
