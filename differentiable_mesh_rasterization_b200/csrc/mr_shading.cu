@@ -119,20 +119,19 @@ struct BlendParams {
     float sigma, gamma, znear, zfar;
 };
 
-// Per-pixel blend state: coverage weights p, depth weights w, the background weight and
-// the normaliser.  Returns false for a pixel with no fragment.
+// Per-pixel blend state from the K slots' face ids, distances and depths: coverage
+// weights p, depth weights w, the background weight wb and the normaliser den.
 template <int KC>
-__device__ __forceinline__ void blend_weights(const int64_t* __restrict__ p2f, const float* __restrict__ dists,
-                                              const float* __restrict__ zbuf, int64_t q, int K, const BlendParams& P,
-                                              bool (&valid)[KC], float (&d)[KC], float (&p)[KC], float (&w)[KC],
-                                              float& wb, float& den) {
+__device__ __forceinline__ void blend_state(const int64_t (&f)[KC], const float (&dist)[KC], const float (&zv)[KC],
+                                            int K, const BlendParams& P, bool (&valid)[KC], float (&d)[KC],
+                                            float (&p)[KC], float (&w)[KC], float& wb, float& den) {
     float zmin = FLT_MAX;
     float z[KC];
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
-        valid[k] = k < K && p2f[q * K + k] >= 0;
-        d[k] = valid[k] ? dists[q * K + k] : 0.f;
-        z[k] = valid[k] ? zbuf[q * K + k] : 0.f;
+        valid[k] = k < K && f[k] >= 0;
+        d[k] = valid[k] ? dist[k] : 0.f;
+        z[k] = valid[k] ? zv[k] : 0.f;
         if (valid[k]) zmin = fminf(zmin, z[k]);
     }
     const float range = P.zfar - P.znear;
@@ -151,6 +150,125 @@ __device__ __forceinline__ void blend_weights(const int64_t* __restrict__ p2f, c
     }
     wb = expf((kBlendEps - (shifted ? s_max : kBlendEps)) / P.gamma);
     den += wb;
+}
+
+// The same from memory (pixel q, K slots, element-wise loads).
+template <int KC>
+__device__ __forceinline__ void blend_weights(const int64_t* __restrict__ p2f, const float* __restrict__ dists,
+                                              const float* __restrict__ zbuf, int64_t q, int K, const BlendParams& P,
+                                              bool (&valid)[KC], float (&d)[KC], float (&p)[KC], float (&w)[KC],
+                                              float& wb, float& den) {
+    int64_t f[KC];
+    float dd[KC], zz[KC];
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+        f[k] = k < K ? p2f[q * K + k] : -1;
+        dd[k] = f[k] >= 0 ? dists[q * K + k] : 0.f;
+        zz[k] = f[k] >= 0 ? zbuf[q * K + k] : 0.f;
+    }
+    blend_state<KC>(f, dd, zz, K, P, valid, d, p, w, wb, den);
+}
+
+// 16-byte loads and stores of N consecutive values (N a multiple of 4 floats or 2 int64;
+// the address 16-byte aligned).
+template <int N>
+__device__ __forceinline__ void ld_vec(const float* __restrict__ a, float (&v)[N]) {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+        const float4 t = reinterpret_cast<const float4*>(a)[i];
+        v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+    }
+}
+template <int N>
+__device__ __forceinline__ void st_vec(float* __restrict__ a, const float (&v)[N]) {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i)
+        reinterpret_cast<float4*>(a)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+template <int N>
+__device__ __forceinline__ void ld_vec(const int64_t* __restrict__ a, int64_t (&v)[N]) {
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+        const longlong2 t = reinterpret_cast<const longlong2*>(a)[i];
+        v[2 * i] = t.x; v[2 * i + 1] = t.y;
+    }
+}
+
+// RGB blend with K == KC (a multiple of 4) and 16-byte aligned arrays: every per-pixel run
+// (ids, distances, depths, 3 KC colours, rgba, gradients) moves in 16-byte accesses.
+template <int KC>
+__global__ void k_blend_fwd_rgb(const int64_t* __restrict__ p2f, const float* __restrict__ colors,
+                                const float* __restrict__ dists, const float* __restrict__ zbuf, int64_t npix,
+                                BlendParams P, float* __restrict__ out) {
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < npix; q += (int64_t)gridDim.x * blockDim.x) {
+        int64_t f[KC];
+        float dd[KC], zz[KC], col[3 * KC];
+        ld_vec<KC>(p2f + q * KC, f);
+        ld_vec<KC>(dists + q * KC, dd);
+        ld_vec<KC>(zbuf + q * KC, zz);
+        ld_vec<3 * KC>(colors + q * 3 * KC, col);
+        bool valid[KC];
+        float d[KC], p[KC], w[KC], wb, den;
+        blend_state<KC>(f, dd, zz, KC, P, valid, d, p, w, wb, den);
+        float o[4];
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+            float acc = wb * P.bg[c];
+#pragma unroll
+            for (int k = 0; k < KC; ++k)
+                if (valid[k]) acc = fmaf(w[k], col[3 * k + c], acc);
+            o[c] = acc / den;
+        }
+        o[3] = silhouette_alpha<KC>(d, valid, KC, P.sigma);
+        st_vec<4>(out + q * 4, o);
+    }
+}
+
+template <int KC>
+__global__ void k_blend_bwd_rgb(const int64_t* __restrict__ p2f, const float* __restrict__ colors,
+                                const float* __restrict__ dists, const float* __restrict__ zbuf, int64_t npix,
+                                BlendParams P, const float* __restrict__ grad_rgba, float* __restrict__ grad_colors,
+                                float* __restrict__ grad_dists, float* __restrict__ grad_zbuf) {
+    const float inv_gz = 1.f / (P.gamma * (P.zfar - P.znear));
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < npix; q += (int64_t)gridDim.x * blockDim.x) {
+        int64_t f[KC];
+        float dd[KC], zz[KC], col[3 * KC], g4[4];
+        ld_vec<KC>(p2f + q * KC, f);
+        ld_vec<KC>(dists + q * KC, dd);
+        ld_vec<KC>(zbuf + q * KC, zz);
+        ld_vec<3 * KC>(colors + q * 3 * KC, col);
+        ld_vec<4>(grad_rgba + q * 4, g4);
+        bool valid[KC];
+        float d[KC], p[KC], w[KC], wb, den;
+        blend_state<KC>(f, dd, zz, KC, P, valid, d, p, w, wb, den);
+        const float inv_den = 1.f / den;
+        float rgb[3];
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+            float acc = wb * P.bg[c];
+#pragma unroll
+            for (int k = 0; k < KC; ++k)
+                if (valid[k]) acc = fmaf(w[k], col[3 * k + c], acc);
+            rgb[c] = acc * inv_den;
+        }
+        float ga[KC], gc[3 * KC], gdv[KC], gzv[KC];
+        silhouette_grad<KC>(d, valid, KC, P.sigma, g4[3], ga);
+#pragma unroll
+        for (int k = 0; k < KC; ++k) {
+            float gw = 0.f;
+#pragma unroll
+            for (int c = 0; c < 3; ++c) {
+                gc[3 * k + c] = valid[k] ? w[k] * inv_den * g4[c] : 0.f;
+                gw = fmaf(col[3 * k + c] - rgb[c], g4[c], gw);
+            }
+            gw *= inv_den;
+            gdv[k] = valid[k] ? gw * w[k] * (-(1.f - p[k]) / P.sigma) + ga[k] : 0.f;
+            gzv[k] = valid[k] ? -gw * w[k] * inv_gz : 0.f;
+        }
+        if (grad_colors) st_vec<3 * KC>(grad_colors + q * 3 * KC, gc);
+        if (grad_dists) st_vec<KC>(grad_dists + q * KC, gdv);
+        if (grad_zbuf) st_vec<KC>(grad_zbuf + q * KC, gzv);
+    }
 }
 
 template <int KC>
@@ -211,6 +329,9 @@ __global__ void k_blend_bwd(const int64_t* __restrict__ p2f, const float* __rest
     }
 }
 
+
+// 16-byte alignment of an optional array (a null pointer does not stop the vector path).
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 int check_blend(int64_t npix, int K, int D, float sigma, float gamma, float znear, float zfar) {
     if (npix < 0 || K < 1 || K > MR_KMAX || D < 1 || D > MR_BLEND_DMAX) {
@@ -319,6 +440,13 @@ int mr_blend_fwd(const int64_t* pix_to_face, const float* colors, const float* d
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int g = mr::grid_for(npix);
     mr::ProfScope ps(MR_STAGE_BLEND_FWD, s);
+    if (D == 3 && (K == 4 || K == 8) && mr::aligned16(pix_to_face) && mr::aligned16(colors) && mr::aligned16(dists) &&
+        mr::aligned16(zbuf) && mr::aligned16(rgba)) {
+        if (K == 4) mr::k_blend_fwd_rgb<4><<<g, 256, 0, s>>>(pix_to_face, colors, dists, zbuf, npix, P, rgba);
+        else mr::k_blend_fwd_rgb<8><<<g, 256, 0, s>>>(pix_to_face, colors, dists, zbuf, npix, P, rgba);
+        MR_CUDA(cudaGetLastError());
+        return MR_OK;
+    }
 #define MR_BF(KC) mr::k_blend_fwd<KC><<<g, 256, 0, s>>>(pix_to_face, colors, dists, zbuf, npix, K, D, P, rgba)
     if (K <= 1) MR_BF(1);
     else if (K <= 2) MR_BF(2);
@@ -346,6 +474,18 @@ int mr_blend_bwd(const int64_t* pix_to_face, const float* colors, const float* d
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int g = mr::grid_for(npix);
     mr::ProfScope ps(MR_STAGE_BLEND_BWD, s);
+    if (D == 3 && (K == 4 || K == 8) && mr::aligned16(pix_to_face) && mr::aligned16(colors) && mr::aligned16(dists) &&
+        mr::aligned16(zbuf) && mr::aligned16(grad_rgba) && mr::aligned16(grad_colors) && mr::aligned16(grad_dists) &&
+        mr::aligned16(grad_zbuf)) {
+        if (K == 4)
+            mr::k_blend_bwd_rgb<4><<<g, 256, 0, s>>>(pix_to_face, colors, dists, zbuf, npix, P, grad_rgba, grad_colors,
+                                                     grad_dists, grad_zbuf);
+        else
+            mr::k_blend_bwd_rgb<8><<<g, 256, 0, s>>>(pix_to_face, colors, dists, zbuf, npix, P, grad_rgba, grad_colors,
+                                                     grad_dists, grad_zbuf);
+        MR_CUDA(cudaGetLastError());
+        return MR_OK;
+    }
 #define MR_BB(KC)                                                                                          \
     mr::k_blend_bwd<KC><<<g, 256, 0, s>>>(pix_to_face, colors, dists, zbuf, npix, K, D, P, grad_rgba, grad_colors, \
                                           grad_dists, grad_zbuf)
