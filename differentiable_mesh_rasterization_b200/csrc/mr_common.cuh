@@ -56,6 +56,31 @@ void scratch_free(void* p, cudaStream_t s);
 // SM of the 148.
 inline int grid_for(int64_t n) { return (int)(n < 148 * 32 * 256 ? (n + 255) / 256 : 148 * 32); }
 
+// 16-byte loads and stores of N consecutive values (N a multiple of 4 floats or 2 int64;
+// the address 16-byte aligned).
+template <int N>
+__device__ __forceinline__ void ld_vec(const float* __restrict__ a, float (&v)[N]) {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+        const float4 t = reinterpret_cast<const float4*>(a)[i];
+        v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+    }
+}
+template <int N>
+__device__ __forceinline__ void st_vec(float* __restrict__ a, const float (&v)[N]) {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i)
+        reinterpret_cast<float4*>(a)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+template <int N>
+__device__ __forceinline__ void ld_vec(const int64_t* __restrict__ a, int64_t (&v)[N]) {
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+        const longlong2 t = reinterpret_cast<const longlong2*>(a)[i];
+        v[2 * i] = t.x; v[2 * i + 1] = t.y;
+    }
+}
+
 // Device-wide sticky error word (asynchronous kernels).
 int* device_error_word();
 

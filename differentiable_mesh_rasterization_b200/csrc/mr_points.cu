@@ -243,22 +243,39 @@ inline Radius2 radius2(float radius) {
 }
 
 // Compositing, thread per pixel.  MODE 0: alpha, 1: norm-weighted.
-template <int KC, int MODE>
+// A pixel's K slot ids and distances: 16-byte loads when VEC (K == KC, a multiple of 4,
+// aligned arrays), else element-wise.
+template <int KC, bool VEC>
+__device__ __forceinline__ void load_slots(const int64_t* __restrict__ idx, const float* __restrict__ dists, int64_t q,
+                                           int K, int64_t (&m)[KC], float (&d)[KC]) {
+    if constexpr (VEC) {
+        ld_vec<KC>(idx + q * KC, m);
+        ld_vec<KC>(dists + q * KC, d);
+    } else {
+#pragma unroll
+        for (int k = 0; k < KC; ++k) {
+            m[k] = k < K ? idx[q * K + k] : -1;
+            d[k] = m[k] >= 0 ? dists[q * K + k] : 0.f;
+        }
+    }
+}
+
+template <int KC, int MODE, bool VEC>
 __global__ void k_composite_fwd(const int64_t* __restrict__ idx, const float* __restrict__ dists, int64_t npix, int K,
                                 const float* __restrict__ feat, int64_t P, int C, Radius2 R,
                                 float* __restrict__ out, int* __restrict__ err) {
     for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < npix; q += (int64_t)gridDim.x * blockDim.x) {
         int64_t m[KC];
-        float w[KC];
+        float w[KC], dv[KC];
         float T = 1.f, wsum = 0.f;
+        load_slots<KC, VEC>(idx, dists, q, K, m, dv);
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
-            m[k] = k < K ? idx[q * K + k] : -1;
             if (m[k] < -1 || m[k] >= P) {
                 atomicOr(err, kErrSlotIndex);
                 m[k] = -1;
             }
-            const float a = m[k] >= 0 ? point_weight(dists[q * K + k], R) : 0.f;
+            const float a = m[k] >= 0 ? point_weight(dv[k], R) : 0.f;
             w[k] = MODE == 0 ? a * T : a;
             T *= 1.f - a;
             wsum += a;
@@ -279,23 +296,23 @@ __global__ void k_composite_fwd(const int64_t* __restrict__ idx, const float* __
 // dL/da_k = T_k ((f_k . g) - R_k) -- no division by 1 - a_k.  Norm-weighted:
 // dL/da_k = (f_k - out) . g / den (den = sum a > floor) or f_k . g / den.  Feature
 // gradients w_k g go to a padded accumulator (float4 per point for C <= 4, else scalars).
-template <int KC, int MODE, bool VEC4>
+template <int KC, int MODE, bool VEC4, bool VEC>
 __global__ void k_composite_bwd(const int64_t* __restrict__ idx, const float* __restrict__ dists, int64_t npix, int K,
                                 const float* __restrict__ feat, int64_t P, int C, Radius2 R,
                                 const float* __restrict__ grad_out, float* __restrict__ gfeat,
                                 float4* __restrict__ gfeat4, float* __restrict__ grad_dists, int* __restrict__ err) {
     for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < npix; q += (int64_t)gridDim.x * blockDim.x) {
         int64_t m[KC];
-        float a[KC], T[KC], fg[KC];
+        float a[KC], T[KC], fg[KC], dv[KC], gdv[KC];
         float t = 1.f, wsum = 0.f;
+        load_slots<KC, VEC>(idx, dists, q, K, m, dv);
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
-            m[k] = k < K ? idx[q * K + k] : -1;
             if (m[k] < -1 || m[k] >= P) {
                 atomicOr(err, kErrSlotIndex);
                 m[k] = -1;
             }
-            a[k] = m[k] >= 0 ? point_weight(dists[q * K + k], R) : 0.f;
+            a[k] = m[k] >= 0 ? point_weight(dv[k], R) : 0.f;
             T[k] = t;
             t *= 1.f - a[k];
             wsum += a[k];
@@ -333,8 +350,10 @@ __global__ void k_composite_bwd(const int64_t* __restrict__ idx, const float* __
                     for (int c = 0; c < C; ++c) atomicAdd(gfeat + m[k] * C + c, wk * grad_out[q * C + c]);
                 }
             }
-            if (grad_dists && k < K) grad_dists[q * K + k] = -ga * R.inv;
+            gdv[k] = -ga * R.inv;
+            if (!VEC && grad_dists && k < K) grad_dists[q * K + k] = gdv[k];
         }
+        if (VEC && grad_dists) st_vec<KC>(grad_dists + q * KC, gdv);
     }
 }
 
@@ -528,16 +547,21 @@ int mr_composite_points_fwd(const int64_t* idx, const float* dists, int64_t npix
     const Radius2 R = radius2(radius);
     const int g = grid_for(npix);
     ProfScope ps(MR_STAGE_COMPOSITE_FWD, s);
-#define MR_CF(KC)                                                                                                \
-    (mode == 0 ? k_composite_fwd<KC, 0><<<g, 256, 0, s>>>(idx, dists, npix, K, features, P, C, R, out, err) \
-               : k_composite_fwd<KC, 1><<<g, 256, 0, s>>>(idx, dists, npix, K, features, P, C, R, out, err))
-    if (K <= 1) MR_CF(1);
+    const bool vec = (K == 4 || K == 8) && ((reinterpret_cast<uintptr_t>(idx) | reinterpret_cast<uintptr_t>(dists)) & 15) == 0;
+#define MR_CF2(KC, V)                                                                                              \
+    (mode == 0 ? k_composite_fwd<KC, 0, V><<<g, 256, 0, s>>>(idx, dists, npix, K, features, P, C, R, out, err) \
+               : k_composite_fwd<KC, 1, V><<<g, 256, 0, s>>>(idx, dists, npix, K, features, P, C, R, out, err))
+#define MR_CF(KC) MR_CF2(KC, false)
+    if (vec && K == 4) MR_CF2(4, true);
+    else if (vec) MR_CF2(8, true);
+    else if (K <= 1) MR_CF(1);
     else if (K <= 2) MR_CF(2);
     else if (K <= 4) MR_CF(4);
     else if (K <= 8) MR_CF(8);
     else if (K <= 16) MR_CF(16);
     else MR_CF(32);
 #undef MR_CF
+#undef MR_CF2
     MR_CUDA(cudaGetLastError());
     return MR_OK;
 }
@@ -578,13 +602,18 @@ int mr_composite_points_bwd(const int64_t* idx, const float* dists, int64_t npix
     const int g = grid_for(npix);
     if (e == cudaSuccess) {
         ProfScope ps(MR_STAGE_COMPOSITE_BWD, s);
-#define MR_CB2(KC, MODE)                                                                                       \
-    (vec4 ? k_composite_bwd<KC, MODE, true><<<g, 256, 0, s>>>(idx, dists, npix, K, features, P, C, R,    \
-                                                              grad_out, nullptr, acc, grad_dists, err)         \
-          : k_composite_bwd<KC, MODE, false><<<g, 256, 0, s>>>(idx, dists, npix, K, features, P, C, R,   \
-                                                               grad_out, grad_features, nullptr, grad_dists, err))
-#define MR_CB(KC) (mode == 0 ? MR_CB2(KC, 0) : MR_CB2(KC, 1))
-        if (K <= 1) MR_CB(1);
+        const bool vec = (K == 4 || K == 8) && ((reinterpret_cast<uintptr_t>(idx) | reinterpret_cast<uintptr_t>(dists) |
+                                                  reinterpret_cast<uintptr_t>(grad_dists)) & 15) == 0;
+#define MR_CB3(KC, MODE, V)                                                                                       \
+    (vec4 ? k_composite_bwd<KC, MODE, true, V><<<g, 256, 0, s>>>(idx, dists, npix, K, features, P, C, R,        \
+                                                                 grad_out, nullptr, acc, grad_dists, err)         \
+          : k_composite_bwd<KC, MODE, false, V><<<g, 256, 0, s>>>(idx, dists, npix, K, features, P, C, R,       \
+                                                                  grad_out, grad_features, nullptr, grad_dists, err))
+#define MR_CB2(KC, V) (mode == 0 ? MR_CB3(KC, 0, V) : MR_CB3(KC, 1, V))
+#define MR_CB(KC) MR_CB2(KC, false)
+        if (vec && K == 4) MR_CB2(4, true);
+        else if (vec) MR_CB2(8, true);
+        else if (K <= 1) MR_CB(1);
         else if (K <= 2) MR_CB(2);
         else if (K <= 4) MR_CB(4);
         else if (K <= 8) MR_CB(8);
@@ -592,6 +621,7 @@ int mr_composite_points_bwd(const int64_t* idx, const float* dists, int64_t npix
         else MR_CB(32);
 #undef MR_CB
 #undef MR_CB2
+#undef MR_CB3
         if (vec4) k_acc4_cols<<<grid_for(P), 256, 0, s>>>(acc, P, C, grad_features);
         e = cudaGetLastError();
     }

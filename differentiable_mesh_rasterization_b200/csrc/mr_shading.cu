@@ -169,31 +169,6 @@ __device__ __forceinline__ void blend_weights(const int64_t* __restrict__ p2f, c
     blend_state<KC>(f, dd, zz, K, P, valid, d, p, w, wb, den);
 }
 
-// 16-byte loads and stores of N consecutive values (N a multiple of 4 floats or 2 int64;
-// the address 16-byte aligned).
-template <int N>
-__device__ __forceinline__ void ld_vec(const float* __restrict__ a, float (&v)[N]) {
-#pragma unroll
-    for (int i = 0; i < N / 4; ++i) {
-        const float4 t = reinterpret_cast<const float4*>(a)[i];
-        v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
-    }
-}
-template <int N>
-__device__ __forceinline__ void st_vec(float* __restrict__ a, const float (&v)[N]) {
-#pragma unroll
-    for (int i = 0; i < N / 4; ++i)
-        reinterpret_cast<float4*>(a)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-}
-template <int N>
-__device__ __forceinline__ void ld_vec(const int64_t* __restrict__ a, int64_t (&v)[N]) {
-#pragma unroll
-    for (int i = 0; i < N / 2; ++i) {
-        const longlong2 t = reinterpret_cast<const longlong2*>(a)[i];
-        v[2 * i] = t.x; v[2 * i + 1] = t.y;
-    }
-}
-
 // RGB blend with K == KC (a multiple of 4) and 16-byte aligned arrays: every per-pixel run
 // (ids, distances, depths, 3 KC colours, rgba, gradients) moves in 16-byte accesses.
 template <int KC>
