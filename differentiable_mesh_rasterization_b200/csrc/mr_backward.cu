@@ -169,9 +169,11 @@ __device__ __forceinline__ bool slot_grad(const float (&x)[3], const float (&y)[
 // (x, y, z, 0) accumulator.  Measured alternatives that lost on this scatter: summing
 // equal vertex ids within a pixel, or along a run of lanes, before the atomics; issuing
 // the K slots' gathers phase by phase (more registers, fewer resident warps); packing the
-// valid slots of a warp's pixels into a shared-memory queue so that no lane idles.
+// valid slots of a warp's pixels into a shared-memory queue so that no lane idles; a
+// per-call table of face records (three 16-byte loads per slot instead of the face ids
+// and nine scalar vertex loads: 1.74 -> 1.71 ms, not worth its 48 bytes per face).
 template <int KC, bool PERSP>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)   // 64 registers: 4 CTAs per SM (measured 1.75 -> 1.63 ms)
 k_raster_bwd(const float* __restrict__ verts, int64_t V, const int64_t* __restrict__ faces, int64_t F,
              const int64_t* __restrict__ p2f, int64_t npix, int H, int W, int K, const float* __restrict__ gz,
              const float* __restrict__ gb, const float* __restrict__ gd, float4* __restrict__ acc,

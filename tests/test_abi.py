@@ -85,3 +85,37 @@ def test_binding_fails_loudly_without_cuda_tensors():
     f = torch.zeros(1, 3, dtype=torch.int64)
     with pytest.raises(ValueError):
         mr.rasterize_fwd(v, f, [0], [1], 8, 8, 0.0, 1)
+
+
+def test_next_row_entry_points_reject_bad_arguments(lib):
+    """Stage-two shading, Phong lighting, point clouds and KNN: host-side validation only."""
+    d = ctypes.c_void_p(16)
+    err = lambda: lib.mr_last_error().decode()
+    assert lib.mr_interpolate_fwd(d, d, 4, 2, d, 1, d, 3, 0, d, None) == -1 and "D=0" in err()
+    bg = np.zeros(9, np.float32)
+    assert lib.mr_blend_fwd(d, d, d, d, 4, 2, 9, bg.ctypes.data, 1e-4, 1e-2, 1.0, 10.0, d, None) == -1
+    assert lib.mr_blend_fwd(d, d, d, d, 4, 2, 3, bg.ctypes.data, 0.0, 1e-2, 1.0, 10.0, d, None) == -1
+    assert lib.mr_blend_bwd(d, d, d, d, 4, 2, 3, bg.ctypes.data, 1e-4, 1e-2, 10.0, 1.0, d, d, d, d, None) == -1
+    prm = np.zeros(16, np.float32)
+    prm[15] = 0.5                                       # shininess below 1
+    assert lib.mr_phong_fwd(d, d, d, 4, prm.ctypes.data, d, None) == -1 and "shininess" in err()
+    prm[15] = 8.0
+    prm[0] = np.nan
+    assert lib.mr_phong_bwd(d, d, d, 4, prm.ctypes.data, d, d, d, d, None) == -1 and "finite" in err()
+    prm[0] = 1.0
+    assert lib.mr_phong_shade_fwd(d, d, 4, 0, d, 1, d, d, d, 3, prm.ctypes.data, d, None) == -1
+    first, num = np.array([0, 5], np.int64), np.array([10, 5], np.int64)     # overlapping clouds
+    assert lib.mr_rasterize_points_fwd(d, 20, first.ctypes.data, num.ctypes.data, 2, 8, 8, 0.1, 4, d, d, d,
+                                       None) == -1 and "not ascending" in err()
+    ok_first, ok_num = np.array([0], np.int64), np.array([20], np.int64)
+    assert lib.mr_rasterize_points_fwd(d, 20, ok_first.ctypes.data, ok_num.ctypes.data, 1, 8, 8, float("nan"), 4,
+                                       d, d, d, None) == -1
+    assert lib.mr_rasterize_points_fwd(d, 20, ok_first.ctypes.data, ok_num.ctypes.data, 1, 8, 8, 0.1, 40, d, d, d,
+                                       None) == -1
+    assert lib.mr_composite_points_fwd(d, d, 4, 2, d, 3, 3, 0.1, 2, d, None) == -1 and "mode=2" in err()
+    assert lib.mr_composite_points_bwd(d, d, 4, 2, d, 3, 3, 0.0, 0, d, d, d, None) == -1
+    assert lib.mr_knn_fwd(d, 10, ok_first.ctypes.data, ok_num.ctypes.data, d, 10, ok_first.ctypes.data,
+                          ok_num.ctypes.data, 1, 5, 4, d, d, None) == -1 and "D=5" in err()
+    assert lib.mr_knn_fwd(d, 20, first.ctypes.data, num.ctypes.data, d, 20, first.ctypes.data, num.ctypes.data, 2,
+                          3, 4, d, d, None) == -1 and "overlap" in err()
+    assert lib.mr_knn_bwd(d, 4, d, 4, 0, 2, d, d, d, d, None) == -1
