@@ -568,7 +568,10 @@ def main():
         result copy."""
         cs = torch.cuda.Stream(device=dev)
         ds = torch.cuda.Stream(device=dev)
-        bufs = [None, None]
+        # device inputs allocated once (two sets), so no allocation sits between the streams
+        bufs = [(torch.empty_like(h_verts, device=dev), torch.empty_like(h_faces, device=dev),
+                 torch.empty_like(h_ga, device=dev)) for _ in range(2)]
+        torch.cuda.synchronize(dev)
         h2d_done = [torch.cuda.Event(), torch.cuda.Event()]
         freed = [None, None]
         e0 = torch.cuda.Event(enable_timing=True)
@@ -579,8 +582,8 @@ def main():
             with torch.cuda.stream(cs):
                 if freed[i] is not None:
                     cs.wait_event(freed[i])
-                bufs[i] = (h_verts.to(dev, non_blocking=True), h_faces.to(dev, non_blocking=True),
-                           h_ga.to(dev, non_blocking=True))
+                for dst, src in zip(bufs[i], (h_verts, h_faces, h_ga)):
+                    dst.copy_(src, non_blocking=True)
                 h2d_done[i].record(cs)
 
         e0.record(cs)
@@ -591,8 +594,6 @@ def main():
                 upload(k + 1)
             stream.wait_event(h2d_done[i])
             dv, df, dg = bufs[i]
-            for t in (dv, df, dg):
-                t.record_stream(stream)
             flush.zero_()
             p2f, _, _, dists, alpha = mr.rasterize_fwd(dv, df, first, num, w.H, w.W, w.blur_radius, w.K,
                                                        w.perspective_correct, sigma=w.sigma)
@@ -618,6 +619,8 @@ def main():
     serial_ms = e2e_serial(args.e2e_steps) if args.e2e_steps > 0 else 0.0
     if world > 1:
         dist.barrier()
+    if args.e2e_steps > 0:
+        e2e_pipelined(3)          # warm-up: the allocator caches the per-step output blocks
     e2e_ms = e2e_pipelined(args.e2e_steps) if args.e2e_steps > 0 else 0.0
     te = torch.tensor([e2e_ms, serial_ms], dtype=torch.float64, device=dev)
     if world > 1:
