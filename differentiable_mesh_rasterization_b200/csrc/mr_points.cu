@@ -154,7 +154,10 @@ __global__ void __launch_bounds__(256) k_point_fine(const float* __restrict__ pt
     __shared__ float4 sp[256];
     const int b = blockIdx.x;
     const int n = b / (nbx * nby), by = (b / nbx) % nby, bx = b % nbx;
-    const int i = by * kPtBin + (threadIdx.x >> 4), j = bx * kPtBin + (threadIdx.x & 15);
+    // each warp takes a 4 x 8 block of the bin (a point's disc meets fewer warps than with
+    // 2 x 16 rows, so fewer warps run the insertion for it)
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = by * kPtBin + (w >> 1) * 4 + (lane >> 3), j = bx * kPtBin + (w & 1) * 8 + (lane & 7);
     // pixel centre as a float pair (hi + lo): the offset to a point is then exact to ~1e-15
     const double pxd = -1.0 + (2.0 * j + 1.0) / W, pyd = 1.0 - (2.0 * i + 1.0) / H;
     const float pxh = (float)pxd, pyh = (float)pyd;
