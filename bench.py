@@ -643,7 +643,10 @@ def main():
     except (OSError, ValueError):
         pass
     sm_mhz_max = float(peaks.get("sm_max_mhz", 1965.0))
-    peak_alu = props.multi_processor_count * FP32_LANES_PER_SM * sm_mhz_max * 1e6 / 1e12   # T inst/s
+    peak_nominal = props.multi_processor_count * FP32_LANES_PER_SM * sm_mhz_max * 1e6 / 1e12   # T inst/s
+    # the denominator is the FFMA issue rate measured on this device in this run (the peaks
+    # file has no FP32 figure); unit counts x the maximum clock are reported beside it
+    peak_alu = mr.measure_fp32_peak(dev) / 1e12
     hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
     hbm_note = "of measured" if "hbm_gbs" in peaks else "of fallback"
     achieved_alu = samples * C_TEST / fine_s / 1e12
@@ -656,8 +659,10 @@ def main():
             "kernel": "k_fine (stage-one fine pass: pixel-face tests and register top-K)",
             "ms_per_step": fine_s * 1e3, "launches_per_step": fine_n // args.steps,
             "samples_per_step": samples, "c_test": C_TEST,
-            "peak_note": f"{props.multi_processor_count} SMs x 128 FP32 lanes x {sm_mhz_max:.0f} MHz "
-                         f"(unit counts and max clock)",
+            "peak_note": "of measured: FFMA-chain probe (mr_measure_fp32_peak) in this run",
+            "peak_nominal": peak_nominal,
+            "peak_nominal_note": f"{props.multi_processor_count} SMs x 128 FP32 lanes x {sm_mhz_max:.0f} MHz",
+            "dense_tests_per_step": int(sum(int(n) for n in batch.num_faces_per_mesh)) * w.H * w.W,
             "hbm_bytes_per_step": fine_bytes,
             "epilogue": {"kernel": "k_epilogue (float64 outputs of the K winners + silhouette)",
                          "bound": "hbm", "ms_per_step": epi_s * 1e3, "bytes_per_step": epi_bytes,

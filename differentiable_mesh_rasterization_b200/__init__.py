@@ -29,7 +29,7 @@ EXPORTS = ("mr_rasterize_fwd", "mr_rasterize_silhouette_fwd", "mr_silhouette_ble
            "mr_rasterize_fwd_noalloc", "mr_interpolate_fwd", "mr_interpolate_bwd", "mr_blend_fwd", "mr_blend_bwd",
            "mr_phong_fwd", "mr_phong_bwd", "mr_phong_shade_fwd", "mr_phong_shade_bwd",
            "mr_rasterize_points_fwd", "mr_rasterize_points_bwd", "mr_composite_points_fwd",
-           "mr_composite_points_bwd", "mr_knn_fwd", "mr_knn_bwd")
+           "mr_composite_points_bwd", "mr_knn_fwd", "mr_knn_bwd", "mr_measure_fp32_peak")
 STAGES = ("face_setup", "bin_count", "bin_scan", "bin_fill", "fine", "silhouette_fwd", "silhouette_bwd",
           "raster_bwd", "silhouette_raster_bwd", "epilogue", "interpolate_fwd", "interpolate_bwd", "blend_fwd",
           "blend_bwd", "phong_fwd", "phong_bwd", "phong_shade_fwd", "phong_shade_bwd",
@@ -80,6 +80,7 @@ def load_library() -> ctypes.CDLL:
         "mr_composite_points_bwd": [P, P, i64, i32, P, i64, i32, f32, i32, P, P, P, P],
         "mr_knn_fwd": [P, i64, P, P, P, i64, P, P, i32, i32, i32, P, P, P],
         "mr_knn_bwd": [P, i64, P, i64, i32, i32, P, P, P, P, P],
+        "mr_measure_fp32_peak": [P, P],
         "mr_profile_enable": [i32],
         "mr_profile_read": [P, P, i32],
     }
@@ -534,6 +535,16 @@ def blend_bwd(pix_to_face, colors, dists, zbuf, background, sigma, gamma, znear,
                                                 bg.ctypes.data, float(sigma), float(gamma), float(znear), float(zfar),
                                                 _ptr(g), _ptr(gc), _ptr(gd), _ptr(gz), _stream(p2f.device)))
     return gc, gd, gz
+
+
+def measure_fp32_peak(device=None) -> float:
+    """Measured FP32 instruction issue rate of the device (``mr_measure_fp32_peak``), inst/s."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    out = ctypes.c_double(0.0)
+    with torch.cuda.device(dev):
+        _check("mr_measure_fp32_peak", lib.mr_measure_fp32_peak(ctypes.byref(out), _stream(dev)))
+    return float(out.value)
 
 
 def device_status(device=None) -> None:

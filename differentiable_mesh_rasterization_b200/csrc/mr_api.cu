@@ -106,6 +106,26 @@ int* device_error_word() {
 
 }  // namespace mr
 
+namespace mr {
+// Independent FFMA chains (8 per thread, each 4 deep per iteration) for the issue-rate
+// probe; the result is stored only if it is exactly zero, which never happens for a
+// multiplier above 1, so nothing is optimised away and nothing is written.
+__global__ void __launch_bounds__(256) k_fma_probe(int iters, float m, float* __restrict__ sink) {
+    float x[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[c] = (float)(threadIdx.x + c) * 1e-3f;
+    for (int it = 0; it < iters; ++it)
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) x[c] = fmaf(x[c], m, 1e-7f);
+    float t = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) t += x[c];
+    if (t == 0.f) sink[blockIdx.x * blockDim.x + threadIdx.x] = t;
+}
+}  // namespace mr
+
 extern "C" {
 
 const char* mr_last_error(void) { return g_last_error; }
@@ -146,6 +166,45 @@ int mr_profile_read(double* stage_ms, int64_t* launches, int32_t nstages) {
 }
 
 int mr_version(void) { return 10000; }
+
+int mr_measure_fp32_peak(double* inst_per_s, void* stream) {
+    if (!inst_per_s) {
+        mr::set_error("null output");
+        return MR_ERR_ARG;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int dev = 0, sms = 0;
+    MR_CUDA(cudaGetDevice(&dev));
+    MR_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    const int blocks = sms * 8, iters = 4096;
+    float* sink = nullptr;
+    int rc = mr::scratch_alloc(reinterpret_cast<void**>(&sink), sizeof(float) * (size_t)blocks * 256, s);
+    if (rc != MR_OK) return rc;
+    cudaEvent_t a = nullptr, b = nullptr;
+    cudaError_t e = cudaEventCreate(&a);
+    if (e == cudaSuccess) e = cudaEventCreate(&b);
+    float ms = 0.f;
+    if (e == cudaSuccess) {
+        mr::k_fma_probe<<<blocks, 256, 0, s>>>(iters, 1.0001f, sink);   // warm-up
+        cudaEventRecord(a, s);
+        mr::k_fma_probe<<<blocks, 256, 0, s>>>(iters, 1.0001f, sink);
+        cudaEventRecord(b, s);
+        e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaEventSynchronize(b);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, a, b);
+    }
+    if (a) cudaEventDestroy(a);
+    if (b) cudaEventDestroy(b);
+    mr::scratch_free(sink, s);
+    if (e != cudaSuccess) return mr::cuda_fail(e, "fp32 probe");
+    if (!(ms > 0.f)) {
+        mr::set_error("fp32 probe: no elapsed time");
+        return MR_ERR_CUDA;
+    }
+    // 8 chains x 4 FFMA per iteration and thread
+    *inst_per_s = (double)blocks * 256.0 * iters * 32.0 / (ms * 1e-3);
+    return MR_OK;
+}
 
 int mr_device_status(void* stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -317,6 +317,15 @@ const char* mr_last_error(void);
 int mr_version(void);
 
 /*
+ * FP32 issue-rate probe (measurement support; no counterpart on the pages): times one
+ * launch of a kernel of independent FFMA chains filling every SM (8 chains per thread,
+ * 148 x 8 CTAs of 256 threads on B200) with CUDA events on `stream` and writes the achieved
+ * FP32 instructions per second to *inst_per_s (HOST).  Synchronises `stream`.  The roofline
+ * of the fine pass divides by this measured figure rather than by unit counts x clock.
+ */
+int mr_measure_fp32_peak(double* inst_per_s, void* stream);
+
+/*
  * Stage timing (the library's own tracing; no counterpart on the pages).  While enabled,
  * every launch of the stages below is bracketed by two CUDA events recorded on the
  * caller's stream; recording adds no synchronisation.  mr_profile_read() waits for the
