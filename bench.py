@@ -24,6 +24,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -33,7 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "pixel-face samples/s and Mpix/s (fwd+bwd) at 1 B200; % of rasterizer roofline"
 UNIT = "pixel-face samples/s"
-C_TEST = 38                 # FP32 instructions per pixel-face test (frozen)
+C_TEST = 38                 # FP32 instructions per pixel-face test in this formulation (frozen)
 FP32_LANES_PER_SM = 128
 L2_FLUSH_BYTES = 256 << 20
 KERNELS_PER_STAGE = {"silhouette_raster_bwd": 2}    # main kernel + (x, y) -> (x, y, z) copy
@@ -88,7 +89,7 @@ class ClockSampler:
     def __init__(self, uuid: str | None):
         self.uuid = uuid
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"mr_clocks_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
