@@ -146,28 +146,26 @@ __global__ void k_order_points(const float* __restrict__ p, const int64_t* __res
     }
 }
 
-// Sorted insertion of (d, id) into a register list of KC entries ordered by (d, id).
+// A neighbour key: the squared distance's bits above the original reference id.  Distances
+// are >= 0 and non-negative floats order like their bits, so one 64-bit compare orders
+// (distance, id); kNone sorts after every reference and reads back as FLT_MAX.
+constexpr unsigned long long kNone = (0x7F7FFFFFull << 32) | 0xFFFFFFFFull;
+
+__device__ __forceinline__ unsigned long long nn_key(float d, int id) {
+    return ((unsigned long long)__float_as_uint(d + 0.f) << 32) | (unsigned)id;
+}
+__device__ __forceinline__ float key_dist(unsigned long long k) { return __uint_as_float((unsigned)(k >> 32)); }
+
+// Sorted insertion into a register list of KC keys (the caller has checked key < the last).
 template <int KC>
-__device__ __forceinline__ void insert_nn(float (&kd)[KC], int (&ki)[KC], float d, int id) {
+__device__ __forceinline__ void insert_nn(unsigned long long (&kk)[KC], unsigned long long key) {
 #pragma unroll
     for (int k = KC - 1; k > 0; --k) {
-        const bool shift = d < kd[k - 1] || (d == kd[k - 1] && id < ki[k - 1]);
-        const bool here = !shift && (d < kd[k] || (d == kd[k] && id < ki[k]));
-        if (shift) {
-            kd[k] = kd[k - 1];
-            ki[k] = ki[k - 1];
-        } else if (here) {
-            kd[k] = d;
-            ki[k] = id;
-        }
+        const bool shift = key < kk[k - 1];
+        kk[k] = shift ? kk[k - 1] : (key < kk[k] ? key : kk[k]);
     }
-    if (d < kd[0] || (d == kd[0] && id < ki[0])) {
-        kd[0] = d;
-        ki[0] = id;
-    }
+    kk[0] = key < kk[0] ? key : kk[0];
 }
-
-__device__ __forceinline__ bool nn_before(float d, int id, float kd, int ki) { return d < kd || (d == kd && id < ki); }
 
 // Boxes of the ordered references: level 0 = groups of 32 consecutive points of one
 // cloud, level 1 = 32 consecutive groups of one cloud.  One warp per box; item t of a
@@ -273,13 +271,9 @@ __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ 
         q[0] = v.x; q[1] = v.y; q[2] = v.z; q[3] = v.w;
         qid = sqid[T.s0 + threadIdx.x];
     }
-    float kd[KC];
-    int ki[KC];
+    unsigned long long kk[KC];
 #pragma unroll
-    for (int k = 0; k < KC; ++k) {
-        kd[k] = FLT_MAX;
-        ki[k] = INT_MAX;
-    }
+    for (int k = 0; k < KC; ++k) kk[k] = kNone;
     const int64_t g0 = gpre[n], s0 = spre[n];
     const int64_t ngr = (rn + 31) >> 5, nsup = (ngr + 31) >> 5;
     int64_t home = 0;
@@ -289,12 +283,12 @@ __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ 
     }
     int64_t up = home + 1, down = home - 1, cur = home;
     for (int64_t it = 0; it < nsup; ++it) {
-        if (__all_sync(0xffffffffu, !live || box_bound<D>(q, slo[s0 + cur], shi[s0 + cur]) > kd[KC - 1])) {
+        if (__all_sync(0xffffffffu, !live || box_bound<D>(q, slo[s0 + cur], shi[s0 + cur]) > key_dist(kk[KC - 1]))) {
             // skipped
         } else {
             const int64_t gb = cur * 32, ge = min(gb + 32, ngr);
             for (int64_t g = gb; g < ge; ++g) {
-                if (__all_sync(0xffffffffu, !live || box_bound<D>(q, glo[g0 + g], ghi[g0 + g]) > kd[KC - 1]))
+                if (__all_sync(0xffffffffu, !live || box_bound<D>(q, glo[g0 + g], ghi[g0 + g]) > key_dist(kk[KC - 1])))
                     continue;
                 const int64_t pb = g * 32;
                 const int cnt = (int)min((int64_t)32, rn - pb);
@@ -320,9 +314,9 @@ __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ 
                     }
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
-                        if (t + u < cnt && d4[u] <= kd[KC - 1]) {
-                            const int id = wid[warp][t + u];
-                            if (nn_before(d4[u], id, kd[KC - 1], ki[KC - 1])) insert_nn<KC>(kd, ki, d4[u], id);
+                        if (t + u < cnt) {
+                            const unsigned long long key = nn_key(d4[u], wid[warp][t + u]);
+                            if (key < kk[KC - 1]) insert_nn<KC>(kk, key);
                         }
                 }
             }
@@ -337,9 +331,9 @@ __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ 
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
         if (k >= K) break;
-        const bool ok = ki[k] != INT_MAX;
-        idx[(int64_t)qid * K + k] = ok ? ki[k] : -1;
-        dists[(int64_t)qid * K + k] = ok ? kd[k] : -1.f;
+        const bool ok = kk[k] != kNone;
+        idx[(int64_t)qid * K + k] = ok ? (int64_t)(unsigned)(kk[k] & 0xffffffffu) : -1;
+        dists[(int64_t)qid * K + k] = ok ? key_dist(kk[k]) : -1.f;
     }
 }
 

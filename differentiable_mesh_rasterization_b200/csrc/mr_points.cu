@@ -78,27 +78,29 @@ __global__ void k_point_bins(const float* __restrict__ pts, int64_t P, const int
     }
 }
 
-// Sorted insertion of (z, id, d2) into a register list of KC entries ordered by (z, id).
+// A slot key: the depth's bits above the point id.  Depths here are >= 0 (negative ones
+// never reach the fine pass and -0 is made +0), and non-negative floats order like their
+// bits, so one 64-bit compare orders (z, id).  kEmpty sorts after every point.
+constexpr unsigned long long kEmpty = (0x7F7FFFFFull << 32) | 0xFFFFFFFFull;
+
+__device__ __forceinline__ unsigned long long point_key(float z, int id) {
+    return ((unsigned long long)__float_as_uint(z + 0.f) << 32) | (unsigned)id;
+}
+
+// Sorted insertion of (key, d2) into a register list of KC entries (the caller has checked
+// key < the list's last key).
 template <int KC>
-__device__ __forceinline__ void insert_point(float (&kz)[KC], int (&kid)[KC], float (&kd)[KC], float z, int id,
+__device__ __forceinline__ void insert_point(unsigned long long (&kk)[KC], float (&kd)[KC], unsigned long long key,
                                              float d2) {
 #pragma unroll
     for (int k = KC - 1; k > 0; --k) {
-        const bool shift = z < kz[k - 1] || (z == kz[k - 1] && id < kid[k - 1]);
-        const bool here = !shift && (z < kz[k] || (z == kz[k] && id < kid[k]));
-        if (shift) {
-            kz[k] = kz[k - 1];
-            kid[k] = kid[k - 1];
-            kd[k] = kd[k - 1];
-        } else if (here) {
-            kz[k] = z;
-            kid[k] = id;
-            kd[k] = d2;
-        }
+        const bool shift = key < kk[k - 1];
+        const bool here = !shift && key < kk[k];
+        kk[k] = shift ? kk[k - 1] : (here ? key : kk[k]);
+        kd[k] = shift ? kd[k - 1] : (here ? d2 : kd[k]);
     }
-    if (z < kz[0] || (z == kz[0] && id < kid[0])) {
-        kz[0] = z;
-        kid[0] = id;
+    if (key < kk[0]) {
+        kk[0] = key;
         kd[0] = d2;
     }
 }
@@ -106,27 +108,27 @@ __device__ __forceinline__ void insert_point(float (&kz)[KC], int (&kid)[KC], fl
 // One pixel's K slots from its register list (16-byte stores when K is a multiple of 4 and
 // the outputs are 16-byte aligned).
 template <int KC>
-__device__ __forceinline__ void write_point_slots(const float (&kz)[KC], const int (&kid)[KC], const float (&kd)[KC],
-                                                  int K, int64_t o, bool vec, int64_t* __restrict__ idx,
+__device__ __forceinline__ void write_point_slots(const unsigned long long (&kk)[KC], const float (&kd)[KC], int K,
+                                                  int64_t o, bool vec, int64_t* __restrict__ idx,
                                                   float* __restrict__ zbuf, float* __restrict__ dists) {
+    long long v[KC];
+    float z[KC], d[KC];
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+        const bool ok = kk[k] != kEmpty;
+        v[k] = ok ? (long long)(unsigned)(kk[k] & 0xffffffffu) : -1;
+        z[k] = ok ? __uint_as_float((unsigned)(kk[k] >> 32)) : -1.f;
+        d[k] = ok ? kd[k] : -1.f;
+    }
     if constexpr (KC >= 4) {
         if (vec && (K & 3) == 0) {
 #pragma unroll
             for (int k = 0; k < KC; k += 4) {
                 if (k >= K) break;
-                long long v[4];
-                float z4[4], d4[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const bool ok = kid[k + u] != INT_MAX;
-                    v[u] = ok ? kid[k + u] : -1;
-                    z4[u] = ok ? kz[k + u] : -1.f;
-                    d4[u] = ok ? kd[k + u] : -1.f;
-                }
-                reinterpret_cast<longlong2*>(idx + o + k)[0] = make_longlong2(v[0], v[1]);
-                reinterpret_cast<longlong2*>(idx + o + k)[1] = make_longlong2(v[2], v[3]);
-                *reinterpret_cast<float4*>(zbuf + o + k) = make_float4(z4[0], z4[1], z4[2], z4[3]);
-                *reinterpret_cast<float4*>(dists + o + k) = make_float4(d4[0], d4[1], d4[2], d4[3]);
+                reinterpret_cast<longlong2*>(idx + o + k)[0] = make_longlong2(v[k], v[k + 1]);
+                reinterpret_cast<longlong2*>(idx + o + k)[1] = make_longlong2(v[k + 2], v[k + 3]);
+                *reinterpret_cast<float4*>(zbuf + o + k) = make_float4(z[k], z[k + 1], z[k + 2], z[k + 3]);
+                *reinterpret_cast<float4*>(dists + o + k) = make_float4(d[k], d[k + 1], d[k + 2], d[k + 3]);
             }
             return;
         }
@@ -134,10 +136,9 @@ __device__ __forceinline__ void write_point_slots(const float (&kz)[KC], const i
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
         if (k >= K) break;
-        const bool ok = kid[k] != INT_MAX;
-        idx[o + k] = ok ? kid[k] : -1;
-        zbuf[o + k] = ok ? kz[k] : -1.f;
-        dists[o + k] = ok ? kd[k] : -1.f;
+        idx[o + k] = v[k];
+        zbuf[o + k] = z[k];
+        dists[o + k] = d[k];
     }
 }
 
@@ -162,12 +163,11 @@ __global__ void __launch_bounds__(256) k_point_fine(const float* __restrict__ pt
     const double pxd = -1.0 + (2.0 * j + 1.0) / W, pyd = 1.0 - (2.0 * i + 1.0) / H;
     const float pxh = (float)pxd, pyh = (float)pyd;
     const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
-    float kz[KC], kd[KC];
-    int kid[KC];
+    unsigned long long kk[KC];
+    float kd[KC];
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
-        kz[k] = FLT_MAX;
-        kid[k] = INT_MAX;
+        kk[k] = kEmpty;
         kd[k] = -1.f;
     }
     const int beg = offsets[b], end = offsets[b + 1];
@@ -184,13 +184,12 @@ __global__ void __launch_bounds__(256) k_point_fine(const float* __restrict__ pt
             const float4 q = sp[t];
             const float dx = (pxh - q.x) + pxl, dy = (pyh - q.y) + pyl;
             const float d2 = fmaf(dx, dx, dy * dy);
-            const int id = __float_as_int(q.w);
-            if (d2 <= r2 && (q.z < kz[KC - 1] || (q.z == kz[KC - 1] && id < kid[KC - 1])))
-                insert_point<KC>(kz, kid, kd, q.z, id, d2);
+            const unsigned long long key = point_key(q.z, __float_as_int(q.w));
+            if (d2 <= r2 && key < kk[KC - 1]) insert_point<KC>(kk, kd, key, d2);
         }
     }
     if (i < H && j < W)
-        write_point_slots<KC>(kz, kid, kd, K, (((int64_t)n * H + i) * W + j) * K, vec, idx, zbuf, dists);
+        write_point_slots<KC>(kk, kd, K, (((int64_t)n * H + i) * W + j) * K, vec, idx, zbuf, dists);
 }
 
 // Backward of the point rasterizer: thread per slot, one float4 (x, y, z, 0) atomic per
