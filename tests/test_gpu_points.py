@@ -241,3 +241,33 @@ def test_knn_backward_matches_oracle(oracle_mod):
     w1, w2 = oracle_mod.knn_bwd(kb.p1, kb.p2, wi, g)
     compare_grad(g1, w1, label="knn grad p1")
     compare_grad(g2, w2, label="knn grad p2")
+
+
+@pytest.mark.parametrize("D,K", [(1, 5), (4, 32)])
+def test_knn_other_dimensions(oracle_mod, D, K):
+    """D = 1 and D = 4 (the widest supported), K up to 32, heterogeneous clouds."""
+    rng = np.random.default_rng(20 + D)
+    sizes = [700, 37, 1500, 5]
+    p2 = rng.normal(size=(sum(sizes), D)).astype(np.float32)
+    p1 = (p2 + 0.05 * rng.normal(size=p2.shape)).astype(np.float32)
+    f = np.cumsum([0] + sizes[:-1]).astype(np.int64)
+    n = np.array(sizes, np.int64)
+    gi, gd = mr.knn_fwd(cuda(p1), f, n, cuda(p2), f, n, K)
+    wi, wd, flags = oracle_mod.knn(p1, f, n, p2, f, n, K)
+    _compare_knn(np_(gi), np_(gd), wi, wd, flags, f"knn D={D} K={K}")
+    g = syn.random_grads(wi.shape, 30 + D)
+    g1, g2 = mr.knn_bwd(cuda(p1), cuda(p2), cuda(wi), cuda(g))
+    w1, w2 = oracle_mod.knn_bwd(p1, p2, wi, g)
+    compare_grad(g1, w1, label=f"knn D={D} grad p1")
+    compare_grad(g2, w2, label=f"knn D={D} grad p2")
+
+
+def test_point_rasterizer_many_slots_and_dense_bins(oracle_mod):
+    """K = 32 and a radius that puts thousands of points in a bin (several 256-point chunks)."""
+    pb = syn.make_point_batch(2, n_clouds=3)             # the third cloud has 2562 points
+    H, W, K, r = 45, 38, 32, np.float32(0.15)
+    got = mr.rasterize_points_fwd(cuda(pb.points), pb.cloud_first_idx, pb.num_points_per_cloud, H, W, r, K)
+    wi, wz, wd, flags = oracle_mod.rasterize_points(pb.points, pb.cloud_first_idx, pb.num_points_per_cloud, H, W,
+                                                    r, K)
+    assert (wi[..., -1] >= 0).mean() > 0.05              # some pixels fill all 32 slots
+    _compare_slots(got, (wi, wz, wd), flags[..., None].repeat(K, -1), "K=32 dense")

@@ -288,3 +288,41 @@ def test_gouraud_lighting_at_vertices_end_to_end(oracle_mod):
     keep = ~vflags
     for name, x, y in (("grad points", gP, oP), ("grad normals", gN, oN), ("grad albedo", gA, oA)):
         compare_grad(np_(x)[keep], y[keep], label=name)
+
+
+def test_shading_full_size_sampled(oracle_mod):
+    """The benchmark batch (64 meshes, 512x512, K=4) through the benchmark's launches:
+    rasterize -> Gouraud colours -> soft RGB blend, and per-fragment Phong shading; sampled
+    pixels against the oracle's chain computed from its own fragments at those pixels."""
+    b = syn.make_batch(5)
+    w = b.workload
+    rng = np.random.default_rng(40)
+    vcol = rng.uniform(size=(b.verts.shape[0], 3)).astype(np.float32)
+    bg = np.array([1.0, 1.0, 1.0], np.float32)
+    kw = dict(sigma=w.sigma, gamma=1e-2, znear=1.0, zfar=10.0)
+    prm = _params(32.0)
+    v, f = cuda(b.verts), cuda(b.faces)
+    p2f, zbuf, bary, dists = mr.rasterize_fwd(v, f, b.mesh_to_face_first_idx, b.num_faces_per_mesh, w.H, w.W,
+                                              w.blur_radius, w.K)
+    col = mr.interpolate_fwd(p2f, bary, f, cuda(vcol))
+    rgba = np_(mr.blend_fwd(p2f, col, dists, zbuf, bg, **kw)).reshape(-1, 4)
+    pcol = np_(mr.phong_shade_fwd(p2f, bary, f, cuda(b.world), cuda(b.normals), cuda(vcol), prm)).reshape(-1, w.K, 3)
+    mr.device_status()
+    covered = np.flatnonzero((np_(p2f)[..., 0] >= 0).reshape(-1))
+    pix = np.concatenate([rng.choice(covered, 1500, replace=False), rng.integers(0, b.N * w.H * w.W, 300)])
+    op2f, oz, ob, od, ex = oracle_mod.rasterize_fwd(b.verts, b.faces, b.mesh_to_face_first_idx,
+                                                    b.num_faces_per_mesh, w.H, w.W, np.float32(w.blur_radius),
+                                                    w.K, False, pixels=pix)
+    ok = ex == 0
+    assert ok.mean() > 0.95
+    ocol = oracle_mod.interpolate_fwd(op2f, ob, b.faces, vcol)
+    orgba = oracle_mod.blend_fwd(op2f, ocol, od, oz, bg, **kw)
+    err = (np.abs(rgba[pix] - orgba) - (1e-4 * np.abs(orgba) + 1e-5))[ok]
+    assert err.max() <= 0, f"rgba off by {err.max():.3g}"
+    opc, pflags = oracle_mod.phong_shade_fwd(op2f, ob, b.faces, b.world, b.normals, vcol, prm.astype(np.float64))
+    sel = ok[:, None] & ~pflags & (op2f >= 0)
+    col_a, _, _ = _rounding_allowance(oracle_mod, op2f, ob, b.faces, b.world, b.normals, vcol,
+                                      prm.astype(np.float64), np.zeros(op2f.shape + (3,)))
+    tol = 1e-4 * np.abs(opc) + 1e-5 + _light_tol(32.0) + 4.0 * col_a
+    perr = (np.abs(pcol[pix] - opc) - tol)[sel]
+    assert perr.max() <= 0, f"Phong colours off by {perr.max():.3g}"
