@@ -231,7 +231,7 @@ __global__ void k_xyzw_to_xyz(const float4* __restrict__ acc, int64_t V, float* 
 // pixels per warp), float32.  Per slot the nearest edge u -> v is recomputed and its two
 // end points receive -2 (p - q)(1 - t) and -2 (p - q) t times dL/ddist.
 template <int KC>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 5)   // 48 registers: 5 CTAs per SM (measured 0.780 -> 0.746 ms)
 k_sil_raster_bwd(const float* __restrict__ verts, int64_t V, const int64_t* __restrict__ faces, int64_t F,
                  const int64_t* __restrict__ p2f, const float* __restrict__ dists,
                  const float* __restrict__ grad_alpha, int64_t npix, int H, int W, int K, float sigma,
