@@ -13,9 +13,10 @@
 // holding its first query's cell, so the K-th distances shrink early; a super-box or a
 // group box beyond the K-th distance of all 32 lanes is skipped (exact: a box bounds every
 // distance in it), a surviving group is staged in the warp's shared memory and each lane
-// tests it four distances at a time, keeping its K best (distance, original id) in
-// registers.  Warps never wait for one another.  The distance is formed from coordinate differences (not |q|^2 + |r|^2 -
-// 2 q.r, which cancels for near neighbours).  Tiles go out largest reference cloud first.
+// tests it four distances at a time, keeping its K best as 64-bit keys (distance bits
+// above the original id) in registers.  Warps never wait for one another.  The distance is
+// formed from coordinate differences (not |q|^2 + |r|^2 - 2 q.r, which cancels for near
+// neighbours).  Tiles go out largest reference cloud first.
 #include <algorithm>
 #include <cfloat>
 #include <climits>
@@ -52,7 +53,7 @@ __device__ __forceinline__ int cell_code(const float* __restrict__ x, const Clou
     for (int e = 0; e < (D < 3 ? D : 3); ++e) {
         const float ext = B.hi[e] - B.lo[e];
         const float t = ext > 0.f ? (x[e] - B.lo[e]) / ext * (float)kGrid : 0.f;
-        c[e] = min(max((int)t, 0), kGrid - 1);       // NaN converts to 0
+        c[e] = (int)fminf(fmaxf(t, 0.f), (float)(kGrid - 1));   // clamped before the cast; NaN -> 0
     }
     int code = 0;
 #pragma unroll
