@@ -37,7 +37,8 @@ UNIT = "pixel-face samples/s"
 C_TEST = 38                 # FP32 instructions per pixel-face test in this formulation (frozen)
 FP32_LANES_PER_SM = 128
 L2_FLUSH_BYTES = 256 << 20
-KERNELS_PER_STAGE = {"silhouette_raster_bwd": 2}    # main kernel + (x, y) -> (x, y, z) copy
+KERNELS_PER_STAGE = {"silhouette_raster_bwd": 2,   # main kernel + (x, y) -> (x, y, z) copy
+                     "bin_scan": 3}                # tile scans, tile totals, tile prefixes added
 
 
 # ----------------------------------------------------------------------------- counting
