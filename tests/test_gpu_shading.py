@@ -345,3 +345,46 @@ def test_shading_full_size_sampled(oracle_mod):
     tol = 1e-4 * np.abs(opc) + 1e-5 + _light_tol(32.0) + 4.0 * col_a
     perr = (np.abs(pcol[pix] - opc) - tol)[sel]
     assert perr.max() <= 0, f"Phong colours off by {perr.max():.3g}"
+
+
+@pytest.mark.parametrize("D", [1, 4])
+def test_blend_other_channel_counts(oracle_mod, frags, D):
+    """The element-wise blend path (D != 3) and a 4-channel attribute, on the oracle's fragments."""
+    b, p2f, zbuf, bary, dists, _ = frags
+    rng = np.random.default_rng(50 + D)
+    kw = dict(sigma=1e-4, gamma=1e-2, znear=1.0, zfar=100.0)
+    bg = rng.uniform(size=D).astype(np.float32)
+    colors = rng.uniform(size=p2f.shape + (D,)).astype(np.float32)
+    got = np_(mr.blend_fwd(cuda(p2f), cuda(colors), cuda(dists), cuda(zbuf), bg, **kw))
+    want = oracle_mod.blend_fwd(p2f, colors, dists, zbuf, bg, **kw)
+    assert np.all(np.abs(got - want) <= 1e-4 * np.abs(want) + 1e-6)
+    g = rng.normal(size=want.shape).astype(np.float32)
+    outs = mr.blend_bwd(cuda(p2f), cuda(colors), cuda(dists), cuda(zbuf), bg, grad_rgba=cuda(g), **kw)
+    wants = oracle_mod.blend_bwd(p2f, colors, dists, zbuf, bg, grad_rgba=g, **kw)
+    for name, x, y in zip(("grad_colors", "grad_dists", "grad_zbuf"), outs, wants):
+        compare_grad(x, y, label=f"D={D} {name}")
+
+
+def test_shading_on_perspective_correct_fragments(oracle_mod):
+    """Interpolation and Phong shading on perspective-correct fragments with K = 16 (the
+    element-wise kernels' widest slot template), against the oracle's own fragments."""
+    b = syn.make_batch(3, n_meshes=2)
+    H = W = 48
+    o = oracle_mod.rasterize_fwd(b.verts, b.faces, b.mesh_to_face_first_idx, b.num_faces_per_mesh, H, W,
+                                 np.float32(b.workload.blur_radius), 16, True)
+    p2f, bary = o[0], o[2].astype(np.float32)
+    assert (p2f[..., 1] >= 0).mean() > 0.05
+    rng = np.random.default_rng(60)
+    attr = rng.uniform(-1, 1, size=(b.verts.shape[0], 4)).astype(np.float32)
+    got = np_(mr.interpolate_fwd(cuda(p2f), cuda(bary), cuda(b.faces), cuda(attr)))
+    want = oracle_mod.interpolate_fwd(p2f, bary, b.faces, attr)
+    scale = oracle_mod.interpolate_fwd(p2f, np.abs(bary), b.faces, np.abs(attr))
+    assert np.all(np.abs(got - want) <= 1e-6 + 2.0 ** -22 * scale)
+    prm = _params(8.0)
+    alb = rng.uniform(size=(b.verts.shape[0], 3)).astype(np.float32)
+    pc = np_(mr.phong_shade_fwd(cuda(p2f), cuda(bary), cuda(b.faces), cuda(b.world), cuda(b.normals), cuda(alb), prm))
+    wc, flags = oracle_mod.phong_shade_fwd(p2f, bary, b.faces, b.world, b.normals, alb, prm.astype(np.float64))
+    col_a, _, _ = _rounding_allowance(oracle_mod, p2f, bary, b.faces, b.world, b.normals, alb,
+                                      prm.astype(np.float64), np.zeros(p2f.shape + (3,)))
+    tol = 1e-4 * np.abs(wc) + 1e-6 + _light_tol(8.0) + 4.0 * col_a
+    assert np.all((np.abs(pc - wc) - tol)[~flags] <= 0)
