@@ -364,10 +364,10 @@ def _timed_steps(mr, torch, dev, stream, flush, steps, step):
     return ms, {name: t / steps for name, (t, n) in st.items() if n}
 
 
-def point_box_samples(pb):
+def point_box_samples(pb, rows=None):
     """Pixel-point samples of a point batch: (pixel, point) pairs of the same image whose pixel
     centre lies in the point's box of half-width radius (exact host count; points behind the
-    camera excluded)."""
+    camera excluded); with ``rows`` only those image rows count."""
     w = pb.workload
     p = pb.points.astype(np.float64)
     r = float(np.float32(w.radius))
@@ -376,7 +376,11 @@ def point_box_samples(pb):
     jh = np.minimum(np.floor((p[:, 0] + r + 1) * w.W / 2 - 0.5), w.W - 1)
     il = np.maximum(np.ceil((1 - p[:, 1] - r) * w.H / 2 - 0.5), 0)
     ih = np.minimum(np.floor((1 - p[:, 1] + r) * w.H / 2 - 0.5), w.H - 1)
-    n = np.clip(jh - jl + 1, 0, None) * np.clip(ih - il + 1, 0, None)
+    if rows is None:
+        n = np.clip(jh - jl + 1, 0, None) * np.clip(ih - il + 1, 0, None)
+    else:
+        rr = np.asarray(rows)
+        n = np.clip(jh - jl + 1, 0, None) * ((rr[None, :] >= il[:, None]) & (rr[None, :] <= ih[:, None])).sum(1)
     return int(np.sum(n[ok]))
 
 
@@ -413,6 +417,92 @@ def points_step_timing(mr, torch, dev, stream, flush, args, hbm_peak, hbm_note):
             "mpix_per_s": npix / (ms / 1e3) / 1e6, "points": int(pb.points.shape[0]), "steps": steps,
             "stages": out, "hbm_peak_note": hbm_note,
             "note": w.description + "; alpha compositing fwd+bwd; L2 flushed per step"}
+
+
+def next_row_oracle_baselines(batch, rows_wanted):
+    """The oracle, as it stands, on a bounded sample of each next row's workload (rank 0,
+    host cores): the same fwd+bwd chain as the timed step on a few whole image rows (one
+    query subset for KNN).  Returns {row: cpu_baseline dict}."""
+    import oracle
+    from differentiable_mesh_rasterization_b200 import synthetic as syn
+    out = {}
+    w = batch.workload
+    H, W, K = w.H, w.W, w.K
+    cores = oracle.default_threads()
+    kw = dict(sigma=w.sigma, gamma=1e-2, znear=1.0, zfar=10.0)
+    bg = np.ones(3)
+    prm = oracle.phong_params([1.0, 1.5, 3.0], [0.0, 0.0, 2.7], [0.1, 0.1, 0.15], [0.6, 0.55, 0.5],
+                              [0.3, 0.3, 0.3], 32.0)
+    alb = np.abs(syn.random_grads((batch.verts.shape[0], 3), 11)).clip(max=1.0)
+    rows = np.unique(np.linspace(0, H - 1, 4).round().astype(np.int64))
+    pix = ((np.arange(batch.N)[:, None, None] * H + rows[None, :, None]) * W + np.arange(W)[None, None, :]).reshape(-1)
+    full = batch.N * H * W
+
+    def scatter(a, fill):
+        z = np.full((full,) + a.shape[1:], fill, a.dtype)
+        z[pix] = a
+        return z.reshape((batch.N, H, W) + a.shape[1:])
+
+    for shading in ("gouraud", "phong"):
+        if shading not in rows_wanted:
+            continue
+        t0 = time.perf_counter()
+        p2f, zb, ba, di, _ = oracle.rasterize_fwd(batch.verts, batch.faces, batch.mesh_to_face_first_idx,
+                                                  batch.num_faces_per_mesh, H, W, np.float32(w.blur_radius), K,
+                                                  False, pixels=pix, exempt=False)
+        g = np.ones((len(pix), 4))
+        if shading == "gouraud":
+            vcol, _ = oracle.phong_fwd(batch.world, batch.normals, alb, prm)
+            col = oracle.interpolate_fwd(p2f, ba, batch.faces, vcol)
+        else:
+            col, _ = oracle.phong_shade_fwd(p2f, ba, batch.faces, batch.world, batch.normals, alb, prm)
+        oracle.blend_fwd(p2f, col, di, zb, bg, **kw)
+        gc, gd, gz = oracle.blend_bwd(p2f, col, di, zb, bg, grad_rgba=g, **kw)
+        if shading == "gouraud":
+            gv, gb = oracle.interpolate_bwd(p2f, ba, batch.faces, vcol, gc)
+            oracle.phong_bwd(batch.world, batch.normals, alb, prm, gv)
+        else:
+            gb = oracle.phong_shade_bwd(p2f, ba, batch.faces, batch.world, batch.normals, alb, prm, gc)[3]
+        oracle.rasterize_bwd(batch.verts, batch.faces, scatter(p2f, -1), False, grad_zbuf=scatter(gz, 0.0),
+                             grad_bary=scatter(gb, 0.0), grad_dists=scatter(gd, 0.0))
+        dt = time.perf_counter() - t0
+        out[shading + "_rgb"] = {"value": count_samples(batch, rows) / dt, "unit": "pixel-face samples/s",
+                                 "cores": cores, "kind": "oracle", "seconds": dt,
+                                 "sample": f"{len(rows)} evenly spaced rows of each of the {batch.N} images"}
+    if "points" in rows_wanted:
+        pb = syn.make_point_batch(5, n_clouds=batch.N)
+        pw = pb.workload
+        r = np.float32(pw.radius)
+        prow = np.array([pw.H // 2])
+        ppix = ((np.arange(pb.N)[:, None, None] * pw.H + prow[None, :, None]) * pw.W +
+                np.arange(pw.W)[None, None, :]).reshape(-1)
+        t0 = time.perf_counter()
+        idx, _, pd, _ = oracle.rasterize_points(pb.points, pb.cloud_first_idx, pb.num_points_per_cloud, pw.H, pw.W,
+                                                r, pw.K, pixels=ppix)
+        oracle.composite_points(idx, pd, pb.features, r)
+        _, gdd = oracle.composite_points_bwd(idx, pd, pb.features, r, np.ones((len(ppix), pw.C)))
+        fi = np.full((pb.N * pw.H * pw.W, pw.K), -1, np.int64)
+        fd = np.zeros((pb.N * pw.H * pw.W, pw.K))
+        fi[ppix] = idx
+        fd[ppix] = gdd
+        oracle.rasterize_points_bwd(pb.points, fi.reshape(pb.N, pw.H, pw.W, pw.K),
+                                    grad_dists=fd.reshape(pb.N, pw.H, pw.W, pw.K))
+        dt = time.perf_counter() - t0
+        out["points_rgb"] = {"value": point_box_samples(pb, prow) / dt, "unit": "pixel-point samples/s",
+                             "cores": 1, "kind": "oracle", "seconds": dt,
+                             "sample": f"the middle row of each of the {pb.N} images"}
+    if "knn" in rows_wanted:
+        kb = syn.make_knn_batch(5, n_clouds=batch.N)
+        sel = np.concatenate([kb.first1[n] + np.arange(min(50, kb.num1[n])) for n in range(kb.N)])
+        n1 = np.array([min(50, kb.num1[n]) for n in range(kb.N)], np.int64)
+        f1 = np.cumsum(np.r_[0, n1[:-1]])
+        t0 = time.perf_counter()
+        ki, kd, _ = oracle.knn(kb.p1[sel], f1, n1, kb.p2, kb.first2, kb.num2, kb.workload.K)
+        oracle.knn_bwd(kb.p1[sel], kb.p2, ki, np.ones(kd.shape))
+        dt = time.perf_counter() - t0
+        out["knn"] = {"value": float(np.sum(n1 * kb.num2)) / dt, "unit": "pairs/s", "cores": 1, "kind": "oracle",
+                      "seconds": dt, "sample": f"the first 50 queries of each of the {kb.N} clouds"}
+    return out
 
 
 KNN_C_PAIR = 7       # FP32 instructions per (query, reference) pair for D=3: 3 FADD, 3 FFMA, 1 compare
@@ -699,6 +789,10 @@ def main():
         rows["knn"] = knn_step_timing(mr, torch, dev, stream, flush, args, peak_alu)
     if rows:
         line["next_rows"] = rows
+        if rank == 0 and not args.no_cpu_baseline:
+            for name, base in next_row_oracle_baselines(batch, args.rows).items():
+                if name in rows:
+                    rows[name]["cpu_baseline"] = base
 
     if rank == 0 and not args.no_cpu_baseline:
         import oracle
