@@ -246,7 +246,9 @@ __device__ __forceinline__ float box_bound(const float (&q)[4], float4 lo4, floa
 // and walks the cloud's super-boxes outward from the one holding its first query's cell
 // (home, home + 1, home - 1, ...).  A super-box or group box beyond every lane's K-th
 // distance is skipped by the whole warp; a group that survives is staged in the warp's
-// shared memory (32 points and ids) and every lane tests it four distances at a time.
+// shared memory (32 points, one array per coordinate, and ids) and every lane tests it
+// four distances at a time, two by two with packed two-lane float32 instructions (each
+// lane rounds as the scalar instruction would, so the distances are the scalar ones).
 template <int KC, int D>
 __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ sq, const int* __restrict__ sqid,
                                                      const short* __restrict__ sqcode, const float4* __restrict__ sr,
@@ -257,8 +259,8 @@ __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ 
                                                      const float4* __restrict__ slo, const float4* __restrict__ shi,
                                                      const KnnTile* __restrict__ tiles, int K,
                                                      int64_t* __restrict__ idx, float* __restrict__ dists) {
-    __shared__ float4 wp[kKnnQueries / 32][32];
-    __shared__ int wid[kKnnQueries / 32][32];
+    __shared__ __align__(16) float wc[kKnnQueries / 32][4][32];
+    __shared__ __align__(16) int wid[kKnnQueries / 32][32];
     const KnnTile T = tiles[blockIdx.x];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (warp * 32 >= T.qn) return;                              // whole warp past the tile: no partner waits
@@ -272,6 +274,9 @@ __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ 
         q[0] = v.x; q[1] = v.y; q[2] = v.z; q[3] = v.w;
         qid = sqid[T.s0 + threadIdx.x];
     }
+    f32x2 qq[D];
+#pragma unroll
+    for (int e = 0; e < D; ++e) qq[e] = pack2(q[e], q[e]);
     unsigned long long kk[KC];
 #pragma unroll
     for (int k = 0; k < KC; ++k) kk[k] = kNone;
@@ -295,28 +300,33 @@ __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ 
                 const int cnt = (int)min((int64_t)32, rn - pb);
                 __syncwarp();
                 if (lane < cnt) {
-                    wp[warp][lane] = sr[r0 + pb + lane];
+                    const float4 r = sr[r0 + pb + lane];
+                    const float rv[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+                    for (int e = 0; e < D; ++e) wc[warp][e][lane] = rv[e];
                     wid[warp][lane] = srid[r0 + pb + lane];
                 }
                 __syncwarp();
+                // slots at or past cnt hold stale values; their distances are computed
+                // (t < cnt <= 32 keeps every read inside the arrays) and never inserted
                 for (int t = 0; t < cnt; t += 4) {
-                    float d4[4];
+                    f32x2 dlo = 0, dhi = 0;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float4 r = wp[warp][min(t + u, 31)];
-                        const float rv[4] = {r.x, r.y, r.z, r.w};
-                        float d = 0.f;
-#pragma unroll
-                        for (int e = 0; e < D; ++e) {
-                            const float w = q[e] - rv[e];
-                            d = fmaf(w, w, d);
-                        }
-                        d4[u] = d;
+                    for (int e = 0; e < D; ++e) {
+                        const ulonglong2 r = *reinterpret_cast<const ulonglong2*>(&wc[warp][e][t]);
+                        const f32x2 wlo = sub2(qq[e], r.x), whi = sub2(qq[e], r.y);
+                        dlo = e == 0 ? mul2(wlo, wlo) : fma2(wlo, wlo, dlo);
+                        dhi = e == 0 ? mul2(whi, whi) : fma2(whi, whi, dhi);
                     }
+                    float d4[4];
+                    unpack2(dlo, d4[0], d4[1]);
+                    unpack2(dhi, d4[2], d4[3]);
+                    const int4 id4 = *reinterpret_cast<const int4*>(&wid[warp][t]);
+                    const int ids[4] = {id4.x, id4.y, id4.z, id4.w};
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
                         if (t + u < cnt) {
-                            const unsigned long long key = nn_key(d4[u], wid[warp][t + u]);
+                            const unsigned long long key = nn_key(d4[u], ids[u]);
                             if (key < kk[KC - 1]) insert_nn<KC>(kk, key);
                         }
                 }
