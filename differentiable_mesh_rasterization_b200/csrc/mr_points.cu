@@ -144,15 +144,20 @@ __device__ __forceinline__ void write_point_slots(const unsigned long long (&kk)
 
 // Fine pass: one CTA of 256 threads per 16 x 16 bin, one thread per pixel; the bin's
 // points are staged in shared memory 256 at a time and every thread keeps its K nearest in
-// registers.  Measured and rejected: a bounded grid walking the bins (load imbalance,
-// 1.45 vs 1.13 ms on the benchmark batch) and sorting each chunk by depth in shared memory
-// so that a full list can stop early (1.53 ms: the warp waits for its slowest lane).
+// registers.  While staging, each point's pixel box (the one that binned it) is tested
+// against the eight 4 x 8 warp tiles of the bin; every warp then compacts the staged
+// points whose box meets its tile (ballot) and tests only those.  Measured and rejected:
+// a bounded grid walking the bins (load imbalance, 1.45 vs 1.13 ms on the benchmark
+// batch) and sorting each chunk by depth in shared memory so that a full list can stop
+// early (1.53 ms: the warp waits for its slowest lane).
 template <int KC>
-__global__ void __launch_bounds__(256) k_point_fine(const float* __restrict__ pts, const int* __restrict__ offsets,
-                                                    const int* __restrict__ list, int H, int W, float r2, int K,
-                                                    int nbx, int nby, int64_t* __restrict__ idx,
+__global__ void __launch_bounds__(256, KC <= 8 ? 5 : 1) k_point_fine(const float* __restrict__ pts, const int* __restrict__ offsets,
+                                                    const int* __restrict__ list, int H, int W, float r, float r2,
+                                                    int K, int nbx, int nby, int64_t* __restrict__ idx,
                                                     float* __restrict__ zbuf, float* __restrict__ dists, bool vec) {
     __shared__ float4 sp[256];
+    __shared__ unsigned char smask[256];          // bit w: the point's box meets warp w's tile
+    __shared__ unsigned char wl[8][256];          // per warp: its staged points, compacted
     const int b = blockIdx.x;
     const int n = b / (nbx * nby), by = (b / nbx) % nby, bx = b % nbx;
     // each warp takes a 4 x 8 block of the bin (a point's disc meets fewer warps than with
@@ -170,18 +175,40 @@ __global__ void __launch_bounds__(256) k_point_fine(const float* __restrict__ pt
         kk[k] = kEmpty;
         kd[k] = -1.f;
     }
+    const unsigned lt_mask = (1u << lane) - 1u;
     const int beg = offsets[b], end = offsets[b + 1];
     for (int c0 = beg; c0 < end; c0 += 256) {
         __syncthreads();
+        unsigned mask = 0;
         if (c0 + (int)threadIdx.x < end) {
             const int p = list[c0 + threadIdx.x];
-            sp[threadIdx.x] = make_float4(pts[3 * (int64_t)p], pts[3 * (int64_t)p + 1], pts[3 * (int64_t)p + 2],
-                                          __int_as_float(p));
+            const float x = pts[3 * (int64_t)p], y = pts[3 * (int64_t)p + 1];
+            sp[threadIdx.x] = make_float4(x, y, pts[3 * (int64_t)p + 2], __int_as_float(p));
+            // pixel ranges whose centres lie within r + 2e-5 of the point, in float32: the
+            // margin (2e-5 NDC) is far above the rounding of these few operations, so the
+            // ranges hold every pixel the test below can accept
+            const float R = r + 2e-5f, hw = 0.5f * W, hh = 0.5f * H;
+            const int j0 = (int)ceilf((x - R + 1.f) * hw - 0.5f), j1 = (int)floorf((x + R + 1.f) * hw - 0.5f);
+            const int i0 = (int)ceilf((1.f - y - R) * hh - 0.5f), i1 = (int)floorf((1.f - y + R) * hh - 0.5f);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const int ti = by * kPtBin + (v >> 1) * 4, tj = bx * kPtBin + (v & 1) * 8;
+                if (j0 <= tj + 7 && j1 >= tj && i0 <= ti + 3 && i1 >= ti) mask |= 1u << v;
+            }
         }
+        smask[threadIdx.x] = (unsigned char)mask;
         __syncthreads();
-        const int cnt = min(256, end - c0);
-        for (int t = 0; t < cnt; ++t) {
-            const float4 q = sp[t];
+        int nw = 0;                               // this warp's points of the chunk
+#pragma unroll
+        for (int s0 = 0; s0 < 256; s0 += 32) {
+            const bool mine = (smask[s0 + lane] >> w) & 1u;
+            const unsigned bal = __ballot_sync(0xffffffffu, mine);
+            if (mine) wl[w][nw + __popc(bal & lt_mask)] = (unsigned char)(s0 + lane);
+            nw += __popc(bal);
+        }
+        __syncwarp();
+        for (int u = 0; u < nw; ++u) {
+            const float4 q = sp[wl[w][u]];
             const float dx = (pxh - q.x) + pxl, dy = (pyh - q.y) + pyl;
             const float d2 = fmaf(dx, dx, dy * dy);
             const unsigned long long key = point_key(q.z, __float_as_int(q.w));
@@ -466,7 +493,7 @@ int mr_rasterize_points_fwd(const float* points, int64_t P, const int64_t* cloud
                          (reinterpret_cast<uintptr_t>(dists) & 15) == 0;
         ProfScope ps(MR_STAGE_POINTS_FINE, s);
 #define MR_PF(KC) \
-    k_point_fine<KC><<<nbins, 256, 0, s>>>(points, offsets, list, H, W, r2, K, nbx, nby, idx, zbuf, dists, vec)
+    k_point_fine<KC><<<nbins, 256, 0, s>>>(points, offsets, list, H, W, radius, r2, K, nbx, nby, idx, zbuf, dists, vec)
         if (K <= 1) MR_PF(1);
         else if (K <= 2) MR_PF(2);
         else if (K <= 4) MR_PF(4);
