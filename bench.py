@@ -147,8 +147,8 @@ def oracle_sample(batch, ga, seconds=15.0):
     t1 = run_oracle(batch, ga, np.array([w.H // 2]))
     R = int(max(1, min(w.H, round(seconds / max(t1, 1e-3)))))
     rows = np.unique(np.linspace(0, w.H - 1, R).round().astype(np.int64))
-    return rows, (f"{len(rows)} evenly spaced rows of each of the {batch.N} images "
-                  f"(fwd + silhouette fwd/bwd + raster bwd on those pixels)")
+    what = "fwd" if w.sigma is None else "fwd + silhouette fwd/bwd + raster bwd"
+    return rows, f"{len(rows)} evenly spaced rows of each of the {batch.N} images ({what} on those pixels)"
 
 
 def run_oracle(batch, ga, rows):
@@ -162,6 +162,8 @@ def run_oracle(batch, ga, rows):
     p2f, zbuf, bary, dists, _ = oracle.rasterize_fwd(batch.verts, batch.faces, batch.mesh_to_face_first_idx,
                                                      batch.num_faces_per_mesh, H, W, np.float32(w.blur_radius), K,
                                                      w.perspective_correct, pixels=pix, exempt=False)
+    if w.sigma is None:                   # forward-only (hard) workload
+        return time.perf_counter() - t0
     sig = np.float32(w.sigma)
     oracle.silhouette_fwd(p2f, dists, sig)
     gd = oracle.silhouette_bwd(ga.reshape(-1)[pix], p2f, dists, sig)
@@ -575,8 +577,7 @@ def main():
 
     batch = syn.make_batch(args.config, seed=rank_seed(args.config, rank), n_meshes=args.images)
     w = batch.workload
-    if w.sigma is None:
-        raise SystemExit("the benchmark step needs a soft-silhouette workload (sigma)")
+    hard = w.sigma is None            # batch 4: hard rasterization, forward only
     samples = count_samples(batch)
     verts = torch.from_numpy(batch.verts).to(dev)
     faces = torch.from_numpy(batch.faces).to(dev)
@@ -586,11 +587,17 @@ def main():
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        p2f, zbuf, bary, dists, alpha = mr.rasterize_fwd(verts, faces, first, num, w.H, w.W, w.blur_radius, w.K,
+    def run(v, f, g):
+        """One step on device inputs; returns the results a caller reads back: alpha and
+        grad_verts, or the depth buffer of a forward-only (hard) workload."""
+        if hard:
+            return (mr.rasterize_fwd(v, f, first, num, w.H, w.W, w.blur_radius, w.K, w.perspective_correct)[1],)
+        p2f, zbuf, bary, dists, alpha = mr.rasterize_fwd(v, f, first, num, w.H, w.W, w.blur_radius, w.K,
                                                          w.perspective_correct, sigma=w.sigma)
-        gv = mr.silhouette_rasterize_bwd(verts, faces, p2f, dists, w.sigma, ga)
-        return alpha, gv
+        return alpha, mr.silhouette_rasterize_bwd(v, f, p2f, dists, w.sigma, g)
+
+    def step():
+        return run(verts, faces, ga)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -626,19 +633,17 @@ def main():
     # end to end through the public API: pinned host inputs in, alpha + grad_verts out
     h_verts = torch.from_numpy(batch.verts).pin_memory()
     h_faces = torch.from_numpy(batch.faces).pin_memory()
-    h_ga = torch.from_numpy(ga_host).pin_memory()
-    h_alpha = torch.empty((w.N, w.H, w.W), dtype=torch.float32).pin_memory()
-    h_gv = torch.empty(batch.verts.shape, dtype=torch.float32).pin_memory()
+    h_ga = torch.from_numpy(np.zeros(0, np.float32) if hard else ga_host).pin_memory()   # nothing to upload when hard
+    h_res = ([torch.empty((w.N, w.H, w.W, w.K), dtype=torch.float32).pin_memory()] if hard else
+             [torch.empty((w.N, w.H, w.W), dtype=torch.float32).pin_memory(),
+              torch.empty(batch.verts.shape, dtype=torch.float32).pin_memory()])
 
     def e2e_step():
         dv = h_verts.to(dev, non_blocking=True)
         df = h_faces.to(dev, non_blocking=True)
         dg = h_ga.to(dev, non_blocking=True)
-        p2f, _, _, dists, alpha = mr.rasterize_fwd(dv, df, first, num, w.H, w.W, w.blur_radius, w.K,
-                                                   w.perspective_correct, sigma=w.sigma)
-        gv = mr.silhouette_rasterize_bwd(dv, df, p2f, dists, w.sigma, dg)
-        h_alpha.copy_(alpha, non_blocking=True)
-        h_gv.copy_(gv, non_blocking=True)
+        for h, d in zip(h_res, run(dv, df, dg)):
+            h.copy_(d, non_blocking=True)
 
     def e2e_serial(n):
         """Copies and compute of every step one after the other on the compute stream."""
@@ -687,18 +692,15 @@ def main():
             stream.wait_event(h2d_done[i])
             dv, df, dg = bufs[i]
             flush.zero_()
-            p2f, _, _, dists, alpha = mr.rasterize_fwd(dv, df, first, num, w.H, w.W, w.blur_radius, w.K,
-                                                       w.perspective_correct, sigma=w.sigma)
-            gv = mr.silhouette_rasterize_bwd(dv, df, p2f, dists, w.sigma, dg)
+            res = run(dv, df, dg)
             done = torch.cuda.Event()
             done.record(stream)
             freed[i] = done
             with torch.cuda.stream(ds):
                 ds.wait_event(done)
-                alpha.record_stream(ds)
-                gv.record_stream(ds)
-                h_alpha.copy_(alpha, non_blocking=True)
-                h_gv.copy_(gv, non_blocking=True)
+                for h, d in zip(h_res, res):
+                    d.record_stream(ds)
+                    h.copy_(d, non_blocking=True)
         e1.record(ds)
         torch.cuda.synchronize(dev)
         return e0.elapsed_time(e1)
@@ -719,7 +721,7 @@ def main():
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
     e2e_value = tot_samples * args.e2e_steps / (float(te[0]) / 1e3) if args.e2e_steps > 0 else None
     h2d = h_verts.numel() * 4 + h_faces.numel() * 8 + h_ga.numel() * 4
-    d2h = h_alpha.numel() * 4 + h_gv.numel() * 4
+    d2h = sum(h.numel() * 4 for h in h_res)
 
     # roofline of the dominant kernel (the fine pass: the pixel-face tests) and of the
     # epilogue (which writes the per-slot outputs)
@@ -744,7 +746,7 @@ def main():
     achieved_alu = samples * C_TEST / fine_s / 1e12
     npix = batch.N * w.H * w.W
     fine_bytes = npix * 4 * w.K                      # the K winning face ids per pixel
-    epi_bytes = npix * (4 * w.K + 28 * w.K + 4)      # ids in; p2f, zbuf, bary, dists, alpha out
+    epi_bytes = npix * (4 * w.K + 28 * w.K + (0 if hard else 4))   # ids in; p2f, zbuf, bary, dists(, alpha) out
     full_batch = args.images is None and args.config == 5
     roof = {"bound": "alu", "achieved": achieved_alu, "peak": peak_alu, "unit": "T FP32-inst/s",
             "frac": achieved_alu / peak_alu, "traffic": measured_traffic("k_fine") if full_batch else None,
@@ -772,12 +774,13 @@ def main():
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": float(te[0]) / max(args.e2e_steps, 1), "pipelined": True,
                     "serial_ms_per_step": float(te[1]) / max(args.e2e_steps, 1),
-                    "note": "pinned host verts, faces, dL/dalpha in; alpha and grad_verts out; the copies of "
+                    "note": ("pinned host verts, faces in; the depth buffer out" if hard else
+                             "pinned host verts, faces, dL/dalpha in; alpha and grad_verts out") + "; the copies of "
                             "step k+1 (in) and step k (out) overlap the compute of step k on two copy streams"},
             "gpu_launches": int(sum(v[1] * KERNELS_PER_STAGE.get(k, 1) for k, v in stages.items())),
             "clocks": clk}
 
-    if args.no_shading:
+    if args.no_shading or hard:           # the next rows run on the soft batch-5 workloads
         args.rows = ""
     rows = {}
     if "gouraud" in args.rows or "phong" in args.rows:
