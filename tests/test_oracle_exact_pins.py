@@ -210,3 +210,33 @@ def test_silhouette_bwd_matches_torch_autograd(oracle_mod):
     ref = dt.grad.numpy()
     assert np.allclose(g, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
     assert np.all(g[p2f < 0] == 0)
+
+
+def test_closed_triangle_counts_its_boundary_as_inside(oracle_mod):
+    """Step 4 takes the closed triangle: vertices and edge points are inside."""
+    tri = np.array([[-0.5, -0.5, 2.0], [0.5, -0.5, 2.0], [0.0, 0.5, 2.0]], np.float64)
+    for px, py in ((-0.5, -0.5), (0.0, -0.5), (0.25, 0.0), (-0.25, 0.0), (0.0, 0.0)):
+        r = oracle_mod.probe(px, py, tri, False)
+        assert r["inside"], (px, py)
+    for px, py in ((0.0, -0.5 - 2.0 ** -20), (0.5, 0.0)):
+        assert not oracle_mod.probe(px, py, tri, False)["inside"]
+
+
+@pytest.mark.parametrize("persp", [False, True])
+def test_equal_depth_ties_go_to_the_lower_face_id(oracle_mod, persp):
+    """Step 10 orders by (z, face id): copies of one face tie exactly in depth."""
+    H = W = 16
+    tri = [[-0.7, -0.6, 2.0], [0.6, -0.5, 2.5], [0.0, 0.7, 3.0]]
+    far = [[-0.7, -0.6, 4.0], [0.6, -0.5, 4.0], [0.0, 0.7, 4.0]]
+    verts = np.array(far + tri + tri + tri, np.float32)           # faces 0 (behind), 1, 2, 3 (copies)
+    faces = np.arange(12, dtype=np.int64).reshape(4, 3)
+    p2f, zbuf, _, _, ex = oracle_mod.rasterize_fwd(verts, faces, np.array([0]), np.array([4]), H, W, 0.0, 4,
+                                                   persp, exempt=False)
+    cov = p2f[0, :, :, 0] >= 0
+    assert cov.sum() > 50
+    assert np.all(p2f[0][cov] == [1, 2, 3, 0])
+    assert np.all(zbuf[0][cov][:, 0] == zbuf[0][cov][:, 2])
+    one, *_ = oracle_mod.rasterize_fwd(verts, faces[::-1].copy(), np.array([0]), np.array([4]), H, W, 0.0, 2,
+                                       persp, exempt=False)
+    # reversed face order: the copies are now faces 0, 1, 2 and the far face is 3
+    assert np.all(one[0][cov] == [0, 1])
