@@ -22,6 +22,18 @@ def centre(i, j):
     return -1 + (2 * j + 1) / W, 1 - (2 * i + 1) / H
 
 
+
+def test_radius_is_inclusive(oracle_mod):
+    """Step 22 keeps a point at distance exactly r (squared distance <= r^2): with r two
+    pixel pitches every quantity is a dyadic rational, so the tie is exact."""
+    x0, y0 = centre(10, 10)
+    r = 2 * PITCH
+    pts = np.array([[x0, y0, 1.0]], np.float32)
+    idx, _, dists, flags = oracle_mod.rasterize_points(pts, [0], [1], H, W, r, 1)
+    for i, j in ((10, 12), (10, 8), (12, 10), (8, 10)):
+        assert idx[0, i, j, 0] == 0 and dists[0, i, j, 0] == r * r and flags[0, i, j]
+    assert idx[0, 10, 13, 0] == -1 and idx[0, 11, 12, 0] == -1
+
 def test_single_point_covers_a_lattice_disc(oracle_mod):
     x0, y0 = centre(13, 17)
     r = 2.5 * PITCH
