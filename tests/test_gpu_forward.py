@@ -86,6 +86,27 @@ def test_degenerate_behind_camera_and_empty_meshes(oracle_mod):
     assert set(np.unique(np_(g[0]))) <= {-1, 1}
 
 
+
+@pytest.mark.parametrize("persp", [False, True])
+def test_exact_depth_ties_go_to_the_lower_face_id(oracle_mod, persp):
+    """Copies of one face tie exactly in depth (identical constants on both sides): the
+    order is by face id, as in the oracle, at every covered pixel."""
+    H = W = 32
+    tri = [[-0.7, -0.6, 2.0], [0.6, -0.5, 2.5], [0.0, 0.7, 3.0]]
+    far = [[-0.7, -0.6, 4.0], [0.6, -0.5, 4.0], [0.0, 0.7, 4.0]]
+    v, f = soup([far, tri, tri, tri])
+    dv, df = to_dev(v, f)
+    g = np_(mr.rasterize_fwd(dv, df, [0], [4], H, W, 0.0, 4, persp)[0])
+    o, _, _, _, ex = oracle_mod.rasterize_fwd(v, f, [0], [4], H, W, 0.0, 4, persp)
+    cov = o[0, :, :, 0] >= 0
+    assert cov.sum() > 150
+    assert np.all(o[0][cov] == [1, 2, 3, 0])
+    # every covered pixel is a depth tie (E1) by construction; only pixels whose coverage
+    # rounding decides (E2: a pixel centre within 1e-6 of an edge) are left out
+    ok = (ex & 2) == 0
+    assert ok.mean() > 0.99
+    assert np.array_equal(g[ok], o[ok])
+
 def test_no_faces_at_all():
     v = torch.zeros((0, 3), device="cuda")
     f = torch.zeros((0, 3), dtype=torch.int64, device="cuda")

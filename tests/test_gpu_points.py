@@ -82,6 +82,20 @@ def test_point_rasterizer_edge_cases(oracle_mod):
     assert int((np_(empty[0]) >= 0).sum()) <= 4            # radius 0: only exact centre hits
 
 
+
+def test_point_at_exactly_the_radius_is_kept(oracle_mod):
+    """Dyadic point and radius (two pixel pitches): the squared distance ties r^2 exactly in
+    float32 too, and the threshold is inclusive on both sides."""
+    H = W = 32
+    x0, y0 = -1 + 21 / W, 1 - 21 / H                # pixel (10, 10)
+    r = 4.0 / W
+    pts = np.array([[x0, y0, 1.0]], np.float32)
+    gi = np_(mr.rasterize_points_fwd(cuda(pts), np.array([0]), np.array([1]), H, W, np.float32(r), 1)[0])
+    wi, *_ = oracle_mod.rasterize_points(pts, [0], [1], H, W, r, 1)
+    assert np.array_equal(gi, wi)
+    for i, j in ((10, 12), (10, 8), (12, 10), (8, 10)):
+        assert gi[0, i, j, 0] == 0
+
 def test_point_rasterizer_full_size_sampled(oracle_mod):
     """The benchmark batch (64 clouds, 1.18 M points, 512x512, K=8) in the benchmark's launch,
     checked at sampled pixels against the oracle and everywhere by properties."""
