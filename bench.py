@@ -44,24 +44,12 @@ KERNELS_PER_STAGE = {"silhouette_raster_bwd": 2,   # main kernel + (x, y) -> (x,
 # ----------------------------------------------------------------------------- counting
 def face_boxes(batch):
     """Per (image, face) pixel boxes grown by sqrt(blur) (exact, float64), degenerate faces dropped."""
+    from differentiable_mesh_rasterization_b200.sharding import face_pixel_boxes
     w = batch.workload
-    r = math.sqrt(w.blur_radius)
-    v = batch.verts.astype(np.float64)
     out = []
     for n in range(batch.N):
         f0, nf = int(batch.mesh_to_face_first_idx[n]), int(batch.num_faces_per_mesh[n])
-        tri = v[batch.faces[f0:f0 + nf]]                        # (nf, 3, 3)
-        a, b, c = tri[:, 0], tri[:, 1], tri[:, 2]
-        area2 = (b[:, 0] - a[:, 0]) * (c[:, 1] - a[:, 1]) - (b[:, 1] - a[:, 1]) * (c[:, 0] - a[:, 0])
-        keep = np.abs(area2) > 1e-12
-        xmin, xmax = tri[:, :, 0].min(1) - r, tri[:, :, 0].max(1) + r
-        ymin, ymax = tri[:, :, 1].min(1) - r, tri[:, :, 1].max(1) + r
-        jl = np.maximum(np.ceil((xmin + 1) * w.W / 2 - 0.5), 0)
-        jh = np.minimum(np.floor((xmax + 1) * w.W / 2 - 0.5), w.W - 1)
-        il = np.maximum(np.ceil((1 - ymax) * w.H / 2 - 0.5), 0)
-        ih = np.minimum(np.floor((1 - ymin) * w.H / 2 - 0.5), w.H - 1)
-        ok = keep & (jl <= jh) & (il <= ih)
-        out.append((jl[ok], jh[ok], il[ok], ih[ok]))
+        out.append(face_pixel_boxes(batch.verts, batch.faces[f0:f0 + nf], w.H, w.W, w.blur_radius))
     return out
 
 
