@@ -3,11 +3,11 @@
  *
  * The operation is the two-stage differentiable mesh rasterizer of PyTorch3D
  * ("Accelerating 3D Deep Learning with PyTorch3D"): stage one keeps, for every pixel,
- * the K nearest faces (method summary: "two-stage rasterization with per-pixel K
- * nearest faces"); stage two blends their influence into a soft silhouette; the
- * backward pass carries pixel gradients back to the vertex positions (tutorial
- * summary, 3:52: "backpropagation of gradients from 2D image pixels back to 3D model
- * parameters").  The batch is heterogeneous and packed (tutorial summary, 1:00).
+ * the K nearest faces (method summary: the rasterizer is split in two stages, the first
+ * choosing K faces per pixel); stage two blends their influence into a soft silhouette;
+ * the backward pass carries pixel gradients back to the vertex positions (tutorial
+ * summary, 3:52: gradients flow from the image back to the mesh).  The batch is
+ * heterogeneous and packed (tutorial summary, 1:00).
  *
  * Conventions shared by every entry point
  * ---------------------------------------

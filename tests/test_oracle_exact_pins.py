@@ -7,8 +7,9 @@ point-segment distance by the perpendicular cross product), and compare.  They a
 the soft silhouette of an axis-aligned square and its gradient against torch float64
 autograd, and the perspective depth of a face whose depth varies along x only.
 
-Source: "Differentiable rendering" pages (PyTorch3D rasterizer: barycentric coordinates,
-signed squared distance, blur radius, perspective_correct; SoftRas silhouette).
+Source: "Accelerating 3D Deep Learning with PyTorch3D" (method: the per-pixel K nearest
+faces with barycentric coordinates, signed squared distance, blur radius and the
+perspective_correct switch; the soft silhouette of the second stage).
 """
 from fractions import Fraction as Fr
 import math
