@@ -107,6 +107,19 @@ def test_exact_depth_ties_go_to_the_lower_face_id(oracle_mod, persp):
     assert ok.mean() > 0.99
     assert np.array_equal(g[ok], o[ok])
 
+
+@pytest.mark.parametrize("H,W", [(1, 3000), (3000, 1), (7, 4099)])
+def test_extreme_aspect_ratios(oracle_mod, H, W):
+    """Single-row and single-column images and a ragged wide one: one bin row or column,
+    partial warp tiles along the short side, non-power-of-two centres (float-pair path)."""
+    b = syn.make_batch(2, n_meshes=2)
+    g, o = run_both(oracle_mod, b.verts, b.faces, b.mesh_to_face_first_idx, b.num_faces_per_mesh, H, W,
+                    2e-3, 4, False, sigma=1e-4)
+    info = compare_forward(g[:4], o, f"{H}x{W}")
+    assert info["valid_slots"] > 100
+    ao = oracle_mod.silhouette_fwd(o[0], o[3], np.float32(1e-4))
+    compare_alpha(g[4], ao, mask=o[4] == 0, label=f"{H}x{W} alpha")
+
 def test_no_faces_at_all():
     v = torch.zeros((0, 3), device="cuda")
     f = torch.zeros((0, 3), dtype=torch.int64, device="cuda")
