@@ -52,9 +52,12 @@ def test_phong_hand_values(oracle_mod):
 
 
 def test_phong_flags_grazing_light(oracle_mod):
-    prm = params(oracle_mod, [1.0, 0.0, 1e-8], [0.0, 0.0, 3.0])
-    _, flag = one(oracle_mod, [0, 0, 0], [0, 0, 1], ALB, prm)
-    assert flag
+    """The flag marks |cos| < 1e-6 only: the light at height h over a unit distance gives
+    cos = h / sqrt(1 + h^2), flagged below h = 1e-6 and not above it."""
+    for h, want in ((1e-8, True), (-5e-7, True), (5e-6, False), (1e-4, False), (-1e-3, False)):
+        prm = params(oracle_mod, [1.0, 0.0, h], [0.0, 0.0, 3.0])
+        _, flag = one(oracle_mod, [0, 0, 0], [0, 0, 1], ALB, prm)
+        assert flag == want, h
 
 
 def test_phong_invariances(oracle_mod):

@@ -437,6 +437,11 @@ def test_exempt_flags(oracle_mod):
     _, _, _, _, ex = oracle_mod.rasterize_fwd(*mesh([tri]), H, W, (1 * s) ** 2, 1)
     assert ex[0, 1, 3] & 2          # one pixel above edge (a, b)
     assert not ex[0, 4, 3]
+    # hard rasterization (blur 0): a pixel centre on an edge has min w = 0 exactly, so its
+    # coverage is rounding's; one a pixel inside is not
+    _, _, _, _, ex = oracle_mod.rasterize_fwd(*mesh([tri]), H, W, 0.0, 1)
+    assert ex[0, 2, 4] & 2 and ex[0, 4, 2] & 2 and ex[0, 4, 4] & 2      # edges ab, ca, bc
+    assert not ex[0, 3, 3] and not ex[0, 0, 0]
 
 
 def test_rejects_bad_arguments(oracle_mod):
