@@ -49,8 +49,8 @@ def mesh_sample_counts(verts, faces, first, num, H: int, W: int, blur_radius: fl
 def partition_meshes(costs, world: int) -> list[np.ndarray]:
     """Split mesh indices 0..N-1 over `world` ranks, balancing the summed cost: meshes in
     decreasing cost (ties: lower index first) each go to the rank with the least cost so
-    far (ties: lower rank) -- the longest-processing-time rule, within 4/3 of the best
-    makespan.  Deterministic, so every rank computes the same split without exchanging
+    far (ties: fewer meshes, then lower rank, so zero-cost meshes spread too) -- the
+    longest-processing-time rule, within 4/3 of the best makespan.  Deterministic, so every rank computes the same split without exchanging
     anything.  Returns per rank its mesh indices in increasing order."""
     if world < 1:
         raise ValueError("world must be >= 1")
@@ -59,7 +59,7 @@ def partition_meshes(costs, world: int) -> list[np.ndarray]:
     load = [0.0] * world
     parts: list[list[int]] = [[] for _ in range(world)]
     for n in order:
-        r = min(range(world), key=lambda q: (load[q], q))
+        r = min(range(world), key=lambda q: (load[q], len(parts[q]), q))
         parts[r].append(n)
         load[r] += costs[n]
     return [np.array(sorted(p), np.int64) for p in parts]

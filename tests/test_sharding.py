@@ -50,6 +50,7 @@ def test_partition_edge_cases():
     assert [p.tolist() for p in sharding.partition_meshes([], 3)] == [[], [], []]
     assert [p.tolist() for p in sharding.partition_meshes([5.0, 5.0], 4)] == [[0], [1], [], []]
     assert [p.tolist() for p in sharding.partition_meshes([1.0, 7.0, 3.0], 1)] == [[0, 1, 2]]
+    assert [p.tolist() for p in sharding.partition_meshes([0.0] * 5, 2)] == [[0, 2, 4], [1, 3]]
     with pytest.raises(ValueError):
         sharding.partition_meshes([1.0], 0)
 
