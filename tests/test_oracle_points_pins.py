@@ -191,6 +191,27 @@ def test_knn_matches_kdtree_on_heterogeneous_clouds(oracle_mod):
         assert np.array_equal(idx[a][ok], (j + b0)[ok])
 
 
+
+@pytest.mark.parametrize("D", [1, 2, 4])
+def test_knn_matches_kdtree_in_other_dimensions(oracle_mod, D):
+    rng = np.random.default_rng(40 + D)
+    num1, num2 = np.array([37, 0, 64]), np.array([50, 9, 130])
+    first1 = np.concatenate([[0], np.cumsum(num1)[:-1]])
+    first2 = np.concatenate([[0], np.cumsum(num2)[:-1]])
+    p1 = rng.normal(size=(num1.sum(), D)).astype(np.float32)
+    p2 = rng.normal(size=(num2.sum(), D)).astype(np.float32)
+    K = 6
+    idx, dists, flags = oracle_mod.knn(p1, first1, num1, p2, first2, num2, K)
+    for n in range(3):
+        a = slice(first1[n], first1[n] + num1[n])
+        if num1[n] == 0:
+            continue
+        tree = cKDTree(p2[first2[n]:first2[n] + num2[n]].astype(np.float64))
+        d, j = tree.query(p1[a].astype(np.float64), k=K)
+        assert np.allclose(dists[a], d ** 2, rtol=1e-12, atol=1e-15)
+        ok = ~flags[a]
+        assert np.array_equal(idx[a][ok], (j + first2[n])[ok])
+
 def test_knn_hand_solved_and_padding(oracle_mod):
     ref = np.array([[0, 0, 0], [1, 0, 0], [3, 0, 0], [6, 0, 0], [10, 0, 0]], np.float32)
     q = np.array([[2.2, 0, 0], [6, 0, 0], [0, 0, 0]], np.float32)
