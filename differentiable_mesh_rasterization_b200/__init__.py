@@ -114,39 +114,65 @@ def _dev(t: torch.Tensor, dtype, name: str) -> torch.Tensor:
     return t.contiguous()
 
 
-def _host_i64(a, name: str) -> np.ndarray:
-    if isinstance(a, torch.Tensor):
-        a = a.detach().cpu().numpy()
-    a = np.ascontiguousarray(a, dtype=np.int64)
-    if a.ndim != 1:
-        raise ValueError(f"{name} must be 1-D")
-    return a
+class _Index:
+    """A per-mesh (per-cloud) index array as the C ABI takes it: a 1-D int64 array in host
+    memory (numpy, a list or a CPU tensor) or a CUDA tensor on the call's device, passed
+    through as a device pointer (the library then reads it with one device-to-host copy on
+    the call's stream)."""
+
+    def __init__(self, a, name: str, device: torch.device):
+        if isinstance(a, torch.Tensor) and a.is_cuda:
+            if a.device != device:
+                raise ValueError(f"{name} is on {a.device}, the call runs on {device}")
+            a = a.detach().to(torch.int64).contiguous()
+            self.ptr = a.data_ptr()
+        else:
+            if isinstance(a, torch.Tensor):
+                a = a.detach().numpy()
+            a = np.ascontiguousarray(a, dtype=np.int64)
+            self.ptr = a.ctypes.data
+        if a.ndim != 1:
+            raise ValueError(f"{name} must be 1-D")
+        self.keep = a
+        self.n = int(a.shape[0])
+
+
+def _mesh_inputs(verts, faces, mesh_to_face_first_idx, num_faces_per_mesh):
+    """Checked arguments of the mesh forward: verts (V, 3) float32 and faces (F, 3) int64 on
+    one CUDA device, two per-mesh index arrays of equal length.  Shapes and lengths are
+    checked first: the library cannot see the extent of a buffer, so a (V, 2) verts or a
+    short per-mesh array would make it read past the end of one."""
+    for t, name in ((verts, "verts"), (faces, "faces")):
+        if not isinstance(t, torch.Tensor) or t.ndim != 2 or t.shape[1] != 3:
+            raise ValueError(f"{name} must be a tensor of shape (n, 3)")
+    first = _Index(mesh_to_face_first_idx, "mesh_to_face_first_idx", verts.device)
+    num = _Index(num_faces_per_mesh, "num_faces_per_mesh", verts.device)
+    if first.n != num.n:
+        raise ValueError("per-mesh arrays differ in length")
+    verts = _dev(verts, torch.float32, "verts")
+    faces = _dev(faces, torch.int64, "faces")
+    if faces.device != verts.device:
+        raise ValueError("verts and faces must be on the same device")
+    return verts, faces, first, num
 
 
 def rasterize_fwd(verts, faces, mesh_to_face_first_idx, num_faces_per_mesh, H, W, blur_radius, K,
                   perspective_correct=False, sigma=None):
     """Stage one (``mr_rasterize_fwd``); with ``sigma`` also the fused silhouette.
 
-    verts (V, 3) float32 CUDA, faces (F, 3) int64 CUDA; the two per-mesh index arrays live
-    on the host (numpy or CPU tensors).  Returns ``pix_to_face (N,H,W,K) int64, zbuf,
+    verts (V, 3) float32 CUDA, faces (F, 3) int64 CUDA; the two per-mesh index arrays in
+    host memory or as CUDA tensors.  Returns ``pix_to_face (N,H,W,K) int64, zbuf,
     bary (N,H,W,K,3), dists`` and, when ``sigma`` is given, ``alpha (N,H,W)``.
     """
     lib = load_library()
-    verts = _dev(verts, torch.float32, "verts")
-    faces = _dev(faces, torch.int64, "faces")
-    if verts.ndim != 2 or verts.shape[1] != 3 or faces.ndim != 2 or faces.shape[1] != 3:
-        raise ValueError("verts and faces must be (V, 3) and (F, 3)")
-    first = _host_i64(mesh_to_face_first_idx, "mesh_to_face_first_idx")
-    num = _host_i64(num_faces_per_mesh, "num_faces_per_mesh")
-    if first.shape != num.shape:
-        raise ValueError("per-mesh arrays differ in length")
-    N = first.shape[0]
+    verts, faces, first, num = _mesh_inputs(verts, faces, mesh_to_face_first_idx, num_faces_per_mesh)
+    N = first.n
     dev = verts.device
     p2f = torch.empty((N, H, W, K), dtype=torch.int64, device=dev)
     zbuf = torch.empty((N, H, W, K), dtype=torch.float32, device=dev)
     bary = torch.empty((N, H, W, K, 3), dtype=torch.float32, device=dev)
     dists = torch.empty((N, H, W, K), dtype=torch.float32, device=dev)
-    args = (_ptr(verts), verts.shape[0], _ptr(faces), faces.shape[0], first.ctypes.data, num.ctypes.data,
+    args = (_ptr(verts), verts.shape[0], _ptr(faces), faces.shape[0], first.ptr, num.ptr,
             N, H, W, float(blur_radius), K, int(bool(perspective_correct)))
     with torch.cuda.device(dev):
         if sigma is None:
@@ -167,11 +193,8 @@ def rasterize_fwd_noalloc(verts, faces, mesh_to_face_first_idx, num_faces_per_me
     torch).  Same outputs as :func:`rasterize_fwd`; batches too large for the array raise.
     """
     lib = load_library()
-    verts = _dev(verts, torch.float32, "verts")
-    faces = _dev(faces, torch.int64, "faces")
-    first = _host_i64(mesh_to_face_first_idx, "mesh_to_face_first_idx")
-    num = _host_i64(num_faces_per_mesh, "num_faces_per_mesh")
-    N = first.shape[0]
+    verts, faces, first, num = _mesh_inputs(verts, faces, mesh_to_face_first_idx, num_faces_per_mesh)
+    N = first.n
     dev = verts.device
     p2f = torch.empty((N, H, W, K), dtype=torch.int64, device=dev)
     zbuf = torch.empty((N, H, W, K), dtype=torch.float32, device=dev)
@@ -180,7 +203,7 @@ def rasterize_fwd_noalloc(verts, faces, mesh_to_face_first_idx, num_faces_per_me
     with torch.cuda.device(dev):
         _check("mr_rasterize_fwd_noalloc",
                lib.mr_rasterize_fwd_noalloc(_ptr(verts), verts.shape[0], _ptr(faces), faces.shape[0],
-                                            first.ctypes.data, num.ctypes.data, N, H, W, float(blur_radius), K,
+                                            first.ptr, num.ptr, N, H, W, float(blur_radius), K,
                                             int(bool(perspective_correct)), _ptr(p2f), _ptr(zbuf), _ptr(bary),
                                             _ptr(dists), _stream(dev)))
     return p2f, zbuf, bary, dists
@@ -396,18 +419,18 @@ def rasterize_points_fwd(points, cloud_first_idx, num_points_per_cloud, H, W, ra
     """K nearest points per pixel (``mr_rasterize_points_fwd``) -> (idx, zbuf, dists), each (N, H, W, K)."""
     lib = load_library()
     pts = _dev(points, torch.float32, "points")
-    first = _host_i64(cloud_first_idx, "cloud_first_idx")
-    num = _host_i64(num_points_per_cloud, "num_points_per_cloud")
-    if pts.ndim != 2 or pts.shape[1] != 3 or first.shape != num.shape:
+    first = _Index(cloud_first_idx, "cloud_first_idx", pts.device)
+    num = _Index(num_points_per_cloud, "num_points_per_cloud", pts.device)
+    if pts.ndim != 2 or pts.shape[1] != 3 or first.n != num.n:
         raise ValueError("points must be (P, 3); cloud_first_idx and num_points_per_cloud of equal length")
-    N = first.shape[0]
+    N = first.n
     dev = pts.device
     idx = torch.empty((N, H, W, K), dtype=torch.int64, device=dev)
     zbuf = torch.empty((N, H, W, K), dtype=torch.float32, device=dev)
     dists = torch.empty((N, H, W, K), dtype=torch.float32, device=dev)
     with torch.cuda.device(dev):
         _check("mr_rasterize_points_fwd",
-               lib.mr_rasterize_points_fwd(_ptr(pts), pts.shape[0], first.ctypes.data, num.ctypes.data, N, H, W,
+               lib.mr_rasterize_points_fwd(_ptr(pts), pts.shape[0], first.ptr, num.ptr, N, H, W,
                                            float(radius), K, _ptr(idx), _ptr(zbuf), _ptr(dists), _stream(dev)))
     return idx, zbuf, dists
 
@@ -470,15 +493,15 @@ def knn_fwd(p1, first1, num1, p2, first2, num2, K):
     lib = load_library()
     a = _dev(p1, torch.float32, "p1")
     b = _dev(p2, torch.float32, "p2")
-    f1, n1, f2, n2 = (_host_i64(x, nm) for x, nm in ((first1, "first1"), (num1, "num1"), (first2, "first2"),
-                                                     (num2, "num2")))
-    if a.ndim != 2 or b.ndim != 2 or a.shape[1] != b.shape[1] or not (f1.shape == n1.shape == f2.shape == n2.shape):
+    f1, n1, f2, n2 = (_Index(x, nm, a.device) for x, nm in ((first1, "first1"), (num1, "num1"), (first2, "first2"),
+                                                            (num2, "num2")))
+    if a.ndim != 2 or b.ndim != 2 or a.shape[1] != b.shape[1] or not (f1.n == n1.n == f2.n == n2.n):
         raise ValueError("p1 (P1, D), p2 (P2, D) and four cloud arrays of equal length expected")
     idx = torch.empty((a.shape[0], K), dtype=torch.int64, device=a.device)
     dists = torch.empty((a.shape[0], K), dtype=torch.float32, device=a.device)
     with torch.cuda.device(a.device):
-        _check("mr_knn_fwd", lib.mr_knn_fwd(_ptr(a), a.shape[0], f1.ctypes.data, n1.ctypes.data, _ptr(b), b.shape[0],
-                                            f2.ctypes.data, n2.ctypes.data, f1.shape[0], a.shape[1], K, _ptr(idx),
+        _check("mr_knn_fwd", lib.mr_knn_fwd(_ptr(a), a.shape[0], f1.ptr, n1.ptr, _ptr(b), b.shape[0],
+                                            f2.ptr, n2.ptr, f1.n, a.shape[1], K, _ptr(idx),
                                             _ptr(dists), _stream(a.device)))
     return idx, dists
 

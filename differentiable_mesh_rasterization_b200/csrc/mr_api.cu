@@ -73,6 +73,29 @@ void scratch_free(void* p, cudaStream_t s) {
     if (p) cudaFreeAsync(p, s);
 }
 
+int host_indices(cudaStream_t s, int64_t n, std::vector<int64_t>& buf,
+                 std::initializer_list<const int64_t**> arrays) {
+    if (n <= 0) return MR_OK;
+    std::vector<const int64_t**> on_device;
+    for (const int64_t** a : arrays) {
+        if (!*a) continue;
+        cudaPointerAttributes at;
+        if (cudaPointerGetAttributes(&at, *a) != cudaSuccess) {
+            cudaGetLastError();          // a pointer CUDA does not know: plain host memory
+            continue;
+        }
+        if (at.type == cudaMemoryTypeDevice) on_device.push_back(a);
+    }
+    if (on_device.empty()) return MR_OK;
+    buf.resize((size_t)n * on_device.size());
+    for (size_t i = 0; i < on_device.size(); ++i)
+        MR_CUDA(cudaMemcpyAsync(buf.data() + i * n, *on_device[i], sizeof(int64_t) * (size_t)n,
+                                cudaMemcpyDeviceToHost, s));
+    MR_CUDA(cudaStreamSynchronize(s));
+    for (size_t i = 0; i < on_device.size(); ++i) *on_device[i] = buf.data() + i * n;
+    return MR_OK;
+}
+
 bool profiling_enabled() { return g_prof_on; }
 
 cudaEvent_t profile_event() {

@@ -5,7 +5,9 @@
 #include <stdint.h>
 
 #include <cstdio>
+#include <initializer_list>
 #include <string>
+#include <vector>
 
 #include "meshrast.h"
 
@@ -79,6 +81,13 @@ int cuda_fail(cudaError_t e, const char* what);
         cudaError_t e_ = (call);                             \
         if (e_ != cudaSuccess) return ::mr::cuda_fail(e_, #call); \
     } while (0)
+
+// Per-mesh (per-cloud) index arrays may be given in host or in device memory.  Each
+// pointer in `arrays` that is device memory is replaced by a host copy of its n entries
+// held in `buf` (one device-to-host copy per array on stream s, then one synchronisation
+// of s); host-readable pointers are left as they are.
+int host_indices(cudaStream_t s, int64_t n, std::vector<int64_t>& buf,
+                 std::initializer_list<const int64_t**> arrays);
 
 // Scratch allocation on the caller's stream (stream-ordered pool).
 int scratch_alloc(void** p, size_t bytes, cudaStream_t s);

@@ -29,6 +29,11 @@ int rasterize_impl(const float* verts, int64_t V, const int64_t* faces, int64_t 
                    const int64_t* num, int32_t N, int32_t H, int32_t W, float blur, int32_t K, int32_t persp,
                    float sigma, bool sil, int64_t* p2f, float* zbuf, float* bary, float* dists, float* alpha,
                    cudaStream_t s) {
+    std::vector<int64_t> staged;
+    if (N > 0) {
+        int rs = host_indices(s, N, staged, {&first, &num});
+        if (rs != MR_OK) return rs;
+    }
     int rc = validate_fwd(verts, V, faces, F, first, num, N, H, W, blur, K, p2f, zbuf, bary, dists);
     if (rc != MR_OK) return rc;
     if (sil && (!(sigma > 0.f) || !std::isfinite(sigma) || (N > 0 && !alpha))) {

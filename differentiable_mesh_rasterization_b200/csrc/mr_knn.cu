@@ -482,10 +482,13 @@ int mr_knn_fwd(const float* p1, int64_t P1, const int64_t* first1, const int64_t
         set_error("null pointer");
         return MR_ERR_ARG;
     }
-    int rc = check_sets(first1, num1, N, P1, "mr_knn_fwd queries");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::vector<int64_t> staged;
+    int rc = host_indices(s, N, staged, {&first1, &num1, &first2, &num2});
+    if (rc != MR_OK) return rc;
+    rc = check_sets(first1, num1, N, P1, "mr_knn_fwd queries");
     if (rc == MR_OK) rc = check_sets(first2, num2, N, P2, "mr_knn_fwd references");
     if (rc != MR_OK) return rc;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     // query clouds must be disjoint; rows outside every cloud are filled with -1
     std::vector<std::pair<int64_t, int64_t>> ranges;
     for (int n = 0; n < N; ++n)

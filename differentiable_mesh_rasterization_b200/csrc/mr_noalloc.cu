@@ -13,7 +13,10 @@
 // The array is MR_NOALLOC_SCRATCH_BYTES (64 MiB) on every device that loads this part
 // of the library and stays there until the process exits.  Its address is looked up
 // once per device, by the first call made on that device with the device current; make
-// that first call before any stream capture.  All calls share the array and it keeps
+// that first call before any stream capture.  Like mr_rasterize_fwd, every call
+// synchronises its stream once, after the bin count, to learn the size of the bin lists
+// (and once before, when the per-mesh arrays are device memory).  All calls share the
+// array and it keeps
 // the previous call's contents (the parts that must start at zero are cleared on every
 // call), so two calls whose work overlaps on the GPU -- on different streams, or from
 // different threads -- race on it; order them on one stream.
@@ -55,6 +58,11 @@ namespace {
 int rasterize_noalloc(const float* verts, int64_t V, const int64_t* faces, int64_t F, const int64_t* first,
                       const int64_t* num, int32_t N, int32_t H, int32_t W, float blur, int32_t K, int32_t persp,
                       int64_t* p2f, float* zbuf, float* bary, float* dists, cudaStream_t s) {
+    std::vector<int64_t> staged;
+    if (N > 0) {
+        int rs = host_indices(s, N, staged, {&first, &num});
+        if (rs != MR_OK) return rs;
+    }
     int rc = validate_fwd(verts, V, faces, F, first, num, N, H, W, blur, K, p2f, zbuf, bary, dists);
     if (rc != MR_OK) return rc;
     if (N == 0) return MR_OK;

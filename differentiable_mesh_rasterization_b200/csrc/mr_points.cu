@@ -424,9 +424,12 @@ int mr_rasterize_points_fwd(const float* points, int64_t P, const int64_t* cloud
         set_error("null pointer");
         return MR_ERR_ARG;
     }
-    int rc = check_clouds(cloud_first_idx, num_points_per_cloud, N, P, "mr_rasterize_points_fwd");
-    if (rc != MR_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::vector<int64_t> staged;
+    int rc = host_indices(s, N, staged, {&cloud_first_idx, &num_points_per_cloud});
+    if (rc != MR_OK) return rc;
+    rc = check_clouds(cloud_first_idx, num_points_per_cloud, N, P, "mr_rasterize_points_fwd");
+    if (rc != MR_OK) return rc;
     const int nbx = (W + kPtBin - 1) / kPtBin, nby = (H + kPtBin - 1) / kPtBin;
     const int64_t nbins64 = (int64_t)N * nbx * nby;
     if (nbins64 >= INT32_MAX / 2) {

@@ -24,7 +24,11 @@
  *    candidate for a pixel iff the pixel centre is inside the closed triangle or
  *    within squared distance blur_radius of it.  Candidates are ordered by (z, face id);
  *    degenerate faces (|2 * area| <= 1e-12) and candidates with z < 0 are dropped.
- *  - Pointers are DEVICE pointers unless marked HOST.  The caller owns every input and
+ *  - Pointers are DEVICE pointers unless marked otherwise.  Per-mesh (per-cloud) index
+ *    arrays are HOST OR DEVICE: the library asks CUDA which one a pointer is and reads a
+ *    device array with one device-to-host copy on `stream`, followed by a
+ *    synchronisation of `stream` (so such an array must be ready in stream order).  The
+ *    caller owns every input and
  *    output; the library allocates its own scratch (stream-ordered, from the device's
  *    default memory pool, released before the call returns) and never frees caller
  *    memory.  stream is a cudaStream_t (NULL = legacy default stream).
@@ -61,8 +65,8 @@ extern "C" {
  *
  *   verts                    V x 3 float32 (device)
  *   faces                    F x 3 int64 (device), every id in [0, V)
- *   mesh_to_face_first_idx   N int64 (HOST)
- *   num_faces_per_mesh       N int64 (HOST); first + num <= F for every mesh
+ *   mesh_to_face_first_idx   N int64 (host or device)
+ *   num_faces_per_mesh       N int64 (host or device); first + num <= F for every mesh
  *   H, W                     1 .. MR_MAX_SIDE
  *   blur_radius              >= 0, finite (squared NDC units)
  *   K                        1 .. MR_KMAX
@@ -73,8 +77,9 @@ extern "C" {
  *   zbuf, dists              N x H x W x K float32 (device, written)
  *   bary                     N x H x W x K x 3 float32 (device, written)
  *
- * Synchronises `stream` once (to size the per-bin face lists).  Returns MR_ERR_DEVICE
- * if a face referenced a vertex outside [0, V) (that face is then ignored).
+ * Synchronises `stream` once to size the per-bin face lists (and once more, before any
+ * launch, when the per-mesh arrays are device memory).  Returns MR_ERR_DEVICE if a face
+ * referenced a vertex outside [0, V) (that face is then ignored).
  */
 int mr_rasterize_fwd(const float* verts, int64_t V, const int64_t* faces, int64_t F,
                      const int64_t* mesh_to_face_first_idx, const int64_t* num_faces_per_mesh,
@@ -95,7 +100,8 @@ int mr_rasterize_fwd(const float* verts, int64_t V, const int64_t* faces, int64_
  *  - Batches whose scratch exceeds the array (face records, per-pixel top-K ids, per-bin
  *    counts and lists) are rejected with MR_ERR_ARG and a message naming the size.
  *  - The first call on a device looks up the array's device address, with that device
- *    current; make that first call before any stream capture.
+ *    current; make that first call before any stream capture.  Every call synchronises
+ *    `stream` once, after the bin count, as mr_rasterize_fwd does.
  *  - All calls share the array and it keeps the last call's contents (what must start
  *    at zero is cleared on every call).  Calls whose work overlaps on the GPU race on
  *    it: issue them in order on one stream.
@@ -250,7 +256,7 @@ int mr_phong_shade_bwd(const int64_t* pix_to_face, const float* bary, int64_t np
  * clouds with the same two stages, over heterogeneous batches; the pages print no formula,
  * so these are the plain definitions that match the mesh path).  points: P x 3 float32
  * (device), screen space (x_ndc, y_ndc, z) like the mesh vertices; cloud n is points
- * [cloud_first_idx[n], + num_points_per_cloud[n]) (HOST arrays of N, ascending, disjoint)
+ * [cloud_first_idx[n], + num_points_per_cloud[n]) (arrays of N in host or device memory, ascending, disjoint)
  * and is drawn into image n.  Pixel centres as for meshes.
  *
  * mr_rasterize_points_fwd: per pixel the K points of its cloud nearest in depth among those
@@ -287,8 +293,8 @@ int mr_composite_points_bwd(const int64_t* idx, const float* dists, int64_t npix
 /*
  * Batched K nearest neighbours (PyTorch3D paper: a custom KNN kernel for heterogeneous
  * batches of point clouds).  p1: P1 x D queries, p2: P2 x D references (float32, device);
- * cloud n of p1 (first1[n], num1[n]; HOST) searches cloud n of p2 (first2[n], num2[n];
- * HOST).  mr_knn_fwd: idx (P1 x K int64: global ids into p2) and dists (P1 x K float32:
+ * cloud n of p1 (first1[n], num1[n]) searches cloud n of p2 (first2[n], num2[n]); all four
+ * in host or device memory.  mr_knn_fwd: idx (P1 x K int64: global ids into p2) and dists (P1 x K float32:
  * squared Euclidean distances), the K nearest ordered by (distance, id); when cloud n of
  * p2 has fewer than K points the rest hold -1 in both; queries in no cloud get -1 rows.
  * 1 <= D <= MR_KNN_DMAX, 1 <= K <= MR_KMAX, P1, P2 < 2^31; MR_ERR_ARG for overlapping query

@@ -45,26 +45,51 @@ def test_version_and_error_string(lib):
     assert isinstance(lib.mr_last_error(), bytes)
 
 
-def _fwd(lib, **kw):
+FORWARDS = ["mr_rasterize_fwd", "mr_rasterize_fwd_noalloc"]
+
+
+def _fwd(lib, entry="mr_rasterize_fwd", **kw):
     a = dict(verts=None, V=3, faces=None, F=1, first=np.array([0], np.int64), num=np.array([1], np.int64),
              N=1, H=8, W=8, blur=0.0, K=1, persp=0)
     a.update(kw)
     dummy = ctypes.c_void_p(16)   # never dereferenced: validation fails first
-    return lib.mr_rasterize_fwd(dummy, a["V"], dummy, a["F"], a["first"].ctypes.data, a["num"].ctypes.data,
-                                a["N"], a["H"], a["W"], a["blur"], a["K"], a["persp"], dummy, dummy, dummy, dummy,
-                                None)
+    return getattr(lib, entry)(dummy, a["V"], dummy, a["F"], a["first"].ctypes.data, a["num"].ctypes.data,
+                               a["N"], a["H"], a["W"], a["blur"], a["K"], a["persp"], dummy, dummy, dummy, dummy,
+                               None)
 
 
+@pytest.mark.parametrize("entry", FORWARDS)
 @pytest.mark.parametrize("kw,msg", [
     (dict(K=0), "K=0"), (dict(K=33), "K=33"), (dict(H=0), "H=0"), (dict(W=40000), "W=40000"),
     (dict(blur=-1.0), "blur_radius"), (dict(blur=float("nan")), "blur_radius"),
     (dict(num=np.array([2], np.int64)), "outside"), (dict(first=np.array([-1], np.int64)), "outside"),
     (dict(F=-1), "F=-1"), (dict(N=-1), "N=-1"),
 ])
-def test_forward_rejects_bad_arguments(lib, kw, msg):
-    rc = _fwd(lib, **kw)
+def test_forward_rejects_bad_arguments(lib, entry, kw, msg):
+    """Both forwards reject bad arguments before any CUDA call (the scratch-free one before
+    it looks up its fixed array)."""
+    rc = _fwd(lib, entry, **kw)
     assert rc == -1
     assert msg in lib.mr_last_error().decode()
+
+
+@pytest.mark.parametrize("entry", FORWARDS)
+def test_forward_with_no_images_is_a_no_op(lib, entry):
+    assert _fwd(lib, entry, N=0, first=np.zeros(0, np.int64), num=np.zeros(0, np.int64)) == 0
+
+
+@pytest.mark.parametrize("fn", ["rasterize_fwd", "rasterize_fwd_noalloc"])
+def test_binding_checks_shapes_before_the_library_sees_them(fn):
+    """A (V, 2) verts, an (F, 2) faces or per-mesh arrays of unequal length would make the
+    kernels or the host plan read past a buffer's end; the binding refuses them."""
+    import torch
+    import differentiable_mesh_rasterization_b200 as mr
+    call = getattr(mr, fn)
+    v3, f3 = torch.zeros(3, 3), torch.zeros(1, 3, dtype=torch.int64)
+    for v, f, first, num in ((torch.zeros(3, 2), f3, [0], [1]), (v3, torch.zeros(1, 2, dtype=torch.int64), [0], [1]),
+                             (v3, f3, [0, 1], [1]), (v3, f3, [[0]], [[1]])):
+        with pytest.raises(ValueError):
+            call(v, f, first, num, 8, 8, 0.0, 1)
 
 
 def test_other_entry_points_reject_bad_arguments(lib):

@@ -6,7 +6,7 @@ import torch
 import differentiable_mesh_rasterization_b200 as mr
 from differentiable_mesh_rasterization_b200 import synthetic as syn
 
-from _parity import compare_alpha, compare_grad, np_
+from _parity import Scene, compare_alpha, compare_forward, compare_grad, np_
 
 pytestmark = pytest.mark.gpu
 
@@ -91,17 +91,10 @@ def test_general_backward_all_outputs(oracle_mod, persp):
     mr.device_status()
 
 
-def _touched_vertices(b, *p2fs):
-    """Vertices of faces sitting in any slot of the given exempt-pixel slot arrays."""
-    fs = np.unique(np.concatenate([p[p >= 0] for p in p2fs]))
-    m = np.zeros(b.verts.shape[0], bool)
-    if fs.size:
-        m[b.faces[fs].reshape(-1)] = True
-    return m
-
-
 def test_end_to_end_batch2(oracle_mod):
-    """verts -> alpha -> grad_verts on both sides from the same seeded inputs."""
+    """verts -> alpha -> grad_verts on both sides from the same seeded inputs. The oracle's
+    backward runs on its own fragments reconciled to the GPU's choice of faces at flagged
+    pixels (the GPU's ids with the oracle's float64 values), so every vertex is compared."""
     b = syn.make_batch(2)
     w = b.workload
     sigma = np.float32(w.sigma)
@@ -110,44 +103,43 @@ def test_end_to_end_batch2(oracle_mod):
     p2f, zb, ba, dists, alpha = mr.rasterize_fwd(v, f, b.mesh_to_face_first_idx, b.num_faces_per_mesh, w.H, w.W,
                                                  w.blur_radius, w.K, sigma=float(sigma))
     got = mr.silhouette_rasterize_bwd(v, f, p2f, dists, float(sigma), cuda(ga))
-    o = oracle_mod.rasterize_fwd(b.verts, b.faces, b.mesh_to_face_first_idx, b.num_faces_per_mesh, w.H, w.W,
-                                 np.float32(w.blur_radius), w.K, False)
-    want = _oracle_chain(oracle_mod, b, o[0], o[3], ga, sigma)
-    ex = o[4] > 0
-    keep = ~_touched_vertices(b, o[0][ex], np_(p2f)[ex])
-    assert keep.mean() > 0.75
-    compare_grad(got, want, mask=keep, label="end-to-end batch2")
-    compare_alpha(alpha, oracle_mod.silhouette_fwd(o[0], o[3], sigma), mask=~ex, label="alpha batch2")
+    sc = Scene(oracle_mod, b.verts, b.faces, b.mesh_to_face_first_idx, b.num_faces_per_mesh, w.H, w.W,
+               w.blur_radius, w.K, False)
+    info = compare_forward((p2f, zb, ba, dists), sc.fwd(), "batch2", scene=sc)
+    rp2f, rd = info["rec"][0], info["rec"][3]
+    want = _oracle_chain(oracle_mod, b, rp2f, rd, ga, sigma)
+    rel = compare_grad(got, want, label="end-to-end batch2")
+    assert rel < 1e-4
+    compare_alpha(alpha, oracle_mod.silhouette_fwd(rp2f, rd, sigma), label="alpha batch2")
 
 
 def test_end_to_end_full_batch5_whole_images(oracle_mod):
-    """The 64-image 512x512 batch on the GPU; the oracle redoes three whole images."""
+    """The 64-image 512x512 batch on the GPU; the oracle redoes three whole images (their
+    meshes own disjoint vertex ranges, so those vertices' gradients are complete)."""
     b = syn.make_batch(5)
     w = b.workload
     sigma = np.float32(w.sigma)
     ga = syn.grad_alpha(b)
     v, f = cuda(b.verts), cuda(b.faces)
-    p2f, _, _, dists, alpha = mr.rasterize_fwd(v, f, b.mesh_to_face_first_idx, b.num_faces_per_mesh, w.H, w.W,
-                                               w.blur_radius, w.K, sigma=float(sigma))
+    p2f, zb, ba, dists, alpha = mr.rasterize_fwd(v, f, b.mesh_to_face_first_idx, b.num_faces_per_mesh, w.H, w.W,
+                                                 w.blur_radius, w.K, sigma=float(sigma))
     got = np_(mr.silhouette_rasterize_bwd(v, f, p2f, dists, float(sigma), cuda(ga)))
     imgs = np.argsort(b.num_faces_per_mesh)[:3]
     pix = np.concatenate([np.arange(n * w.H * w.W, (n + 1) * w.H * w.W) for n in imgs])
-    o = oracle_mod.rasterize_fwd(b.verts, b.faces, b.mesh_to_face_first_idx, b.num_faces_per_mesh, w.H, w.W,
-                                 np.float32(w.blur_radius), w.K, False, pixels=pix)
+    sc = Scene(oracle_mod, b.verts, b.faces, b.mesh_to_face_first_idx, b.num_faces_per_mesh, w.H, w.W,
+               w.blur_radius, w.K, False, pix)
+    sel = lambda x: np_(x).reshape((-1,) + tuple(x.shape[3:]))[pix]
+    info = compare_forward(tuple(sel(x) for x in (p2f, zb, ba, dists)), sc.fwd(), "batch5 images", scene=sc)
     P2F = np.full((b.N, w.H, w.W, w.K), -1, np.int64)
     D = np.full((b.N, w.H, w.W, w.K), -1.0)
-    P2F.reshape(-1, w.K)[pix] = o[0]
-    D.reshape(-1, w.K)[pix] = o[3]
+    P2F.reshape(-1, w.K)[pix] = info["rec"][0]
+    D.reshape(-1, w.K)[pix] = info["rec"][3]
     want = _oracle_chain(oracle_mod, b, P2F, D, ga, sigma)
-    exm = o[4] > 0
-    gp = np_(p2f).reshape(-1, w.K)[pix]
-    keep = ~_touched_vertices(b, o[0][exm], gp[exm])
     for n in imgs:
         v0, nv = b.mesh_to_vert_first_idx[n], b.num_verts_per_mesh[n]
-        sel = np.zeros(b.verts.shape[0], bool)
-        sel[v0:v0 + nv] = True
-        compare_grad(got, want, mask=sel & keep, label=f"batch5 image {n}")
-    compare_alpha(np_(alpha).reshape(-1)[pix], oracle_mod.silhouette_fwd(o[0], o[3], sigma), mask=~exm,
+        rel = compare_grad(got[v0:v0 + nv], want[v0:v0 + nv], label=f"batch5 image {n}")
+        assert rel < 1e-4
+    compare_alpha(np_(alpha).reshape(-1)[pix], oracle_mod.silhouette_fwd(info["rec"][0], info["rec"][3], sigma),
                   label="batch5 alpha")
 
 

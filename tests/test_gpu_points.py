@@ -285,3 +285,22 @@ def test_point_rasterizer_many_slots_and_dense_bins(oracle_mod):
                                                     r, K)
     assert (wi[..., -1] >= 0).mean() > 0.05              # some pixels fill all 32 slots
     _compare_slots(got, (wi, wz, wd), flags[..., None].repeat(K, -1), "K=32 dense")
+
+
+def test_device_resident_cloud_arrays_match_host_ones():
+    """Per-cloud index arrays given as CUDA tensors: the point rasterizer and KNN read them
+    with one device-to-host copy and give identical outputs."""
+    pb = syn.make_point_batch(2)
+    w = pb.workload
+    dev = lambda a: torch.as_tensor(np.asarray(a, np.int64)).cuda()
+    P = cuda(pb.points)
+    want = mr.rasterize_points_fwd(P, pb.cloud_first_idx, pb.num_points_per_cloud, w.H, w.W, w.radius, w.K)
+    got = mr.rasterize_points_fwd(P, dev(pb.cloud_first_idx), dev(pb.num_points_per_cloud), w.H, w.W, w.radius, w.K)
+    for x, y in zip(got, want):
+        assert torch.equal(x, y)
+    kb = syn.make_knn_batch(2)
+    a, b = cuda(kb.p1), cuda(kb.p2)
+    want = mr.knn_fwd(a, kb.first1, kb.num1, b, kb.first2, kb.num2, 8)
+    got = mr.knn_fwd(a, dev(kb.first1), kb.num1, b, dev(kb.first2), dev(kb.num2), 8)
+    for x, y in zip(got, want):
+        assert torch.equal(x, y)

@@ -194,6 +194,9 @@ def test_knn_matches_kdtree_on_heterogeneous_clouds(oracle_mod):
 
 @pytest.mark.parametrize("D", [1, 2, 4])
 def test_knn_matches_kdtree_in_other_dimensions(oracle_mod, D):
+    """Heterogeneous clouds (one query cloud empty) against scipy's KD-tree.  The tie flag is
+    pinned too: a query is flagged exactly when two of its K+1 nearest KD-tree distances
+    (squared) lie within 1e-6 of each other, relative to the larger."""
     rng = np.random.default_rng(40 + D)
     num1, num2 = np.array([37, 0, 64]), np.array([50, 9, 130])
     first1 = np.concatenate([[0], np.cumsum(num1)[:-1]])
@@ -207,10 +210,15 @@ def test_knn_matches_kdtree_in_other_dimensions(oracle_mod, D):
         if num1[n] == 0:
             continue
         tree = cKDTree(p2[first2[n]:first2[n] + num2[n]].astype(np.float64))
-        d, j = tree.query(p1[a].astype(np.float64), k=K)
-        assert np.allclose(dists[a], d ** 2, rtol=1e-12, atol=1e-15)
+        d, j = tree.query(p1[a].astype(np.float64), k=K + 1)
+        d2 = d ** 2
+        assert np.allclose(dists[a], d2[:, :K], rtol=1e-12, atol=1e-15)
+        # (a cloud smaller than K + 1 pads the KD-tree's answer with inf: no tie there)
+        tied = (np.isfinite(d2[:, 1:]) & ((d2[:, 1:] - d2[:, :-1]) <= 1e-6 * d2[:, 1:])).any(1)
+        assert np.array_equal(flags[a].astype(bool), tied)
         ok = ~flags[a]
-        assert np.array_equal(idx[a][ok], (j + first2[n])[ok])
+        assert np.array_equal(idx[a][ok], (j[:, :K] + first2[n])[ok])
+
 
 def test_knn_hand_solved_and_padding(oracle_mod):
     ref = np.array([[0, 0, 0], [1, 0, 0], [3, 0, 0], [6, 0, 0], [10, 0, 0]], np.float32)

@@ -68,3 +68,32 @@ def test_noalloc_rejects_batches_beyond_its_scratch():
     with pytest.raises(mr.MeshRastError) as e:
         mr.rasterize_fwd_noalloc(v, f, b.mesh_to_face_first_idx, b.num_faces_per_mesh, 1024, 1024, 1e-5, 16, True)
     assert e.value.code == -1 and "scratch" in str(e.value)
+
+
+
+def test_noalloc_rejects_bin_lists_beyond_its_scratch_and_recovers():
+    """The second limit: the fixed part of the scratch fits (one 2048x2048 image, K=1), but
+    the per-bin face lists found by the count pass do not (a blur radius of 1.4 in NDC puts
+    each of the 1280 faces into all 16384 bins).  The call has already run kernels on the
+    shared array when it refuses; the next call must still match mr_rasterize_fwd."""
+    verts, faces = syn.icosphere(3)
+    v = torch.from_numpy(syn.project(verts * 0.5).astype(np.float32)).cuda()
+    f = torch.from_numpy(faces.astype(np.int64)).cuda()
+    with pytest.raises(mr.MeshRastError) as e:
+        mr.rasterize_fwd_noalloc(v, f, [0], [faces.shape[0]], 2048, 2048, 2.0, 1, False)
+    assert e.value.code == -1 and "bin lists" in str(e.value)
+    args = _inputs(2, None)
+    want = mr.rasterize_fwd(*args)
+    got = mr.rasterize_fwd_noalloc(*args)
+    torch.cuda.synchronize()
+    _same(got, want, "after the refused call")
+
+
+def test_noalloc_takes_device_resident_mesh_arrays():
+    v, f, first, num, H, W, blur, K, persp = _inputs(2, None)
+    want = mr.rasterize_fwd(v, f, first, num, H, W, blur, K, persp)
+    got = mr.rasterize_fwd_noalloc(v, f, torch.as_tensor(first).cuda(), torch.as_tensor(num).cuda(), H, W, blur, K,
+                                   persp)
+    torch.cuda.synchronize()
+    _same(got, want, "device-resident per-mesh arrays")
+
