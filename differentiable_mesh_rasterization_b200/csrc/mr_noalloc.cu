@@ -16,10 +16,9 @@
 // that first call before any stream capture.  Like mr_rasterize_fwd, every call
 // synchronises its stream once, after the bin count, to learn the size of the bin lists
 // (and once before, when the per-mesh arrays are device memory).  All calls share the
-// array and it keeps
-// the previous call's contents (the parts that must start at zero are cleared on every
-// call), so two calls whose work overlaps on the GPU -- on different streams, or from
-// different threads -- race on it; order them on one stream.
+// array and it keeps the previous call's contents (the parts that must start at zero are
+// cleared on every call), so two calls whose work overlaps on the GPU -- on different
+// streams, or from different threads -- race on it; order them on one stream.
 #include <mutex>
 
 #include "mr_forward_kernels.cuh"
