@@ -29,7 +29,7 @@ EXPORTS = ("mr_rasterize_fwd", "mr_rasterize_silhouette_fwd", "mr_silhouette_ble
            "mr_rasterize_fwd_noalloc", "mr_interpolate_fwd", "mr_interpolate_bwd", "mr_blend_fwd", "mr_blend_bwd",
            "mr_phong_fwd", "mr_phong_bwd", "mr_phong_shade_fwd", "mr_phong_shade_bwd",
            "mr_rasterize_points_fwd", "mr_rasterize_points_bwd", "mr_composite_points_fwd",
-           "mr_composite_points_bwd", "mr_knn_fwd", "mr_knn_bwd", "mr_measure_fp32_peak")
+           "mr_composite_points_bwd", "mr_knn_fwd", "mr_knn_bwd", "mr_measure_fp32_peak", "mr_knn_count_pairs")
 STAGES = ("face_setup", "bin_count", "bin_scan", "bin_fill", "fine", "silhouette_fwd", "silhouette_bwd",
           "raster_bwd", "silhouette_raster_bwd", "epilogue", "interpolate_fwd", "interpolate_bwd", "blend_fwd",
           "blend_bwd", "phong_fwd", "phong_bwd", "phong_shade_fwd", "phong_shade_bwd",
@@ -80,6 +80,7 @@ def load_library() -> ctypes.CDLL:
         "mr_composite_points_bwd": [P, P, i64, i32, P, i64, i32, f32, i32, P, P, P, P],
         "mr_knn_fwd": [P, i64, P, P, P, i64, P, P, i32, i32, i32, P, P, P],
         "mr_knn_bwd": [P, i64, P, i64, i32, i32, P, P, P, P, P],
+        "mr_knn_count_pairs": [P, i64, P, P, P, i64, P, P, i32, i32, i32, P, P, P, P],
         "mr_measure_fp32_peak": [P, P],
         "mr_profile_enable": [i32],
         "mr_profile_read": [P, P, i32],
@@ -504,6 +505,26 @@ def knn_fwd(p1, first1, num1, p2, first2, num2, K):
                                             f2.ptr, n2.ptr, f1.n, a.shape[1], K, _ptr(idx),
                                             _ptr(dists), _stream(a.device)))
     return idx, dists
+
+
+def knn_count_pairs(p1, first1, num1, p2, first2, num2, K):
+    """The (query, reference) pairs the KNN search evaluates (``mr_knn_count_pairs``): the
+    search's real work, for its roofline.  Returns (pairs, idx, dists)."""
+    lib = load_library()
+    a = _dev(p1, torch.float32, "p1")
+    b = _dev(p2, torch.float32, "p2")
+    f1, n1, f2, n2 = (_Index(x, nm, a.device) for x, nm in ((first1, "first1"), (num1, "num1"), (first2, "first2"),
+                                                            (num2, "num2")))
+    if a.ndim != 2 or b.ndim != 2 or a.shape[1] != b.shape[1] or not (f1.n == n1.n == f2.n == n2.n):
+        raise ValueError("p1 (P1, D), p2 (P2, D) and four cloud arrays of equal length expected")
+    idx = torch.empty((a.shape[0], K), dtype=torch.int64, device=a.device)
+    dists = torch.empty((a.shape[0], K), dtype=torch.float32, device=a.device)
+    out = np.zeros(1, np.int64)
+    with torch.cuda.device(a.device):
+        _check("mr_knn_count_pairs",
+               lib.mr_knn_count_pairs(_ptr(a), a.shape[0], f1.ptr, n1.ptr, _ptr(b), b.shape[0], f2.ptr, n2.ptr, f1.n,
+                                      a.shape[1], K, _ptr(idx), _ptr(dists), out.ctypes.data, _stream(a.device)))
+    return int(out[0]), idx, dists
 
 
 def knn_bwd(p1, p2, idx, grad_dists):

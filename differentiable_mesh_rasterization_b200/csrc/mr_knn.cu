@@ -249,7 +249,9 @@ __device__ __forceinline__ float box_bound(const float (&q)[4], float4 lo4, floa
 // shared memory (32 points, one array per coordinate, and ids) and every lane tests it
 // four distances at a time, two by two with packed two-lane float32 instructions (each
 // lane rounds as the scalar instruction would, so the distances are the scalar ones).
-template <int KC, int D>
+// COUNT adds, per warp, the (live query, reference) pairs whose distance it evaluates to
+// *work (one atomic per warp at the end): the search's real work, for measurement.
+template <int KC, int D, bool COUNT>
 __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ sq, const int* __restrict__ sqid,
                                                      const short* __restrict__ sqcode, const float4* __restrict__ sr,
                                                      const int* __restrict__ srid, const int* __restrict__ roff,
@@ -258,7 +260,8 @@ __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ 
                                                      const float4* __restrict__ glo, const float4* __restrict__ ghi,
                                                      const float4* __restrict__ slo, const float4* __restrict__ shi,
                                                      const KnnTile* __restrict__ tiles, int K,
-                                                     int64_t* __restrict__ idx, float* __restrict__ dists) {
+                                                     int64_t* __restrict__ idx, float* __restrict__ dists,
+                                                     unsigned long long* __restrict__ work) {
     __shared__ __align__(16) float wc[kKnnQueries / 32][4][32];
     __shared__ __align__(16) int wid[kKnnQueries / 32][32];
     const KnnTile T = tiles[blockIdx.x];
@@ -288,6 +291,8 @@ __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ 
         home = min(max(h, (int64_t)0), rn - 1) >> 10;           // super-box of the first query's cell
     }
     int64_t up = home + 1, down = home - 1, cur = home;
+    unsigned long long evaluated = 0;
+    const unsigned live_lanes = COUNT ? (unsigned)__popc(__ballot_sync(0xffffffffu, live)) : 0u;
     for (int64_t it = 0; it < nsup; ++it) {
         if (__all_sync(0xffffffffu, !live || box_bound<D>(q, slo[s0 + cur], shi[s0 + cur]) > key_dist(kk[KC - 1]))) {
             // skipped
@@ -298,6 +303,7 @@ __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ 
                     continue;
                 const int64_t pb = g * 32;
                 const int cnt = (int)min((int64_t)32, rn - pb);
+                if (COUNT) evaluated += (unsigned long long)cnt * live_lanes;
                 __syncwarp();
                 if (lane < cnt) {
                     const float4 r = sr[r0 + pb + lane];
@@ -338,6 +344,7 @@ __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ 
         else if (down >= 0) cur = down--;
         else cur = up++;
     }
+    if (COUNT && lane == 0) atomicAdd(work, evaluated);
     if (!live) return;
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
@@ -407,7 +414,8 @@ cudaError_t run_knn(int N, int K, const float* p1, const float* p2, const int64_
                     const int64_t* d_spre, int64_t S1, int64_t S2, int64_t G, int64_t NS, CloudBox* box, int* counts1,
                     int* counts2, int* off1, int* off2, long long* tile1, long long* tile2, float4* sq, int* sqid,
                     short* sqcode, float4* sr, int* srid, short* srcode, float4* glo, float4* ghi, float4* slo,
-                    float4* shi, const KnnTile* tiles, int ntiles, int64_t* idx, float* dists, cudaStream_t s) {
+                    float4* shi, const KnnTile* tiles, int ntiles, int64_t* idx, float* dists,
+                    unsigned long long* work, cudaStream_t s) {
     const int nb = N * kCells, nt = (nb + kScanTile - 1) / kScanTile;
     cudaError_t e;
     k_cloud_box<D><<<N, 256, 0, s>>>(p2, d_first2, d_num2, box);
@@ -440,15 +448,21 @@ cudaError_t run_knn(int N, int K, const float* p1, const float* p2, const int64_
                                                                                      G, slo, shi);
     }
     if ((e = cudaGetLastError())) return e;
-#define MR_KNN(KC)                                                                                                 \
-    k_knn<KC, D><<<ntiles, kKnnQueries, 0, s>>>(sq, sqid, sqcode, sr, srid, off2, d_pre2, d_num2, d_gpre, d_spre, glo, \
-                                                ghi, slo, shi, tiles, K, idx, dists)
-    if (K <= 1) MR_KNN(1);
-    else if (K <= 2) MR_KNN(2);
-    else if (K <= 4) MR_KNN(4);
-    else if (K <= 8) MR_KNN(8);
-    else if (K <= 16) MR_KNN(16);
-    else MR_KNN(32);
+#define MR_KNN(KC)                                                                                            \
+    if (work)                                                                                                 \
+        k_knn<KC, D, true><<<ntiles, kKnnQueries, 0, s>>>(sq, sqid, sqcode, sr, srid, off2, d_pre2, d_num2,   \
+                                                          d_gpre, d_spre, glo, ghi, slo, shi, tiles, K, idx, \
+                                                          dists, work);                                       \
+    else                                                                                                      \
+        k_knn<KC, D, false><<<ntiles, kKnnQueries, 0, s>>>(sq, sqid, sqcode, sr, srid, off2, d_pre2, d_num2,  \
+                                                           d_gpre, d_spre, glo, ghi, slo, shi, tiles, K, idx, \
+                                                           dists, nullptr)
+    if (K <= 1) { MR_KNN(1); }
+    else if (K <= 2) { MR_KNN(2); }
+    else if (K <= 4) { MR_KNN(4); }
+    else if (K <= 8) { MR_KNN(8); }
+    else if (K <= 16) { MR_KNN(16); }
+    else { MR_KNN(32); }
 #undef MR_KNN
     return cudaGetLastError();
 }
@@ -463,15 +477,12 @@ int check_sets(const int64_t* first, const int64_t* num, int N, int64_t P, const
     return MR_OK;
 }
 
-}  // namespace
-}  // namespace mr
-
-extern "C" {
-
-int mr_knn_fwd(const float* p1, int64_t P1, const int64_t* first1, const int64_t* num1, const float* p2, int64_t P2,
-               const int64_t* first2, const int64_t* num2, int32_t N, int32_t D, int32_t K, int64_t* idx,
-               float* dists, void* stream) {
-    using namespace mr;
+// The whole search; with `evaluated` (host) also the number of (query, reference) pairs
+// whose distance the search evaluated (one more stream synchronisation).
+int knn_impl(const float* p1, int64_t P1, const int64_t* first1, const int64_t* num1, const float* p2, int64_t P2,
+             const int64_t* first2, const int64_t* num2, int32_t N, int32_t D, int32_t K, int64_t* idx, float* dists,
+             int64_t* evaluated, void* stream) {
+    if (evaluated) *evaluated = 0;
     if (N < 0 || D < 1 || D > MR_KNN_DMAX || K < 1 || K > MR_KMAX || P1 < 0 || P2 < 0 || P1 > INT32_MAX ||
         P2 > INT32_MAX) {
         set_error("invalid arguments N=%d D=%d K=%d P1=%lld P2=%lld", N, D, K, (long long)P1, (long long)P2);
@@ -549,14 +560,14 @@ int mr_knn_fwd(const float* p1, int64_t P1, const int64_t* first1, const int64_t
     // ordered sets, the tiles
     const int nb = N * kCells, nt = (nb + kScanTile - 1) / kScanTile;
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    size_t sz[12] = {sizeof(int64_t) * host.size(), sizeof(CloudBox) * (size_t)N, sizeof(int) * (size_t)nb,
+    size_t sz[13] = {sizeof(int64_t) * host.size(), sizeof(CloudBox) * (size_t)N, sizeof(int) * (size_t)nb,
                      sizeof(int) * (size_t)nb, sizeof(int) * ((size_t)nb + 1), sizeof(int) * ((size_t)nb + 1),
                      sizeof(long long) * ((size_t)nt + 1), sizeof(long long) * ((size_t)nt + 1),
                      (sizeof(float4) + sizeof(int) + sizeof(short)) * (size_t)S1,
                      (sizeof(float4) + sizeof(int) + sizeof(short)) * (size_t)S2, sizeof(KnnTile) * tiles.size(),
-                     sizeof(float4) * 2 * (size_t)(G + NS)};
-    size_t total = 0, at[12];
-    for (int i = 0; i < 12; ++i) {
+                     sizeof(float4) * 2 * (size_t)(G + NS), sizeof(unsigned long long)};
+    size_t total = 0, at[13];
+    for (int i = 0; i < 13; ++i) {
         at[i] = total;
         total += up(sz[i]);
     }
@@ -582,8 +593,10 @@ int mr_knn_fwd(const float* p1, int64_t P1, const int64_t* first1, const int64_t
     float4* ghi = glo + G;
     float4* slo = ghi + G;
     float4* shi = slo + NS;
+    unsigned long long* work = evaluated ? reinterpret_cast<unsigned long long*>(base + at[12]) : nullptr;
     cudaError_t e = cudaMemcpyAsync(plan, host.data(), sz[0], cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess) e = cudaMemcpyAsync(dt, tiles.data(), sz[10], cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && work) e = cudaMemsetAsync(work, 0, sizeof(unsigned long long), s);
     if (e == cudaSuccess) {
         ProfScope ps(MR_STAGE_KNN, s);
         const int ntl = (int)tiles.size();
@@ -591,7 +604,7 @@ int mr_knn_fwd(const float* p1, int64_t P1, const int64_t* first1, const int64_t
         const int64_t *gp = plan + 5 * N, *sp = plan + 6 * N;
 #define MR_RUN(DD)                                                                                                   \
     run_knn<DD>(N, K, p1, p2, f1, f2, pr1, pr2, n2, gp, sp, S1, S2, G, NS, box, counts1, counts2, off1, off2, tile1, \
-                tile2, sq, sqid, sqcode, sr, srid, srcode, glo, ghi, slo, shi, dt, ntl, idx, dists, s)
+                tile2, sq, sqid, sqcode, sr, srid, srcode, glo, ghi, slo, shi, dt, ntl, idx, dists, work, s)
         switch (D) {
             case 1: e = MR_RUN(1); break;
             case 2: e = MR_RUN(2); break;
@@ -600,10 +613,37 @@ int mr_knn_fwd(const float* p1, int64_t P1, const int64_t* first1, const int64_t
         }
 #undef MR_RUN
     }
+    unsigned long long count = 0;
+    if (e == cudaSuccess && work) {
+        e = cudaMemcpyAsync(&count, work, sizeof(count), cudaMemcpyDeviceToHost, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    }
     // (copies from pageable host memory return once the data is staged: the vectors may go)
     scratch_free(base, s);
     if (e != cudaSuccess) return cuda_fail(e, "knn");
+    if (evaluated) *evaluated = (int64_t)count;
     return MR_OK;
+}
+
+}  // namespace
+}  // namespace mr
+
+extern "C" {
+
+int mr_knn_fwd(const float* p1, int64_t P1, const int64_t* first1, const int64_t* num1, const float* p2, int64_t P2,
+               const int64_t* first2, const int64_t* num2, int32_t N, int32_t D, int32_t K, int64_t* idx,
+               float* dists, void* stream) {
+    return mr::knn_impl(p1, P1, first1, num1, p2, P2, first2, num2, N, D, K, idx, dists, nullptr, stream);
+}
+
+int mr_knn_count_pairs(const float* p1, int64_t P1, const int64_t* first1, const int64_t* num1, const float* p2,
+                       int64_t P2, const int64_t* first2, const int64_t* num2, int32_t N, int32_t D, int32_t K,
+                       int64_t* idx, float* dists, int64_t* evaluated_pairs, void* stream) {
+    if (!evaluated_pairs) {
+        mr::set_error("null evaluated_pairs");
+        return MR_ERR_ARG;
+    }
+    return mr::knn_impl(p1, P1, first1, num1, p2, P2, first2, num2, N, D, K, idx, dists, evaluated_pairs, stream);
 }
 
 int mr_knn_bwd(const float* p1, int64_t P1, const float* p2, int64_t P2, int32_t D, int32_t K, const int64_t* idx,

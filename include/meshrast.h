@@ -311,6 +311,20 @@ int mr_knn_fwd(const float* p1, int64_t P1, const int64_t* first1, const int64_t
 int mr_knn_bwd(const float* p1, int64_t P1, const float* p2, int64_t P2, int32_t D, int32_t K,
                const int64_t* idx, const float* grad_dists, float* grad_p1, float* grad_p2, void* stream);
 
+/*
+ * Work count of the KNN search (measurement support; no counterpart on the pages): runs
+ * mr_knn_fwd's search (same arguments, same outputs) in a counting build of its kernel and
+ * writes to *evaluated_pairs (HOST) the number of (query, reference) pairs whose distance
+ * the search evaluated -- the pairs of every group staged for a warp times its live
+ * queries; the groups bounded away by their boxes are not counted.  This is the work the
+ * KNN roofline divides by; the search is exact, so the count is at most sum_n num1 * num2
+ * and usually far below it.  Synchronises `stream`.
+ */
+int mr_knn_count_pairs(const float* p1, int64_t P1, const int64_t* first1, const int64_t* num1,
+                       const float* p2, int64_t P2, const int64_t* first2, const int64_t* num2,
+                       int32_t N, int32_t D, int32_t K, int64_t* idx, float* dists,
+                       int64_t* evaluated_pairs, void* stream);
+
 /* Synchronises `stream`, then returns MR_ERR_DEVICE (and clears the word) if any
  * asynchronous kernel of this library flagged an out-of-range index on the current
  * device since the last call, else MR_OK (or MR_ERR_CUDA). */

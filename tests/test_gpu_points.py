@@ -304,3 +304,27 @@ def test_device_resident_cloud_arrays_match_host_ones():
     got = mr.knn_fwd(a, dev(kb.first1), kb.num1, b, dev(kb.first2), dev(kb.num2), 8)
     for x, y in zip(got, want):
         assert torch.equal(x, y)
+
+
+def test_knn_pair_count_is_the_work_of_the_search():
+    """mr_knn_count_pairs returns the same neighbours as mr_knn_fwd and the pairs the search
+    evaluated: exactly num1 x num2 when every cloud holds at most 32 references (one group,
+    nothing to prune: the first group is always staged), and below the exhaustive count on
+    the full-size batch, where whole groups are bounded away."""
+    rng = np.random.default_rng(70)
+    num1, num2 = np.array([50, 7, 0, 33]), np.array([20, 32, 5, 1])
+    f1 = np.concatenate([[0], np.cumsum(num1)[:-1]])
+    f2 = np.concatenate([[0], np.cumsum(num2)[:-1]])
+    a = cuda(rng.normal(size=(num1.sum(), 3)).astype(np.float32))
+    b = cuda(rng.normal(size=(num2.sum(), 3)).astype(np.float32))
+    count, ci, cd = mr.knn_count_pairs(a, f1, num1, b, f2, num2, 4)
+    gi, gd = mr.knn_fwd(a, f1, num1, b, f2, num2, 4)
+    assert torch.equal(ci, gi) and torch.equal(cd, gd)
+    assert count == int(np.sum(num1 * num2))
+    kb = syn.make_knn_batch(5, n_clouds=8)
+    A, B = cuda(kb.p1), cuda(kb.p2)
+    count, ci, cd = mr.knn_count_pairs(A, kb.first1, kb.num1, B, kb.first2, kb.num2, 8)
+    gi, gd = mr.knn_fwd(A, kb.first1, kb.num1, B, kb.first2, kb.num2, 8)
+    assert torch.equal(ci, gi) and torch.equal(cd, gd)
+    exhaustive = int(np.sum(kb.num1.astype(np.int64) * kb.num2))
+    assert int(kb.p1.shape[0]) * 8 <= count < exhaustive
