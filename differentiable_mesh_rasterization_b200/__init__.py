@@ -29,7 +29,8 @@ EXPORTS = ("mr_rasterize_fwd", "mr_rasterize_silhouette_fwd", "mr_silhouette_ble
            "mr_rasterize_fwd_noalloc", "mr_interpolate_fwd", "mr_interpolate_bwd", "mr_blend_fwd", "mr_blend_bwd",
            "mr_phong_fwd", "mr_phong_bwd", "mr_phong_shade_fwd", "mr_phong_shade_bwd",
            "mr_rasterize_points_fwd", "mr_rasterize_points_bwd", "mr_composite_points_fwd",
-           "mr_composite_points_bwd", "mr_knn_fwd", "mr_knn_bwd", "mr_measure_fp32_peak", "mr_knn_count_pairs")
+           "mr_composite_points_bwd", "mr_knn_fwd", "mr_knn_bwd", "mr_measure_fp32_peak", "mr_knn_count_pairs",
+           "mr_inject_fault", "mr_scratch_in_use")
 STAGES = ("face_setup", "bin_count", "bin_scan", "bin_fill", "fine", "silhouette_fwd", "silhouette_bwd",
           "raster_bwd", "silhouette_raster_bwd", "epilogue", "interpolate_fwd", "interpolate_bwd", "blend_fwd",
           "blend_bwd", "phong_fwd", "phong_bwd", "phong_shade_fwd", "phong_shade_bwd",
@@ -82,6 +83,8 @@ def load_library() -> ctypes.CDLL:
         "mr_knn_bwd": [P, i64, P, i64, i32, i32, P, P, P, P, P],
         "mr_knn_count_pairs": [P, i64, P, P, P, i64, P, P, i32, i32, i32, P, P, P, P],
         "mr_measure_fp32_peak": [P, P],
+        "mr_inject_fault": [i32, i32],
+        "mr_scratch_in_use": [P],
         "mr_profile_enable": [i32],
         "mr_profile_read": [P, P, i32],
     }
@@ -579,6 +582,24 @@ def blend_bwd(pix_to_face, colors, dists, zbuf, background, sigma, gamma, znear,
                                                 bg.ctypes.data, float(sigma), float(gamma), float(znear), float(zfar),
                                                 _ptr(g), _ptr(gc), _ptr(gd), _ptr(gz), _stream(p2f.device)))
     return gc, gd, gz
+
+
+INJECT = {"off": 0, "oom": 1, "cuda": 2}
+
+
+def inject_fault(kind: str = "off", skip: int = 0) -> None:
+    """Arm (``"oom"``, ``"cuda"``) or disarm (``"off"``) a one-shot failure of the library's
+    scratch allocator after ``skip`` successful allocations (``mr_inject_fault``)."""
+    _check("mr_inject_fault", load_library().mr_inject_fault(INJECT[kind], int(skip)))
+
+
+def scratch_in_use(device=None) -> int:
+    """Bytes allocated from the device's default memory pool (``mr_scratch_in_use``)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    out = ctypes.c_int64(0)
+    with torch.cuda.device(dev):
+        _check("mr_scratch_in_use", load_library().mr_scratch_in_use(ctypes.byref(out)))
+    return int(out.value)
 
 
 def measure_fp32_peak(device=None) -> float:

@@ -337,10 +337,33 @@ const char* mr_last_error(void);
 int mr_version(void);
 
 /*
- * FP32 issue-rate probe (measurement support; no counterpart on the pages): times one
- * launch of a kernel of independent FFMA chains filling every SM (8 chains per thread,
- * 148 x 8 CTAs of 256 threads on B200) with CUDA events on `stream` and writes the achieved
- * FP32 instructions per second to *inst_per_s (HOST).  Synchronises `stream`.  The roofline
+ * Host-side fault injection, for testing callers' and the library's error paths (no
+ * counterpart on the pages).  kind = MR_INJECT_OOM or MR_INJECT_CUDA arms a one-shot
+ * failure of the library's scratch allocator: the first `skip` allocations after this call
+ * succeed, the next one returns MR_ERR_OOM or MR_ERR_CUDA (the message says "injected")
+ * without allocating, and the hook disarms itself.  The entry point that meets it frees any
+ * scratch it already holds and returns that code; nothing fails on the GPU.  MR_INJECT_OFF
+ * disarms.  Process-wide (all threads and devices).  MR_ERR_ARG for another kind or skip < 0.
+ */
+#define MR_INJECT_OFF 0
+#define MR_INJECT_OOM 1
+#define MR_INJECT_CUDA 2
+int mr_inject_fault(int32_t kind, int32_t skip);
+
+/*
+ * Bytes currently allocated from the current device's default memory pool (its
+ * used-memory counter), where the library's scratch comes from; *bytes is HOST.  The
+ * scratch of a call is released in stream order, so read this after synchronising the
+ * call's stream.  For tests of the library's cleanup.
+ */
+int mr_scratch_in_use(int64_t* bytes);
+
+/*
+ * FP32 issue-rate probe (measurement support; no counterpart on the pages): times five
+ * launches (after a warm-up) of a kernel of independent FFMA chains filling every SM
+ * (8 chains per thread, 148 x 8 CTAs of 256 threads on B200, ~11 ms each) with CUDA events
+ * on `stream` and writes the FP32 instructions per second of the fastest launch to
+ * *inst_per_s (HOST).  Synchronises `stream`; takes about 70 ms.  The roofline
  * of the fine pass divides by this measured figure rather than by unit counts x clock.
  */
 int mr_measure_fp32_peak(double* inst_per_s, void* stream);

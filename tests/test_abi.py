@@ -144,3 +144,20 @@ def test_next_row_entry_points_reject_bad_arguments(lib):
     assert lib.mr_knn_fwd(d, 20, first.ctypes.data, num.ctypes.data, d, 20, first.ctypes.data, num.ctypes.data, 2,
                           3, 4, d, d, None) == -1 and "overlap" in err()
     assert lib.mr_knn_bwd(d, 4, d, 4, 0, 2, d, d, d, d, None) == -1
+
+
+@pytest.mark.parametrize("kind,code", [(1, -2), (2, -3)])
+def test_injected_allocation_failure_returns_its_code_and_disarms(lib, kind, code):
+    """The one-shot hook fails the library's first scratch allocation before anything is
+    launched (valid arguments, so the call gets that far); the next call no longer meets it."""
+    assert lib.mr_inject_fault(kind, 0) == 0
+    rc = _fwd(lib)
+    assert rc == code and "injected" in lib.mr_last_error().decode()
+    rc = _fwd(lib)            # disarmed: without a GPU the real allocator path fails differently
+    assert "injected" not in lib.mr_last_error().decode()
+    assert lib.mr_inject_fault(0, 0) == 0
+
+
+def test_fault_injection_rejects_bad_arguments(lib):
+    assert lib.mr_inject_fault(3, 0) == -1 and "kind=3" in lib.mr_last_error().decode()
+    assert lib.mr_inject_fault(1, -1) == -1
