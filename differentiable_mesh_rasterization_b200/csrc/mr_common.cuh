@@ -54,6 +54,17 @@ __device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
     return d;
 }
 
+// Asynchronous 16-byte global -> shared copies (no register round trip); a thread sees
+// its own copies after cp_wait_all, the other lanes' after a following __syncwarp.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_wait_all() {
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+}
+
 // Device error bits.
 constexpr int kErrFaceIndex = 1;    // a face vertex id outside [0, V)
 constexpr int kErrSlotIndex = 2;    // a pix_to_face entry outside [-1, F)

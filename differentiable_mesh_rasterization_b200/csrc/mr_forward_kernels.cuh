@@ -267,7 +267,7 @@ template <int KC, bool PERSP, bool EXACT>
 __global__ void __launch_bounds__(kFineThreads, KC <= 4 ? 6 : 4)
 k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const int* __restrict__ offsets,
        const int* __restrict__ list, int nbx, int nby, int H, int W, int K, float blur, int* __restrict__ topk) {
-    __shared__ float4 s_c[kWarpsPerBin][32][kConstF4];
+    __shared__ __align__(16) float4 s_c[kWarpsPerBin][32][kConstF4];
 
     const int bin = blockIdx.x;
     const int bxi = bin % nbx;
@@ -321,8 +321,9 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
             const int slot = __popc(m & lt_mask);
             const float4* src = fconst + (int64_t)kConstF4 * fid;
 #pragma unroll
-            for (int u = 0; u < kConstF4; ++u) slots[slot][u] = __ldg(src + u);
+            for (int u = 0; u < kConstF4; ++u) cp_async16(&slots[slot][u], src + u);
         }
+        cp_wait_all();
         __syncwarp();
         const int nh = __popc(m);
         for (int qi = 0; qi < nh; ++qi) {
@@ -420,23 +421,35 @@ __device__ __forceinline__ void slot_outputs(const FaceGeom& g, double pxd, doub
 }
 
 // One thread per pixel: the K winners' outputs (and the fused silhouette), written
-// contiguously per pixel with 16-byte stores when K is a multiple of 4.
-template <int KC, bool PERSP, bool SIL>
+// contiguously per pixel; VEC (K == KC, a multiple of 4, 16-byte aligned outputs) with
+// 16-byte loads and stores.  Pixels are taken in 16 x 16 tiles (one tile per 256
+// consecutive work items), so the threads of a block gather the faces of one screen
+// region and the geometry reads hit L1.
+template <int KC, bool PERSP, bool SIL, bool VEC>
 __global__ void __launch_bounds__(256, 4)
-k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int64_t npix, int H, int W, int K,
-           float sigma, bool vec_ok, int64_t* __restrict__ p2f, float* __restrict__ zbuf, float* __restrict__ bary,
-           float* __restrict__ dists, float* __restrict__ alpha) {
-    for (int64_t pix = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; pix < npix;
-         pix += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t rem = pix % ((int64_t)H * W);
-        const int i = (int)(rem / W), j = (int)(rem % W);
+k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int N, int H, int W, int K, float sigma,
+           int64_t* __restrict__ p2f, float* __restrict__ zbuf, float* __restrict__ bary, float* __restrict__ dists,
+           float* __restrict__ alpha) {
+    const int tw = (W + kBin - 1) / kBin, th = (H + kBin - 1) / kBin;
+    const int64_t items = (int64_t)N * th * tw * (kBin * kBin);
+    for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < items;
+         it += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t tile = it / (kBin * kBin);
+        const int r = (int)(it % (kBin * kBin));
+        const int tx = (int)(tile % tw);
+        const int64_t t2 = tile / tw;
+        const int ty = (int)(t2 % th);
+        const int64_t n = t2 / th;
+        const int i = ty * kBin + r / kBin, j = tx * kBin + r % kBin;
+        if (i >= H || j >= W) continue;
+        const int64_t pix = (n * H + i) * W + j;
         const double pxd = -1.0 + (2.0 * j + 1.0) / W;
         const double pyd = 1.0 - (2.0 * i + 1.0) / H;
         const float pxh = (float)pxd, pyh = (float)pyd;
         const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
         float dsil[KC];
         bool vsil[KC];
-        if (vec_ok && (KC % 4) == 0 && K == KC) {
+        if (VEC) {
 #pragma unroll
             for (int k4 = 0; k4 < KC; k4 += 4) {
                 const int4 f4 = *reinterpret_cast<const int4*>(topk + pix * KC + k4);
@@ -502,17 +515,21 @@ void launch_fine(bool persp, bool exact, int nbins, cudaStream_t s, const float4
 }
 
 template <int KC>
-void launch_epilogue(bool persp, bool sil, int64_t npix, cudaStream_t s, const FaceGeom* geom, const int* topk,
-                     int H, int W, int K, float sigma, bool vec_ok, int64_t* p2f, float* zbuf, float* bary,
-                     float* dists, float* alpha) {
-    const int grid = (int)std::min<int64_t>((npix + 255) / 256, 148 * 16);
-#define MR_EPI(P, S) \
-    k_epilogue<KC, P, S><<<grid, 256, 0, s>>>(geom, topk, npix, H, W, K, sigma, vec_ok, p2f, zbuf, bary, dists, alpha)
+void launch_epilogue(bool persp, bool sil, bool vec, int N, int H, int W, cudaStream_t s, const FaceGeom* geom,
+                     const int* topk, int K, float sigma, int64_t* p2f, float* zbuf, float* bary, float* dists,
+                     float* alpha) {
+    const int64_t items = (int64_t)N * ceil_div(H, kBin) * ceil_div(W, kBin) * (kBin * kBin);
+    const int grid = (int)std::min<int64_t>((items + 255) / 256, 148 * 32);
+#define MR_EPI(P, S, V) \
+    k_epilogue<KC, P, S, V><<<grid, 256, 0, s>>>(geom, topk, N, H, W, K, sigma, p2f, zbuf, bary, dists, alpha)
+#define MR_EPI2(P, S) \
+    if (vec) MR_EPI(P, S, true); else MR_EPI(P, S, false)
     if (persp) {
-        if (sil) MR_EPI(true, true); else MR_EPI(true, false);
+        if (sil) { MR_EPI2(true, true); } else { MR_EPI2(true, false); }
     } else {
-        if (sil) MR_EPI(false, true); else MR_EPI(false, false);
+        if (sil) { MR_EPI2(false, true); } else { MR_EPI2(false, false); }
     }
+#undef MR_EPI2
 #undef MR_EPI
 }
 
@@ -529,10 +546,11 @@ void dispatch_fine(int KC, bool persp, bool exact, int nbins, cudaStream_t s, co
     }
 }
 
-void dispatch_epilogue(int KC, bool persp, bool sil, int64_t npix, cudaStream_t s, const FaceGeom* geom,
-                       const int* topk, int H, int W, int K, float sigma, bool vec_ok, int64_t* p2f, float* zbuf,
+void dispatch_epilogue(int KC, bool persp, bool sil, bool vec_ok, int N, int H, int W, cudaStream_t s,
+                       const FaceGeom* geom, const int* topk, int K, float sigma, int64_t* p2f, float* zbuf,
                        float* bary, float* dists, float* alpha) {
-#define MR_E(KCV) launch_epilogue<KCV>(persp, sil, npix, s, geom, topk, H, W, K, sigma, vec_ok, p2f, zbuf, bary, dists, alpha)
+    const bool vec = vec_ok && K == KC && (KC % 4) == 0;
+#define MR_E(KCV) launch_epilogue<KCV>(persp, sil, vec, N, H, W, s, geom, topk, K, sigma, p2f, zbuf, bary, dists, alpha)
     switch (KC) {
         case 1: MR_E(1); break;
         case 2: MR_E(2); break;
@@ -723,7 +741,7 @@ inline cudaError_t fwd_enqueue_rest(const FwdPlan& P, const FwdBufs& B, int* lis
     if ((e = cudaGetLastError())) return e;
     {
         ProfScope ps(MR_STAGE_EPILOGUE, s);
-        dispatch_epilogue(P.KC, P.persp != 0, sil, P.npix, s, B.geom, B.topk, P.H, P.W, P.K, sigma, vec_ok, p2f, zbuf,
+        dispatch_epilogue(P.KC, P.persp != 0, sil, vec_ok, P.N, P.H, P.W, s, B.geom, B.topk, P.K, sigma, p2f, zbuf,
                           bary, dists, alpha);
     }
     return cudaGetLastError();
