@@ -8,7 +8,8 @@ rasterizer backward to the vertex positions, with dL/dalpha ~ N(0, 1).  The defa
 workload is the 64-image 512x512 heterogeneous batch (32 icospheres of levels 3-6 and
 32 tori, K=4, sigma=1e-4).  Under torchrun every rank renders its own batch (seed offset
 by rank: weak scaling; no collective on the data path) and the reported time is the
-maximum over ranks.
+maximum over ranks; with --split the ranks share ONE batch, split by whole meshes balanced
+by their pixel-face samples (strong scaling; still no collective on the data path).
 
 A pixel-face sample is a (pixel, face) pair of the same image whose pixel centre lies in
 the face's 2-D box grown by sqrt(blur_radius): the tests the method must make.  It is
@@ -196,7 +197,8 @@ def workload_config(w, args):
     return {"workload": w.name, "description": w.description, "batch": w.N, "H": w.H, "W": w.W, "K": w.K,
             "blur_radius": w.blur_radius, "sigma": w.sigma, "perspective_correct": w.perspective_correct,
             "passes": "fwd+bwd" if w.backward else "fwd", "l2": "flushed (256 MiB write) between timed steps",
-            "parallelism": f"independent batch per GPU x{args.gpus}"}
+            "parallelism": (f"one batch split by whole meshes over {args.gpus} GPUs" if args.split else
+                            f"independent batch per GPU x{args.gpus}")}
 
 
 # ----------------------------------------------------------------------------- ncu traffic
@@ -283,7 +285,7 @@ def shading_step_timing(mr, torch, dev, stream, batch, verts, faces, first, num,
         _, _, _, gbary = mr.phong_shade_bwd(p2f, bary, faces, P, N, alb, prm, gcol)
         mr.rasterize_bwd(verts, faces, p2f, w.perspective_correct, grad_zbuf=gz, grad_bary=gbary, grad_dists=gd)
 
-    npix = batch.N * w.H * w.W
+    npix = n_img * w.H * w.W
     K = w.K
     # algorithmic bytes of the stage-two kernels (slot = K per pixel; colours D = 3): each
     # per-slot input read once, each output written once; vertex gathers hit L2 and are
@@ -564,6 +566,9 @@ def main():
     ap.add_argument("--no-shading", action="store_true", help="skip the Gouraud, Phong, point-cloud and KNN measurements")
     ap.add_argument("--rows", default="gouraud,phong,points,knn",
                     help="comma-separated next-row measurements after the main step (gouraud, phong, points, knn)")
+    ap.add_argument("--split", action="store_true",
+                    help="under torchrun, split ONE batch over the ranks by whole meshes, balanced by their "
+                         "pixel-face samples (strong scaling), instead of one batch per rank (weak scaling)")
     ap.add_argument("--images", type=int, default=None,
                     help="render only the first N meshes of the batch, clouds of the point and KNN batches "
                          "(small profiling case)")
@@ -587,15 +592,30 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    batch = syn.make_batch(args.config, seed=rank_seed(args.config, rank), n_meshes=args.images)
+    batch = syn.make_batch(args.config, seed=rank_seed(args.config, 0 if args.split else rank),
+                           n_meshes=args.images)
     w = batch.workload
     hard = w.sigma is None            # batch 4: hard rasterization, forward only
-    samples = count_samples(batch)
-    verts = torch.from_numpy(batch.verts).to(dev)
-    faces = torch.from_numpy(batch.faces).to(dev)
     ga_host = syn.grad_alpha(batch)
-    ga = torch.from_numpy(ga_host).to(dev)
+    h_v, h_f = batch.verts, batch.faces
     first, num = batch.mesh_to_face_first_idx, batch.num_faces_per_mesh
+    n_img = batch.N
+    if args.split:
+        # this rank's meshes of the one batch: every rank computes the same split from the
+        # same inputs, so nothing is exchanged
+        from differentiable_mesh_rasterization_b200 import sharding
+        costs = sharding.mesh_sample_counts(h_v, h_f, first, num, w.H, w.W, w.blur_radius)
+        mine = sharding.partition_meshes(costs, world)[rank]
+        sh = sharding.Shard(h_f, first, num, mine)
+        h_v, h_f, first, num = np.ascontiguousarray(h_v[sh.vert_ids]), sh.faces, sh.first, sh.num
+        ga_host = np.ascontiguousarray(ga_host[mine])
+        n_img = len(mine)
+        samples = int(costs[mine].sum())
+    else:
+        samples = count_samples(batch)
+    verts = torch.from_numpy(h_v).to(dev)
+    faces = torch.from_numpy(h_f).to(dev)
+    ga = torch.from_numpy(ga_host).to(dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -637,18 +657,18 @@ def main():
         dist.barrier()
     stages = mr.profile_read()
     dev_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    dev_ms, tot_samples, tot_pix = combine_ranks(dev_ms, float(samples), float(batch.N * w.H * w.W), dev)
+    dev_ms, tot_samples, tot_pix = combine_ranks(dev_ms, float(samples), float(n_img * w.H * w.W), dev)
     sec = dev_ms / 1e3
     value = tot_samples * args.steps / sec
     mpix = tot_pix * args.steps / sec / 1e6
 
     # end to end through the public API: pinned host inputs in, alpha + grad_verts out
-    h_verts = torch.from_numpy(batch.verts).pin_memory()
-    h_faces = torch.from_numpy(batch.faces).pin_memory()
+    h_verts = torch.from_numpy(h_v).pin_memory()
+    h_faces = torch.from_numpy(h_f).pin_memory()
     h_ga = torch.from_numpy(np.zeros(0, np.float32) if hard else ga_host).pin_memory()   # nothing to upload when hard
-    h_res = ([torch.empty((w.N, w.H, w.W, w.K), dtype=torch.float32).pin_memory()] if hard else
-             [torch.empty((w.N, w.H, w.W), dtype=torch.float32).pin_memory(),
-              torch.empty(batch.verts.shape, dtype=torch.float32).pin_memory()])
+    h_res = ([torch.empty((n_img, w.H, w.W, w.K), dtype=torch.float32).pin_memory()] if hard else
+             [torch.empty((n_img, w.H, w.W), dtype=torch.float32).pin_memory(),
+              torch.empty(h_v.shape, dtype=torch.float32).pin_memory()])
 
     def e2e_step():
         dv = h_verts.to(dev, non_blocking=True)
@@ -756,7 +776,7 @@ def main():
     hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
     hbm_note = "of measured" if "hbm_gbs" in peaks else "of fallback"
     achieved_alu = samples * C_TEST / fine_s / 1e12
-    npix = batch.N * w.H * w.W
+    npix = n_img * w.H * w.W
     fine_bytes = npix * 4 * w.K                      # the K winning face ids per pixel
     epi_bytes = npix * (4 * w.K + 28 * w.K + (0 if hard else 4))   # ids in; p2f, zbuf, bary, dists(, alpha) out
     full_batch = args.images is None and args.config == 5
@@ -768,7 +788,7 @@ def main():
             "peak_note": "of measured: FFMA-chain probe (mr_measure_fp32_peak) in this run",
             "peak_nominal": peak_nominal,
             "peak_nominal_note": f"{props.multi_processor_count} SMs x 128 FP32 lanes x {sm_mhz_max:.0f} MHz",
-            "dense_tests_per_step": int(sum(int(n) for n in batch.num_faces_per_mesh)) * w.H * w.W,
+            "dense_tests_per_step": int(sum(int(n) for n in num)) * w.H * w.W,
             "hbm_bytes_per_step": fine_bytes,
             "a3a4": a3a4_roofline(samples, fine_s, epi_s, epi_bytes, peak_alu, hbm_peak, hbm_note),
             "epilogue": {"kernel": "k_epilogue (float64 outputs of the K winners + silhouette)",
@@ -779,7 +799,7 @@ def main():
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dev_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded icospheres and tori)",
+            "scaling": "strong" if args.split else "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded icospheres and tori)",
             "config": workload_config(w, args), "mpix_per_s": mpix,
             "samples_per_step": tot_samples,
             "stages_ms_per_step": {k: v[0] / args.steps for k, v in stages.items() if v[1]},

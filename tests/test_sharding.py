@@ -132,3 +132,16 @@ def test_two_ranks_reproduce_the_whole_batch(oracle_mod):
         assert np.array_equal(P, p2f)
         assert np.array_equal(A, alpha)
         assert np.allclose(G, gv, rtol=1e-10, atol=1e-12 * np.abs(gv).max())
+
+
+@pytest.mark.parametrize("cfg", [2, 5])
+def test_shard_costs_add_up_to_the_benchmark_sample_count(cfg):
+    """The cost model of the split and the benchmark's sample count are written separately;
+    summed over meshes they must agree, so a split run reports the same total work."""
+    sys.path.insert(0, ROOT)
+    import bench
+    b = syn.make_batch(cfg)
+    w = b.workload
+    costs = sharding.mesh_sample_counts(b.verts, b.faces, b.mesh_to_face_first_idx, b.num_faces_per_mesh, w.H, w.W,
+                                        w.blur_radius)
+    assert int(costs.sum()) == bench.count_samples(b)
