@@ -39,7 +39,8 @@ C_TEST = 38                 # FP32 instructions per pixel-face test in this form
 FP32_LANES_PER_SM = 128
 L2_FLUSH_BYTES = 256 << 20
 KERNELS_PER_STAGE = {"silhouette_raster_bwd": 2,   # main kernel + (x, y) -> (x, y, z) copy
-                     "bin_scan": 3}                # tile scans, tile totals, tile prefixes added
+                     "bin_scan": 5}                # tile scans, tile totals, tile prefixes added; the bins'
+                                                   # length histogram and longest-first order
 
 
 # ----------------------------------------------------------------------------- counting

@@ -240,6 +240,57 @@ __global__ void k_bin_pairs(const FaceBox* __restrict__ box, const int64_t* __re
     }
 }
 
+// ------------------------------------------------------------------ launch order of the bins
+// The fine pass's time is set by its longest bin lists when they start late (a crowded
+// bin's warps walk its whole list); the bins are therefore launched longest first: a
+// histogram of the list lengths in 33 classes (0, then 2^(c-1) <= length < 2^c), then each
+// bin written to its class's next place, classes from the longest down.  Order inside a
+// class is free; the outputs do not depend on the order.
+constexpr int kLenClasses = 33;
+
+__device__ __forceinline__ int len_class(int len) { return len > 0 ? 32 - __clz(len) : 0; }
+
+__global__ void k_bin_hist(const int* __restrict__ offsets, int nbins, int* __restrict__ hist) {
+    __shared__ int h[kLenClasses];
+    for (int c = threadIdx.x; c < kLenClasses; c += blockDim.x) h[c] = 0;
+    __syncthreads();
+    for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < nbins; b += gridDim.x * blockDim.x)
+        atomicAdd(&h[len_class(offsets[(b + 1) * kDepthBuckets] - offsets[b * kDepthBuckets])], 1);
+    __syncthreads();
+    for (int c = threadIdx.x; c < kLenClasses; c += blockDim.x)
+        if (h[c]) atomicAdd(&hist[c], h[c]);
+}
+
+// Rounds of blockDim bins: ranks inside the round from shared-memory atomics, then one
+// global atomic per class and round reserves the round's places in that class.
+__global__ void k_bin_order(const int* __restrict__ offsets, int nbins, const int* __restrict__ hist,
+                            int* __restrict__ cursor, int* __restrict__ order) {
+    __shared__ int start[kLenClasses], cnt[kLenClasses], base[kLenClasses];
+    if (threadIdx.x == 0) {
+        int at = 0;
+        for (int c = kLenClasses - 1; c >= 0; --c) {
+            start[c] = at;
+            at += hist[c];
+        }
+    }
+    for (int b0 = blockIdx.x * blockDim.x; b0 < nbins; b0 += gridDim.x * blockDim.x) {
+        for (int c = threadIdx.x; c < kLenClasses; c += blockDim.x) cnt[c] = 0;
+        __syncthreads();
+        const int b = b0 + threadIdx.x;
+        int c = 0, r = 0;
+        if (b < nbins) {
+            c = len_class(offsets[(b + 1) * kDepthBuckets] - offsets[b * kDepthBuckets]);
+            r = atomicAdd(&cnt[c], 1);
+        }
+        __syncthreads();
+        for (int k = threadIdx.x; k < kLenClasses; k += blockDim.x)
+            base[k] = cnt[k] ? start[k] + atomicAdd(&cursor[k], cnt[k]) : 0;
+        __syncthreads();
+        if (b < nbins) order[base[c] + r] = b;
+        __syncthreads();
+    }
+}
+
 // ------------------------------------------------------------------ fine pass
 template <int KC>
 __device__ __forceinline__ void topk_insert(float (&kk)[KC], int (&ff)[KC], float key, int fid) {
@@ -266,10 +317,11 @@ __device__ __forceinline__ void topk_insert(float (&kk)[KC], int (&ff)[KC], floa
 template <int KC, bool PERSP, bool EXACT>
 __global__ void __launch_bounds__(kFineThreads, KC <= 4 ? 6 : 4)
 k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const int* __restrict__ offsets,
-       const int* __restrict__ list, int nbx, int nby, int H, int W, int K, float blur, int* __restrict__ topk) {
+       const int* __restrict__ list, const int* __restrict__ order, int nbx, int nby, int H, int W, int K, float blur,
+       int* __restrict__ topk) {
     __shared__ __align__(16) float4 s_c[kWarpsPerBin][32][kConstF4];
 
-    const int bin = blockIdx.x;
+    const int bin = order[blockIdx.x];
     const int bxi = bin % nbx;
     const int byi = (bin / nbx) % nby;
     const int n = bin / (nbx * nby);
@@ -503,9 +555,10 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int 
 
 template <int KC>
 void launch_fine(bool persp, bool exact, int nbins, cudaStream_t s, const float4* fconst, const FaceBox* box,
-                 const int* offsets, const int* list, int nbx, int nby, int H, int W, int K, float blur, int* topk) {
+                 const int* order, const int* offsets, const int* list, int nbx, int nby, int H, int W, int K,
+                 float blur, int* topk) {
 #define MR_FINE(P, E) \
-    k_fine<KC, P, E><<<nbins, kFineThreads, 0, s>>>(fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk)
+    k_fine<KC, P, E><<<nbins, kFineThreads, 0, s>>>(fconst, box, offsets, list, order, nbx, nby, H, W, K, blur, topk)
     if (persp) {
         if (exact) MR_FINE(true, true); else MR_FINE(true, false);
     } else {
@@ -534,16 +587,19 @@ void launch_epilogue(bool persp, bool sil, bool vec, int N, int H, int W, cudaSt
 }
 
 void dispatch_fine(int KC, bool persp, bool exact, int nbins, cudaStream_t s, const float4* fconst,
-                   const FaceBox* box, const int* offsets, const int* list, int nbx, int nby, int H, int W, int K,
-                   float blur, int* topk) {
+                   const FaceBox* box, const int* order, const int* offsets, const int* list, int nbx, int nby, int H,
+                   int W, int K, float blur, int* topk) {
+#define MR_F(KCV) \
+    launch_fine<KCV>(persp, exact, nbins, s, fconst, box, order, offsets, list, nbx, nby, H, W, K, blur, topk)
     switch (KC) {
-        case 1: launch_fine<1>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
-        case 2: launch_fine<2>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
-        case 4: launch_fine<4>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
-        case 8: launch_fine<8>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
-        case 16: launch_fine<16>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
-        default: launch_fine<32>(persp, exact, nbins, s, fconst, box, offsets, list, nbx, nby, H, W, K, blur, topk); break;
+        case 1: MR_F(1); break;
+        case 2: MR_F(2); break;
+        case 4: MR_F(4); break;
+        case 8: MR_F(8); break;
+        case 16: MR_F(16); break;
+        default: MR_F(32); break;
     }
+#undef MR_F
 }
 
 void dispatch_epilogue(int KC, bool persp, bool sil, bool vec_ok, int N, int H, int W, cudaStream_t s,
@@ -608,7 +664,7 @@ struct FwdPlan {
     int64_t V, F, pairs, npix;
     int N, H, W, K, KC, persp, nbx, nby, nbins, nslots, ntiles;
     float blur;
-    size_t geom, box, con, top, cnt, off, tsum, rng, pre, fst, tot, err, bytes;
+    size_t geom, box, con, top, cnt, off, tsum, rng, pre, fst, tot, err, ord, hist, bytes;
 };
 
 inline int fwd_plan(int64_t V, int64_t F, const int64_t* num, int N, int H, int W, float blur, int K, int persp,
@@ -641,7 +697,9 @@ inline int fwd_plan(int64_t V, int64_t F, const int64_t* num, int N, int H, int 
     P.fst = P.pre + up(sizeof(int64_t) * (size_t)(N + 1));
     P.tot = P.fst + up(sizeof(int64_t) * (size_t)N);
     P.err = P.tot + 256;
-    P.bytes = P.err + 256;
+    P.ord = P.err + 256;
+    P.hist = P.ord + up(sizeof(int) * (size_t)P.nbins);
+    P.bytes = P.hist + up(sizeof(int) * 2 * kLenClasses);
     return MR_OK;
 }
 
@@ -656,6 +714,8 @@ struct FwdBufs {
     int64_t *prefix, *first;
     long long* total;
     int* err;
+    int* order;       // bins, longest list first
+    int* hist;        // kLenClasses class counts, then kLenClasses cursors
 };
 
 inline FwdBufs fwd_bufs(char* ws, const FwdPlan& P) {
@@ -672,6 +732,8 @@ inline FwdBufs fwd_bufs(char* ws, const FwdPlan& P) {
     B.first = reinterpret_cast<int64_t*>(ws + P.fst);
     B.total = reinterpret_cast<long long*>(ws + P.tot);
     B.err = reinterpret_cast<int*>(ws + P.err);
+    B.order = reinterpret_cast<int*>(ws + P.ord);
+    B.hist = reinterpret_cast<int*>(ws + P.hist);
     return B;
 }
 
@@ -713,6 +775,11 @@ inline cudaError_t fwd_enqueue_count(const FwdPlan& P, const FwdBufs& B, const f
         k_scan_tops<<<1, 1024, 0, s>>>(B.tile_sum, P.ntiles, B.total);
         k_scan_add<<<std::min(ceil_div(P.nslots + 1, 256), 148 * 8), 256, 0, s>>>(B.offsets, P.nslots, B.tile_sum,
                                                                                   B.total);
+        // the fine pass's launch order: longest bin lists first
+        if ((e = cudaMemsetAsync(B.hist, 0, sizeof(int) * 2 * kLenClasses, s))) return e;
+        const int og = std::min(ceil_div(P.nbins, 256), 148 * 4);
+        k_bin_hist<<<og, 256, 0, s>>>(B.offsets, P.nbins, B.hist);
+        k_bin_order<<<og, 256, 0, s>>>(B.offsets, P.nbins, B.hist, B.hist + kLenClasses, B.order);
     }
     if ((e = cudaGetLastError())) return e;
     if ((e = cudaMemcpyAsync(host_total, B.total, sizeof(long long), cudaMemcpyDeviceToHost, s))) return e;
@@ -735,8 +802,8 @@ inline cudaError_t fwd_enqueue_rest(const FwdPlan& P, const FwdBufs& B, int* lis
     const bool exact = (P.H & (P.H - 1)) == 0 && (P.W & (P.W - 1)) == 0;
     {
         ProfScope ps(MR_STAGE_FINE, s);
-        dispatch_fine(P.KC, P.persp != 0, exact, P.nbins, s, B.fconst, B.box, B.offsets, list, P.nbx, P.nby, P.H, P.W,
-                      P.K, P.blur, B.topk);
+        dispatch_fine(P.KC, P.persp != 0, exact, P.nbins, s, B.fconst, B.box, B.order, B.offsets, list, P.nbx, P.nby,
+                      P.H, P.W, P.K, P.blur, B.topk);
     }
     if ((e = cudaGetLastError())) return e;
     {
