@@ -208,8 +208,9 @@ KERNEL_SOURCE = os.path.join(ROOT, "differentiable_mesh_rasterization_b200", "cs
 
 
 def measured_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu capture of this workload,
-    or None when there is none or the kernel source changed since it was taken."""
+    """DRAM bytes per launch of `kernel` from the committed ncu capture (a smaller case of
+    this workload, scaled to it by the units the kernel processes), or None when there is
+    none or the kernel source changed since it was taken."""
     import hashlib
     try:
         rec = json.load(open(TRAFFIC_FILE))
@@ -219,7 +220,7 @@ def measured_traffic(kernel: str):
     if rec.get("source_sha256") != sha:
         return None
     k = rec.get("kernels", {}).get(kernel)
-    return None if k is None else k["dram_read_bytes"] + k["dram_write_bytes"]
+    return None if k is None else (k["dram_read_bytes"] + k["dram_write_bytes"]) * k.get("scale", 1.0)
 
 
 # ----------------------------------------------------------------------------- ranks
