@@ -287,7 +287,7 @@ def shading_step_timing(mr, torch, dev, stream, batch, verts, faces, first, num,
         _, _, _, gbary = mr.phong_shade_bwd(p2f, bary, faces, P, N, alb, prm, gcol)
         mr.rasterize_bwd(verts, faces, p2f, w.perspective_correct, grad_zbuf=gz, grad_bary=gbary, grad_dists=gd)
 
-    npix = n_img * w.H * w.W
+    npix = batch.N * w.H * w.W
     K = w.K
     # algorithmic bytes of the stage-two kernels (slot = K per pixel; colours D = 3): each
     # per-slot input read once, each output written once; vertex gathers hit L2 and are
@@ -815,7 +815,7 @@ def main():
             "gpu_launches": int(sum(v[1] * KERNELS_PER_STAGE.get(k, 1) for k, v in stages.items())),
             "clocks": clk}
 
-    if args.no_shading or hard:           # the next rows run on the soft batch-5 workloads
+    if args.no_shading or hard or args.split:   # the next rows run on the whole soft batch-5 workloads
         args.rows = ""
     rows = {}
     if "gouraud" in args.rows or "phong" in args.rows:
