@@ -646,6 +646,8 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    mr.scratch_peak(dev, reset=True)
     mr.profile_enable(True)
     with ClockSampler(uuid or None) as clocks:
         for k in range(args.steps):
@@ -655,6 +657,10 @@ def main():
             ends[k].record(stream)
         torch.cuda.synchronize(dev)
     mr.profile_enable(False)
+    memory = {"scratch_peak_bytes": mr.scratch_peak(dev), "torch_peak_bytes": int(torch.cuda.max_memory_allocated(dev)),
+              "l2_flush_bytes": L2_FLUSH_BYTES,
+              "note": "over the timed steps: the library's scratch (high-water mark of the device's default "
+                      "memory pool) and torch's allocations (inputs, the outputs of each step, the L2-flush buffer)"}
     if world > 1:
         dist.barrier()
     stages = mr.profile_read()
@@ -812,6 +818,7 @@ def main():
                     "note": ("pinned host verts, faces in; the depth buffer out" if hard else
                              "pinned host verts, faces, dL/dalpha in; alpha and grad_verts out") + "; the copies of "
                             "step k+1 (in) and step k (out) overlap the compute of step k on two copy streams"},
+            "memory": memory,
             "gpu_launches": int(sum(v[1] * KERNELS_PER_STAGE.get(k, 1) for k, v in stages.items())),
             "clocks": clk}
 

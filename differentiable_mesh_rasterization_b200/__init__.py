@@ -30,7 +30,7 @@ EXPORTS = ("mr_rasterize_fwd", "mr_rasterize_silhouette_fwd", "mr_silhouette_ble
            "mr_phong_fwd", "mr_phong_bwd", "mr_phong_shade_fwd", "mr_phong_shade_bwd",
            "mr_rasterize_points_fwd", "mr_rasterize_points_bwd", "mr_composite_points_fwd",
            "mr_composite_points_bwd", "mr_knn_fwd", "mr_knn_bwd", "mr_measure_fp32_peak", "mr_knn_count_pairs",
-           "mr_inject_fault", "mr_scratch_in_use")
+           "mr_inject_fault", "mr_scratch_in_use", "mr_scratch_peak")
 STAGES = ("face_setup", "bin_count", "bin_scan", "bin_fill", "fine", "silhouette_fwd", "silhouette_bwd",
           "raster_bwd", "silhouette_raster_bwd", "epilogue", "interpolate_fwd", "interpolate_bwd", "blend_fwd",
           "blend_bwd", "phong_fwd", "phong_bwd", "phong_shade_fwd", "phong_shade_bwd",
@@ -85,6 +85,7 @@ def load_library() -> ctypes.CDLL:
         "mr_measure_fp32_peak": [P, P],
         "mr_inject_fault": [i32, i32],
         "mr_scratch_in_use": [P],
+        "mr_scratch_peak": [P, i32],
         "mr_profile_enable": [i32],
         "mr_profile_read": [P, P, i32],
     }
@@ -599,6 +600,16 @@ def scratch_in_use(device=None) -> int:
     out = ctypes.c_int64(0)
     with torch.cuda.device(dev):
         _check("mr_scratch_in_use", load_library().mr_scratch_in_use(ctypes.byref(out)))
+    return int(out.value)
+
+
+def scratch_peak(device=None, reset: bool = False) -> int:
+    """High-water mark of the device's default memory pool, where the library's scratch
+    comes from (``mr_scratch_peak``); ``reset`` restarts it after reading."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    out = ctypes.c_int64(0)
+    with torch.cuda.device(dev):
+        _check("mr_scratch_peak", load_library().mr_scratch_peak(ctypes.byref(out), int(bool(reset))))
     return int(out.value)
 
 

@@ -113,6 +113,16 @@ int host_indices(cudaStream_t s, int64_t n, std::vector<int64_t>& buf,
 
 bool profiling_enabled() { return g_prof_on; }
 
+const char* stage_name(int stage) {
+    static const char* const names[MR_NUM_STAGES] = {
+        "mr:face_setup", "mr:bin_count", "mr:bin_scan", "mr:bin_fill", "mr:fine", "mr:silhouette_fwd",
+        "mr:silhouette_bwd", "mr:raster_bwd", "mr:silhouette_raster_bwd", "mr:epilogue", "mr:interpolate_fwd",
+        "mr:interpolate_bwd", "mr:blend_fwd", "mr:blend_bwd", "mr:phong_fwd", "mr:phong_bwd", "mr:phong_shade_fwd",
+        "mr:phong_shade_bwd", "mr:points_bin", "mr:points_fine", "mr:points_bwd", "mr:composite_fwd",
+        "mr:composite_bwd", "mr:knn", "mr:knn_bwd"};
+    return stage >= 0 && stage < MR_NUM_STAGES ? names[stage] : "mr:stage";
+}
+
 cudaEvent_t profile_event() {
     std::lock_guard<std::mutex> g(g_prof_mutex);
     if (!g_prof_free.empty()) {
@@ -213,6 +223,25 @@ int mr_inject_fault(int32_t kind, int32_t skip) {
     g_inject_kind.store(MR_INJECT_OFF);
     g_inject_skip.store(skip);
     g_inject_kind.store(kind);
+    return MR_OK;
+}
+
+int mr_scratch_peak(int64_t* bytes, int32_t reset) {
+    if (!bytes) {
+        mr::set_error("null output");
+        return MR_ERR_ARG;
+    }
+    int dev = 0;
+    MR_CUDA(cudaGetDevice(&dev));
+    cudaMemPool_t pool;
+    MR_CUDA(cudaDeviceGetDefaultMemPool(&pool, dev));
+    uint64_t high = 0;
+    MR_CUDA(cudaMemPoolGetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &high));
+    *bytes = (int64_t)high;
+    if (reset) {
+        uint64_t zero = 0;
+        MR_CUDA(cudaMemPoolSetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &zero));
+    }
     return MR_OK;
 }
 

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include <cstdio>
@@ -141,11 +142,15 @@ int* device_error_word();
 bool profiling_enabled();
 void profile_record(int stage, cudaEvent_t start, cudaEvent_t stop);
 cudaEvent_t profile_event();
+// Each scope is also an NVTX range named after its stage (host-side enqueue of the stage's
+// launches; free unless a tracing tool is attached).
+const char* stage_name(int stage);
 struct ProfScope {
     int stage;
     cudaStream_t s;
     cudaEvent_t a = nullptr, b = nullptr;
     ProfScope(int st, cudaStream_t str) : stage(st), s(str) {
+        nvtxRangePushA(stage_name(st));
         if (profiling_enabled()) {
             a = profile_event();
             b = profile_event();
@@ -157,6 +162,7 @@ struct ProfScope {
             cudaEventRecord(b, s);
             profile_record(stage, a, b);
         }
+        nvtxRangePop();
     }
 };
 

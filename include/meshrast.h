@@ -359,6 +359,16 @@ int mr_inject_fault(int32_t kind, int32_t skip);
 int mr_scratch_in_use(int64_t* bytes);
 
 /*
+ * High-water mark of the bytes allocated from the current device's default memory pool
+ * since it was last reset (the peak of the library's scratch, and of anything else the
+ * process takes from that pool); *bytes is HOST.  reset != 0 clears the mark after reading
+ * it (CUDA resets it to zero; it then follows the allocations made from then on).  For
+ * memory measurements (the pages compare renderers'
+ * memory; no other counterpart there).
+ */
+int mr_scratch_peak(int64_t* bytes, int32_t reset);
+
+/*
  * FP32 issue-rate probe (measurement support; no counterpart on the pages): times five
  * launches (after a warm-up) of a kernel of independent FFMA chains filling every SM
  * (8 chains per thread, 148 x 8 CTAs of 256 threads on B200, ~11 ms each) with CUDA events
@@ -371,7 +381,9 @@ int mr_measure_fp32_peak(double* inst_per_s, void* stream);
 /*
  * Stage timing (the library's own tracing; no counterpart on the pages).  While enabled,
  * every launch of the stages below is bracketed by two CUDA events recorded on the
- * caller's stream; recording adds no synchronisation.  mr_profile_read() waits for the
+ * caller's stream; recording adds no synchronisation.  Independently of this switch, the
+ * host-side enqueue of each stage is an NVTX range named "mr:<stage>" (free unless a
+ * tracing tool is attached).  mr_profile_read() waits for the
  * recorded events, writes the summed milliseconds and launch counts per stage into
  * stage_ms[0..nstages) and launches[0..nstages) (either may be NULL), and forgets them.
  * Process-wide; intended for one device and one thread at a time.
