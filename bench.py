@@ -785,8 +785,8 @@ def main():
     hbm_note = "of measured" if "hbm_gbs" in peaks else "of fallback"
     achieved_alu = samples * C_TEST / fine_s / 1e12
     npix = n_img * w.H * w.W
-    fine_bytes = npix * 4 * w.K                      # the K winning face ids per pixel
-    epi_bytes = npix * (4 * w.K + 28 * w.K + (0 if hard else 4))   # ids in; p2f, zbuf, bary, dists(, alpha) out
+    fine_bytes = npix * 8 * w.K                      # the K winning face ids per pixel, written as pix_to_face
+    epi_bytes = npix * (8 * w.K + 20 * w.K + (0 if hard else 4))   # ids in; zbuf, bary, dists(, alpha) out
     full_batch = args.images is None and args.config == 5
     roof = {"bound": "alu", "achieved": achieved_alu, "peak": peak_alu, "unit": "T FP32-inst/s",
             "frac": achieved_alu / peak_alu, "traffic": measured_traffic("k_fine") if full_batch else None,

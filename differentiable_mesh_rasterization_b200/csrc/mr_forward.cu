@@ -16,7 +16,8 @@
 //   fine         one CTA per bin, eight independent warps (8x4 pixel tiles): ballot-
 //                compacted per-warp face lists staged in shared memory, a warp-wide
 //                depth pre-test, the full candidacy test, and a register-resident
-//                insertion-sorted top-K per pixel; writes the K winning face ids.
+//                insertion-sorted top-K per pixel; writes the K winning face ids
+//                straight into pix_to_face.
 //   epilogue     one thread per pixel: barycentrics, z and signed squared distance of
 //                the K winners recomputed in float64 from the original vertices, the
 //                fused soft silhouette, 16-byte stores.

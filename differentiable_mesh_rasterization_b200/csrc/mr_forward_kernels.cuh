@@ -318,7 +318,7 @@ template <int KC, bool PERSP, bool EXACT>
 __global__ void __launch_bounds__(kFineThreads, KC <= 4 ? 6 : 4)
 k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const int* __restrict__ offsets,
        const int* __restrict__ list, const int* __restrict__ order, int nbx, int nby, int H, int W, int K, float blur,
-       int* __restrict__ topk) {
+       bool vec, int64_t* __restrict__ p2f) {
     __shared__ __align__(16) float4 s_c[kWarpsPerBin][32][kConstF4];
 
     const int bin = order[blockIdx.x];
@@ -409,17 +409,18 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
         __syncwarp();
     }
     if (!in_img) return;
+    // the winners go straight into pix_to_face (global face ids, -1 past the candidates);
+    // the epilogue reads them back from there
     const int64_t pix = ((int64_t)n * H + i) * W + j;
-    if (K == KC && (KC % 4) == 0) {
+    if ((KC % 2) == 0 && K == KC && vec) {
 #pragma unroll
-        for (int k4 = 0; k4 < KC; k4 += 4)
-            *reinterpret_cast<int4*>(topk + pix * KC + k4) =
-                make_int4(ff[k4] == INT_MAX ? -1 : ff[k4], ff[k4 + 1] == INT_MAX ? -1 : ff[k4 + 1],
-                          ff[k4 + 2] == INT_MAX ? -1 : ff[k4 + 2], ff[k4 + 3] == INT_MAX ? -1 : ff[k4 + 3]);
+        for (int k2 = 0; k2 < KC; k2 += 2)
+            *reinterpret_cast<longlong2*>(p2f + pix * KC + k2) =
+                make_longlong2(ff[k2] == INT_MAX ? -1 : ff[k2], ff[k2 + 1] == INT_MAX ? -1 : ff[k2 + 1]);
     } else {
 #pragma unroll
         for (int k = 0; k < KC; ++k)
-            if (k < K) topk[pix * K + k] = ff[k] == INT_MAX ? -1 : ff[k];
+            if (k < K) p2f[pix * K + k] = ff[k] == INT_MAX ? -1 : ff[k];
     }
 }
 
@@ -479,9 +480,8 @@ __device__ __forceinline__ void slot_outputs(const FaceGeom& g, double pxd, doub
 // region and the geometry reads hit L1.
 template <int KC, bool PERSP, bool SIL, bool VEC>
 __global__ void __launch_bounds__(256, 4)
-k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int N, int H, int W, int K, float sigma,
-           int64_t* __restrict__ p2f, float* __restrict__ zbuf, float* __restrict__ bary, float* __restrict__ dists,
-           float* __restrict__ alpha) {
+k_epilogue(const FaceGeom* __restrict__ geom, const int64_t* __restrict__ p2f, int N, int H, int W, int K, float sigma,
+           float* __restrict__ zbuf, float* __restrict__ bary, float* __restrict__ dists, float* __restrict__ alpha) {
     const int tw = (W + kBin - 1) / kBin, th = (H + kBin - 1) / kBin;
     const int64_t items = (int64_t)N * th * tw * (kBin * kBin);
     for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < items;
@@ -504,10 +504,10 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int 
         if (VEC) {
 #pragma unroll
             for (int k4 = 0; k4 < KC; k4 += 4) {
-                const int4 f4 = *reinterpret_cast<const int4*>(topk + pix * KC + k4);
-                const int fk[4] = {f4.x, f4.y, f4.z, f4.w};
+                const longlong2 fa = reinterpret_cast<const longlong2*>(p2f + pix * KC + k4)[0];
+                const longlong2 fb = reinterpret_cast<const longlong2*>(p2f + pix * KC + k4)[1];
+                const int fk[4] = {(int)fa.x, (int)fa.y, (int)fb.x, (int)fb.y};
                 float zz[4], bb[12], dd[4];
-                long long pf[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     if (fk[u] >= 0) {
@@ -515,13 +515,10 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int 
                     } else {
                         zz[u] = -1.f; dd[u] = -1.f; bb[3 * u] = bb[3 * u + 1] = bb[3 * u + 2] = -1.f;
                     }
-                    pf[u] = fk[u];
                     dsil[k4 + u] = dd[u];
                     vsil[k4 + u] = fk[u] >= 0;
                 }
                 const int64_t s = pix * KC + k4;
-                reinterpret_cast<longlong2*>(p2f + s)[0] = make_longlong2(pf[0], pf[1]);
-                reinterpret_cast<longlong2*>(p2f + s)[1] = make_longlong2(pf[2], pf[3]);
                 *reinterpret_cast<float4*>(zbuf + s) = make_float4(zz[0], zz[1], zz[2], zz[3]);
                 *reinterpret_cast<float4*>(dists + s) = make_float4(dd[0], dd[1], dd[2], dd[3]);
                 float4* bp = reinterpret_cast<float4*>(bary + 3 * s);
@@ -534,14 +531,13 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int 
             for (int k = 0; k < KC; ++k) {
                 if (k >= K) break;
                 const int64_t s = pix * K + k;
-                const int fk = topk[s];
+                const int fk = (int)p2f[s];
                 float zz, bb[3], dd;
                 if (fk >= 0) {
                     slot_outputs<PERSP>(geom[fk], pxd, pyd, pxh, pxl, pyh, pyl, &zz, bb, &dd);
                 } else {
                     zz = -1.f; dd = -1.f; bb[0] = bb[1] = bb[2] = -1.f;
                 }
-                p2f[s] = fk;
                 zbuf[s] = zz;
                 dists[s] = dd;
                 bary[3 * s] = bb[0]; bary[3 * s + 1] = bb[1]; bary[3 * s + 2] = bb[2];
@@ -556,9 +552,10 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ topk, int 
 template <int KC>
 void launch_fine(bool persp, bool exact, int nbins, cudaStream_t s, const float4* fconst, const FaceBox* box,
                  const int* order, const int* offsets, const int* list, int nbx, int nby, int H, int W, int K,
-                 float blur, int* topk) {
+                 float blur, bool vec, int64_t* p2f) {
 #define MR_FINE(P, E) \
-    k_fine<KC, P, E><<<nbins, kFineThreads, 0, s>>>(fconst, box, offsets, list, order, nbx, nby, H, W, K, blur, topk)
+    k_fine<KC, P, E><<<nbins, kFineThreads, 0, s>>>(fconst, box, offsets, list, order, nbx, nby, H, W, K, blur, vec, \
+                                                     p2f)
     if (persp) {
         if (exact) MR_FINE(true, true); else MR_FINE(true, false);
     } else {
@@ -569,12 +566,12 @@ void launch_fine(bool persp, bool exact, int nbins, cudaStream_t s, const float4
 
 template <int KC>
 void launch_epilogue(bool persp, bool sil, bool vec, int N, int H, int W, cudaStream_t s, const FaceGeom* geom,
-                     const int* topk, int K, float sigma, int64_t* p2f, float* zbuf, float* bary, float* dists,
+                     const int64_t* p2f, int K, float sigma, float* zbuf, float* bary, float* dists,
                      float* alpha) {
     const int64_t items = (int64_t)N * ceil_div(H, kBin) * ceil_div(W, kBin) * (kBin * kBin);
     const int grid = (int)std::min<int64_t>((items + 255) / 256, 148 * 32);
 #define MR_EPI(P, S, V) \
-    k_epilogue<KC, P, S, V><<<grid, 256, 0, s>>>(geom, topk, N, H, W, K, sigma, p2f, zbuf, bary, dists, alpha)
+    k_epilogue<KC, P, S, V><<<grid, 256, 0, s>>>(geom, p2f, N, H, W, K, sigma, zbuf, bary, dists, alpha)
 #define MR_EPI2(P, S) \
     if (vec) MR_EPI(P, S, true); else MR_EPI(P, S, false)
     if (persp) {
@@ -588,9 +585,9 @@ void launch_epilogue(bool persp, bool sil, bool vec, int N, int H, int W, cudaSt
 
 void dispatch_fine(int KC, bool persp, bool exact, int nbins, cudaStream_t s, const float4* fconst,
                    const FaceBox* box, const int* order, const int* offsets, const int* list, int nbx, int nby, int H,
-                   int W, int K, float blur, int* topk) {
+                   int W, int K, float blur, bool vec, int64_t* p2f) {
 #define MR_F(KCV) \
-    launch_fine<KCV>(persp, exact, nbins, s, fconst, box, order, offsets, list, nbx, nby, H, W, K, blur, topk)
+    launch_fine<KCV>(persp, exact, nbins, s, fconst, box, order, offsets, list, nbx, nby, H, W, K, blur, vec, p2f)
     switch (KC) {
         case 1: MR_F(1); break;
         case 2: MR_F(2); break;
@@ -603,10 +600,10 @@ void dispatch_fine(int KC, bool persp, bool exact, int nbins, cudaStream_t s, co
 }
 
 void dispatch_epilogue(int KC, bool persp, bool sil, bool vec_ok, int N, int H, int W, cudaStream_t s,
-                       const FaceGeom* geom, const int* topk, int K, float sigma, int64_t* p2f, float* zbuf,
+                       const FaceGeom* geom, const int64_t* p2f, int K, float sigma, float* zbuf,
                        float* bary, float* dists, float* alpha) {
     const bool vec = vec_ok && K == KC && (KC % 4) == 0;
-#define MR_E(KCV) launch_epilogue<KCV>(persp, sil, vec, N, H, W, s, geom, topk, K, sigma, p2f, zbuf, bary, dists, alpha)
+#define MR_E(KCV) launch_epilogue<KCV>(persp, sil, vec, N, H, W, s, geom, p2f, K, sigma, zbuf, bary, dists, alpha)
     switch (KC) {
         case 1: MR_E(1); break;
         case 2: MR_E(2); break;
@@ -664,7 +661,7 @@ struct FwdPlan {
     int64_t V, F, pairs, npix;
     int N, H, W, K, KC, persp, nbx, nby, nbins, nslots, ntiles;
     float blur;
-    size_t geom, box, con, top, cnt, off, tsum, rng, pre, fst, tot, err, ord, hist, bytes;
+    size_t geom, box, con, cnt, off, tsum, rng, pre, fst, tot, err, ord, hist, bytes;
 };
 
 inline int fwd_plan(int64_t V, int64_t F, const int64_t* num, int N, int H, int W, float blur, int K, int persp,
@@ -688,8 +685,7 @@ inline int fwd_plan(int64_t V, int64_t F, const int64_t* num, int N, int H, int 
     P.geom = 0;
     P.box = P.geom + up(sizeof(FaceGeom) * (size_t)F);
     P.con = P.box + up(sizeof(FaceBox) * (size_t)F);
-    P.top = P.con + up(sizeof(float4) * kConstF4 * (size_t)F);
-    P.cnt = P.top + up(sizeof(int) * (size_t)P.npix * (size_t)K);
+    P.cnt = P.con + up(sizeof(float4) * kConstF4 * (size_t)F);
     P.off = P.cnt + up(sizeof(int) * (size_t)P.nslots);
     P.tsum = P.off + up(sizeof(int) * (size_t)(P.nslots + 1));
     P.rng = P.tsum + up(sizeof(long long) * (size_t)P.ntiles);
@@ -708,7 +704,7 @@ struct FwdBufs {
     FaceGeom* geom;
     FaceBox* box;
     float4* fconst;
-    int *topk, *counts, *offsets;
+    int *counts, *offsets;
     long long* tile_sum;
     unsigned* krange;
     int64_t *prefix, *first;
@@ -723,7 +719,6 @@ inline FwdBufs fwd_bufs(char* ws, const FwdPlan& P) {
     B.geom = reinterpret_cast<FaceGeom*>(ws + P.geom);
     B.box = reinterpret_cast<FaceBox*>(ws + P.box);
     B.fconst = reinterpret_cast<float4*>(ws + P.con);
-    B.topk = reinterpret_cast<int*>(ws + P.top);
     B.counts = reinterpret_cast<int*>(ws + P.cnt);
     B.offsets = reinterpret_cast<int*>(ws + P.off);
     B.tile_sum = reinterpret_cast<long long*>(ws + P.tsum);
@@ -803,13 +798,13 @@ inline cudaError_t fwd_enqueue_rest(const FwdPlan& P, const FwdBufs& B, int* lis
     {
         ProfScope ps(MR_STAGE_FINE, s);
         dispatch_fine(P.KC, P.persp != 0, exact, P.nbins, s, B.fconst, B.box, B.order, B.offsets, list, P.nbx, P.nby,
-                      P.H, P.W, P.K, P.blur, B.topk);
+                      P.H, P.W, P.K, P.blur, aligned16(p2f), p2f);
     }
     if ((e = cudaGetLastError())) return e;
     {
         ProfScope ps(MR_STAGE_EPILOGUE, s);
-        dispatch_epilogue(P.KC, P.persp != 0, sil, vec_ok, P.N, P.H, P.W, s, B.geom, B.topk, P.K, sigma, p2f, zbuf,
-                          bary, dists, alpha);
+        dispatch_epilogue(P.KC, P.persp != 0, sil, vec_ok, P.N, P.H, P.W, s, B.geom, p2f, P.K, sigma, zbuf, bary,
+                          dists, alpha);
     }
     return cudaGetLastError();
 }

@@ -6,7 +6,7 @@
 // carving out more, a latency-critical loop where an allocation could block or fail
 // under memory pressure, or a plugin that runs inside someone else's memory budget.
 // For them this entry point runs the same kernels as mr_rasterize_fwd, but every byte
-// of scratch (face records, per-bin counts and lists, the top-K face ids) comes from
+// of scratch (face records, per-bin counts, their launch order and the bin lists) comes from
 // one file-scope device array of fixed size.  The caller still provides the inputs and
 // the outputs.
 //

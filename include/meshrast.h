@@ -97,8 +97,8 @@ int mr_rasterize_fwd(const float* verts, int64_t V, const int64_t* faces, int64_
  * of its scratch from one fixed device array of MR_NOALLOC_SCRATCH_BYTES that the
  * library holds on each device using it until the process exits; it calls no cudaMalloc,
  * cudaFree or other allocating routine.  The caller still provides inputs and outputs.
- *  - Batches whose scratch exceeds the array (face records, per-pixel top-K ids, per-bin
- *    counts and lists) are rejected with MR_ERR_ARG and a message naming the size.
+ *  - Batches whose scratch exceeds the array (face records, per-bin counts and lists)
+ *    are rejected with MR_ERR_ARG and a message naming the size.
  *  - The first call on a device looks up the array's device address, with that device
  *    current; make that first call before any stream capture.  Every call synchronises
  *    `stream` once, after the bin count, as mr_rasterize_fwd does.

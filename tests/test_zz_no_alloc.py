@@ -62,11 +62,14 @@ def test_noalloc_matches_allocating_forward_on_two_calls():
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch():
-    b = syn.make_batch(4)                  # 1024x1024 with K=16 needs > 64 MiB of top-K ids
+    """The first limit: the 64 meshes of the 512x512 batch hold 2.35 M faces, whose records
+    (160 bytes each) alone exceed the fixed array; rejected before anything is launched
+    (a small image keeps the outputs small)."""
+    b = syn.make_batch(5)
     v = torch.from_numpy(b.verts).cuda()
     f = torch.from_numpy(b.faces).cuda()
     with pytest.raises(mr.MeshRastError) as e:
-        mr.rasterize_fwd_noalloc(v, f, b.mesh_to_face_first_idx, b.num_faces_per_mesh, 1024, 1024, 1e-5, 16, True)
+        mr.rasterize_fwd_noalloc(v, f, b.mesh_to_face_first_idx, b.num_faces_per_mesh, 32, 32, 1e-5, 4, False)
     assert e.value.code == -1 and "scratch" in str(e.value)
 
 
