@@ -101,6 +101,19 @@ int cuda_fail(cudaError_t e, const char* what);
 int host_indices(cudaStream_t s, int64_t n, std::vector<int64_t>& buf,
                  std::initializer_list<const int64_t**> arrays);
 
+// A mapped (zero-copy) pinned host buffer of two 64-bit words, one per calling thread and
+// device: the values a call reads back in the middle (a list total, the device error
+// word) are written there by a kernel, so reading them needs no copy engine -- a copy
+// would queue behind the caller's own large transfers on that engine.  dev is nullptr when
+// no such buffer can be had; the caller then copies instead.
+struct Mailbox {
+    volatile long long* host;
+    long long* dev;
+};
+Mailbox host_mailbox();
+// Enqueues on s: out[0] = *total, out[1] = err ? *err : 0 (out: a Mailbox's dev pointer).
+cudaError_t post_counts(const long long* total, const int* err, long long* out, cudaStream_t s);
+
 // Scratch allocation on the caller's stream (stream-ordered pool).
 int scratch_alloc(void** p, size_t bytes, cudaStream_t s);
 void scratch_free(void* p, cudaStream_t s);

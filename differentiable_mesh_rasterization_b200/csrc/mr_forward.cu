@@ -60,9 +60,14 @@ int rasterize_impl(const float* verts, int64_t V, const int64_t* faces, int64_t 
     };
     long long total = 0;
     int herr = 0;
-    cudaError_t e = fwd_enqueue_count(P, B, verts, faces, prefix.data(), first, s, &total, &herr);
+    const Mailbox mb = host_mailbox();
+    cudaError_t e = fwd_enqueue_count(P, B, verts, faces, prefix.data(), first, s, &total, &herr, mb.dev);
     if (e != cudaSuccess) return finish(cuda_fail(e, "forward: face setup and binning"));
     if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return finish(cuda_fail(e, "cudaStreamSynchronize"));
+    if (mb.dev) {
+        total = mb.host[0];
+        herr = (int)mb.host[1];
+    }
     if (total >= INT32_MAX) {
         set_error("bin lists too long (%lld entries)", total);
         return finish(MR_ERR_ARG);

@@ -736,10 +736,11 @@ inline int pair_blocks(int64_t pairs) { return (int)std::min<int64_t>((pairs + 2
 
 // Up to the bin counts: per-mesh arrays to the device, clears, face setup (with the
 // images' key ranges), bin count and scan, and the read-back of the list total and the
-// error word into host_total / host_err (valid after the stream is synchronised).
+// error word (valid after the stream is synchronised): written by a kernel into mailbox
+// (a Mailbox's dev pointer) when one is given, else copied into host_total / host_err.
 inline cudaError_t fwd_enqueue_count(const FwdPlan& P, const FwdBufs& B, const float* verts, const int64_t* faces,
                                      const int64_t* host_prefix, const int64_t* host_first, cudaStream_t s,
-                                     long long* host_total, int* host_err) {
+                                     long long* host_total, int* host_err, long long* mailbox = nullptr) {
     cudaError_t e;
     if ((e = cudaMemcpyAsync(B.prefix, host_prefix, sizeof(int64_t) * (P.N + 1), cudaMemcpyHostToDevice, s))) return e;
     if ((e = cudaMemcpyAsync(B.first, host_first, sizeof(int64_t) * P.N, cudaMemcpyHostToDevice, s))) return e;
@@ -777,6 +778,7 @@ inline cudaError_t fwd_enqueue_count(const FwdPlan& P, const FwdBufs& B, const f
         k_bin_order<<<og, 256, 0, s>>>(B.offsets, P.nbins, B.hist, B.hist + kLenClasses, B.order);
     }
     if ((e = cudaGetLastError())) return e;
+    if (mailbox) return post_counts(B.total, B.err, mailbox, s);
     if ((e = cudaMemcpyAsync(host_total, B.total, sizeof(long long), cudaMemcpyDeviceToHost, s))) return e;
     return cudaMemcpyAsync(host_err, B.err, sizeof(int), cudaMemcpyDeviceToHost, s);
 }

@@ -470,8 +470,14 @@ int mr_rasterize_points_fwd(const float* points, int64_t P, const int64_t* cloud
         k_scan_add<<<std::min((nbins + 256) / 256, 148 * 8), 256, 0, s>>>(offsets, nbins, tile, total_d);
         e = cudaGetLastError();
     }
-    if (e == cudaSuccess) e = cudaMemcpyAsync(&total, total_d, sizeof(long long), cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(s);   // the one sync: the list's size
+    // the one sync: the list's size, read back without a copy engine when a mapped host
+    // word is at hand
+    const Mailbox mb = host_mailbox();
+    if (e == cudaSuccess)
+        e = mb.dev ? post_counts(total_d, nullptr, mb.dev, s)
+                   : cudaMemcpyAsync(&total, total_d, sizeof(long long), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess && mb.dev) total = mb.host[0];
     if (e == cudaSuccess && total > INT32_MAX) {
         scratch_free(base, s);
         set_error("%lld point-bin entries exceed the int32 list (radius too large for this batch)", total);

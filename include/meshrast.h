@@ -78,8 +78,13 @@ extern "C" {
  *   bary                     N x H x W x K x 3 float32 (device, written)
  *
  * Synchronises `stream` once to size the per-bin face lists (and once more, before any
- * launch, when the per-mesh arrays are device memory).  Returns MR_ERR_DEVICE if a face
- * referenced a vertex outside [0, V) (that face is then ignored).
+ * launch, when the per-mesh arrays are device memory).  The list size and the device
+ * error word come back through 64 bytes of mapped pinned host memory, allocated on a
+ * thread's first call for the current device and kept for the life of the thread; that
+ * read-back uses no copy engine, so it does not wait behind the caller's own transfers
+ * (where the mapped memory cannot be had, it falls back to a device-to-host copy on
+ * `stream`).  Returns MR_ERR_DEVICE if a face referenced a vertex outside [0, V) (that
+ * face is then ignored).
  */
 int mr_rasterize_fwd(const float* verts, int64_t V, const int64_t* faces, int64_t F,
                      const int64_t* mesh_to_face_first_idx, const int64_t* num_faces_per_mesh,
@@ -263,7 +268,8 @@ int mr_phong_shade_bwd(const int64_t* pix_to_face, const float* bary, int64_t np
  *   with z >= 0 and squared 2-D distance to the pixel centre <= radius^2, ordered by
  *   (z, point id): idx (global point id, int64), zbuf (= z), dists (squared distance), all
  *   N x H x W x K, -1 in empty slots.  Bins points into 16 x 16-pixel tiles; performs one
- *   stream synchronisation (the bin list's size).  MR_ERR_ARG also when the bin list would
+ *   stream synchronisation (the bin list's size, read back through the same mapped host
+ *   word as mr_rasterize_fwd's).  MR_ERR_ARG also when the bin list would
  *   exceed 2^31 entries (a radius far larger than the image).
  * mr_rasterize_points_bwd: grad_points (P x 3, overwritten) from grad_zbuf and grad_dists
  *   (each nullable): d dists / d (x, y) = -2 (pixel centre - (x, y)), d zbuf / d z = 1.
