@@ -482,18 +482,30 @@ template <int KC, bool PERSP, bool SIL, bool VEC>
 __global__ void __launch_bounds__(256, 4)
 k_epilogue(const FaceGeom* __restrict__ geom, const int64_t* __restrict__ p2f, int N, int H, int W, int K, float sigma,
            float* __restrict__ zbuf, float* __restrict__ bary, float* __restrict__ dists, float* __restrict__ alpha) {
+    static_assert(kBin == 16, "the tile arithmetic below takes 16 x 16 tiles");
     const int tw = (W + kBin - 1) / kBin, th = (H + kBin - 1) / kBin;
     const int64_t items = (int64_t)N * th * tw * (kBin * kBin);
+    const bool small = (int64_t)N * th * tw <= 0x7fffffff;   // tile ids fit 32-bit division
+    const bool ragged = (H % kBin) != 0 || (W % kBin) != 0;   // some tiles stick out of the image
     for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < items;
          it += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t tile = it / (kBin * kBin);
-        const int r = (int)(it % (kBin * kBin));
-        const int tx = (int)(tile % tw);
-        const int64_t t2 = tile / tw;
-        const int ty = (int)(t2 % th);
-        const int64_t n = t2 / th;
-        const int i = ty * kBin + r / kBin, j = tx * kBin + r % kBin;
-        if (i >= H || j >= W) continue;
+        const int64_t tile = it >> 8;                           // kBin * kBin = 256 items per tile
+        const int r = (int)(it & 255);
+        int tx, ty;
+        int64_t n;
+        if (small) {
+            const unsigned t = (unsigned)tile, t2 = t / (unsigned)tw;
+            tx = (int)(t - t2 * (unsigned)tw);
+            ty = (int)(t2 % (unsigned)th);
+            n = t2 / (unsigned)th;
+        } else {
+            tx = (int)(tile % tw);
+            const int64_t t2 = tile / tw;
+            ty = (int)(t2 % th);
+            n = t2 / th;
+        }
+        const int i = ty * kBin + (r >> 4), j = tx * kBin + (r & 15);
+        if (ragged && (i >= H || j >= W)) continue;
         const int64_t pix = (n * H + i) * W + j;
         const double pxd = -1.0 + (2.0 * j + 1.0) / W;
         const double pyd = 1.0 - (2.0 * i + 1.0) / H;
@@ -545,7 +557,7 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int64_t* __restrict__ p2f, i
                 vsil[k] = fk >= 0;
             }
         }
-        if (SIL) alpha[pix] = silhouette_alpha<KC>(dsil, vsil, K, sigma);
+        if (SIL) alpha[pix] = silhouette_alpha<KC>(dsil, vsil, VEC ? KC : K, sigma);   // VEC implies K == KC
     }
 }
 
