@@ -379,9 +379,15 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
         const FaceBox b = nbox;
         // tile depth cull: the farthest K-th key over the warp's pixels; a face whose lowest
         // key over its box lies beyond it cannot enter any lane's top K
-        float zfar = in_img ? kk[KC - 1] : -FLT_MAX;
+        float zfar;
+        if constexpr (!PERSP) {
+            // keys >= 0 order as their bit patterns: one warp reduction (off-image lanes give 0)
+            zfar = __uint_as_float(__reduce_max_sync(0xffffffffu, in_img ? __float_as_uint(kk[KC - 1]) : 0u));
+        } else {
+            zfar = in_img ? kk[KC - 1] : -FLT_MAX;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) zfar = fmaxf(zfar, __shfl_xor_sync(0xffffffffu, zfar, o));
+            for (int o = 16; o > 0; o >>= 1) zfar = fmaxf(zfar, __shfl_xor_sync(0xffffffffu, zfar, o));
+        }
         const bool hit = base + lane < cnt && b.x0 <= tj0 + kWarpTileW - 1 && b.x1 >= tj0 &&
                          b.y0 <= ti0 + kWarpTileH - 1 && b.y1 >= ti0 && b.kmin <= zfar;
         if (base + 32 + lane < cnt) {

@@ -9,16 +9,26 @@
 
 namespace mr {
 
-// alpha evaluated as -expm1(sum_k log(1 - p_k)) with log(1 - p_k) = -log1p(exp(-d_k / sigma)):
-// full relative accuracy both for alpha near 0 (far blur ring) and near 1 (interior).
+// alpha = 1 - prod_k (1 - p_k) = 1 - 1 / P with P = prod_k (1 + e_k), e_k = exp(-d_k / sigma),
+// because 1 - p_k = 1 / (1 + e_k).  P - 1 is carried as its own running value,
+// (P - 1)' = (P - 1) + e + (P - 1) e, so alpha = (P - 1) / P keeps full relative accuracy
+// for alpha near 0 (far blur ring), and one exponential per slot is the only
+// transcendental.  The exponent is capped at 80 and P - 1 at 1e30 (alpha is then 1 in
+// float32 either way), so an interior slot (e huge) next to a far one (e = 0) cannot form
+// inf * 0.
 template <int KC>
 __device__ __forceinline__ float silhouette_alpha(const float (&d)[KC], const bool (&valid)[KC], int K,
                                                   float sigma) {
-    float s = 0.f;
+    const float inv_sigma = 1.f / sigma;
+    float pm1 = 0.f;
 #pragma unroll
     for (int k = 0; k < KC; ++k)
-        if (k < K && valid[k]) s -= log1pf(expf(-(d[k] / sigma)));
-    return -expm1f(s);
+        if (k < K && valid[k]) {
+            const float e = expf(fminf(-d[k] * inv_sigma, 80.f));
+            pm1 = fminf(fmaf(pm1, e, pm1 + e), 1e30f);
+        }
+    const float r = 1.f / (1.f + pm1);
+    return pm1 <= 1.f ? pm1 * r : 1.f - r;
 }
 
 // dL/dd_k = -dL/dalpha * prod_{j != k} (1 - p_j) * p_k (1 - p_k) / sigma; 0 for empty slots.
