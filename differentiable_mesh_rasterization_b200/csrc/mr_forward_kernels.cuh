@@ -459,7 +459,7 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
 // because extrapolated blur-ring faces reach |w| in the hundreds, where float32 cannot
 // hold them to 1e-5.  The squared distance only needs float32: the nearest-edge
 // distance in face-local differences is good to ~1e-10 in NDC^2.
-template <bool PERSP>
+template <bool PERSP, bool EXACT = false>
 __device__ __forceinline__ void slot_outputs(const FaceGeom& g, double pxd, double pyd, float pxh, float pxl,
                                              float pyh, float pyl, float* z_out, float* b_out, float* d_out) {
     const double inv_area2 = (double)g.a.w + (double)g.b.w;
@@ -481,9 +481,14 @@ __device__ __forceinline__ void slot_outputs(const FaceGeom& g, double pxd, doub
     } else {
         z = w0 * z0 + w1 * z1 + w2 * z2;
     }
-    // squared distance to the nearest edge, float32, pixel - vertex differences
-    const float qx[3] = {(pxh - g.a.x) + pxl, (pxh - g.b.x) + pxl, (pxh - g.c.x) + pxl};
-    const float qy[3] = {(pyh - g.a.y) + pyl, (pyh - g.b.y) + pyl, (pyh - g.c.y) + pyl};
+    // squared distance to the nearest edge, float32, pixel - vertex differences; the segment
+    // parameter t takes the fast division (len2 is a normal float32 of an edge the setup kept:
+    // its error of a few ulp moves d2 far below the 1e-5 of the outputs)
+    // EXACT: the pixel centre is an exact float32 (H, W powers of two), its low part is 0
+    const float qx[3] = {EXACT ? pxh - g.a.x : (pxh - g.a.x) + pxl, EXACT ? pxh - g.b.x : (pxh - g.b.x) + pxl,
+                         EXACT ? pxh - g.c.x : (pxh - g.c.x) + pxl};
+    const float qy[3] = {EXACT ? pyh - g.a.y : (pyh - g.a.y) + pyl, EXACT ? pyh - g.b.y : (pyh - g.b.y) + pyl,
+                         EXACT ? pyh - g.c.y : (pyh - g.c.y) + pyl};
     const float vx[3] = {g.a.x, g.b.x, g.c.x}, vy[3] = {g.a.y, g.b.y, g.c.y};
     float d2 = FLT_MAX;
 #pragma unroll
@@ -491,7 +496,7 @@ __device__ __forceinline__ void slot_outputs(const FaceGeom& g, double pxd, doub
         const int k1 = k == 2 ? 0 : k + 1;
         const float ex = vx[k1] - vx[k], ey = vy[k1] - vy[k];
         const float len2 = fmaf(ex, ex, ey * ey);
-        const float t = len2 > 0.f ? __saturatef(fmaf(qx[k], ex, qy[k] * ey) * __frcp_rn(len2)) : 0.f;
+        const float t = len2 > 0.f ? __saturatef(__fdividef(fmaf(qx[k], ex, qy[k] * ey), len2)) : 0.f;
         const float rx = fmaf(-t, ex, qx[k]), ry = fmaf(-t, ey, qy[k]);
         d2 = fminf(d2, fmaf(rx, rx, ry * ry));
     }
@@ -507,7 +512,7 @@ __device__ __forceinline__ void slot_outputs(const FaceGeom& g, double pxd, doub
 // 16-byte loads and stores.  Pixels are taken in 16 x 16 tiles (one tile per 256
 // consecutive work items), so the threads of a block gather the faces of one screen
 // region and the geometry reads hit L1.
-template <int KC, bool PERSP, bool SIL, bool VEC>
+template <int KC, bool PERSP, bool SIL, bool VEC, bool EXACT>
 __global__ void __launch_bounds__(256, 4)
 k_epilogue(const FaceGeom* __restrict__ geom, const int64_t* __restrict__ p2f, int N, int H, int W, int K, float sigma,
            float* __restrict__ zbuf, float* __restrict__ bary, float* __restrict__ dists, float* __restrict__ alpha) {
@@ -552,7 +557,8 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int64_t* __restrict__ p2f, i
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     if (fk[u] >= 0) {
-                        slot_outputs<PERSP>(geom[fk[u]], pxd, pyd, pxh, pxl, pyh, pyl, &zz[u], &bb[3 * u], &dd[u]);
+                        slot_outputs<PERSP, EXACT>(geom[fk[u]], pxd, pyd, pxh, pxl, pyh, pyl, &zz[u], &bb[3 * u],
+                                                   &dd[u]);
                     } else {
                         zz[u] = -1.f; dd[u] = -1.f; bb[3 * u] = bb[3 * u + 1] = bb[3 * u + 2] = -1.f;
                     }
@@ -575,7 +581,7 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int64_t* __restrict__ p2f, i
                 const int fk = (int)p2f[s];
                 float zz, bb[3], dd;
                 if (fk >= 0) {
-                    slot_outputs<PERSP>(geom[fk], pxd, pyd, pxh, pxl, pyh, pyl, &zz, bb, &dd);
+                    slot_outputs<PERSP, EXACT>(geom[fk], pxd, pyd, pxh, pxl, pyh, pyl, &zz, bb, &dd);
                 } else {
                     zz = -1.f; dd = -1.f; bb[0] = bb[1] = bb[2] = -1.f;
                 }
@@ -606,15 +612,17 @@ void launch_fine(bool persp, bool exact, int nbins, cudaStream_t s, const float4
 }
 
 template <int KC>
-void launch_epilogue(bool persp, bool sil, bool vec, int N, int H, int W, cudaStream_t s, const FaceGeom* geom,
-                     const int64_t* p2f, int K, float sigma, float* zbuf, float* bary, float* dists,
-                     float* alpha) {
+void launch_epilogue(bool persp, bool sil, bool vec, bool exact, int N, int H, int W, cudaStream_t s,
+                     const FaceGeom* geom, const int64_t* p2f, int K, float sigma, float* zbuf, float* bary,
+                     float* dists, float* alpha) {
     const int64_t items = (int64_t)N * ceil_div(H, kBin) * ceil_div(W, kBin) * (kBin * kBin);
     const int grid = (int)std::min<int64_t>((items + 255) / 256, 148 * 32);
-#define MR_EPI(P, S, V) \
-    k_epilogue<KC, P, S, V><<<grid, 256, 0, s>>>(geom, p2f, N, H, W, K, sigma, zbuf, bary, dists, alpha)
-#define MR_EPI2(P, S) \
-    if (vec) MR_EPI(P, S, true); else MR_EPI(P, S, false)
+#define MR_EPI(P, S, V, X) \
+    k_epilogue<KC, P, S, V, X><<<grid, 256, 0, s>>>(geom, p2f, N, H, W, K, sigma, zbuf, bary, dists, alpha)
+#define MR_EPI2(P, S)                           \
+    if (vec && exact) MR_EPI(P, S, true, true); \
+    else if (vec) MR_EPI(P, S, true, false);    \
+    else MR_EPI(P, S, false, false)
     if (persp) {
         if (sil) { MR_EPI2(true, true); } else { MR_EPI2(true, false); }
     } else {
@@ -640,11 +648,12 @@ void dispatch_fine(int KC, bool persp, bool exact, int nbins, cudaStream_t s, co
 #undef MR_F
 }
 
-void dispatch_epilogue(int KC, bool persp, bool sil, bool vec_ok, int N, int H, int W, cudaStream_t s,
+void dispatch_epilogue(int KC, bool persp, bool sil, bool vec_ok, bool exact, int N, int H, int W, cudaStream_t s,
                        const FaceGeom* geom, const int64_t* p2f, int K, float sigma, float* zbuf,
                        float* bary, float* dists, float* alpha) {
     const bool vec = vec_ok && K == KC && (KC % 4) == 0;
-#define MR_E(KCV) launch_epilogue<KCV>(persp, sil, vec, N, H, W, s, geom, p2f, K, sigma, zbuf, bary, dists, alpha)
+#define MR_E(KCV) \
+    launch_epilogue<KCV>(persp, sil, vec, exact, N, H, W, s, geom, p2f, K, sigma, zbuf, bary, dists, alpha)
     switch (KC) {
         case 1: MR_E(1); break;
         case 2: MR_E(2); break;
@@ -846,8 +855,8 @@ inline cudaError_t fwd_enqueue_rest(const FwdPlan& P, const FwdBufs& B, int* lis
     if ((e = cudaGetLastError())) return e;
     {
         ProfScope ps(MR_STAGE_EPILOGUE, s);
-        dispatch_epilogue(P.KC, P.persp != 0, sil, vec_ok, P.N, P.H, P.W, s, B.geom, p2f, P.K, sigma, zbuf, bary,
-                          dists, alpha);
+        dispatch_epilogue(P.KC, P.persp != 0, sil, vec_ok, exact, P.N, P.H, P.W, s, B.geom, p2f, P.K, sigma, zbuf,
+                          bary, dists, alpha);
     }
     return cudaGetLastError();
 }

@@ -13,18 +13,18 @@ namespace mr {
 // because 1 - p_k = 1 / (1 + e_k).  P - 1 is carried as its own running value,
 // (P - 1)' = (P - 1) + e + (P - 1) e, so alpha = (P - 1) / P keeps full relative accuracy
 // for alpha near 0 (far blur ring), and one exponential per slot is the only
-// transcendental.  The exponent is capped at 80 and P - 1 at 1e30 (alpha is then 1 in
+// transcendental.  The exponent is capped at 2^115 and P - 1 at 1e30 (alpha is then 1 in
 // float32 either way), so an interior slot (e huge) next to a far one (e = 0) cannot form
 // inf * 0.
 template <int KC>
 __device__ __forceinline__ float silhouette_alpha(const float (&d)[KC], const bool (&valid)[KC], int K,
                                                   float sigma) {
-    const float inv_sigma = 1.f / sigma;
+    const float c = 1.4426950408889634f / sigma;   // log2(e) / sigma: e_k = 2^(-d_k c)
     float pm1 = 0.f;
 #pragma unroll
     for (int k = 0; k < KC; ++k)
         if (k < K && valid[k]) {
-            const float e = expf(fminf(-d[k] * inv_sigma, 80.f));
+            const float e = exp2f(fminf(-d[k] * c, 115.f));
             pm1 = fminf(fmaf(pm1, e, pm1 + e), 1e30f);
         }
     const float r = 1.f / (1.f + pm1);
