@@ -90,9 +90,10 @@ void scratch_free(void* p, cudaStream_t s) {
 
 namespace {
 __global__ void k_post_counts(const long long* __restrict__ total, const int* __restrict__ err,
-                              long long* __restrict__ out) {
+                              const int* __restrict__ extra, long long* __restrict__ out) {
     out[0] = *total;
     out[1] = err ? (long long)*err : 0;
+    out[2] = extra ? (long long)*extra : 0;
     __threadfence_system();
 }
 
@@ -125,8 +126,8 @@ Mailbox host_mailbox() {
     return g_mail.m[dev];
 }
 
-cudaError_t post_counts(const long long* total, const int* err, long long* out, cudaStream_t s) {
-    k_post_counts<<<1, 1, 0, s>>>(total, err, out);
+cudaError_t post_counts(const long long* total, const int* err, const int* extra, long long* out, cudaStream_t s) {
+    k_post_counts<<<1, 1, 0, s>>>(total, err, extra, out);
     return cudaGetLastError();
 }
 

@@ -111,8 +111,9 @@ struct Mailbox {
     long long* dev;
 };
 Mailbox host_mailbox();
-// Enqueues on s: out[0] = *total, out[1] = err ? *err : 0 (out: a Mailbox's dev pointer).
-cudaError_t post_counts(const long long* total, const int* err, long long* out, cudaStream_t s);
+// Enqueues on s: out[0] = *total, out[1] = err ? *err : 0, out[2] = extra ? *extra : 0 (out: a
+// Mailbox's dev pointer).
+cudaError_t post_counts(const long long* total, const int* err, const int* extra, long long* out, cudaStream_t s);
 
 // Scratch allocation on the caller's stream (stream-ordered pool).
 int scratch_alloc(void** p, size_t bytes, cudaStream_t s);

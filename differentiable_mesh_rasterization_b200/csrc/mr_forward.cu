@@ -59,14 +59,15 @@ int rasterize_impl(const float* verts, int64_t V, const int64_t* faces, int64_t 
         return code;
     };
     long long total = 0;
-    int herr = 0;
+    int herr = 0, empty = 0;
     const Mailbox mb = host_mailbox();
-    cudaError_t e = fwd_enqueue_count(P, B, verts, faces, prefix.data(), first, s, &total, &herr, mb.dev);
+    cudaError_t e = fwd_enqueue_count(P, B, verts, faces, prefix.data(), first, s, &total, &herr, &empty, mb.dev);
     if (e != cudaSuccess) return finish(cuda_fail(e, "forward: face setup and binning"));
     if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return finish(cuda_fail(e, "cudaStreamSynchronize"));
     if (mb.dev) {
         total = mb.host[0];
         herr = (int)mb.host[1];
+        empty = (int)mb.host[2];
     }
     if (total >= INT32_MAX) {
         set_error("bin lists too long (%lld entries)", total);
@@ -76,7 +77,7 @@ int rasterize_impl(const float* verts, int64_t V, const int64_t* faces, int64_t 
         rc = scratch_alloc(reinterpret_cast<void**>(&list), sizeof(int) * (size_t)total, s);
         if (rc != MR_OK) return finish(rc);
     }
-    e = fwd_enqueue_rest(P, B, list, total, sil, sigma, p2f, zbuf, bary, dists, alpha, s);
+    e = fwd_enqueue_rest(P, B, list, total, empty, sil, sigma, p2f, zbuf, bary, dists, alpha, s);
     if (e != cudaSuccess) return finish(cuda_fail(e, "forward: fine pass"));
     if (herr != 0) {
         set_error("a face references a vertex id outside [0, V=%lld); it was ignored", (long long)V);

@@ -514,8 +514,9 @@ __device__ __forceinline__ void slot_outputs(const FaceGeom& g, double pxd, doub
 // region and the geometry reads hit L1.
 template <int KC, bool PERSP, bool SIL, bool VEC, bool EXACT>
 __global__ void __launch_bounds__(256, 4)
-k_epilogue(const FaceGeom* __restrict__ geom, const int64_t* __restrict__ p2f, int N, int H, int W, int K, float sigma,
-           float* __restrict__ zbuf, float* __restrict__ bary, float* __restrict__ dists, float* __restrict__ alpha) {
+k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ offsets, int64_t* __restrict__ p2f, int N,
+           int H, int W, int K, float sigma, float* __restrict__ zbuf, float* __restrict__ bary,
+           float* __restrict__ dists, float* __restrict__ alpha) {
     static_assert(kBin == 16, "the tile arithmetic below takes 16 x 16 tiles");
     const int tw = (W + kBin - 1) / kBin, th = (H + kBin - 1) / kBin;
     const int64_t items = (int64_t)N * th * tw * (kBin * kBin);
@@ -540,6 +541,8 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int64_t* __restrict__ p2f, i
         }
         const int i = ty * kBin + (r >> 4), j = tx * kBin + (r & 15);
         if (ragged && (i >= H || j >= W)) continue;
+        // a tile is a bin: the fine pass did not run for an empty one, whose pixels get -1 here
+        const bool empty = offsets[(tile + 1) * kDepthBuckets] == offsets[tile * kDepthBuckets];
         const int64_t pix = (n * H + i) * W + j;
         const double pxd = -1.0 + (2.0 * j + 1.0) / W;
         const double pyd = 1.0 - (2.0 * i + 1.0) / H;
@@ -550,8 +553,14 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int64_t* __restrict__ p2f, i
         if (VEC) {
 #pragma unroll
             for (int k4 = 0; k4 < KC; k4 += 4) {
-                const longlong2 fa = reinterpret_cast<const longlong2*>(p2f + pix * KC + k4)[0];
-                const longlong2 fb = reinterpret_cast<const longlong2*>(p2f + pix * KC + k4)[1];
+                longlong2 fa = make_longlong2(-1, -1), fb = fa;
+                if (empty) {
+                    reinterpret_cast<longlong2*>(p2f + pix * KC + k4)[0] = fa;
+                    reinterpret_cast<longlong2*>(p2f + pix * KC + k4)[1] = fb;
+                } else {
+                    fa = reinterpret_cast<const longlong2*>(p2f + pix * KC + k4)[0];
+                    fb = reinterpret_cast<const longlong2*>(p2f + pix * KC + k4)[1];
+                }
                 const int fk[4] = {(int)fa.x, (int)fa.y, (int)fb.x, (int)fb.y};
                 float zz[4], bb[12], dd[4];
 #pragma unroll
@@ -578,7 +587,8 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int64_t* __restrict__ p2f, i
             for (int k = 0; k < KC; ++k) {
                 if (k >= K) break;
                 const int64_t s = pix * K + k;
-                const int fk = (int)p2f[s];
+                if (empty) p2f[s] = -1;
+                const int fk = empty ? -1 : (int)p2f[s];
                 float zz, bb[3], dd;
                 if (fk >= 0) {
                     slot_outputs<PERSP, EXACT>(geom[fk], pxd, pyd, pxh, pxl, pyh, pyl, &zz, bb, &dd);
@@ -613,12 +623,12 @@ void launch_fine(bool persp, bool exact, int nbins, cudaStream_t s, const float4
 
 template <int KC>
 void launch_epilogue(bool persp, bool sil, bool vec, bool exact, int N, int H, int W, cudaStream_t s,
-                     const FaceGeom* geom, const int64_t* p2f, int K, float sigma, float* zbuf, float* bary,
-                     float* dists, float* alpha) {
+                     const FaceGeom* geom, const int* offsets, int64_t* p2f, int K, float sigma, float* zbuf,
+                     float* bary, float* dists, float* alpha) {
     const int64_t items = (int64_t)N * ceil_div(H, kBin) * ceil_div(W, kBin) * (kBin * kBin);
     const int grid = (int)std::min<int64_t>((items + 255) / 256, 148 * 64);   // 148 x 64: 0.425 -> 0.420 ms
 #define MR_EPI(P, S, V, X) \
-    k_epilogue<KC, P, S, V, X><<<grid, 256, 0, s>>>(geom, p2f, N, H, W, K, sigma, zbuf, bary, dists, alpha)
+    k_epilogue<KC, P, S, V, X><<<grid, 256, 0, s>>>(geom, offsets, p2f, N, H, W, K, sigma, zbuf, bary, dists, alpha)
 #define MR_EPI2(P, S)                           \
     if (vec && exact) MR_EPI(P, S, true, true); \
     else if (vec) MR_EPI(P, S, true, false);    \
@@ -649,11 +659,11 @@ void dispatch_fine(int KC, bool persp, bool exact, int nbins, cudaStream_t s, co
 }
 
 void dispatch_epilogue(int KC, bool persp, bool sil, bool vec_ok, bool exact, int N, int H, int W, cudaStream_t s,
-                       const FaceGeom* geom, const int64_t* p2f, int K, float sigma, float* zbuf,
+                       const FaceGeom* geom, const int* offsets, int64_t* p2f, int K, float sigma, float* zbuf,
                        float* bary, float* dists, float* alpha) {
     const bool vec = vec_ok && K == KC && (KC % 4) == 0;
 #define MR_E(KCV) \
-    launch_epilogue<KCV>(persp, sil, vec, exact, N, H, W, s, geom, p2f, K, sigma, zbuf, bary, dists, alpha)
+    launch_epilogue<KCV>(persp, sil, vec, exact, N, H, W, s, geom, offsets, p2f, K, sigma, zbuf, bary, dists, alpha)
     switch (KC) {
         case 1: MR_E(1); break;
         case 2: MR_E(2); break;
@@ -785,12 +795,14 @@ inline FwdBufs fwd_bufs(char* ws, const FwdPlan& P) {
 inline int pair_blocks(int64_t pairs) { return (int)std::min<int64_t>((pairs + 255) / 256, 148 * 16); }
 
 // Up to the bin counts: per-mesh arrays to the device, clears, face setup (with the
-// images' key ranges), bin count and scan, and the read-back of the list total and the
-// error word (valid after the stream is synchronised): written by a kernel into mailbox
-// (a Mailbox's dev pointer) when one is given, else copied into host_total / host_err.
+// images' key ranges), bin count and scan, the bins' longest-first order, and the read-back
+// of the list total, the error word and the number of empty bins (valid after the stream is
+// synchronised): written by a kernel into mailbox (a Mailbox's dev pointer, words 0-2) when
+// one is given, else copied into host_total / host_err / host_empty.
 inline cudaError_t fwd_enqueue_count(const FwdPlan& P, const FwdBufs& B, const float* verts, const int64_t* faces,
                                      const int64_t* host_prefix, const int64_t* host_first, cudaStream_t s,
-                                     long long* host_total, int* host_err, long long* mailbox = nullptr) {
+                                     long long* host_total, int* host_err, int* host_empty,
+                                     long long* mailbox = nullptr) {
     cudaError_t e;
     if ((e = cudaMemcpyAsync(B.prefix, host_prefix, sizeof(int64_t) * (P.N + 1), cudaMemcpyHostToDevice, s))) return e;
     if ((e = cudaMemcpyAsync(B.first, host_first, sizeof(int64_t) * P.N, cudaMemcpyHostToDevice, s))) return e;
@@ -828,15 +840,20 @@ inline cudaError_t fwd_enqueue_count(const FwdPlan& P, const FwdBufs& B, const f
         k_bin_order<<<og, 256, 0, s>>>(B.offsets, P.nbins, B.hist, B.hist + kLenClasses, B.order);
     }
     if ((e = cudaGetLastError())) return e;
-    if (mailbox) return post_counts(B.total, B.err, mailbox, s);
+    // hist[0]: the bins of length class 0, i.e. the empty ones (they come last in the order)
+    if (mailbox) return post_counts(B.total, B.err, B.hist, mailbox, s);
     if ((e = cudaMemcpyAsync(host_total, B.total, sizeof(long long), cudaMemcpyDeviceToHost, s))) return e;
+    if ((e = cudaMemcpyAsync(host_empty, B.hist, sizeof(int), cudaMemcpyDeviceToHost, s))) return e;
     return cudaMemcpyAsync(host_err, B.err, sizeof(int), cudaMemcpyDeviceToHost, s);
 }
 
 // Bin fill into `list` (total entries), fine pass and epilogue.
-inline cudaError_t fwd_enqueue_rest(const FwdPlan& P, const FwdBufs& B, int* list, long long total, bool sil,
-                                    float sigma, int64_t* p2f, float* zbuf, float* bary, float* dists, float* alpha,
-                                    cudaStream_t s) {
+// The fine pass runs one CTA per non-empty bin (the first nbins - empty entries of the
+// longest-first order); the epilogue writes the padding of the empty bins' pixels, their
+// pix_to_face included.
+inline cudaError_t fwd_enqueue_rest(const FwdPlan& P, const FwdBufs& B, int* list, long long total, int empty,
+                                    bool sil, float sigma, int64_t* p2f, float* zbuf, float* bary, float* dists,
+                                    float* alpha, cudaStream_t s) {
     cudaError_t e;
     if (total > 0) {
         if ((e = cudaMemsetAsync(B.counts, 0, sizeof(int) * (size_t)P.nslots, s))) return e;
@@ -847,16 +864,18 @@ inline cudaError_t fwd_enqueue_rest(const FwdPlan& P, const FwdBufs& B, int* lis
     }
     const bool vec_ok = aligned16(p2f) && aligned16(zbuf) && aligned16(bary) && aligned16(dists);
     const bool exact = (P.H & (P.H - 1)) == 0 && (P.W & (P.W - 1)) == 0;
+    const int busy = P.nbins - std::min(std::max(empty, 0), P.nbins);
     {
         ProfScope ps(MR_STAGE_FINE, s);
-        dispatch_fine(P.KC, P.persp != 0, exact, P.nbins, s, B.fconst, B.box, B.order, B.offsets, list, P.nbx, P.nby,
-                      P.H, P.W, P.K, P.blur, aligned16(p2f), p2f);
+        if (busy > 0)
+            dispatch_fine(P.KC, P.persp != 0, exact, busy, s, B.fconst, B.box, B.order, B.offsets, list, P.nbx,
+                          P.nby, P.H, P.W, P.K, P.blur, aligned16(p2f), p2f);
     }
     if ((e = cudaGetLastError())) return e;
     {
         ProfScope ps(MR_STAGE_EPILOGUE, s);
-        dispatch_epilogue(P.KC, P.persp != 0, sil, vec_ok, exact, P.N, P.H, P.W, s, B.geom, p2f, P.K, sigma, zbuf,
-                          bary, dists, alpha);
+        dispatch_epilogue(P.KC, P.persp != 0, sil, vec_ok, exact, P.N, P.H, P.W, s, B.geom, B.offsets, p2f, P.K,
+                          sigma, zbuf, bary, dists, alpha);
     }
     return cudaGetLastError();
 }

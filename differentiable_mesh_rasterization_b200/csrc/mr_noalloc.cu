@@ -81,8 +81,8 @@ int rasterize_noalloc(const float* verts, int64_t V, const int64_t* faces, int64
     const FwdBufs B = fwd_bufs(ws, P);
     int* list = reinterpret_cast<int*>(ws + P.bytes);     // the bin lists follow the fixed block
     long long total = 0;
-    int herr = 0;
-    MR_CUDA(fwd_enqueue_count(P, B, verts, faces, prefix.data(), first, s, &total, &herr));
+    int herr = 0, empty = 0;
+    MR_CUDA(fwd_enqueue_count(P, B, verts, faces, prefix.data(), first, s, &total, &herr, &empty));
     MR_CUDA(cudaStreamSynchronize(s));
     if (total < 0 || P.bytes + sizeof(int) * (size_t)total > (size_t)MR_NOALLOC_SCRATCH_BYTES) {
         set_error("mr_rasterize_fwd_noalloc: the bin lists need %lld entries, more than the %zu left of the "
@@ -90,7 +90,7 @@ int rasterize_noalloc(const float* verts, int64_t V, const int64_t* faces, int64
                   ((size_t)MR_NOALLOC_SCRATCH_BYTES - P.bytes) / sizeof(int), MR_NOALLOC_SCRATCH_BYTES);
         return MR_ERR_ARG;
     }
-    MR_CUDA(fwd_enqueue_rest(P, B, list, total, false, 0.f, p2f, zbuf, bary, dists, nullptr, s));
+    MR_CUDA(fwd_enqueue_rest(P, B, list, total, empty, false, 0.f, p2f, zbuf, bary, dists, nullptr, s));
     if (herr != 0) {
         set_error("a face references a vertex id outside [0, V=%lld); it was ignored", (long long)V);
         return MR_ERR_DEVICE;

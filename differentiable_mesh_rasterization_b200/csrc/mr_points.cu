@@ -474,7 +474,7 @@ int mr_rasterize_points_fwd(const float* points, int64_t P, const int64_t* cloud
     // word is at hand
     const Mailbox mb = host_mailbox();
     if (e == cudaSuccess)
-        e = mb.dev ? post_counts(total_d, nullptr, mb.dev, s)
+        e = mb.dev ? post_counts(total_d, nullptr, nullptr, mb.dev, s)
                    : cudaMemcpyAsync(&total, total_d, sizeof(long long), cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e == cudaSuccess && mb.dev) total = mb.host[0];
