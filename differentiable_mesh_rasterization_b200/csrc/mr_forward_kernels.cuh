@@ -522,6 +522,7 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ offsets, i
     const int64_t items = (int64_t)N * th * tw * (kBin * kBin);
     const bool small = (int64_t)N * th * tw <= 0x7fffffff;   // tile ids fit 32-bit division
     const bool ragged = (H % kBin) != 0 || (W % kBin) != 0;   // some tiles stick out of the image
+    const double inv_w = 1.0 / W, inv_h = 1.0 / H;
     for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < items;
          it += (int64_t)gridDim.x * blockDim.x) {
         const int64_t tile = it >> 8;                           // kBin * kBin = 256 items per tile
@@ -541,11 +542,40 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ offsets, i
         }
         const int i = ty * kBin + (r >> 4), j = tx * kBin + (r & 15);
         if (ragged && (i >= H || j >= W)) continue;
-        // a tile is a bin: the fine pass did not run for an empty one, whose pixels get -1 here
-        const bool empty = offsets[(tile + 1) * kDepthBuckets] == offsets[tile * kDepthBuckets];
         const int64_t pix = (n * H + i) * W + j;
-        const double pxd = -1.0 + (2.0 * j + 1.0) / W;
-        const double pyd = 1.0 - (2.0 * i + 1.0) / H;
+        // a tile is a bin: the fine pass did not run for an empty one, whose pixels get the
+        // padding here (-1 in every slot, alpha 0)
+        if (offsets[(tile + 1) * kDepthBuckets] == offsets[tile * kDepthBuckets]) {
+            if (VEC) {
+                const float4 m1 = make_float4(-1.f, -1.f, -1.f, -1.f);
+#pragma unroll
+                for (int k4 = 0; k4 < KC; k4 += 4) {
+                    const int64_t s = pix * KC + k4;
+                    reinterpret_cast<longlong2*>(p2f + s)[0] = make_longlong2(-1, -1);
+                    reinterpret_cast<longlong2*>(p2f + s)[1] = make_longlong2(-1, -1);
+                    *reinterpret_cast<float4*>(zbuf + s) = m1;
+                    *reinterpret_cast<float4*>(dists + s) = m1;
+                    float4* bp = reinterpret_cast<float4*>(bary + 3 * s);
+                    bp[0] = m1;
+                    bp[1] = m1;
+                    bp[2] = m1;
+                }
+            } else {
+                for (int k = 0; k < K; ++k) {
+                    const int64_t s = pix * K + k;
+                    p2f[s] = -1;
+                    zbuf[s] = -1.f;
+                    dists[s] = -1.f;
+                    bary[3 * s] = bary[3 * s + 1] = bary[3 * s + 2] = -1.f;
+                }
+            }
+            if (SIL) alpha[pix] = 0.f;
+            continue;
+        }
+        // EXACT (H, W powers of two): 1/W and 1/H are exact, so the centre is one exact
+        // product instead of a division (the same float64 value)
+        const double pxd = EXACT ? (double)(2 * j + 1 - W) * inv_w : -1.0 + (2.0 * j + 1.0) / W;
+        const double pyd = EXACT ? (double)(H - 2 * i - 1) * inv_h : 1.0 - (2.0 * i + 1.0) / H;
         const float pxh = (float)pxd, pyh = (float)pyd;
         const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
         float dsil[KC];
@@ -553,14 +583,8 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ offsets, i
         if (VEC) {
 #pragma unroll
             for (int k4 = 0; k4 < KC; k4 += 4) {
-                longlong2 fa = make_longlong2(-1, -1), fb = fa;
-                if (empty) {
-                    reinterpret_cast<longlong2*>(p2f + pix * KC + k4)[0] = fa;
-                    reinterpret_cast<longlong2*>(p2f + pix * KC + k4)[1] = fb;
-                } else {
-                    fa = reinterpret_cast<const longlong2*>(p2f + pix * KC + k4)[0];
-                    fb = reinterpret_cast<const longlong2*>(p2f + pix * KC + k4)[1];
-                }
+                const longlong2 fa = reinterpret_cast<const longlong2*>(p2f + pix * KC + k4)[0];
+                const longlong2 fb = reinterpret_cast<const longlong2*>(p2f + pix * KC + k4)[1];
                 const int fk[4] = {(int)fa.x, (int)fa.y, (int)fb.x, (int)fb.y};
                 float zz[4], bb[12], dd[4];
 #pragma unroll
@@ -587,8 +611,7 @@ k_epilogue(const FaceGeom* __restrict__ geom, const int* __restrict__ offsets, i
             for (int k = 0; k < KC; ++k) {
                 if (k >= K) break;
                 const int64_t s = pix * K + k;
-                if (empty) p2f[s] = -1;
-                const int fk = empty ? -1 : (int)p2f[s];
+                const int fk = (int)p2f[s];
                 float zz, bb[3], dd;
                 if (fk >= 0) {
                     slot_outputs<PERSP, EXACT>(geom[fk], pxd, pyd, pxh, pxl, pyh, pyl, &zz, bb, &dd);
