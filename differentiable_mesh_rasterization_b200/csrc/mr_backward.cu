@@ -277,13 +277,20 @@ k_sil_raster_bwd(const float* __restrict__ verts, int64_t V, const int64_t* __re
         bool v[KC];
         int64_t fk[KC];
         int ebits = 0;   // error flags of this pixel, set in the device word once at the end
+        bool work = false;
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
-            const bool in = live && k < K;
-            fk[k] = in ? p2f[q * K + k] : -1;
+            fk[k] = live && k < K ? p2f[q * K + k] : -1;
+            work |= fk[k] != -1;
+        }
+        // a warp of pixels with every slot empty (background) has nothing to add: skip its
+        // distance and dL/dalpha reads and the arithmetic
+        if (!__any_sync(0xffffffffu, work)) continue;
+#pragma unroll
+        for (int k = 0; k < KC; ++k) {
             if (fk[k] < -1) ebits |= kErrSlotIndex;
             v[k] = fk[k] >= 0;
-            d[k] = in ? dists[q * K + k] : 0.f;
+            d[k] = live && k < K ? dists[q * K + k] : 0.f;
         }
         const float ga = live ? grad_alpha[q] : 0.f;
         silhouette_grad<KC>(d, v, K, sigma, ga, g);
