@@ -37,23 +37,26 @@ template <int KC>
 __device__ __forceinline__ void silhouette_grad(const float (&d)[KC], const bool (&valid)[KC], int K, float sigma,
                                                 float grad_alpha, float (&g)[KC]) {
     float q[KC], p[KC];
+    const float inv_sigma = 1.f / sigma;
+    const float c = 1.4426950408889634f * inv_sigma;   // log2(e) / sigma
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
         // one exponential per slot: with e = exp(-|x|) and r = 1 / (1 + e) the two
-        // sigmoids are r and e * r, assigned by the sign of x (no overflow either way)
-        const float x = d[k] / sigma;
-        const float e = expf(-fabsf(x));
-        const float r = 1.f / (1.f + e);
-        q[k] = x >= 0.f ? r : e * r;    // 1 - p_k
-        p[k] = x >= 0.f ? e * r : r;
+        // sigmoids are r and e * r, assigned by the sign of x (no overflow either way);
+        // 1 + e lies in (1, 2], where the fast reciprocal is good to about an ulp
+        const float e = exp2f(-fabsf(d[k]) * c);
+        const float r = __fdividef(1.f, 1.f + e);
+        q[k] = d[k] >= 0.f ? r : e * r;    // 1 - p_k
+        p[k] = d[k] >= 0.f ? e * r : r;
     }
+    const float ga = -grad_alpha * inv_sigma;
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
         float others = 1.f;
 #pragma unroll
         for (int j = 0; j < KC; ++j)
             if (j != k && j < K && valid[j]) others *= q[j];
-        g[k] = (k < K && valid[k]) ? -grad_alpha * others * p[k] * q[k] / sigma : 0.f;
+        g[k] = (k < K && valid[k]) ? ga * others * p[k] * q[k] : 0.f;
     }
 }
 
