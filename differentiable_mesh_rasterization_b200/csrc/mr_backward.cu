@@ -211,10 +211,11 @@ k_raster_bwd(const float* __restrict__ verts, int64_t V, const int64_t* __restri
              const float* __restrict__ gb, const float* __restrict__ gd, float4* __restrict__ acc,
              int* __restrict__ err) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const double inv_w = 1.0 / W, inv_h = 1.0 / H;
     for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < npix; q += stride) {
-        const int64_t rem = q % ((int64_t)H * W);
-        const int i = (int)(rem / W), j = (int)(rem % W);
-        const double pxd = -1.0 + (2.0 * j + 1.0) / W, pyd = 1.0 - (2.0 * i + 1.0) / H;
+        int i, j;
+        pixel_rc(q, H, W, i, j);
+        const double pxd = pixel_x(j, W, inv_w), pyd = pixel_y(i, H, inv_h);
         const float pxh = (float)pxd, pyh = (float)pyd;
         const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
 #pragma unroll

@@ -123,6 +123,30 @@ void scratch_free(void* p, cudaStream_t s);
 // SM of the 148.
 inline int grid_for(int64_t n) { return (int)(n < 148 * 32 * 256 ? (n + 255) / 256 : 148 * 32); }
 
+// Row i and column j of flat pixel index q (images of H x W, row-major): 32-bit division
+// when q fits (64-bit division costs several times more).
+__device__ __forceinline__ void pixel_rc(int64_t q, int H, int W, int& i, int& j) {
+    if (q <= 0x7fffffff) {
+        const unsigned r = (unsigned)q % ((unsigned)H * (unsigned)W);
+        i = (int)(r / (unsigned)W);
+        j = (int)(r - (unsigned)i * (unsigned)W);
+    } else {
+        const int64_t r = q % ((int64_t)H * W);
+        i = (int)(r / W);
+        j = (int)(r % W);
+    }
+}
+
+// Centre of pixel column j in NDC, -1 + (2j + 1) / W, in float64; inv_w = 1.0 / W.  For W a
+// power of two 1/W is exact and so is the product: the same value without a division.
+__device__ __forceinline__ double pixel_x(int j, int W, double inv_w) {
+    return (W & (W - 1)) == 0 ? (double)(2 * j + 1 - W) * inv_w : -1.0 + (2.0 * j + 1.0) / W;
+}
+// Centre of pixel row i, 1 - (2i + 1) / H.
+__device__ __forceinline__ double pixel_y(int i, int H, double inv_h) {
+    return (H & (H - 1)) == 0 ? (double)(H - 2 * i - 1) * inv_h : 1.0 - (2.0 * i + 1.0) / H;
+}
+
 // 16-byte loads and stores of N consecutive values (N a multiple of 4 floats or 2 int64;
 // the address 16-byte aligned).
 template <int N>
