@@ -137,6 +137,31 @@ def test_no_faces_at_all():
     assert torch.all(alpha == 0)
 
 
+@pytest.mark.parametrize("H,W,K", [(64, 64, 4), (48, 80, 4), (37, 53, 2), (64, 64, 3)])
+def test_every_output_element_is_written(H, W, K):
+    """Outputs pre-filled with a sentinel: a small triangle leaves most 16 x 16 bins empty
+    (the fine pass skips those and the epilogue pads them) and the rest partly covered; the
+    vector path (K = 4, H and W multiples of 16) and the general one both write every
+    element, and the results equal a call into fresh buffers."""
+    v, f = to_dev(*soup([[[-0.2, -0.1, 2.0], [0.15, -0.2, 2.1], [0.0, 0.25, 2.2]]]))
+    lib = mr.load_library()
+    ref = mr.rasterize_fwd(v, f, [0], [1], H, W, 2e-3, K, sigma=1e-4)
+    p2f = torch.full((1, H, W, K), 123456, dtype=torch.int64, device="cuda")
+    zbuf, dists = (torch.full((1, H, W, K), 7.5, device="cuda") for _ in range(2))
+    bary = torch.full((1, H, W, K, 3), 7.5, device="cuda")
+    alpha = torch.full((1, H, W), 7.5, device="cuda")
+    first, num = np.array([0], np.int64), np.array([1], np.int64)
+    rc = lib.mr_rasterize_silhouette_fwd(v.data_ptr(), v.shape[0], f.data_ptr(), f.shape[0], first.ctypes.data,
+                                         num.ctypes.data, 1, H, W, 2e-3, K, 0, 1e-4, p2f.data_ptr(),
+                                         zbuf.data_ptr(), bary.data_ptr(), dists.data_ptr(), alpha.data_ptr(),
+                                         torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert rc == 0
+    for got, want in zip((p2f, zbuf, bary, dists, alpha), ref):
+        assert torch.equal(got, want)
+    assert (ref[0] >= 0).any() and (ref[0][..., 0] == -1).float().mean() > 0.5
+
+
 def test_face_covering_the_whole_image_and_crowded_bin(oracle_mod):
     H = W = 64
     big = [[-3.0, -3.0, 2.5], [3.0, -3.0, 2.5], [0.0, 3.0, 2.6]]
