@@ -496,10 +496,53 @@ def next_row_oracle_baselines(batch, rows_wanted):
         dt = time.perf_counter() - t0
         out["knn"] = {"value": float(np.sum(n1 * kb.num2)) / dt, "unit": "pairs/s", "cores": 1, "kind": "oracle",
                       "seconds": dt, "sample": f"the first 50 queries of each of the {kb.N} clouds"}
+    if "subpixel" in rows_wanted:
+        sb = syn.make_batch(4)
+        sw = sb.workload
+        srow = np.array([sw.H // 2])
+        spix = (srow[:, None] * sw.W + np.arange(sw.W)[None, :]).reshape(-1)
+        t0 = time.perf_counter()
+        oracle.rasterize_fwd(sb.verts, sb.faces, sb.mesh_to_face_first_idx, sb.num_faces_per_mesh, sw.H, sw.W,
+                             np.float32(sw.blur_radius), sw.K, sw.perspective_correct, pixels=spix, exempt=False)
+        dt = time.perf_counter() - t0
+        out["subpixel_1024px"] = {"value": count_samples(sb, srow) / dt, "unit": "pixel-face samples/s",
+                                  "cores": cores, "kind": "oracle", "seconds": dt,
+                                  "sample": "the middle row of the image (forward)"}
     return out
 
 
 KNN_C_PAIR = 7       # FP32 instructions per (query, reference) pair for D=3: 3 FADD, 3 FFMA, 1 compare
+
+
+def subpixel_step_timing(mr, torch, dev, stream, flush, args, peak_alu, hbm_peak, hbm_note):
+    """The single-image sub-pixel workload (one 1024x1024 image of an icosphere of level 7:
+    327,680 faces, most smaller than a pixel; K=8, blur 1e-5, perspective-correct; hard
+    rasterization, so a step is the forward): step time, and the fine pass and the fine pass
+    with its epilogue against the same rooflines as the main workload."""
+    from differentiable_mesh_rasterization_b200 import synthetic as syn
+    batch = syn.make_batch(4)
+    w = batch.workload
+    verts = torch.from_numpy(batch.verts).to(dev)
+    faces = torch.from_numpy(batch.faces).to(dev)
+    first, num = batch.mesh_to_face_first_idx, batch.num_faces_per_mesh
+
+    def step():
+        mr.rasterize_fwd(verts, faces, first, num, w.H, w.W, w.blur_radius, w.K, w.perspective_correct)
+
+    steps = max(3, args.steps // 5)
+    ms, stages = _timed_steps(mr, torch, dev, stream, flush, steps, step)
+    samples = float(count_samples(batch))
+    npix = batch.N * w.H * w.W
+    fine_s, epi_s = stages["fine"] / 1e3, stages["epilogue"] / 1e3
+    achieved = samples * C_TEST / fine_s / 1e12
+    return {"workload": w.name, "ms_per_step": ms, "samples_per_s": samples / (ms / 1e3),
+            "mpix_per_s": npix / (ms / 1e3) / 1e6, "samples_per_step": samples, "steps": steps,
+            "stages": {s: {"ms_per_step": t} for s, t in stages.items()},
+            "roofline": {"bound": "alu", "kernel": "k_fine", "achieved": achieved, "peak": peak_alu,
+                         "unit": "T FP32-inst/s", "frac": achieved / peak_alu, "c_test": C_TEST,
+                         "a3a4": a3a4_roofline(samples, fine_s, epi_s, npix * 28 * w.K, peak_alu, hbm_peak,
+                                               hbm_note)},
+            "note": w.description + "; forward (hard rasterization); L2 flushed per step"}
 
 
 def knn_step_timing(mr, torch, dev, stream, flush, args, peak_alu):
@@ -566,8 +609,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-shading", action="store_true", help="skip the Gouraud, Phong, point-cloud and KNN measurements")
-    ap.add_argument("--rows", default="gouraud,phong,points,knn",
-                    help="comma-separated next-row measurements after the main step (gouraud, phong, points, knn)")
+    ap.add_argument("--rows", default="gouraud,phong,points,knn,subpixel",
+                    help="comma-separated next-row measurements after the main step (gouraud, phong, points, knn, "
+                         "subpixel: the one-image 1024x1024 workload of sub-pixel faces)")
     ap.add_argument("--split", action="store_true",
                     help="under torchrun, split ONE batch over the ranks by whole meshes, balanced by their "
                          "pixel-face samples (strong scaling), instead of one batch per rank (weak scaling)")
@@ -832,6 +876,9 @@ def main():
         rows["points_rgb"] = points_step_timing(mr, torch, dev, stream, flush, args, hbm_peak, hbm_note)
     if "knn" in args.rows:
         rows["knn"] = knn_step_timing(mr, torch, dev, stream, flush, args, peak_alu)
+    if "subpixel" in args.rows:
+        rows["subpixel_1024px"] = subpixel_step_timing(mr, torch, dev, stream, flush, args, peak_alu, hbm_peak,
+                                                       hbm_note)
     if rows:
         line["next_rows"] = rows
         if rank == 0 and not args.no_cpu_baseline:
