@@ -292,37 +292,26 @@ __global__ void k_bin_order(const int* __restrict__ offsets, int nbins, const in
 }
 
 // ------------------------------------------------------------------ fine pass
+// The K nearest candidates of a lane in registers, sorted by (key, face id).  Keys are held
+// as unsigned images that order like the float keys: without perspective correction the
+// keys are depths >= 0, whose bit patterns already do; with it they are negative, and
+// float_order maps them.  (key, face id) then compares as one unsigned 64-bit value: all K
+// compares first (independent of each other), then each slot takes its left neighbour, the
+// new entry or itself.  On the 64-image batch the fine pass took 1.483 instead of 1.548 ms
+// with this form over a serial chain of float compares with an id tie-break, results the
+// same bit for bit.
 template <int KC>
-__device__ __forceinline__ void topk_insert(float (&kk)[KC], int (&ff)[KC], float key, int fid) {
-#pragma unroll
-    for (int k = 0; k < KC; ++k) {
-        bool lt = key < kk[k] || (key == kk[k] && fid < ff[k]);
-        float tk = lt ? kk[k] : key;
-        int tf = lt ? ff[k] : fid;
-        kk[k] = lt ? key : kk[k];
-        ff[k] = lt ? fid : ff[k];
-        key = tk;
-        fid = tf;
-    }
-}
-
-// The same insertion for keys >= 0 (no perspective correction), whose float order is the
-// order of their bit patterns: (key, face id) compares as one unsigned 64-bit value, all K
-// compares first (independent of each other), then each slot takes its left neighbour,
-// the new entry or itself.  Same results bit for bit; on the 64-image batch the fine pass
-// takes 1.483 instead of 1.548 ms.
-template <int KC>
-__device__ __forceinline__ void topk_insert_bits(float (&kk)[KC], int (&ff)[KC], float key, int fid) {
-    const unsigned long long x = ((unsigned long long)__float_as_uint(key) << 32) | (unsigned)fid;
+__device__ __forceinline__ void topk_insert(unsigned (&kb)[KC], int (&ff)[KC], unsigned key, int fid) {
+    const unsigned long long x = ((unsigned long long)key << 32) | (unsigned)fid;
     bool c[KC];
 #pragma unroll
-    for (int k = 0; k < KC; ++k) c[k] = x < (((unsigned long long)__float_as_uint(kk[k]) << 32) | (unsigned)ff[k]);
+    for (int k = 0; k < KC; ++k) c[k] = x < (((unsigned long long)kb[k] << 32) | (unsigned)ff[k]);
 #pragma unroll
     for (int k = KC - 1; k > 0; --k) {
-        kk[k] = c[k - 1] ? kk[k - 1] : (c[k] ? key : kk[k]);
+        kb[k] = c[k - 1] ? kb[k - 1] : (c[k] ? key : kb[k]);
         ff[k] = c[k - 1] ? ff[k - 1] : (c[k] ? fid : ff[k]);
     }
-    kk[0] = c[0] ? key : kk[0];
+    kb[0] = c[0] ? key : kb[0];
     ff[0] = c[0] ? fid : ff[0];
 }
 
@@ -357,11 +346,12 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
     const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
     const unsigned lt_mask = (1u << lane) - 1u;
 
-    float kk[KC];
+    unsigned kb[KC];   // the keys' order images (see topk_insert); off-image lanes are never written
     int ff[KC];
+    const unsigned far_key = PERSP ? float_order(FLT_MAX) : __float_as_uint(FLT_MAX);
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
-        kk[k] = in_img ? FLT_MAX : (PERSP ? -FLT_MAX : 0.f);   // off-image lanes are never written
+        kb[k] = in_img ? far_key : 0u;
         ff[k] = INT_MAX;
     }
 
@@ -379,15 +369,9 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
         const FaceBox b = nbox;
         // tile depth cull: the farthest K-th key over the warp's pixels; a face whose lowest
         // key over its box lies beyond it cannot enter any lane's top K
-        float zfar;
-        if constexpr (!PERSP) {
-            // keys >= 0 order as their bit patterns: one warp reduction (off-image lanes give 0)
-            zfar = __uint_as_float(__reduce_max_sync(0xffffffffu, in_img ? __float_as_uint(kk[KC - 1]) : 0u));
-        } else {
-            zfar = in_img ? kk[KC - 1] : -FLT_MAX;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) zfar = fmaxf(zfar, __shfl_xor_sync(0xffffffffu, zfar, o));
-        }
+        // one warp reduction over the order images (off-image lanes give 0, the lowest)
+        const unsigned zfar_b = __reduce_max_sync(0xffffffffu, in_img ? kb[KC - 1] : 0u);
+        const float zfar = PERSP ? order_float(zfar_b) : __uint_as_float(zfar_b);
         const bool hit = base + lane < cnt && b.x0 <= tj0 + kWarpTileW - 1 && b.x1 >= tj0 &&
                          b.y0 <= ti0 + kWarpTileH - 1 && b.y1 >= ti0 && b.kmin <= zfar;
         if (base + 32 + lane < cnt) {
@@ -412,8 +396,8 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
             // admissible: in front of the camera and not behind the lane's K-th key.  Without
             // perspective the keys are depths >= 0, whose float order is their bit order,
             // so one unsigned compare does both (negative keys wrap to huge values).
-            const bool maybe = PERSP ? (key < 0.f && key <= kk[KC - 1])
-                                     : (__float_as_uint(key) <= __float_as_uint(kk[KC - 1]));
+            const unsigned kbits = PERSP ? float_order(key) : __float_as_uint(key);
+            const bool maybe = PERSP ? (key < 0.f && kbits <= kb[KC - 1]) : kbits <= kb[KC - 1];
             if (!__any_sync(0xffffffffu, maybe)) continue;
             const float4 e0 = slots[qi][2], e1 = slots[qi][3], e2 = slots[qi][4], q5 = slots[qi][5];
             const float c0 = fmaf(-e0.y, dx, fmaf(e0.x, dy, e0.z));
@@ -430,10 +414,7 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
             const float d2 = fmaf(o2, o2, c2 * c2);
             const bool inside = fminf(c0, fminf(c1, c2)) >= 0.f;
             const float dmin = fminf(d0, fminf(d1, d2));
-            if (maybe && (inside || dmin <= blur)) {
-                if constexpr (PERSP) topk_insert<KC>(kk, ff, key, __float_as_int(q5.y));
-                else topk_insert_bits<KC>(kk, ff, key, __float_as_int(q5.y));
-            }
+            if (maybe && (inside || dmin <= blur)) topk_insert<KC>(kb, ff, kbits, __float_as_int(q5.y));
         }
         __syncwarp();
     }
