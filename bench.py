@@ -39,8 +39,10 @@ C_TEST = 38                 # FP32 instructions per pixel-face test in this form
 FP32_LANES_PER_SM = 128
 L2_FLUSH_BYTES = 256 << 20
 KERNELS_PER_STAGE = {"silhouette_raster_bwd": 2,   # main kernel + (x, y) -> (x, y, z) copy
-                     "bin_scan": 5}                # tile scans, tile totals, tile prefixes added; the bins'
-                                                   # length histogram and longest-first order
+                     "bin_scan": 6}                # tile scans, tile totals, tile prefixes added; the bins'
+                                                   # length histogram and longest-first order; and right
+                                                   # after the stage the one-thread read-back of the list
+                                                   # total, error word and empty-bin count (k_post_counts)
 
 
 # ----------------------------------------------------------------------------- counting
