@@ -83,8 +83,9 @@ __device__ __forceinline__ void phong_point_bwd(f3 P, f3 N, f3 c, f3 g, const Ph
             g.z * fmaf(Q.dif[2], S.td, Q.amb[2]));
     const float g_td = fmaf(g.x, Q.dif[0] * c.x, fmaf(g.y, Q.dif[1] * c.y, g.z * Q.dif[2] * c.z));
     const float g_ts = fmaf(g.x, Q.spe[0], fmaf(g.y, Q.spe[1], g.z * Q.spe[2]));
-    // d rv^s / d rv = s rv^(s - 1) = s ts / rv (rv > 0 where the term is on)
-    const float g_rv = S.shiny ? g_ts * Q.shine * powf(S.rv, Q.shine - 1.f) : 0.f;
+    // d rv^s / d rv = s rv^(s - 1) = s ts / rv (rv > 0 where the term is on): the power
+    // already formed for the colour, divided once, instead of a second powf
+    const float g_rv = S.shiny ? g_ts * Q.shine * __fdividef(S.ts, S.rv) : 0.f;
     const float g_cos = (S.lit ? g_td : 0.f) + 2.f * g_rv * S.nv;
     const float g_nv = 2.f * g_rv * S.cos;
     const float g_lv = -g_rv;
