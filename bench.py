@@ -694,7 +694,7 @@ def main():
     torch.cuda.synchronize(dev)
     torch.cuda.reset_peak_memory_stats(dev)
     mr.scratch_peak(dev, reset=True)
-    mr.profile_enable(True)
+    mr.profile_enable(False)
     with ClockSampler(uuid or None) as clocks:
         for k in range(args.steps):
             flush.zero_()
@@ -702,11 +702,20 @@ def main():
             step()
             ends[k].record(stream)
         torch.cuda.synchronize(dev)
-    mr.profile_enable(False)
     memory = {"scratch_peak_bytes": mr.scratch_peak(dev), "torch_peak_bytes": int(torch.cuda.max_memory_allocated(dev)),
               "l2_flush_bytes": L2_FLUSH_BYTES,
               "note": "over the timed steps: the library's scratch (high-water mark of the device's default "
                       "memory pool) and torch's allocations (inputs, the outputs of each step, the L2-flush buffer)"}
+    # Per-stage times (and from them the kernels' rooflines and the launch count): a second
+    # pass of the same steps with the library's stage events on.  They are kept out of the
+    # timed steps above, where their 14 event records per step would add about 0.04 ms.
+    mr.profile_read()
+    mr.profile_enable(True)
+    for k in range(args.steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    mr.profile_enable(False)
     if world > 1:
         dist.barrier()
     stages = mr.profile_read()
@@ -857,6 +866,8 @@ def main():
             "config": workload_config(w, args), "mpix_per_s": mpix,
             "samples_per_step": tot_samples,
             "stages_ms_per_step": {k: v[0] / args.steps for k, v in stages.items() if v[1]},
+            "stages_note": ("per-stage times from a second pass of the same steps with the library's CUDA events "
+                            "around each stage on the launching stream; the timed steps run without them"),
             "roofline": roof,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": float(te[0]) / max(args.e2e_steps, 1), "pipelined": True,

@@ -1,5 +1,6 @@
 // Host-side plumbing of the C ABI: error reporting, stream-ordered scratch, the device
 // error word and the status query.
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdint>
@@ -124,6 +125,36 @@ Mailbox host_mailbox() {
         }
     }
     return g_mail.m[dev];
+}
+
+namespace {
+struct StagingSlots {
+    void* p[64] = {};
+    size_t cap[64] = {};
+};
+thread_local StagingSlots g_stage;
+}  // namespace
+
+void* host_staging(size_t bytes) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (g_stage.cap[dev] < bytes) {
+        if (g_stage.p[dev]) cudaFreeHost(g_stage.p[dev]);
+        g_stage.p[dev] = nullptr;
+        g_stage.cap[dev] = 0;
+        const size_t want = std::max<size_t>(bytes, 4096);
+        void* h = nullptr;
+        if (cudaHostAlloc(&h, want, cudaHostAllocPortable) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        g_stage.p[dev] = h;
+        g_stage.cap[dev] = want;
+    }
+    return g_stage.p[dev];
 }
 
 cudaError_t post_counts(const long long* total, const int* err, const int* extra, long long* out, cudaStream_t s) {

@@ -111,6 +111,14 @@ struct Mailbox {
     long long* dev;
 };
 Mailbox host_mailbox();
+// Pinned host memory of at least `bytes`, one growing buffer per calling thread and
+// device, or nullptr when it cannot be had.  Host-to-device copies of small per-call arrays
+// go through it: a copy from pageable memory may first synchronise the stream (to stage
+// the data), which leaves the GPU idle until the call has launched its first kernel.  The
+// buffer may be rewritten by the thread's next call, so a caller only uses it for copies
+// that its own stream synchronisation has completed before it returns.
+void* host_staging(size_t bytes);
+
 // Enqueues on s: out[0] = *total, out[1] = err ? *err : 0, out[2] = extra ? *extra : 0 (out: a
 // Mailbox's dev pointer).
 cudaError_t post_counts(const long long* total, const int* err, const int* extra, long long* out, cudaStream_t s);

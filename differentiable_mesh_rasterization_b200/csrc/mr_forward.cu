@@ -61,7 +61,9 @@ int rasterize_impl(const float* verts, int64_t V, const int64_t* faces, int64_t 
     long long total = 0;
     int herr = 0, empty = 0;
     const Mailbox mb = host_mailbox();
-    cudaError_t e = fwd_enqueue_count(P, B, verts, faces, prefix.data(), first, s, &total, &herr, &empty, mb.dev);
+    int64_t* staging = static_cast<int64_t*>(host_staging(sizeof(int64_t) * (2 * (size_t)N + 1)));
+    cudaError_t e = fwd_enqueue_count(P, B, verts, faces, prefix.data(), first, s, &total, &herr, &empty, mb.dev,
+                                      staging);
     if (e != cudaSuccess) return finish(cuda_fail(e, "forward: face setup and binning"));
     if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return finish(cuda_fail(e, "cudaStreamSynchronize"));
     if (mb.dev) {

@@ -451,12 +451,19 @@ int mr_rasterize_points_fwd(const float* points, int64_t P, const int64_t* cloud
     int* offsets = reinterpret_cast<int*>(base + up(sz_cl) + up(sz_cnt));
     long long* tile = reinterpret_cast<long long*>(base + up(sz_cl) + up(sz_cnt) + up(sz_off));
     long long* total_d = tile + ntiles;
-    std::vector<int64_t> host(2 * (size_t)N);
-    std::copy(cloud_first_idx, cloud_first_idx + N, host.begin());
-    std::copy(num_points_per_cloud, num_points_per_cloud + N, host.begin() + N);
+    // the per-cloud arrays through pinned staging when it can be had (a copy from pageable
+    // memory may first wait for the stream); the synchronisation below completes the copy
+    std::vector<int64_t> host;
+    int64_t* hs = static_cast<int64_t*>(host_staging(sizeof(int64_t) * 2 * (size_t)N));
+    if (!hs) {
+        host.resize(2 * (size_t)N);
+        hs = host.data();
+    }
+    std::copy(cloud_first_idx, cloud_first_idx + N, hs);
+    std::copy(num_points_per_cloud, num_points_per_cloud + N, hs + N);
     int* list = nullptr;
     long long total = 0;
-    cudaError_t e = cudaMemcpyAsync(cl, host.data(), sz_cl, cudaMemcpyHostToDevice, s);
+    cudaError_t e = cudaMemcpyAsync(cl, hs, sz_cl, cudaMemcpyHostToDevice, s);
     const float r2 = radius * radius;
     const int gp = grid_for(std::max<int64_t>(P, 1));
     if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, sz_cnt, s);
