@@ -304,19 +304,7 @@ def shading_step_timing(mr, torch, dev, stream, batch, verts, faces, first, num,
             step()
         torch.cuda.synchronize(dev)
         steps = max(3, args.steps // 5)
-        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-        ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-        mr.profile_read()
-        mr.profile_enable(True)
-        for k in range(steps):
-            flush.zero_()
-            starts[k].record(stream)
-            step()
-            ends[k].record(stream)
-        torch.cuda.synchronize(dev)
-        mr.profile_enable(False)
-        st = mr.profile_read()
-        ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / steps
+        ms, st = _timed_and_staged(mr, torch, dev, stream, flush, steps, step)
         stages = {}
         for name, (t, n) in st.items():
             if n:
@@ -338,25 +326,36 @@ def shading_step_timing(mr, torch, dev, stream, batch, verts, faces, first, num,
     return out
 
 
-def _timed_steps(mr, torch, dev, stream, flush, steps, step):
-    """Warm-up, then ``steps`` timed calls of ``step`` (L2 flushed before each, CUDA events on
-    the launching stream, library stage timing on): (ms per step, stage dict)."""
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize(dev)
+def _timed_and_staged(mr, torch, dev, stream, flush, steps, step):
+    """``steps`` timed calls of ``step`` (L2 flushed before each, CUDA events on the launching
+    stream), then the same number again with the library's stage events on: (ms per step,
+    {stage: (ms, launches)} of the second pass)."""
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    mr.profile_read()
-    mr.profile_enable(True)
     for k in range(steps):
         flush.zero_()
         starts[k].record(stream)
         step()
         ends[k].record(stream)
     torch.cuda.synchronize(dev)
-    mr.profile_enable(False)
-    st = mr.profile_read()
     ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / steps
+    mr.profile_read()
+    mr.profile_enable(True)
+    for k in range(steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    mr.profile_enable(False)
+    return ms, mr.profile_read()
+
+
+def _timed_steps(mr, torch, dev, stream, flush, steps, step):
+    """Warm-up, then ``steps`` timed calls of ``step`` and a second pass for the library's
+    stage times (see _timed_and_staged): (ms per step, stage dict)."""
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    ms, st = _timed_and_staged(mr, torch, dev, stream, flush, steps, step)
     return ms, {name: t / steps for name, (t, n) in st.items() if n}
 
 
