@@ -321,8 +321,8 @@ __device__ __forceinline__ void topk_insert(unsigned (&kb)[KC], int (&ff)[KC], u
     ff[0] = c[0] ? fid : ff[0];
 }
 
-// One CTA per 16x16 bin; each of its eight warps owns an 8x4 pixel tile and runs on its
-// own (no block barriers).  A warp reads the bin's face list 32 ids at a time, tests
+// Two CTAs of four warps per 16x16 bin; each of the bin's eight warps owns an 8x4 pixel
+// tile and runs on its own (no block barriers).  A warp reads the bin's face list 32 ids at a time, tests
 // each face's pixel box against its tile, compacts the hits with a ballot and copies
 // their constants into its shared-memory slots.  For each staged face the warp first
 // evaluates the depth key alone; if no lane could admit the face into its top-K (face
@@ -330,17 +330,18 @@ __device__ __forceinline__ void topk_insert(unsigned (&kb)[KC], int (&ff)[KC], u
 // every lane runs the full candidacy test.  EXACT: the pixel centres are exact float32
 // values (H and W powers of two), so the float-float low parts vanish.
 template <int KC, bool PERSP, bool EXACT>
-__global__ void __launch_bounds__(kFineThreads, KC <= 4 ? 6 : 4)
+__global__ void __launch_bounds__(kFineThreads, (KC <= 4 ? 6 : 4) * kFineCtasPerBin)
 k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const int* __restrict__ offsets,
        const int* __restrict__ list, const int* __restrict__ order, int nbx, int nby, int H, int W, int K, float blur,
        bool vec, int64_t* __restrict__ p2f) {
-    __shared__ __align__(16) float4 s_c[kWarpsPerBin][32][kConstF4];
+    __shared__ __align__(16) float4 s_c[kFineWarps][32][kConstF4];
 
-    const int bin = order[blockIdx.x];
+    const int bin = order[blockIdx.x / kFineCtasPerBin];
     const int bxi = bin % nbx;
     const int byi = (bin / nbx) % nby;
     const int n = bin / (nbx * nby);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int lwarp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = (blockIdx.x % kFineCtasPerBin) * kFineWarps + lwarp;   // the warp tile within the bin
     const int tj0 = bxi * kBin + (warp & 1) * kWarpTileW;
     const int ti0 = byi * kBin + (warp >> 1) * kWarpTileH;
     if (tj0 >= W || ti0 >= H) return;                        // tile entirely off the image
@@ -362,7 +363,7 @@ k_fine(const float4* __restrict__ fconst, const FaceBox* __restrict__ box, const
     }
 
     const int beg = offsets[bin * kDepthBuckets], cnt = offsets[(bin + 1) * kDepthBuckets] - beg;
-    float4(*slots)[kConstF4] = s_c[warp];
+    float4(*slots)[kConstF4] = s_c[lwarp];
     // the next batch's face id and box are loaded while the current batch is tested
     int nfid = 0;
     FaceBox nbox = {1, 0, 1, 0, 0.f, 0};
@@ -620,9 +621,9 @@ template <int KC>
 void launch_fine(bool persp, bool exact, int nbins, cudaStream_t s, const float4* fconst, const FaceBox* box,
                  const int* order, const int* offsets, const int* list, int nbx, int nby, int H, int W, int K,
                  float blur, bool vec, int64_t* p2f) {
-#define MR_FINE(P, E) \
-    k_fine<KC, P, E><<<nbins, kFineThreads, 0, s>>>(fconst, box, offsets, list, order, nbx, nby, H, W, K, blur, vec, \
-                                                     p2f)
+#define MR_FINE(P, E)                                                                                          \
+    k_fine<KC, P, E><<<nbins * kFineCtasPerBin, kFineThreads, 0, s>>>(fconst, box, offsets, list, order, nbx, nby, \
+                                                                       H, W, K, blur, vec, p2f)
     if (persp) {
         if (exact) MR_FINE(true, true); else MR_FINE(true, false);
     } else {
