@@ -154,7 +154,8 @@ template <int KC>
 __global__ void __launch_bounds__(256, KC <= 8 ? 5 : 1) k_point_fine(const float* __restrict__ pts, const int* __restrict__ offsets,
                                                     const int* __restrict__ list, int H, int W, float r, float r2,
                                                     int K, int nbx, int nby, int64_t* __restrict__ idx,
-                                                    float* __restrict__ zbuf, float* __restrict__ dists, bool vec) {
+                                                    float* __restrict__ zbuf, float* __restrict__ dists, bool vec,
+                                                    double inv_w, double inv_h) {
     __shared__ float4 sp[256];
     __shared__ unsigned char smask[256];          // bit w: the point's box meets warp w's tile
     __shared__ unsigned char wl[8][256];          // per warp: its staged points, compacted
@@ -164,10 +165,6 @@ __global__ void __launch_bounds__(256, KC <= 8 ? 5 : 1) k_point_fine(const float
     // 2 x 16 rows, so fewer warps run the insertion for it)
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int i = by * kPtBin + (w >> 1) * 4 + (lane >> 3), j = bx * kPtBin + (w & 1) * 8 + (lane & 7);
-    // pixel centre as a float pair (hi + lo): the offset to a point is then exact to ~1e-15
-    const double pxd = -1.0 + (2.0 * j + 1.0) / W, pyd = 1.0 - (2.0 * i + 1.0) / H;
-    const float pxh = (float)pxd, pyh = (float)pyd;
-    const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
     unsigned long long kk[KC];
     float kd[KC];
 #pragma unroll
@@ -175,8 +172,17 @@ __global__ void __launch_bounds__(256, KC <= 8 ? 5 : 1) k_point_fine(const float
         kk[k] = kEmpty;
         kd[k] = -1.f;
     }
-    const unsigned lt_mask = (1u << lane) - 1u;
     const int beg = offsets[b], end = offsets[b + 1];
+    if (beg == end) {                             // an empty bin (the whole CTA): padding only
+        if (i < H && j < W)
+            write_point_slots<KC>(kk, kd, K, (((int64_t)n * H + i) * W + j) * K, vec, idx, zbuf, dists);
+        return;
+    }
+    // pixel centre as a float pair (hi + lo): the offset to a point is then exact to ~1e-15
+    const double pxd = pixel_x(j, W, inv_w), pyd = pixel_y(i, H, inv_h);
+    const float pxh = (float)pxd, pyh = (float)pyd;
+    const float pxl = (float)(pxd - (double)pxh), pyl = (float)(pyd - (double)pyh);
+    const unsigned lt_mask = (1u << lane) - 1u;
     for (int c0 = beg; c0 < end; c0 += 256) {
         __syncthreads();
         unsigned mask = 0;
@@ -509,7 +515,8 @@ int mr_rasterize_points_fwd(const float* points, int64_t P, const int64_t* cloud
                          (reinterpret_cast<uintptr_t>(dists) & 15) == 0;
         ProfScope ps(MR_STAGE_POINTS_FINE, s);
 #define MR_PF(KC) \
-    k_point_fine<KC><<<nbins, 256, 0, s>>>(points, offsets, list, H, W, radius, r2, K, nbx, nby, idx, zbuf, dists, vec)
+    k_point_fine<KC><<<nbins, 256, 0, s>>>(points, offsets, list, H, W, radius, r2, K, nbx, nby, idx, zbuf, dists, vec, \
+                                           1.0 / W, 1.0 / H)
         if (K <= 1) MR_PF(1);
         else if (K <= 2) MR_PF(2);
         else if (K <= 4) MR_PF(4);
