@@ -329,9 +329,12 @@ __global__ void __launch_bounds__(kKnnQueries) k_knn(const float4* __restrict__ 
                     unpack2(dhi, d4[2], d4[3]);
                     const int4 id4 = *reinterpret_cast<const int4*>(&wid[warp][t]);
                     const int ids[4] = {id4.x, id4.y, id4.z, id4.w};
+                    // a float compare with the K-th distance screens first (distances >= 0 order
+                    // like their bits; the 64-bit key then settles an equal distance by id)
+                    const float dlast = key_dist(kk[KC - 1]);
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
-                        if (t + u < cnt) {
+                        if (t + u < cnt && d4[u] <= dlast) {
                             const unsigned long long key = nn_key(d4[u], ids[u]);
                             if (key < kk[KC - 1]) insert_nn<KC>(kk, key);
                         }
