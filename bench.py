@@ -666,13 +666,15 @@ def main():
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def run(v, f, g):
+    def run(v, f, g, before_backward=None):
         """One step on device inputs; returns the results a caller reads back: alpha and
         grad_verts, or the depth buffer of a forward-only (hard) workload."""
         if hard:
             return (mr.rasterize_fwd(v, f, first, num, w.H, w.W, w.blur_radius, w.K, w.perspective_correct)[1],)
         p2f, zbuf, bary, dists, alpha = mr.rasterize_fwd(v, f, first, num, w.H, w.W, w.blur_radius, w.K,
                                                          w.perspective_correct, sigma=w.sigma)
+        if before_backward is not None:
+            before_backward()
         return alpha, mr.silhouette_rasterize_bwd(v, f, p2f, dists, w.sigma, g)
 
     def step():
@@ -755,15 +757,17 @@ def main():
         """The same steps with the host-to-device copy of step k+1 on one copy stream and the
         device-to-host copy of step k on another (one copy engine each way), overlapping the
         compute of step k (double-buffered device inputs; events order every copy against
-        the compute that uses it).  Timed from before the first input copy to after the last
-        result copy."""
+        the compute that uses it: a step's forward waits for its verts and faces, its
+        backward also for its dL/dalpha, which is copied last).  Timed from before the first
+        input copy to after the last result copy."""
         cs = torch.cuda.Stream(device=dev)
         ds = torch.cuda.Stream(device=dev)
         # device inputs allocated once (two sets), so no allocation sits between the streams
         bufs = [(torch.empty_like(h_verts, device=dev), torch.empty_like(h_faces, device=dev),
                  torch.empty_like(h_ga, device=dev)) for _ in range(2)]
         torch.cuda.synchronize(dev)
-        h2d_done = [torch.cuda.Event(), torch.cuda.Event()]
+        geo_done = [torch.cuda.Event(), torch.cuda.Event()]     # verts and faces of a step arrived
+        h2d_done = [torch.cuda.Event(), torch.cuda.Event()]     # and its dL/dalpha
         freed = [None, None]
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -773,8 +777,10 @@ def main():
             with torch.cuda.stream(cs):
                 if freed[i] is not None:
                     cs.wait_event(freed[i])
-                for dst, src in zip(bufs[i], (h_verts, h_faces, h_ga)):
+                for dst, src in zip(bufs[i][:2], (h_verts, h_faces)):
                     dst.copy_(src, non_blocking=True)
+                geo_done[i].record(cs)
+                bufs[i][2].copy_(h_ga, non_blocking=True)
                 h2d_done[i].record(cs)
 
         e0.record(cs)
@@ -783,10 +789,11 @@ def main():
             i = k % 2
             if k + 1 < n:
                 upload(k + 1)
-            stream.wait_event(h2d_done[i])
+            # the forward needs only the geometry; the backward waits for dL/dalpha as well
+            stream.wait_event(geo_done[i])
             dv, df, dg = bufs[i]
             flush.zero_()
-            res = run(dv, df, dg)
+            res = run(dv, df, dg, before_backward=lambda: stream.wait_event(h2d_done[i]))
             done = torch.cuda.Event()
             done.record(stream)
             freed[i] = done
@@ -873,7 +880,8 @@ def main():
                     "serial_ms_per_step": float(te[1]) / max(args.e2e_steps, 1),
                     "note": ("pinned host verts, faces in; the depth buffer out" if hard else
                              "pinned host verts, faces, dL/dalpha in; alpha and grad_verts out") + "; the copies of "
-                            "step k+1 (in) and step k (out) overlap the compute of step k on two copy streams"},
+                            "step k+1 (in) and step k (out) overlap the compute of step k on two copy streams; a "
+                            "step's forward waits for its geometry, its backward for its dL/dalpha"},
             "memory": memory,
             "gpu_launches": int(sum(v[1] * KERNELS_PER_STAGE.get(k, 1) for k, v in stages.items())),
             "clocks": clk}
