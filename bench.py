@@ -789,17 +789,26 @@ def main():
             i = k % 2
             if k + 1 < n:
                 upload(k + 1)
-            # the forward needs only the geometry; the backward waits for dL/dalpha as well
+            # the forward needs only the geometry; the backward waits for dL/dalpha as well;
+            # alpha is final once the forward is done and goes out while the backward runs
             stream.wait_event(geo_done[i])
             dv, df, dg = bufs[i]
             flush.zero_()
-            res = run(dv, df, dg, before_backward=lambda: stream.wait_event(h2d_done[i]))
+            fwd_done = []
+
+            def between():
+                ev = torch.cuda.Event()
+                ev.record(stream)
+                fwd_done.append(ev)
+                stream.wait_event(h2d_done[i])
+
+            res = run(dv, df, dg, before_backward=between)
             done = torch.cuda.Event()
             done.record(stream)
             freed[i] = done
             with torch.cuda.stream(ds):
-                ds.wait_event(done)
-                for h, d in zip(h_res, res):
+                for j, (h, d) in enumerate(zip(h_res, res)):
+                    ds.wait_event(fwd_done[0] if j == 0 and fwd_done else done)
                     d.record_stream(ds)
                     h.copy_(d, non_blocking=True)
         e1.record(ds)
