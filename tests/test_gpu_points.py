@@ -83,6 +83,28 @@ def test_point_rasterizer_edge_cases(oracle_mod):
 
 
 
+@pytest.mark.parametrize("H,W,K", [(64, 64, 8), (40, 72, 4), (37, 53, 3)])
+def test_point_outputs_are_fully_written(H, W, K):
+    """Outputs pre-filled with a sentinel: a few points leave most 16 x 16 bins empty (those
+    write their padding before any pixel arithmetic); every element is written and equals
+    a call into fresh buffers."""
+    rng = np.random.default_rng(5)
+    pts = np.concatenate([rng.uniform(-0.15, 0.15, (40, 2)), rng.uniform(1.0, 3.0, (40, 1))], 1).astype(np.float32)
+    p = torch.from_numpy(pts).cuda()
+    ref = mr.rasterize_points_fwd(p, [0], [40], H, W, 0.05, K)
+    idx = torch.full((1, H, W, K), 987654, dtype=torch.int64, device="cuda")
+    zbuf, dists = (torch.full((1, H, W, K), 7.5, device="cuda") for _ in range(2))
+    first, num = np.array([0], np.int64), np.array([40], np.int64)
+    rc = mr.load_library().mr_rasterize_points_fwd(p.data_ptr(), 40, first.ctypes.data, num.ctypes.data, 1, H, W,
+                                                   0.05, K, idx.data_ptr(), zbuf.data_ptr(), dists.data_ptr(),
+                                                   torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert rc == 0
+    for got, want in zip((idx, zbuf, dists), ref):
+        assert torch.equal(got, want)
+    assert (ref[0] >= 0).any() and (ref[0][..., 0] == -1).float().mean() > 0.5
+
+
 def test_point_at_exactly_the_radius_is_kept(oracle_mod):
     """Dyadic point and radius (two pixel pitches): the squared distance ties r^2 exactly in
     float32 too, and the threshold is inclusive on both sides."""
