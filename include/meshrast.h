@@ -83,7 +83,9 @@ extern "C" {
  * thread's first call for the current device and kept for the life of the thread; that
  * read-back uses no copy engine, so it does not wait behind the caller's own transfers
  * (where the mapped memory cannot be had, it falls back to a device-to-host copy on
- * `stream`).  Returns MR_ERR_DEVICE if a face referenced a vertex outside [0, V) (that
+ * `stream`).  The per-mesh arrays go to the device through a pinned host buffer of the
+ * same lifetime (2N + 1 int64, grown when a call needs more), so that their copy does not
+ * first wait for the stream's earlier work.  Returns MR_ERR_DEVICE if a face referenced a vertex outside [0, V) (that
  * face is then ignored).
  */
 int mr_rasterize_fwd(const float* verts, int64_t V, const int64_t* faces, int64_t F,
