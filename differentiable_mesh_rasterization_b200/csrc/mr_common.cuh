@@ -106,9 +106,9 @@ int cuda_fail(cudaError_t e, const char* what);
 int host_indices(cudaStream_t s, int64_t n, std::vector<int64_t>& buf,
                  std::initializer_list<const int64_t**> arrays);
 
-// A mapped (zero-copy) pinned host buffer of two 64-bit words, one per calling thread and
-// device: the values a call reads back in the middle (a list total, the device error
-// word) are written there by a kernel, so reading them needs no copy engine -- a copy
+// A mapped (zero-copy) pinned host buffer of 64 bytes (three 64-bit words in use), one per
+// calling thread and device: the values a call reads back in the middle (a list total, the
+// device error word, a count) are written there by a kernel, so reading them needs no copy engine -- a copy
 // would queue behind the caller's own large transfers on that engine.  dev is nullptr when
 // no such buffer can be had; the caller then copies instead.
 struct Mailbox {

@@ -8,19 +8,23 @@
 //                lower bound of the depth key over the box, the face's plane constants
 //                for the fine pass (float64, rounded once), and the image's key range.
 //   bin count    one thread per pair: count the 16x16 screen bins the box touches, per
-//                depth bucket of the face within its image (warp-aggregated atomics).
-//   bin scan     exclusive scan of the per-(bin, bucket) counts -> list offsets, total.
-//   (host)       one stream synchronisation to size the face lists.
+//                depth bucket of the face within its image (one atomic per run of equal
+//                slots in neighbouring lanes).
+//   bin scan     exclusive scan of the per-(bin, bucket) counts -> list offsets, total;
+//                the bins' longest-first order and the number of empty bins.
+//   (host)       one stream synchronisation to size the face lists (the total, the error
+//                word and the empty-bin count come back through mapped host memory).
 //   bin fill     second pass of the pair loop: scatter face ids into the bin lists, so
 //                each bin's list runs from its nearest depth bucket to its farthest.
-//   fine         one CTA per bin, eight independent warps (8x4 pixel tiles): ballot-
-//                compacted per-warp face lists staged in shared memory, a warp-wide
-//                depth pre-test, the full candidacy test, and a register-resident
-//                insertion-sorted top-K per pixel; writes the K winning face ids
+//   fine         two CTAs of four warps per non-empty bin, eight independent warps in all
+//                (8x4 pixel tiles): ballot-compacted per-warp face lists staged in shared
+//                memory, a warp-wide depth pre-test, the full candidacy test, and a
+//                register-resident sorted top-K per pixel; writes the K winning face ids
 //                straight into pix_to_face.
 //   epilogue     one thread per pixel: barycentrics, z and signed squared distance of
 //                the K winners recomputed in float64 from the original vertices, the
-//                fused soft silhouette, 16-byte stores.
+//                fused soft silhouette, 16-byte stores; the pixels of empty bins get their
+//                padding (pix_to_face included) without reads.
 #include "mr_forward_kernels.cuh"
 
 namespace mr {
