@@ -756,24 +756,26 @@ def main():
     def e2e_pipelined(n):
         """The same steps with the host-to-device copy of step k+1 on one copy stream and the
         device-to-host copy of step k on another (one copy engine each way), overlapping the
-        compute of step k (double-buffered device inputs; events order every copy against
+        compute of step k (triple-buffered device inputs; events order every copy against
         the compute that uses it: a step's forward waits for its verts and faces, its
         backward also for its dL/dalpha, which is copied last).  Timed from before the first
         input copy to after the last result copy."""
         cs = torch.cuda.Stream(device=dev)
         ds = torch.cuda.Stream(device=dev)
-        # device inputs allocated once (two sets), so no allocation sits between the streams
+        NBUF = 3
+        # device inputs allocated once (three sets, so a step's upload never waits for the
+        # compute just before it), so no allocation sits between the streams
         bufs = [(torch.empty_like(h_verts, device=dev), torch.empty_like(h_faces, device=dev),
-                 torch.empty_like(h_ga, device=dev)) for _ in range(2)]
+                 torch.empty_like(h_ga, device=dev)) for _ in range(NBUF)]
         torch.cuda.synchronize(dev)
-        geo_done = [torch.cuda.Event(), torch.cuda.Event()]     # verts and faces of a step arrived
-        h2d_done = [torch.cuda.Event(), torch.cuda.Event()]     # and its dL/dalpha
-        freed = [None, None]
+        geo_done = [torch.cuda.Event() for _ in range(NBUF)]     # verts and faces of a step arrived
+        h2d_done = [torch.cuda.Event() for _ in range(NBUF)]     # and its dL/dalpha
+        freed = [None] * NBUF
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
 
         def upload(k):
-            i = k % 2
+            i = k % NBUF
             with torch.cuda.stream(cs):
                 if freed[i] is not None:
                     cs.wait_event(freed[i])
@@ -786,7 +788,7 @@ def main():
         e0.record(cs)
         upload(0)
         for k in range(n):
-            i = k % 2
+            i = k % NBUF
             if k + 1 < n:
                 upload(k + 1)
             # the forward needs only the geometry; the backward waits for dL/dalpha as well;
