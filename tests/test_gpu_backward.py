@@ -143,6 +143,36 @@ def test_end_to_end_full_batch5_whole_images(oracle_mod):
                   label="batch5 alpha")
 
 
+@pytest.mark.parametrize("hw", [200, 256])
+def test_fused_backward_vector_and_scalar_loads(oracle_mod, hw):
+    """With K = 4 the fused backward reads each pixel's ids and distances in 16-byte loads
+    when both arrays start on a 16-byte boundary, one by one otherwise. Both forms agree
+    (up to the order of the atomics) and match the oracle's backward on the same fragments,
+    with H, W a power of two (exact pixel centres) and not."""
+    b = syn.make_batch(5, n_meshes=2)
+    w = b.workload
+    sigma = np.float32(w.sigma)
+    v, f = cuda(b.verts), cuda(b.faces)
+    p2f, _, _, dists, _ = mr.rasterize_fwd(v, f, b.mesh_to_face_first_idx, b.num_faces_per_mesh, hw, hw,
+                                           w.blur_radius, 4, sigma=float(sigma))
+    assert (p2f >= 0).sum().item() > 1000
+    ga = np.random.default_rng(hw).normal(size=(b.N, hw, hw)).astype(np.float32)
+    assert p2f.data_ptr() % 16 == 0 and dists.data_ptr() % 16 == 0
+    got = mr.silhouette_rasterize_bwd(v, f, p2f, dists, float(sigma), cuda(ga))
+    # the same contiguous arrays, 8 (ids) and 4 (distances) bytes past a 16-byte boundary
+    p2f_u = torch.empty(p2f.numel() + 1, dtype=torch.int64, device="cuda")[1:].view(p2f.shape)
+    d_u = torch.empty(dists.numel() + 1, dtype=torch.float32, device="cuda")[1:].view(dists.shape)
+    p2f_u.copy_(p2f)
+    d_u.copy_(dists)
+    assert p2f_u.data_ptr() % 16 == 8 and d_u.data_ptr() % 16 == 4
+    got_u = mr.silhouette_rasterize_bwd(v, f, p2f_u, d_u, float(sigma), cuda(ga))
+    diff = ((got - got_u).norm() / got.norm()).item()
+    assert diff < 1e-5, diff
+    want = _oracle_chain(oracle_mod, b, np_(p2f), np_(dists).astype(np.float64), ga, sigma)
+    assert compare_grad(got, want, label=f"fused bwd 16-byte loads {hw}px") < 1e-4
+    assert compare_grad(got_u, want, label=f"fused bwd scalar loads {hw}px") < 1e-4
+
+
 def test_backward_rejects_bad_slots():
     v = cuda(np.array([[-0.5, -0.5, 2.0], [0.5, -0.5, 2.0], [0.0, 0.5, 2.0]], np.float32))
     f = cuda(np.array([[0, 1, 2]], np.int64))
