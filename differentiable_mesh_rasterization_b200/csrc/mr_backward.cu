@@ -13,9 +13,9 @@
 //   squared distance to the nearest edge u -> v at q = u + t (v - u):
 //       dd2/du = -2 (p - q)(1 - t),  dd2/dv = -2 (p - q) t;   dist = -d2 inside, +d2 outside.
 //
-// Contributions are scattered with float32 atomics (red.global.add): the general kernel
-// adds into grad_verts (zeroed first); the fused silhouette kernel adds (x, y) pairs into
-// a float2 accumulator that a final pass copies to grad_verts.
+// Contributions are scattered with float32 vector atomics (red.global.add): the general
+// kernel adds (x, y, z, 0) rows into a float4 accumulator, the fused silhouette kernel
+// (x, y) pairs into a float2 one; a final pass copies either to grad_verts.
 #include <algorithm>
 #include <cfloat>
 #include <cmath>
