@@ -836,8 +836,8 @@ def main():
     d2h = sum(h.numel() * 4 for h in h_res)
 
     # roofline of the dominant kernel (the fine pass: the pixel-face tests) and of the
-    # epilogue (which writes the per-slot outputs)
-    # per step: the fine pass and the epilogue run as several chunk launches each
+    # epilogue (which writes the per-slot outputs); the stage times and launch counts are
+    # totals over the steps of the second pass
     fine_ms, fine_n = stages["fine"]
     fine_s = fine_ms / 1e3 / args.steps
     epi_ms, epi_n = stages["epilogue"]
