@@ -129,6 +129,7 @@ def test_extreme_aspect_ratios(oracle_mod, H, W):
     assert info["valid_slots"] > 100
     compare_alpha(g[4], alpha_of(oracle_mod, info, 1e-4), label=f"{H}x{W} alpha")
 
+
 def test_no_faces_at_all():
     v = torch.zeros((0, 3), device="cuda")
     f = torch.zeros((0, 3), dtype=torch.int64, device="cuda")
