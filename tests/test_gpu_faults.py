@@ -6,7 +6,6 @@ with its message, that the scratch it had already taken is released (the default
 used bytes return to their level before the call), and that the next call succeeds and
 matches a clean run.
 """
-import numpy as np
 import pytest
 import torch
 

@@ -6,7 +6,6 @@ triangle, ray-plane intersection depths in 3-D, exact translation / permutation 
 batching invariants, finite differences of its own forward (for the backward), and
 the sigmoid closed forms of the blur radius used by the benchmark batches.
 """
-import math
 
 import numpy as np
 import pytest
